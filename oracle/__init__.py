@@ -1,0 +1,159 @@
+"""fp64 CPU oracle for paged attention (test infrastructure only).
+
+Only ``tests/``, ``__graft_entry__.smoke()`` and the ``cpu_baseline`` /
+``--impl reference`` legs of ``bench.py`` may import this package.  The
+product library (``scatter_kv_b200``) never imports it, and this package
+imports nothing from there.
+
+The arithmetic lives in ``pa_oracle.c`` (plain C, fp64); this module only
+compiles it with gcc, loads it with ctypes and marshals numpy arrays.  See
+that file's header for the definitions it follows (FlexAttention operator
+doc, "FlexAttention Computation" and "Grouped Query Attention (GQA)"; ONNX
+Runtime PR "[WebGPU] Initial PagedAttention implementation (1/n)", section
+"FlashAttention: optional seqlens_q input").
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import subprocess
+
+import numpy as np
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+_SRC = os.path.join(_HERE, "pa_oracle.c")
+_LIB = os.path.join(_HERE, "libpa_oracle.so")
+_lib = None
+
+F16 = 0
+F64 = 1
+
+
+def build(force: bool = False) -> str:
+    """Compile pa_oracle.c into libpa_oracle.so (gcc, -O2, OpenMP)."""
+    if force or not os.path.exists(_LIB) or os.path.getmtime(_LIB) < os.path.getmtime(_SRC):
+        tmp = _LIB + f".tmp{os.getpid()}"
+        subprocess.check_call(["gcc", "-O2", "-fopenmp", "-fPIC", "-shared", "-std=c11",
+                               "-o", tmp, _SRC, "-lm"])
+        os.replace(tmp, _LIB)
+    return _LIB
+
+
+def _load():
+    global _lib
+    if _lib is None:
+        lib = ctypes.CDLL(build())
+        P = ctypes.c_void_p
+        i32, i64 = ctypes.c_int32, ctypes.c_int64
+        lib.oracle_half_to_double.argtypes = [ctypes.c_uint16]
+        lib.oracle_half_to_double.restype = ctypes.c_double
+        lib.oracle_scatter_kv.argtypes = [P, P, P, P, P, i64, ctypes.c_int, ctypes.c_int,
+                                          ctypes.c_int, ctypes.c_int]
+        lib.oracle_slot_mapping.argtypes = [P, P, P, ctypes.c_int, ctypes.c_int, ctypes.c_int,
+                                            i64, P]
+        lib.oracle_kv_slots.argtypes = [P, P, ctypes.c_int, ctypes.c_int, ctypes.c_int, P]
+        lib.oracle_kv_slots.restype = i64
+        lib.oracle_attention.argtypes = [P, P, P, P, P, P, ctypes.c_int, i64, ctypes.c_int,
+                                         ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_int,
+                                         ctypes.c_double, ctypes.c_int, ctypes.c_int, P, i64,
+                                         P, i64, P]
+        lib.oracle_max_threads.restype = ctypes.c_int
+        _lib = lib
+    return _lib
+
+
+def _ptr(a: np.ndarray):
+    return a.ctypes.data_as(ctypes.c_void_p)
+
+
+def _c(a, dtype):
+    return np.ascontiguousarray(a, dtype=dtype)
+
+
+def max_threads() -> int:
+    """Threads the oracle's OpenMP loop uses (OMP_NUM_THREADS, else all cores)."""
+    return int(_load().oracle_max_threads())
+
+
+def half_to_double(bits: int) -> float:
+    return float(_load().oracle_half_to_double(int(bits) & 0xFFFF))
+
+
+def scatter_kv(key, value, slot_mapping, key_cache, value_cache) -> None:
+    """In place: key_cache[slot // bs, slot % bs] = key[t] (and value), slot >= 0."""
+    lib = _load()
+    assert key_cache.flags.c_contiguous and value_cache.flags.c_contiguous
+    assert key_cache.dtype == key.dtype == value.dtype == value_cache.dtype
+    key = _c(key, key.dtype)
+    value = _c(value, value.dtype)
+    slots = _c(slot_mapping, np.int32)
+    nb, bs, kvh, d = key_cache.shape
+    lib.oracle_scatter_kv(_ptr(key), _ptr(value), _ptr(slots), _ptr(key_cache), _ptr(value_cache),
+                          key.shape[0], kvh, d, bs, key.dtype.itemsize)
+
+
+def slot_mapping(block_table, cu_seqlens_q, seqlens_kv, block_size: int) -> np.ndarray:
+    lib = _load()
+    bt = _c(block_table, np.int32)
+    cu = _c(cu_seqlens_q, np.int32)
+    skv = _c(seqlens_kv, np.int32)
+    token_count = int(cu[-1])
+    out = np.empty(token_count, dtype=np.int32)
+    lib.oracle_slot_mapping(_ptr(bt), _ptr(cu), _ptr(skv), len(skv), bt.shape[1], block_size,
+                            token_count, _ptr(out))
+    return out
+
+
+def kv_slots(block_table, seqlens_kv, block_size: int) -> np.ndarray:
+    """Slots of logical positions [0, seqlens_kv[b]) for every sequence b."""
+    lib = _load()
+    bt = _c(block_table, np.int32)
+    skv = _c(seqlens_kv, np.int32)
+    out = np.empty(int(skv.astype(np.int64).sum()), dtype=np.int32)
+    n = lib.oracle_kv_slots(_ptr(bt), _ptr(skv), len(skv), bt.shape[1], block_size, _ptr(out))
+    assert n == out.size
+    return out
+
+
+def attention(query, key_cache, value_cache, block_table, cu_seqlens_q, seqlens_kv,
+              scale: float, causal: bool = True, rows=None) -> np.ndarray:
+    """fp64 paged attention.
+
+    query [token_count, q_heads, head_size]; caches [num_blocks, block_size,
+    kv_heads, head_size]; all float16 or all float64.  ``rows``: optional
+    int64 [n, 2] array of (token, q_head) pairs to compute; the result is
+    then [n, head_size], else [token_count, q_heads, head_size] (float64).
+    """
+    lib = _load()
+    if query.dtype == np.float16:
+        dtype = F16
+    elif query.dtype == np.float64:
+        dtype = F64
+    else:
+        raise TypeError("oracle takes float16 or float64 arrays")
+    assert key_cache.dtype == value_cache.dtype == query.dtype
+    q = _c(query, query.dtype)
+    kc = key_cache if key_cache.flags.c_contiguous else np.ascontiguousarray(key_cache)
+    vc = value_cache if value_cache.flags.c_contiguous else np.ascontiguousarray(value_cache)
+    bt = _c(block_table, np.int32)
+    cu = _c(cu_seqlens_q, np.int32)
+    skv = _c(seqlens_kv, np.int32)
+    token_count, q_heads, head_size = q.shape
+    nb, bs, kv_heads, d2 = kc.shape
+    assert d2 == head_size
+    max_keys = max(1, int(skv.max()) if skv.size else 1)
+    nthreads = max_threads()
+    scratch = np.empty(nthreads * max_keys, dtype=np.float64)
+    if rows is None:
+        out = np.empty((token_count, q_heads, head_size), dtype=np.float64)
+        rows_p, nrows = None, token_count * q_heads
+    else:
+        rows = _c(rows, np.int64).reshape(-1, 2)
+        out = np.empty((rows.shape[0], head_size), dtype=np.float64)
+        rows_p, nrows = _ptr(rows), rows.shape[0]
+    if nrows:
+        lib.oracle_attention(_ptr(q), _ptr(kc), _ptr(vc), _ptr(bt), _ptr(cu), _ptr(skv), len(skv),
+                             token_count, q_heads, kv_heads, head_size, bs, bt.shape[1],
+                             float(scale), 1 if causal else 0, dtype, rows_p, nrows,
+                             _ptr(scratch), max_keys, _ptr(out))
+    return out

@@ -1,0 +1,223 @@
+/*
+ * pa_oracle.c -- plain, slow, fp64 CPU oracle for paged attention with a
+ * block-table KV cache (continuous batching).
+ *
+ * TEST INFRASTRUCTURE ONLY.  Only the test suite, the smoke check and the
+ * CPU-baseline leg of the benchmark may load this file's library.  It shares
+ * no code, header, table or helper with the CUDA library under
+ * scatter_kv_b200/, and it includes nothing from there.
+ *
+ * What it computes, and where that is defined:
+ *
+ *  - Attention.  FlexAttention operator doc (ONNX ai.onnx.preview),
+ *    "FlexAttention Computation":  Scores = (Q @ K^T) * scale;
+ *    Probs = Softmax(Scores, axis=-1);  Y = Probs @ V.
+ *    Same doc, "Grouped Query Attention (GQA)": query head h reads K/V head
+ *    floor(h / group_size), group_size = q_num_heads / kv_num_heads.
+ *    Same doc, "Modifier Subgraphs": masking writes -inf into masked scores;
+ *    here a masked key is simply left out of the sum, which is the same
+ *    thing in exact arithmetic (exp(-inf) = 0).
+ *
+ *  - Causal bound under continuous batching.  ONNX Runtime PR "[WebGPU]
+ *    Initial PagedAttention implementation (1/n)", section "FlashAttention:
+ *    optional seqlens_q input": past_len_b = total_kv_b - seqlens_q[b]; and
+ *    the review's list "Things I specifically checked": query i of sequence
+ *    b sees seq_causal_length = past_len_b + i + 1 keys, i.e. logical key
+ *    positions [0, past_len_b + i].
+ *
+ *  - Paged cache addressing (the same PR, "Description": scatter K/V into
+ *    the paged cache; review: "scatter block addressing").  Logical key
+ *    position j of sequence b lives in physical block block_table[b][j / bs]
+ *    at row j % bs; a cache is [num_blocks, block_size, kv_heads, head_size].
+ *    A token's slot is block * block_size + row.
+ *
+ *  - Token -> sequence lookup for the slot mapping (review, "Things I
+ *    specifically checked"): the sequence of packed token t is the first b
+ *    with cu_seqlens_q[b+1] > t, which skips zero-length sequences.
+ *
+ * Arithmetic: every floating-point value is taken to fp64 exactly (binary16
+ * and binary32 are subsets of binary64) and all sums run in increasing key
+ * order, so the result does not depend on where pages sit in the pool.
+ * Scores use fp64 throughout; the maximum is subtracted before exp() as the
+ * textbook softmax does (it changes nothing in exact arithmetic).
+ *
+ * No validation: the oracle is only called on inputs the tests built to be
+ * valid.  OpenMP (when compiled with -fopenmp) splits the independent output
+ * rows across threads; it does not change any row's arithmetic.
+ */
+#include <math.h>
+#include <stdint.h>
+#include <string.h>
+
+#define ORACLE_F16 0
+#define ORACLE_F64 1
+
+/* IEEE 754 binary16 -> binary64, written from the format's definition:
+ * 1 sign bit, 5 exponent bits (bias 15), 10 fraction bits. */
+double oracle_half_to_double(uint16_t h)
+{
+    int sign = (h >> 15) & 1;
+    int e = (h >> 10) & 0x1f;
+    int f = h & 0x3ff;
+    double v;
+    if (e == 0) {
+        v = ldexp((double)f, -24);               /* zero / subnormal: f * 2^-24 */
+    } else if (e == 31) {
+        v = (f == 0) ? INFINITY : NAN;
+    } else {
+        v = ldexp((double)(1024 + f), e - 25);   /* (1 + f/1024) * 2^(e-15) */
+    }
+    return sign ? -v : v;
+}
+
+static double load(const void *base, int64_t idx, int dtype)
+{
+    if (dtype == ORACLE_F64) return ((const double *)base)[idx];
+    return oracle_half_to_double(((const uint16_t *)base)[idx]);
+}
+
+/* Scatter new K/V tokens into the paged caches.
+ * key/value: [token_count, kv_heads, head_size] elements of elem_bytes bytes.
+ * key_cache/value_cache: [num_blocks, block_size, kv_heads, head_size].
+ * slot_mapping[t] = block * block_size + row; a negative slot skips token t.
+ * A plain element copy: the result must match the GPU bit for bit. */
+void oracle_scatter_kv(const void *key, const void *value, const int32_t *slot_mapping,
+                       void *key_cache, void *value_cache, int64_t token_count,
+                       int kv_heads, int head_size, int block_size, int elem_bytes)
+{
+    int64_t row_bytes = (int64_t)kv_heads * head_size * elem_bytes;
+    for (int64_t t = 0; t < token_count; ++t) {
+        int32_t slot = slot_mapping[t];
+        if (slot < 0) continue;
+        int64_t block = slot / block_size;
+        int64_t row = slot % block_size;
+        int64_t dst = (block * block_size + row) * row_bytes;
+        memcpy((char *)key_cache + dst, (const char *)key + t * row_bytes, (size_t)row_bytes);
+        memcpy((char *)value_cache + dst, (const char *)value + t * row_bytes, (size_t)row_bytes);
+    }
+}
+
+/* Sequence of packed token t: the first b with cu_seqlens_q[b+1] > t. */
+static int seq_of_token(const int32_t *cu_seqlens_q, int batch, int64_t t)
+{
+    for (int b = 0; b < batch; ++b)
+        if (cu_seqlens_q[b + 1] > t) return b;
+    return -1;
+}
+
+/* Slot of each new token: token t of sequence b (local index i = t - cu[b])
+ * sits at logical position p = past_len_b + i, past_len_b = seqlens_kv[b] -
+ * q_len_b; its slot is block_table[b][p / bs] * bs + p % bs. */
+void oracle_slot_mapping(const int32_t *block_table, const int32_t *cu_seqlens_q,
+                         const int32_t *seqlens_kv, int batch, int max_blocks_per_seq,
+                         int block_size, int64_t token_count, int32_t *slot_mapping)
+{
+    for (int64_t t = 0; t < token_count; ++t) {
+        int b = seq_of_token(cu_seqlens_q, batch, t);
+        int64_t q_len = cu_seqlens_q[b + 1] - cu_seqlens_q[b];
+        int64_t past = seqlens_kv[b] - q_len;
+        int64_t p = past + (t - cu_seqlens_q[b]);
+        int64_t block = block_table[(int64_t)b * max_blocks_per_seq + p / block_size];
+        slot_mapping[t] = (int32_t)(block * block_size + p % block_size);
+    }
+}
+
+/* Slots holding logical positions [0, seqlens_kv[b]) of every sequence, in
+ * (b, position) order; returns how many were written.  The tests use it to
+ * find the cache rows attention may read (everything else may be poisoned). */
+int64_t oracle_kv_slots(const int32_t *block_table, const int32_t *seqlens_kv, int batch,
+                        int max_blocks_per_seq, int block_size, int32_t *slots)
+{
+    int64_t n = 0;
+    for (int b = 0; b < batch; ++b)
+        for (int64_t j = 0; j < seqlens_kv[b]; ++j) {
+            int64_t block = block_table[(int64_t)b * max_blocks_per_seq + j / block_size];
+            slots[n++] = (int32_t)(block * block_size + j % block_size);
+        }
+    return n;
+}
+
+/* One output row: packed token t (of sequence b, local index i) and query
+ * head h.  Writes head_size doubles to y. */
+static void attention_row(const void *query, const void *key_cache, const void *value_cache,
+                          const int32_t *block_table, const int32_t *cu_seqlens_q,
+                          const int32_t *seqlens_kv, int batch, int q_heads, int kv_heads,
+                          int head_size, int block_size, int max_blocks_per_seq, double scale,
+                          int causal, int dtype, int64_t t, int h, double *scores, double *y)
+{
+    int b = seq_of_token(cu_seqlens_q, batch, t);
+    int64_t q_len = cu_seqlens_q[b + 1] - cu_seqlens_q[b];
+    int64_t total = seqlens_kv[b];
+    int64_t past = total - q_len;
+    int64_t i = t - cu_seqlens_q[b];
+    int64_t nkeys = causal ? past + i + 1 : total;       /* keys [0, nkeys) */
+    int group = q_heads / kv_heads;
+    int kvh = h / group;
+    int64_t qbase = (t * q_heads + h) * (int64_t)head_size;
+
+    double m = -INFINITY;
+    for (int64_t j = 0; j < nkeys; ++j) {
+        int64_t block = block_table[(int64_t)b * max_blocks_per_seq + j / block_size];
+        int64_t kbase = ((block * block_size + j % block_size) * kv_heads + kvh) * (int64_t)head_size;
+        double s = 0.0;
+        for (int d = 0; d < head_size; ++d)
+            s += load(query, qbase + d, dtype) * load(key_cache, kbase + d, dtype);
+        s *= scale;
+        scores[j] = s;
+        if (s > m) m = s;
+    }
+    double denom = 0.0;
+    for (int d = 0; d < head_size; ++d) y[d] = 0.0;
+    for (int64_t j = 0; j < nkeys; ++j) {
+        double p = exp(scores[j] - m);
+        denom += p;
+        int64_t block = block_table[(int64_t)b * max_blocks_per_seq + j / block_size];
+        int64_t vbase = ((block * block_size + j % block_size) * kv_heads + kvh) * (int64_t)head_size;
+        for (int d = 0; d < head_size; ++d) y[d] += p * load(value_cache, vbase + d, dtype);
+    }
+    for (int d = 0; d < head_size; ++d) y[d] /= denom;
+}
+
+/* Attention rows.  query: [token_count, q_heads, head_size]; caches
+ * [num_blocks, block_size, kv_heads, head_size]; elements are binary16 bit
+ * patterns (dtype 0) or doubles (dtype 1).  rows: nrows (token, head) pairs
+ * as int64 [nrows, 2]; rows == NULL means every (token, head) in order.
+ * out: [nrows, head_size] doubles.  scratch: max_keys doubles per thread
+ * (callers pass max_keys >= the longest sequence).  causal = 0 attends to all
+ * seqlens_kv[b] keys (only used for the FlexAttention worked examples). */
+void oracle_attention(const void *query, const void *key_cache, const void *value_cache,
+                      const int32_t *block_table, const int32_t *cu_seqlens_q,
+                      const int32_t *seqlens_kv, int batch, int64_t token_count, int q_heads,
+                      int kv_heads, int head_size, int block_size, int max_blocks_per_seq,
+                      double scale, int causal, int dtype, const int64_t *rows, int64_t nrows,
+                      double *scratch, int64_t max_keys, double *out)
+{
+    if (rows == NULL) nrows = token_count * q_heads;
+#pragma omp parallel
+    {
+        int tid = 0;
+#ifdef _OPENMP
+        extern int omp_get_thread_num(void);
+        tid = omp_get_thread_num();
+#endif
+        double *scores = scratch + (int64_t)tid * max_keys;
+#pragma omp for schedule(dynamic, 1)
+        for (int64_t r = 0; r < nrows; ++r) {
+            int64_t t = rows ? rows[2 * r] : r / q_heads;
+            int h = rows ? (int)rows[2 * r + 1] : (int)(r % q_heads);
+            attention_row(query, key_cache, value_cache, block_table, cu_seqlens_q, seqlens_kv,
+                          batch, q_heads, kv_heads, head_size, block_size, max_blocks_per_seq,
+                          scale, causal, dtype, t, h, scores, out + r * head_size);
+        }
+    }
+}
+
+int oracle_max_threads(void)
+{
+#ifdef _OPENMP
+    extern int omp_get_max_threads(void);
+    return omp_get_max_threads();
+#else
+    return 1;
+#endif
+}
