@@ -1,0 +1,448 @@
+"""Benchmark of the paged-attention hot path on B200.
+
+One step = one pass of the whole path over one synthetic continuous batch:
+slot mapping, scatter of the new K/V into the paged cache, attention
+(split-KV decode + combine, and the tcgen05 prefill kernel when the batch has
+longer queries).  Default workload: the decode-heavy GQA batch (64 sequences,
+q_len 1, past U[512, 4096], 32/8 heads, head size 128, block size 16,
+20000-block pool); metric: algorithmic HBM bytes of the step per second.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME] [--impl reference]
+
+Multi-GPU (torchrun, one rank per GPU): the path does not shard inside one
+batch, so every rank runs its own replica of the workload; times are the max
+over ranks and ``value`` counts the bytes of all ranks (weak scaling).
+
+``--impl reference`` times the fp64 CPU oracle on this host's cores over a
+bounded sample of the same workload (there is no other implementation of
+this path to run).
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import math
+import os
+import re
+import subprocess
+import sys
+import threading
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+import workloads  # noqa: E402
+
+METRIC = "paged attn: decode KV GB/s & prefill TFLOP/s, % of B200 roofline"
+L2_BYTES = 126 * 1024 * 1024
+
+
+# ----------------------------------------------------------------- work counts
+
+def algorithmic_counts(spec: workloads.Spec) -> dict:
+    """Bytes and FLOPs the method must move / compute for one step.
+
+    attention bytes: every K/V row of a sequence read once per KV head, plus
+    Q read and O written; FLOPs: 4 * q_heads * d per visible (query, key)
+    pair, causal; scatter bytes: new K/V read and written, slots read."""
+    T = spec.seqlens_kv.astype(np.int64)
+    d, kvh, qh = spec.head_size, spec.kv_heads, spec.q_heads
+    kv_bytes = int((T * kvh * d * 2 * 2).sum())
+    q_bytes = spec.token_count * qh * d * 2
+    o_bytes = q_bytes
+    flops = 0
+    for ql, past in zip(spec.q_lens.astype(np.int64), spec.past.astype(np.int64)):
+        # sum over i < ql of (past + i + 1) visible keys
+        flops += 4 * qh * d * int(ql * past + ql * (ql + 1) // 2)
+    scatter_bytes = 4 * spec.token_count * kvh * d * 2 + 4 * spec.token_count
+    is_decode = bool(spec.q_lens.max() <= 4)
+    return dict(kv_bytes=kv_bytes, q_bytes=q_bytes, o_bytes=o_bytes, flops=flops,
+                scatter_bytes=scatter_bytes,
+                step_bytes=kv_bytes + q_bytes + o_bytes + scatter_bytes, decode=is_decode)
+
+
+def load_peaks() -> dict:
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(path):
+        with open(path) as f:
+            p = json.load(f)
+        return dict(hbm_gbs=float(p["hbm_gbs"]), tflops=float(p["bf16_tflops"]),
+                    tflops_sustained=float(p["bf16_tflops_sustained"]), source="measured")
+    return dict(hbm_gbs=6650.0, tflops=1590.0, tflops_sustained=1400.0, source="fallback")
+
+
+# ----------------------------------------------------------------- clocks
+
+class ClockSampler:
+    """nvidia-smi samples (every 200 ms) while the timed region runs."""
+
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int):
+        self.gpu = gpu_index
+        self.proc = None
+        self.lines = []
+        self.thread = None
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(self.gpu), f"--query-gpu={self.FIELDS}",
+                 "--format=csv,noheader,nounits", "-lms", "200"],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except OSError:
+            self.proc = None
+            return
+        self.thread = threading.Thread(target=self._read, daemon=True)
+        self.thread.start()
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.lines.append(line.strip())
+
+    def stop(self) -> dict:
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        time.sleep(0.25)
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+        sm, smax, reasons = [], [], set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for ln in self.lines:
+            parts = [p.strip() for p in ln.split(",")]
+            if len(parts) < 9:
+                continue
+            try:
+                sm.append(float(parts[1]))
+                smax.append(float(parts[2]))
+            except ValueError:
+                continue
+            for n, v in zip(names, parts[5:9]):
+                if v.lower() == "active":
+                    reasons.add(n)
+        return {"sm_mhz": float(np.median(sm)) if sm else None,
+                "sm_max_mhz": max(smax) if smax else None,
+                "samples": len(sm), "reasons": sorted(reasons)}
+
+
+# ----------------------------------------------------------------- distributed
+
+def dist_setup(n_gpus: int):
+    """(rank, world, local_rank); initialises torch.distributed for N > 1."""
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        backend = os.environ.get("PA_BENCH_BACKEND", "nccl")
+        dist.init_process_group(backend=backend, timeout=datetime.timedelta(seconds=120))
+    return rank, world, local
+
+
+def max_over_ranks(value: float, world: int, device=None) -> float:
+    if world <= 1:
+        return value
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([value], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def barrier(world: int, device=None):
+    if world > 1:
+        import torch
+        import torch.distributed as dist
+        if device is not None and dist.get_backend() == "nccl":
+            dist.barrier(device_ids=[torch.cuda.current_device()])
+        else:
+            dist.barrier()
+
+
+# ----------------------------------------------------------------- oracle timing
+
+def time_oracle(spec: workloads.Spec, x: dict, target_s: float, seed: int = 0):
+    """Run the fp64 oracle over a sample of (sequence, KV head) units of the
+    workload for about target_s seconds.  Returns (GB/s, seconds, sample text,
+    threads).  Bytes counted are the same algorithmic bytes as the GPU's."""
+    import oracle
+    rng = np.random.default_rng(seed)
+    units = [(b, h) for b in range(spec.batch) for h in range(spec.kv_heads) if spec.q_lens[b] > 0]
+    order = rng.permutation(len(units))
+    cu = np.concatenate([[0], np.cumsum(spec.q_lens)])
+    g = spec.q_heads // spec.kv_heads
+    scale = 1.0 / math.sqrt(spec.head_size)
+    done_bytes, done_units, rows_done = 0, 0, 0
+    t0 = time.perf_counter()
+    i = 0
+    while i < len(order) and time.perf_counter() - t0 < target_s:
+        b, h = units[order[i]]
+        i += 1
+        rows = np.array([(t, h * g + j) for t in range(cu[b], cu[b + 1]) for j in range(g)],
+                        dtype=np.int64)
+        oracle.attention(x["query"], x["key_cache"], x["value_cache"], x["block_table"],
+                         x["cu_seqlens_q"], x["seqlens_kv"], scale, rows=rows)
+        T = int(spec.seqlens_kv[b])
+        done_bytes += T * spec.head_size * 2 * 2 + 2 * rows.shape[0] * spec.head_size * 2
+        done_units += 1
+        rows_done += rows.shape[0]
+    dt = time.perf_counter() - t0
+    sample = (f"{done_units} of {len(units)} (sequence, KV head) units, {rows_done} output rows, "
+              f"fp64 oracle attention, {dt:.1f} s")
+    return done_bytes / dt / 1e9, dt, sample, oracle.max_threads()
+
+
+# ----------------------------------------------------------------- profiles
+
+def kernel_source_hash() -> str:
+    h = hashlib.sha256()
+    for name in sorted(os.listdir(os.path.join(ROOT, "scatter_kv_b200", "csrc"))):
+        with open(os.path.join(ROOT, "scatter_kv_b200", "csrc", name), "rb") as f:
+            h.update(name.encode() + f.read())
+    return h.hexdigest()[:16]
+
+
+def profiled_traffic(kernel: str, workload: str):
+    """dram bytes per launch from a committed ncu summary, if it was taken
+    on the current kernel sources (else None)."""
+    path = os.path.join(ROOT, "profiles", f"{kernel}_{workload}.md")
+    if not os.path.exists(path):
+        return None
+    text = open(path).read()
+    m = re.search(r"traffic_bytes_per_launch:\s*([0-9.eE+]+)", text)
+    h = re.search(r"source_hash:\s*([0-9a-f]+)", text)
+    if not m or not h or h.group(1) != kernel_source_hash():
+        return None
+    return float(m.group(1))
+
+
+# ----------------------------------------------------------------- main arms
+
+def run_reference(args, spec, rank, world):
+    if rank != 0:
+        return
+    x = workloads.generate(spec)
+    import oracle
+    # The new tokens must be in the cache before attention reads them.
+    slots = oracle.slot_mapping(x["block_table"], x["cu_seqlens_q"], x["seqlens_kv"],
+                                spec.block_size)
+    oracle.scatter_kv(x["key"], x["value"], slots, x["key_cache"], x["value_cache"])
+    per_step = max(2.0, min(15.0, 150.0 / max(1, args.steps + args.warmup)))
+    for w in range(args.warmup):
+        time_oracle(spec, x, min(per_step, 2.0), seed=1000 + w)
+    vals, secs, samples = [], [], []
+    for k in range(args.steps):
+        v, dt, sample, cores = time_oracle(spec, x, per_step, seed=k)
+        vals.append(v)
+        secs.append(dt)
+        samples.append(sample)
+    value = float(np.median(vals))
+    line = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": "GB/s",
+        "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": float(np.mean(secs)) * 1e3, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": {"workload": spec.name, "l2": "n/a (host)"},
+        "cpu_baseline": {"value": value, "unit": "GB/s", "cores": cores, "kind": "oracle",
+                         "sample": samples[-1]},
+        "e2e": {"value": value, "unit": "GB/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+
+
+def run_gpu(args, spec, rank, world, local):
+    import torch
+    import scatter_kv_b200 as pa
+
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    counts = algorithmic_counts(spec)
+    peaks = load_peaks()
+    x = workloads.generate(spec)
+    d = {k: torch.from_numpy(np.ascontiguousarray(v)).to(dev) for k, v in x.items()}
+    dims = pa.make_dims(batch=spec.batch, token_count=spec.token_count, q_heads=spec.q_heads,
+                        kv_heads=spec.kv_heads, head_size=spec.head_size,
+                        num_blocks=spec.num_blocks, block_size=spec.block_size,
+                        max_blocks_per_seq=x["block_table"].shape[1],
+                        max_seqlen_q=int(spec.q_lens.max()), max_seqlen_kv=int(spec.seqlens_kv.max()))
+    bufs = pa.allocate(dims, device=dev)
+    scale = pa.default_scale(spec.head_size)
+    stream = torch.cuda.Stream(device=dev)
+    flush = torch.empty(2 * L2_BYTES // 4, dtype=torch.int32, device=dev)
+
+    def step():
+        pa.step(d["query"], d["key"], d["value"], d["key_cache"], d["value_cache"],
+                d["block_table"], d["cu_seqlens_q"], d["seqlens_kv"], scale, dims, bufs, stream)
+
+    with torch.cuda.stream(stream):
+        for _ in range(max(3, args.warmup)):
+            step()
+        stream.synchronize()
+        status = int(bufs.status[0].item())
+        if status != 0:
+            raise RuntimeError(f"device status {status:#x} on the benchmark inputs")
+
+        # ---- device-timed region: K steps, L2 flushed between steps
+        ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+              for _ in range(args.steps)]
+        pa.pa_trace_read()
+        pa.pa_trace_enable(True)
+        clocks = ClockSampler(local)
+        clocks.start()
+        barrier(world, dev)
+        torch.cuda.synchronize()
+        for k in range(args.steps):
+            flush.fill_(k)
+            ev[k][0].record(stream)
+            step()
+            ev[k][1].record(stream)
+        torch.cuda.synchronize()
+        barrier(world, dev)
+        clk = clocks.stop()
+        pa.pa_trace_enable(False)
+        trace = pa.pa_trace_read()
+        ms = sum(a.elapsed_time(b) for a, b in ev)
+        ms = max_over_ranks(ms, world, dev)
+
+        # ---- end-to-end through the public API with host buffers
+        host = {k: torch.from_numpy(np.ascontiguousarray(x[k])).pin_memory()
+                for k in ("query", "key", "value", "block_table", "cu_seqlens_q", "seqlens_kv")}
+        out_host = torch.empty(bufs.out.shape, dtype=bufs.out.dtype).pin_memory()
+        h2d = sum(t.numel() * t.element_size() for t in host.values())
+        d2h = out_host.numel() * out_host.element_size()
+        ev2 = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+               for _ in range(args.steps)]
+        barrier(world, dev)
+        torch.cuda.synchronize()
+        for k in range(args.steps):
+            flush.fill_(k)
+            ev2[k][0].record(stream)
+            for name, t in host.items():
+                d[name].copy_(t, non_blocking=True)
+            step()
+            out_host.copy_(bufs.out, non_blocking=True)
+            ev2[k][1].record(stream)
+        torch.cuda.synchronize()
+        barrier(world, dev)
+        ms_e2e = max_over_ranks(sum(a.elapsed_time(b) for a, b in ev2), world, dev)
+
+    # ---- roofline of the dominant kernel (from the live trace)
+    per_kernel = {}
+    for name, t in trace:
+        per_kernel.setdefault(name, []).append(t)
+    launches = sum(len(v) for v in per_kernel.values())
+    total_k = sum(sum(v) for v in per_kernel.values())
+    dominant = max(per_kernel, key=lambda n: sum(per_kernel[n]))
+    avg_ms = float(np.mean(per_kernel[dominant]))
+    wl_key = args.workload
+    if dominant == "prefill_tcgen05":
+        achieved = counts["flops"] / (avg_ms * 1e-3) / 1e12
+        roof = {"bound": "tensor", "achieved": achieved, "peak": peaks["tflops"], "unit": "TFLOP/s",
+                "frac": achieved / peaks["tflops"],
+                "traffic": profiled_traffic(dominant, wl_key),
+                "kernel": dominant, "peak_source": f"{peaks['source']} bf16 burst (fp16 same rate)"}
+    else:
+        alg = counts["kv_bytes"] + counts["q_bytes"]
+        if dominant == "scatter_kv":
+            alg = counts["scatter_bytes"]
+        achieved = alg / (avg_ms * 1e-3) / 1e9
+        roof = {"bound": "hbm", "achieved": achieved, "peak": peaks["hbm_gbs"], "unit": "GB/s",
+                "frac": achieved / peaks["hbm_gbs"],
+                "traffic": profiled_traffic(dominant, wl_key),
+                "kernel": dominant, "peak_source": f"{peaks['source']} copy bandwidth"}
+    roof["kernel_ms"] = avg_ms
+    roof["share_of_kernel_time"] = sum(per_kernel[dominant]) / total_k if total_k else None
+
+    if counts["decode"]:
+        unit, value = "GB/s", counts["step_bytes"] * world / (ms / args.steps * 1e-3) / 1e9
+        e2e_value = counts["step_bytes"] * world / (ms_e2e / args.steps * 1e-3) / 1e9
+    else:
+        unit, value = "TFLOP/s", counts["flops"] * world / (ms / args.steps * 1e-3) / 1e12
+        e2e_value = counts["flops"] * world / (ms_e2e / args.steps * 1e-3) / 1e12
+
+    line = None
+    if rank == 0:
+        cpu = None
+        if world == 1 and not args.no_cpu_baseline:
+            import oracle  # noqa: F401
+            gbs, dt, sample, cores = time_oracle(spec, x_with_scatter(x, spec), args.cpu_seconds)
+            if counts["decode"]:
+                cpu = {"value": gbs, "unit": "GB/s", "cores": cores, "kind": "oracle", "sample": sample}
+            else:
+                # Same sample expressed in the step's unit: FLOPs of the rows run per second.
+                cpu = {"value": gbs * counts["flops"] / max(1, counts["kv_bytes"] + 2 * counts["q_bytes"]) / 1e3,
+                       "unit": "TFLOP/s", "cores": cores, "kind": "oracle",
+                       "sample": sample + " (rate scaled by the workload's FLOP/byte ratio)"}
+        line = {
+            "metric": METRIC, "value": value, "unit": unit, "n_gpus": world, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": ms / args.steps, "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "f16", "data": "synthetic",
+            "config": {"workload": spec.name, "batch": spec.batch, "tokens": spec.token_count,
+                       "q_heads": spec.q_heads, "kv_heads": spec.kv_heads,
+                       "head_size": spec.head_size, "block_size": spec.block_size,
+                       "num_blocks": spec.num_blocks, "seed": spec.seed,
+                       "l2": "flushed between steps (256 MB write outside the timed events)",
+                       "parallelism": f"replicas x{world}"},
+            "roofline": roof,
+            "cpu_baseline": cpu,
+            "e2e": {"value": e2e_value, "unit": unit, "h2d_bytes_per_step": h2d,
+                    "d2h_bytes_per_step": d2h},
+            "gpu_launches": launches,
+            "kernels": {n: {"launches": len(v), "avg_ms": float(np.mean(v))} for n, v in per_kernel.items()},
+            "algorithmic": {k: v for k, v in counts.items() if k != "decode"},
+            "clocks": clk,
+        }
+        print(json.dumps(line), flush=True)
+    return line
+
+
+def x_with_scatter(x, spec):
+    """The workload as the oracle sees it after the step's scatter."""
+    import oracle
+    y = dict(x)
+    y["key_cache"] = x["key_cache"].copy()
+    y["value_cache"] = x["value_cache"].copy()
+    slots = oracle.slot_mapping(x["block_table"], x["cu_seqlens_q"], x["seqlens_kv"],
+                                spec.block_size)
+    oracle.scatter_kv(x["key"], x["value"], slots, y["key_cache"], y["value_cache"])
+    return y
+
+
+def main(argv=None):
+    ap = argparse.ArgumentParser(description=__doc__.split("\n")[0])
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--workload", default="decode", choices=sorted(workloads.CONFIG_KEYS))
+    ap.add_argument("--cpu-seconds", type=float, default=10.0)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args(argv)
+    if args.warmup < 3 and args.impl == "ours":
+        args.warmup = 3
+    spec = workloads.CONFIGS[workloads.CONFIG_KEYS[args.workload]]()
+    rank, world, local = dist_setup(args.gpus)
+    try:
+        if args.impl == "reference":
+            run_reference(args, spec, rank, world)
+        else:
+            run_gpu(args, spec, rank, world, local)
+    finally:
+        if world > 1:
+            import torch.distributed as dist
+            dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

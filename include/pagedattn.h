@@ -1,0 +1,187 @@
+/*
+ * pagedattn.h -- C ABI of the B200 (sm_100a) paged-attention library
+ * (libpagedattn.so): scatter of new K/V tokens into a block-table KV cache,
+ * and fused causal grouped-query attention over packed variable-length
+ * queries, as used by continuous batching.
+ *
+ * Definitions the calls follow:
+ *   - ONNX Runtime PR "[WebGPU] Initial PagedAttention implementation (1/n)":
+ *     "Description" (scatter K/V into the paged cache, then attention over
+ *     packed varlen Q with output packed as (token_count, hidden_size));
+ *     "FlashAttention: optional seqlens_q input" (past_len_b = total_kv_b -
+ *     seqlens_q[b]); the review's "Things I specifically checked" (query i
+ *     sees past_len_b + i + 1 keys; the token -> sequence lookup skips
+ *     zero-length sequences; the cache update happens before the
+ *     token_count == 0 early return).
+ *   - ONNX preview FlexAttention operator doc: "FlexAttention Computation"
+ *     (Y = softmax(Q K^T * scale) V), "Grouped Query Attention (GQA)" (query
+ *     head h reads K/V head floor(h / (q_heads / kv_heads))), and softmax in
+ *     float32 for non-double inputs ("Modifier Subgraphs").
+ *
+ * Conventions for every call:
+ *   - Pointers named as tensors are DEVICE pointers, caller-owned, dense
+ *     row-major, 16-byte aligned.  The library allocates no device memory,
+ *     keeps no per-call state, and never reads data back to the host.
+ *   - `stream` is a cudaStream_t (NULL = legacy default stream).  Every call
+ *     is asynchronous on it; host-side argument errors are returned before
+ *     anything is launched.
+ *   - Floating-point tensors are IEEE binary16 (PA_DTYPE_F16); accumulation
+ *     and softmax run in fp32; outputs are rounded to nearest-even.
+ *   - `dev_status` (may be NULL) is a device int32 the caller zeroes; kernels
+ *     OR PA_DEV_* bits into it when the device-side metadata is invalid.  A
+ *     sequence with invalid metadata gets all-zero output rows; no kernel
+ *     traps.  Read it with pa_get_status().
+ */
+#ifndef PAGEDATTN_H
+#define PAGEDATTN_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+    PA_OK = 0,
+    PA_ERR_INVALID_ARGUMENT = 1,   /* bad pointer, shape, alignment or workspace size */
+    PA_ERR_NOT_IMPLEMENTED = 2,    /* valid per the pages but not built (bf16, head sizes) */
+    PA_ERR_CUDA = 3                /* a CUDA runtime call failed (launch, driver entry point) */
+} pa_status;
+
+typedef enum {
+    PA_DTYPE_F16 = 0,
+    PA_DTYPE_BF16 = 1              /* rejected with PA_ERR_NOT_IMPLEMENTED, as the PR's v1 does */
+} pa_dtype;
+
+/* Bits OR-ed into *dev_status by the kernels. */
+enum {
+    PA_DEV_BAD_CU_SEQLENS = 1 << 0,  /* cu_seqlens_q[0] != 0, decreasing, or last != token_count */
+    PA_DEV_QLEN_GT_KV     = 1 << 1,  /* q_len_b > seqlens_kv[b] (negative past) */
+    PA_DEV_KV_TOO_LONG    = 1 << 2,  /* seqlens_kv[b] > max_blocks_per_seq * block_size */
+    PA_DEV_BAD_BLOCK      = 1 << 3,  /* a block_table entry in use is outside [0, num_blocks) */
+    PA_DEV_BAD_SLOT       = 1 << 4,  /* a slot_mapping entry >= num_blocks * block_size */
+    PA_DEV_TIMEOUT        = 1 << 5,  /* a bounded in-kernel wait gave up (never expected) */
+    PA_DEV_HINT_EXCEEDED  = 1 << 6   /* a sequence is longer than max_seqlen_q_hint or
+                                        max_seqlen_kv_hint */
+};
+
+/* Problem dimensions, all host-known.  token_count = cu_seqlens_q[batch].
+ * head_size must be 16, 32, 64 or 128; block_size a power of two in
+ * [16, 256]; q_heads a multiple of kv_heads with q_heads / kv_heads <= 32;
+ * num_blocks * block_size < 2^31.
+ * The hints are optional upper bounds (0 = unknown): max_seqlen_q_hint
+ * bounds every q_len_b, max_seqlen_kv_hint every seqlens_kv[b].  They size
+ * grids and workspace; a sequence that exceeds a hint is treated as invalid
+ * (PA_DEV_HINT_EXCEEDED, zero output rows). */
+typedef struct {
+    int32_t batch;
+    int64_t token_count;
+    int32_t q_heads;
+    int32_t kv_heads;
+    int32_t head_size;
+    int64_t num_blocks;
+    int32_t block_size;
+    int32_t max_blocks_per_seq;
+    int32_t max_seqlen_q_hint;
+    int32_t max_seqlen_kv_hint;
+    int32_t dtype;                 /* pa_dtype */
+} pa_dims;
+
+/* pa_scatter_kv -- write the new tokens' keys and values into the paged caches.
+ * PR "[WebGPU] Initial PagedAttention implementation (1/n)", "Description"
+ * (scatter K/V into the paged cache); the cache update is in place.
+ *   key, value:   [token_count, kv_heads, head_size] f16, read only.
+ *   slot_mapping: [token_count] int32; token t goes to block slot / block_size,
+ *                 row slot % block_size.  A negative slot skips the token; a
+ *                 slot >= num_blocks * block_size is skipped and flagged
+ *                 PA_DEV_BAD_SLOT.  Duplicate slots: which write lands is
+ *                 unspecified.
+ *   key_cache, value_cache: [num_blocks, block_size, kv_heads, head_size] f16,
+ *                 updated in place.
+ * token_count == 0 is a valid no-op.  Bytes are copied unchanged. */
+pa_status pa_scatter_kv(const void* key, const void* value, const int32_t* slot_mapping,
+                        void* key_cache, void* value_cache, const pa_dims* dims,
+                        int32_t* dev_status, void* stream);
+
+/* pa_compute_slot_mapping -- slot of every new token.  Token t belongs to the
+ * first sequence b with cu_seqlens_q[b+1] > t (zero-length sequences are
+ * skipped; review "Things I specifically checked"); its logical position is
+ * p = past_len_b + (t - cu_seqlens_q[b]) with past_len_b = seqlens_kv[b] -
+ * q_len_b; slot = block_table[b][p / block_size] * block_size + p % block_size.
+ *   block_table:  [batch, max_blocks_per_seq] int32.
+ *   cu_seqlens_q: [batch + 1] int32.  seqlens_kv: [batch] int32 (totals, past
+ *                 plus new tokens).
+ *   slot_mapping: [token_count] int32 output; -1 for a token whose sequence
+ *                 fails the device checks (the matching PA_DEV_* bit is set). */
+pa_status pa_compute_slot_mapping(const int32_t* block_table, const int32_t* cu_seqlens_q,
+                                  const int32_t* seqlens_kv, int32_t* slot_mapping,
+                                  const pa_dims* dims, int32_t* dev_status, void* stream);
+
+/* pa_attention_workspace_size -- device workspace bytes pa_attention needs for
+ * these dims (split-KV partial results of the decode path).  *bytes may be 0. */
+pa_status pa_attention_workspace_size(const pa_dims* dims, size_t* bytes);
+
+/* pa_attention -- causal GQA attention over the paged cache.
+ * FlexAttention "FlexAttention Computation" and "Grouped Query Attention
+ * (GQA)"; causal bound from PR "[WebGPU] Initial PagedAttention
+ * implementation (1/n)", "FlashAttention: optional seqlens_q input": query i
+ * of sequence b (q_len_b = cu_seqlens_q[b+1] - cu_seqlens_q[b]) attends to
+ * logical key positions [0, seqlens_kv[b] - q_len_b + i].
+ *   query: [token_count, q_heads, head_size] f16, packed by sequence.
+ *   key_cache, value_cache: as for pa_scatter_kv (read only here; call
+ *          pa_scatter_kv first, on the same stream).  Cache rows that no
+ *          sequence's visible keys map to are never used, whatever they hold.
+ *   block_table, cu_seqlens_q, seqlens_kv: as for pa_compute_slot_mapping.
+ *   scale: multiplier of Q K^T; 0 selects 1 / sqrt(head_size).
+ *   out:   [token_count, q_heads, head_size] f16, written for every token.
+ *   workspace: device buffer of at least pa_attention_workspace_size() bytes
+ *          (may be NULL when that is 0); contents need no initialisation.
+ * Sequences with q_len_b <= 4 take the split-KV decode kernels, longer ones
+ * the tensor-core prefill kernel; both write disjoint rows of `out`. */
+pa_status pa_attention(const void* query, const void* key_cache, const void* value_cache,
+                       const int32_t* block_table, const int32_t* cu_seqlens_q,
+                       const int32_t* seqlens_kv, float scale, void* out, const pa_dims* dims,
+                       void* workspace, size_t workspace_bytes, int32_t* dev_status,
+                       void* stream);
+
+/* pa_get_status -- synchronise `stream` and copy *dev_status to *host_code.
+ * For tests and debugging; it blocks the host. */
+pa_status pa_get_status(const int32_t* dev_status, int32_t* host_code, void* stream);
+
+/* pa_status_string -- static text for a pa_status value. */
+const char* pa_status_string(pa_status status);
+
+/* pa_last_error -- static text describing the last host-side error of the
+ * calling thread ("" if none). */
+const char* pa_last_error(void);
+
+/* Kernel tracing: when enabled, every launch the library makes is bracketed
+ * by a pair of CUDA events on its stream; pa_trace_read() waits for them and
+ * returns (kernel id, milliseconds) records in launch order, then clears.
+ * Off by default; a bounded ring (PA_TRACE_CAPACITY launches) that drops
+ * records once full.  Not thread-safe. */
+#define PA_TRACE_CAPACITY 4096
+typedef struct {
+    int32_t kernel;                /* PA_KERNEL_* */
+    float ms;
+} pa_trace_record;
+
+enum {
+    PA_KERNEL_SCATTER = 0,
+    PA_KERNEL_SLOT_MAPPING = 1,
+    PA_KERNEL_DECODE = 2,
+    PA_KERNEL_COMBINE = 3,
+    PA_KERNEL_PREFILL = 4,
+    PA_KERNEL_COUNT = 5
+};
+
+pa_status pa_trace_enable(int on);
+int pa_trace_read(pa_trace_record* records, int max_records);
+const char* pa_kernel_name(int32_t kernel);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* PAGEDATTN_H */

@@ -1,0 +1,257 @@
+"""Paged attention for continuous batching on NVIDIA B200 (sm_100a).
+
+A thin ctypes binding of ``libpagedattn.so`` (declared in
+``include/pagedattn.h``): the functions below carry the C names and only
+marshal arguments -- shapes and raw device pointers of torch tensors -- into
+the C calls.  All computation runs in the library's CUDA kernels; there is
+no Python or CPU fallback, and importing this package fails loudly when the
+library has not been built (``python scatter_kv_b200/build.py``).
+
+Calls:
+  pa_scatter_kv            new K/V tokens -> paged cache (in place)
+  pa_compute_slot_mapping  cache slot of every new token
+  pa_attention             causal GQA attention over the paged cache
+  pa_attention_workspace_size, pa_get_status, pa_trace_*  (plumbing)
+"""
+from __future__ import annotations
+
+import ctypes
+import math
+import os
+from dataclasses import dataclass
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libpagedattn.so")
+
+PA_OK = 0
+PA_ERR_INVALID_ARGUMENT = 1
+PA_ERR_NOT_IMPLEMENTED = 2
+PA_ERR_CUDA = 3
+
+PA_DTYPE_F16 = 0
+PA_DTYPE_BF16 = 1
+
+PA_DEV_BAD_CU_SEQLENS = 1 << 0
+PA_DEV_QLEN_GT_KV = 1 << 1
+PA_DEV_KV_TOO_LONG = 1 << 2
+PA_DEV_BAD_BLOCK = 1 << 3
+PA_DEV_BAD_SLOT = 1 << 4
+PA_DEV_TIMEOUT = 1 << 5
+PA_DEV_HINT_EXCEEDED = 1 << 6
+
+PA_KERNEL_SCATTER = 0
+PA_KERNEL_SLOT_MAPPING = 1
+PA_KERNEL_DECODE = 2
+PA_KERNEL_COMBINE = 3
+PA_KERNEL_PREFILL = 4
+PA_TRACE_CAPACITY = 4096
+
+
+class pa_dims(ctypes.Structure):
+    _fields_ = [
+        ("batch", ctypes.c_int32),
+        ("token_count", ctypes.c_int64),
+        ("q_heads", ctypes.c_int32),
+        ("kv_heads", ctypes.c_int32),
+        ("head_size", ctypes.c_int32),
+        ("num_blocks", ctypes.c_int64),
+        ("block_size", ctypes.c_int32),
+        ("max_blocks_per_seq", ctypes.c_int32),
+        ("max_seqlen_q_hint", ctypes.c_int32),
+        ("max_seqlen_kv_hint", ctypes.c_int32),
+        ("dtype", ctypes.c_int32),
+    ]
+
+
+class pa_trace_record(ctypes.Structure):
+    _fields_ = [("kernel", ctypes.c_int32), ("ms", ctypes.c_float)]
+
+
+class PagedAttentionError(RuntimeError):
+    def __init__(self, status: int, message: str):
+        super().__init__(f"{_status_name(status)}: {message}")
+        self.status = status
+
+
+EXPORTS = [
+    "pa_scatter_kv", "pa_compute_slot_mapping", "pa_attention_workspace_size", "pa_attention",
+    "pa_get_status", "pa_status_string", "pa_last_error", "pa_trace_enable", "pa_trace_read",
+    "pa_kernel_name",
+]
+
+
+def _load():
+    if not os.path.exists(LIB_PATH):
+        raise ImportError(
+            f"{LIB_PATH} is missing: build it with `python scatter_kv_b200/build.py` "
+            "(there is no fallback implementation)")
+    lib = ctypes.CDLL(LIB_PATH)
+    P, I32P = ctypes.c_void_p, ctypes.POINTER(ctypes.c_int32)
+    D = ctypes.POINTER(pa_dims)
+    lib.pa_scatter_kv.argtypes = [P, P, P, P, P, D, P, P]
+    lib.pa_scatter_kv.restype = ctypes.c_int
+    lib.pa_compute_slot_mapping.argtypes = [P, P, P, P, D, P, P]
+    lib.pa_compute_slot_mapping.restype = ctypes.c_int
+    lib.pa_attention_workspace_size.argtypes = [D, ctypes.POINTER(ctypes.c_size_t)]
+    lib.pa_attention_workspace_size.restype = ctypes.c_int
+    lib.pa_attention.argtypes = [P, P, P, P, P, P, ctypes.c_float, P, D, P, ctypes.c_size_t, P, P]
+    lib.pa_attention.restype = ctypes.c_int
+    lib.pa_get_status.argtypes = [P, I32P, P]
+    lib.pa_get_status.restype = ctypes.c_int
+    lib.pa_status_string.argtypes = [ctypes.c_int]
+    lib.pa_status_string.restype = ctypes.c_char_p
+    lib.pa_last_error.argtypes = []
+    lib.pa_last_error.restype = ctypes.c_char_p
+    lib.pa_trace_enable.argtypes = [ctypes.c_int]
+    lib.pa_trace_enable.restype = ctypes.c_int
+    lib.pa_trace_read.argtypes = [ctypes.POINTER(pa_trace_record), ctypes.c_int]
+    lib.pa_trace_read.restype = ctypes.c_int
+    lib.pa_kernel_name.argtypes = [ctypes.c_int32]
+    lib.pa_kernel_name.restype = ctypes.c_char_p
+    return lib
+
+
+lib = _load()
+
+
+def _status_name(st: int) -> str:
+    return lib.pa_status_string(int(st)).decode()
+
+
+def _check(st: int):
+    if st != PA_OK:
+        raise PagedAttentionError(st, lib.pa_last_error().decode())
+
+
+def _ptr(t):
+    """Device (or host) address of a torch tensor; None -> NULL; ints pass through."""
+    if t is None:
+        return None
+    if isinstance(t, int):
+        return t
+    return t.data_ptr()
+
+
+def _stream(stream):
+    if stream is None:
+        import torch
+        return torch.cuda.current_stream().cuda_stream
+    if isinstance(stream, int):
+        return stream
+    return stream.cuda_stream
+
+
+def make_dims(query=None, key_cache=None, block_table=None, cu_seqlens_q=None, *, batch=None,
+              token_count=None, q_heads=None, kv_heads=None, head_size=None, num_blocks=None,
+              block_size=None, max_blocks_per_seq=None, max_seqlen_q=0, max_seqlen_kv=0,
+              dtype=PA_DTYPE_F16) -> pa_dims:
+    """pa_dims from tensor shapes (query [T, qh, d], cache [nb, bs, kvh, d],
+    block table [B, maxblk], cu_seqlens_q [B + 1]); keywords override."""
+    d = pa_dims()
+    if query is not None:
+        d.token_count, d.q_heads, d.head_size = query.shape
+    if key_cache is not None:
+        d.num_blocks, d.block_size, d.kv_heads, hs = key_cache.shape
+        d.head_size = hs
+    if block_table is not None:
+        d.batch, d.max_blocks_per_seq = block_table.shape
+    if cu_seqlens_q is not None:
+        d.batch = cu_seqlens_q.shape[0] - 1
+    for name, val in (("batch", batch), ("token_count", token_count), ("q_heads", q_heads),
+                      ("kv_heads", kv_heads), ("head_size", head_size), ("num_blocks", num_blocks),
+                      ("block_size", block_size), ("max_blocks_per_seq", max_blocks_per_seq)):
+        if val is not None:
+            setattr(d, name, int(val))
+    d.max_seqlen_q_hint = int(max_seqlen_q)
+    d.max_seqlen_kv_hint = int(max_seqlen_kv)
+    d.dtype = int(dtype)
+    return d
+
+
+def pa_scatter_kv(key, value, slot_mapping, key_cache, value_cache, dims: pa_dims,
+                  dev_status=None, stream=None) -> None:
+    _check(lib.pa_scatter_kv(_ptr(key), _ptr(value), _ptr(slot_mapping), _ptr(key_cache),
+                             _ptr(value_cache), ctypes.byref(dims), _ptr(dev_status),
+                             _stream(stream)))
+
+
+def pa_compute_slot_mapping(block_table, cu_seqlens_q, seqlens_kv, slot_mapping, dims: pa_dims,
+                            dev_status=None, stream=None) -> None:
+    _check(lib.pa_compute_slot_mapping(_ptr(block_table), _ptr(cu_seqlens_q), _ptr(seqlens_kv),
+                                       _ptr(slot_mapping), ctypes.byref(dims), _ptr(dev_status),
+                                       _stream(stream)))
+
+
+def pa_attention_workspace_size(dims: pa_dims) -> int:
+    n = ctypes.c_size_t(0)
+    _check(lib.pa_attention_workspace_size(ctypes.byref(dims), ctypes.byref(n)))
+    return int(n.value)
+
+
+def pa_attention(query, key_cache, value_cache, block_table, cu_seqlens_q, seqlens_kv, scale,
+                 out, dims: pa_dims, workspace=None, workspace_bytes=None, dev_status=None,
+                 stream=None) -> None:
+    if workspace_bytes is None:
+        workspace_bytes = 0 if workspace is None or isinstance(workspace, int) else \
+            workspace.numel() * workspace.element_size()
+    _check(lib.pa_attention(_ptr(query), _ptr(key_cache), _ptr(value_cache), _ptr(block_table),
+                            _ptr(cu_seqlens_q), _ptr(seqlens_kv), float(scale), _ptr(out),
+                            ctypes.byref(dims), _ptr(workspace), int(workspace_bytes),
+                            _ptr(dev_status), _stream(stream)))
+
+
+def pa_get_status(dev_status, stream=None) -> int:
+    code = ctypes.c_int32(0)
+    _check(lib.pa_get_status(_ptr(dev_status), ctypes.byref(code), _stream(stream)))
+    return int(code.value)
+
+
+def pa_trace_enable(on: bool = True) -> None:
+    _check(lib.pa_trace_enable(1 if on else 0))
+
+
+def pa_trace_read():
+    """[(kernel name, ms), ...] of the launches since the last read."""
+    buf = (pa_trace_record * PA_TRACE_CAPACITY)()
+    n = lib.pa_trace_read(buf, PA_TRACE_CAPACITY)
+    return [(lib.pa_kernel_name(buf[i].kernel).decode(), float(buf[i].ms)) for i in range(n)]
+
+
+def default_scale(head_size: int) -> float:
+    return 1.0 / math.sqrt(head_size)
+
+
+@dataclass
+class Workspace:
+    """Device buffers one paged-attention call needs, sized for ``dims``."""
+
+    out: object
+    workspace: object
+    status: object
+    slot_mapping: object
+
+
+def allocate(dims: pa_dims, device="cuda", out=None):
+    """Allocate output, workspace, status word and slot-mapping buffers with torch."""
+    import torch
+    nbytes = pa_attention_workspace_size(dims)
+    if out is None:
+        out = torch.empty((dims.token_count, dims.q_heads, dims.head_size), dtype=torch.float16,
+                          device=device)
+    ws = torch.empty(max(nbytes, 16), dtype=torch.uint8, device=device)
+    status = torch.zeros(4, dtype=torch.int32, device=device)
+    slots = torch.empty(max(dims.token_count, 1), dtype=torch.int32, device=device)
+    return Workspace(out, ws, status, slots)
+
+
+def step(query, key, value, key_cache, value_cache, block_table, cu_seqlens_q, seqlens_kv,
+         scale, dims: pa_dims, buffers: Workspace, stream=None):
+    """One pass of the hot path: slot mapping, scatter of the new K/V, then
+    attention.  Returns ``buffers.out``."""
+    pa_compute_slot_mapping(block_table, cu_seqlens_q, seqlens_kv, buffers.slot_mapping, dims,
+                            buffers.status, stream)
+    pa_scatter_kv(key, value, buffers.slot_mapping, key_cache, value_cache, dims, buffers.status,
+                  stream)
+    pa_attention(query, key_cache, value_cache, block_table, cu_seqlens_q, seqlens_kv, scale,
+                 buffers.out, dims, buffers.workspace, None, buffers.status, stream)
+    return buffers.out

@@ -1,0 +1,420 @@
+// pa_api.cu -- the extern "C" boundary of libpagedattn.so: host-side
+// argument checks, TMA tensor-map construction, launch planning, kernel
+// tracing.  Nothing here touches tensor data; every step of the computation
+// runs in the kernels of pa_scatter.cu, pa_decode.cu and pa_prefill.cu.
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <math.h>
+#include <stdarg.h>
+#include <stdio.h>
+#include <string.h>
+
+#include <mutex>
+
+#include "pa_internal.h"
+#include "pagedattn.h"
+
+namespace {
+
+thread_local char g_last_error[512] = "";
+
+pa_status fail(pa_status st, const char* fmt, ...) {
+    va_list ap;
+    va_start(ap, fmt);
+    vsnprintf(g_last_error, sizeof(g_last_error), fmt, ap);
+    va_end(ap);
+    return st;
+}
+
+pa_status cuda_fail(cudaError_t e, const char* what) {
+    return fail(PA_ERR_CUDA, "%s: %s", what, cudaGetErrorString(e));
+}
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+bool is_pow2(long long v) { return v > 0 && (v & (v - 1)) == 0; }
+
+// ------------------------------------------------------------------ device info
+
+int num_sms_of_current_device() {
+    static int cache[64] = {0};
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return 148;
+    if (cache[dev] == 0) {
+        int n = 0;
+        if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0)
+            n = 148;
+        cache[dev] = n;
+    }
+    return cache[dev];
+}
+
+// ------------------------------------------------------------------ tensor maps
+
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
+                                  const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
+                                  const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
+                                  CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn() {
+    static EncodeTiledFn fn = nullptr;
+    static std::once_flag once;
+    std::call_once(once, [] {
+        void* p = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) ==
+                cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<EncodeTiledFn>(p);
+    });
+    return fn;
+}
+
+CUtensorMapSwizzle swizzle_for(int head_size) {
+    const int row_bytes = (head_size < 64 ? head_size : 64) * 2;
+    return row_bytes == 128 ? CU_TENSOR_MAP_SWIZZLE_128B
+         : row_bytes == 64  ? CU_TENSOR_MAP_SWIZZLE_64B
+                            : CU_TENSOR_MAP_SWIZZLE_32B;
+}
+
+// Cache [num_blocks, block_size, kv_heads, head_size] seen as the 4-D tensor
+// (head_size, kv_heads, block_size, num_blocks); a box is `rows` rows of one
+// KV head of one page, 64 (or head_size, if smaller) elements wide.
+pa_status make_cache_map(CUtensorMap* m, const void* base, const pa_dims& d, int rows) {
+    EncodeTiledFn fn = encode_fn();
+    if (!fn) return fail(PA_ERR_CUDA, "cuTensorMapEncodeTiled entry point unavailable");
+    const int A = d.head_size < 64 ? d.head_size : 64;
+    cuuint64_t dims[4] = {(cuuint64_t)d.head_size, (cuuint64_t)d.kv_heads, (cuuint64_t)d.block_size,
+                          (cuuint64_t)d.num_blocks};
+    cuuint64_t strides[3] = {(cuuint64_t)d.head_size * 2, (cuuint64_t)d.kv_heads * d.head_size * 2,
+                             (cuuint64_t)d.block_size * d.kv_heads * d.head_size * 2};
+    cuuint32_t box[4] = {(cuuint32_t)A, 1, (cuuint32_t)rows, 1};
+    cuuint32_t estr[4] = {1, 1, 1, 1};
+    CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 4, const_cast<void*>(base), dims, strides,
+                    box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, swizzle_for(d.head_size),
+                    CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    if (r != CUDA_SUCCESS) return fail(PA_ERR_CUDA, "cuTensorMapEncodeTiled(cache) failed: %d", (int)r);
+    return PA_OK;
+}
+
+// Query [token_count, q_heads, head_size] seen as (head_size, q_heads,
+// token_count); a box is 128 / group tokens x group heads = 128 rows.
+pa_status make_query_map(CUtensorMap* m, const void* base, const pa_dims& d) {
+    EncodeTiledFn fn = encode_fn();
+    if (!fn) return fail(PA_ERR_CUDA, "cuTensorMapEncodeTiled entry point unavailable");
+    const int A = d.head_size < 64 ? d.head_size : 64;
+    const int g = d.q_heads / d.kv_heads;
+    cuuint64_t dims[3] = {(cuuint64_t)d.head_size, (cuuint64_t)d.q_heads, (cuuint64_t)d.token_count};
+    cuuint64_t strides[2] = {(cuuint64_t)d.head_size * 2, (cuuint64_t)d.q_heads * d.head_size * 2};
+    cuuint32_t box[3] = {(cuuint32_t)A, (cuuint32_t)g, (cuuint32_t)(pa::kPrefillRows / g)};
+    cuuint32_t estr[3] = {1, 1, 1};
+    CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 3, const_cast<void*>(base), dims, strides,
+                    box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, swizzle_for(d.head_size),
+                    CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    if (r != CUDA_SUCCESS) return fail(PA_ERR_CUDA, "cuTensorMapEncodeTiled(query) failed: %d", (int)r);
+    return PA_OK;
+}
+
+// ------------------------------------------------------------------ tracing
+
+struct TraceState {
+    bool on = false;
+    int n = 0;
+    int kernel[PA_TRACE_CAPACITY];
+    cudaEvent_t ev0[PA_TRACE_CAPACITY];
+    cudaEvent_t ev1[PA_TRACE_CAPACITY];
+    bool created[PA_TRACE_CAPACITY] = {false};
+};
+TraceState g_trace;
+
+struct TraceScope {
+    int slot = -1;
+    cudaStream_t stream;
+    TraceScope(int kernel, cudaStream_t s) : stream(s) {
+        if (!g_trace.on || g_trace.n >= PA_TRACE_CAPACITY) return;
+        slot = g_trace.n++;
+        if (!g_trace.created[slot]) {
+            cudaEventCreate(&g_trace.ev0[slot]);
+            cudaEventCreate(&g_trace.ev1[slot]);
+            g_trace.created[slot] = true;
+        }
+        g_trace.kernel[slot] = kernel;
+        cudaEventRecord(g_trace.ev0[slot], stream);
+    }
+    ~TraceScope() {
+        if (slot >= 0) cudaEventRecord(g_trace.ev1[slot], stream);
+    }
+};
+
+// ------------------------------------------------------------------ validation
+
+pa_status check_dims(const pa_dims* dp) {
+    if (dp == nullptr) return fail(PA_ERR_INVALID_ARGUMENT, "dims is NULL");
+    const pa_dims& d = *dp;
+    if (d.dtype == PA_DTYPE_BF16)
+        return fail(PA_ERR_NOT_IMPLEMENTED, "bfloat16 is not implemented (f16 only)");
+    if (d.dtype != PA_DTYPE_F16) return fail(PA_ERR_INVALID_ARGUMENT, "unknown dtype %d", d.dtype);
+    if (d.batch < 0 || d.token_count < 0)
+        return fail(PA_ERR_INVALID_ARGUMENT, "negative batch or token_count");
+    if (d.q_heads <= 0 || d.kv_heads <= 0 || d.q_heads % d.kv_heads != 0)
+        return fail(PA_ERR_INVALID_ARGUMENT, "q_heads (%d) must be a positive multiple of kv_heads (%d)",
+                    d.q_heads, d.kv_heads);
+    const int g = d.q_heads / d.kv_heads;
+    if (!is_pow2(g) || g > 32)
+        return fail(PA_ERR_NOT_IMPLEMENTED, "q_heads / kv_heads = %d: only powers of two up to 32", g);
+    if (d.head_size <= 0 || d.head_size % 8 != 0)
+        return fail(PA_ERR_INVALID_ARGUMENT, "head_size %d must be a positive multiple of 8", d.head_size);
+    if (d.head_size != 16 && d.head_size != 32 && d.head_size != 64 && d.head_size != 128)
+        return fail(PA_ERR_NOT_IMPLEMENTED, "head_size %d: only 16, 32, 64, 128", d.head_size);
+    if (!is_pow2(d.block_size) || d.block_size < 16 || d.block_size > 256)
+        return fail(PA_ERR_INVALID_ARGUMENT, "block_size %d must be a power of two in [16, 256]",
+                    d.block_size);
+    if (d.num_blocks <= 0 || d.max_blocks_per_seq <= 0)
+        return fail(PA_ERR_INVALID_ARGUMENT, "num_blocks and max_blocks_per_seq must be positive");
+    if (d.num_blocks * (long long)d.block_size >= (1ll << 31))
+        return fail(PA_ERR_INVALID_ARGUMENT, "num_blocks * block_size must be < 2^31");
+    if ((long long)d.max_blocks_per_seq * d.block_size >= (1ll << 31))
+        return fail(PA_ERR_INVALID_ARGUMENT, "max_blocks_per_seq * block_size must be < 2^31");
+    if (d.token_count >= (1ll << 31))
+        return fail(PA_ERR_INVALID_ARGUMENT, "token_count must be < 2^31");
+    if (d.max_seqlen_q_hint < 0 || d.max_seqlen_kv_hint < 0)
+        return fail(PA_ERR_INVALID_ARGUMENT, "negative hint");
+    return PA_OK;
+}
+
+#define PA_REQUIRE_PTR(p)                                                                    \
+    do {                                                                                     \
+        if ((p) == nullptr) return fail(PA_ERR_INVALID_ARGUMENT, "%s is NULL", #p);          \
+        if (!aligned16(p)) return fail(PA_ERR_INVALID_ARGUMENT, "%s is not 16-byte aligned", #p); \
+    } while (0)
+
+#define PA_REQUIRE_IPTR(p)                                                                   \
+    do {                                                                                     \
+        if ((p) == nullptr) return fail(PA_ERR_INVALID_ARGUMENT, "%s is NULL", #p);          \
+        if ((reinterpret_cast<uintptr_t>(p) & 3u) != 0)                                      \
+            return fail(PA_ERR_INVALID_ARGUMENT, "%s is not 4-byte aligned", #p);            \
+    } while (0)
+
+}  // namespace
+
+extern "C" {
+
+pa_status pa_scatter_kv(const void* key, const void* value, const int32_t* slot_mapping,
+                        void* key_cache, void* value_cache, const pa_dims* dims,
+                        int32_t* dev_status, void* stream) {
+    g_last_error[0] = 0;
+    pa_status st = check_dims(dims);
+    if (st != PA_OK) return st;
+    if (dims->token_count == 0) return PA_OK;
+    PA_REQUIRE_PTR(key);
+    PA_REQUIRE_PTR(value);
+    PA_REQUIRE_IPTR(slot_mapping);
+    PA_REQUIRE_PTR(key_cache);
+    PA_REQUIRE_PTR(value_cache);
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    TraceScope tr(PA_KERNEL_SCATTER, s);
+    cudaError_t e = pa::launch_scatter(key, value, slot_mapping, key_cache, value_cache, *dims,
+                                       dev_status, s, num_sms_of_current_device());
+    return e == cudaSuccess ? PA_OK : cuda_fail(e, "scatter launch");
+}
+
+pa_status pa_compute_slot_mapping(const int32_t* block_table, const int32_t* cu_seqlens_q,
+                                  const int32_t* seqlens_kv, int32_t* slot_mapping,
+                                  const pa_dims* dims, int32_t* dev_status, void* stream) {
+    g_last_error[0] = 0;
+    pa_status st = check_dims(dims);
+    if (st != PA_OK) return st;
+    if (dims->token_count == 0) return PA_OK;
+    if (dims->batch == 0) return fail(PA_ERR_INVALID_ARGUMENT, "token_count > 0 with batch 0");
+    PA_REQUIRE_IPTR(block_table);
+    PA_REQUIRE_IPTR(cu_seqlens_q);
+    PA_REQUIRE_IPTR(seqlens_kv);
+    PA_REQUIRE_IPTR(slot_mapping);
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    TraceScope tr(PA_KERNEL_SLOT_MAPPING, s);
+    cudaError_t e = pa::launch_slot_mapping(block_table, cu_seqlens_q, seqlens_kv, slot_mapping,
+                                            *dims, dev_status, s);
+    return e == cudaSuccess ? PA_OK : cuda_fail(e, "slot mapping launch");
+}
+
+pa_status pa_attention_workspace_size(const pa_dims* dims, size_t* bytes) {
+    g_last_error[0] = 0;
+    if (bytes == nullptr) return fail(PA_ERR_INVALID_ARGUMENT, "bytes is NULL");
+    pa_status st = check_dims(dims);
+    if (st != PA_OK) return st;
+    *bytes = pa::plan_decode(*dims, num_sms_of_current_device()).workspace_bytes;
+    return PA_OK;
+}
+
+pa_status pa_attention(const void* query, const void* key_cache, const void* value_cache,
+                       const int32_t* block_table, const int32_t* cu_seqlens_q,
+                       const int32_t* seqlens_kv, float scale, void* out, const pa_dims* dims,
+                       void* workspace, size_t workspace_bytes, int32_t* dev_status,
+                       void* stream) {
+    g_last_error[0] = 0;
+    pa_status st = check_dims(dims);
+    if (st != PA_OK) return st;
+    const pa_dims& d = *dims;
+    if (d.token_count == 0) return PA_OK;
+    if (d.batch == 0) return fail(PA_ERR_INVALID_ARGUMENT, "token_count > 0 with batch 0");
+    if (!(scale >= 0.f) || isinf(scale))
+        return fail(PA_ERR_INVALID_ARGUMENT, "scale must be finite and >= 0");
+    PA_REQUIRE_PTR(query);
+    PA_REQUIRE_PTR(key_cache);
+    PA_REQUIRE_PTR(value_cache);
+    PA_REQUIRE_PTR(out);
+    PA_REQUIRE_IPTR(block_table);
+    PA_REQUIRE_IPTR(cu_seqlens_q);
+    PA_REQUIRE_IPTR(seqlens_kv);
+    const int nsm = num_sms_of_current_device();
+    const pa::DecodePlan plan = pa::plan_decode(d, nsm);
+    if (workspace_bytes < plan.workspace_bytes)
+        return fail(PA_ERR_INVALID_ARGUMENT, "workspace of %zu bytes is smaller than the %zu needed",
+                    workspace_bytes, plan.workspace_bytes);
+    if (plan.workspace_bytes > 0) PA_REQUIRE_PTR(workspace);
+    if (scale == 0.f) scale = 1.f / sqrtf((float)d.head_size);
+    const float scale_log2 = scale * 1.4426950408889634f;
+    const int g = d.q_heads / d.kv_heads;
+    const int kv_cap = d.max_blocks_per_seq * d.block_size;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+
+    // Decode (split-KV) part: sequences with q_len <= plan.decode_max_q.
+    {
+        CUtensorMap tk, tv;
+        const int rows = d.block_size < pa::kDecodeKeys ? d.block_size : pa::kDecodeKeys;
+        if ((st = make_cache_map(&tk, key_cache, d, rows)) != PA_OK) return st;
+        if ((st = make_cache_map(&tv, value_cache, d, rows)) != PA_OK) return st;
+        pa::DecodeParams p{};
+        p.query = static_cast<const __half*>(query);
+        p.out = static_cast<__half*>(out);
+        const size_t rows_total = (size_t)d.batch * d.kv_heads * plan.max_splits * (16 * plan.mtiles);
+        p.part_o = static_cast<float*>(workspace);
+        p.part_lse = plan.workspace_bytes ? static_cast<float*>(workspace) + rows_total * d.head_size
+                                          : nullptr;
+        p.block_table = block_table;
+        p.cu_seqlens_q = cu_seqlens_q;
+        p.seqlens_kv = seqlens_kv;
+        p.status = dev_status;
+        p.token_count = d.token_count;
+        p.num_blocks = d.num_blocks;
+        p.batch = d.batch;
+        p.q_heads = d.q_heads;
+        p.kv_heads = d.kv_heads;
+        p.group = g;
+        p.block_size = d.block_size;
+        p.max_blocks = d.max_blocks_per_seq;
+        p.kv_cap = kv_cap;
+        p.kv_hint = d.max_seqlen_kv_hint;
+        p.q_hint = d.max_seqlen_q_hint;
+        p.decode_max_q = plan.decode_max_q;
+        p.chunk = plan.chunk;
+        p.max_splits = plan.max_splits;
+        p.rmax = 16 * plan.mtiles;
+        p.scale_log2 = scale_log2;
+        {
+            TraceScope tr(PA_KERNEL_DECODE, s);
+            cudaError_t e = pa::launch_decode(tk, tv, p, d.head_size, plan.mtiles, s);
+            if (e != cudaSuccess) return cuda_fail(e, "decode launch");
+        }
+        if (plan.max_splits > 1) {
+            TraceScope tr(PA_KERNEL_COMBINE, s);
+            cudaError_t e = pa::launch_combine(p, d.head_size, s);
+            if (e != cudaSuccess) return cuda_fail(e, "combine launch");
+        }
+    }
+
+    // Prefill part: sequences with q_len > plan.decode_max_q.
+    if (d.max_seqlen_q_hint == 0 || d.max_seqlen_q_hint > plan.decode_max_q) {
+        const long long longer = d.token_count / (plan.decode_max_q + 1);
+        const long long slots = (d.token_count * g + pa::kPrefillRows - 1) / pa::kPrefillRows +
+                                (longer < d.batch ? longer : d.batch);
+        if (slots > 0) {
+            if (slots > 65535) return fail(PA_ERR_NOT_IMPLEMENTED, "too many query tiles (%lld)", slots);
+            CUtensorMap tq, tk, tv;
+            const int rows = d.block_size < 64 ? d.block_size : 64;
+            if ((st = make_query_map(&tq, query, d)) != PA_OK) return st;
+            if ((st = make_cache_map(&tk, key_cache, d, rows)) != PA_OK) return st;
+            if ((st = make_cache_map(&tv, value_cache, d, rows)) != PA_OK) return st;
+            pa::PrefillParams p{};
+            p.out = static_cast<__half*>(out);
+            p.block_table = block_table;
+            p.cu_seqlens_q = cu_seqlens_q;
+            p.seqlens_kv = seqlens_kv;
+            p.status = dev_status;
+            p.token_count = d.token_count;
+            p.num_blocks = d.num_blocks;
+            p.batch = d.batch;
+            p.q_heads = d.q_heads;
+            p.kv_heads = d.kv_heads;
+            p.group = g;
+            p.block_size = d.block_size;
+            p.max_blocks = d.max_blocks_per_seq;
+            p.kv_cap = kv_cap;
+            p.kv_hint = d.max_seqlen_kv_hint;
+            p.q_hint = d.max_seqlen_q_hint;
+            p.decode_max_q = plan.decode_max_q;
+            p.num_slots = (int)slots;
+            p.scale_log2 = scale_log2;
+            TraceScope tr(PA_KERNEL_PREFILL, s);
+            cudaError_t e = pa::launch_prefill(tq, tk, tv, p, d.head_size, s);
+            if (e != cudaSuccess) return cuda_fail(e, "prefill launch");
+        }
+    }
+    return PA_OK;
+}
+
+pa_status pa_get_status(const int32_t* dev_status, int32_t* host_code, void* stream) {
+    g_last_error[0] = 0;
+    if (dev_status == nullptr || host_code == nullptr)
+        return fail(PA_ERR_INVALID_ARGUMENT, "NULL pointer");
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    cudaError_t e = cudaMemcpyAsync(host_code, dev_status, sizeof(int32_t), cudaMemcpyDeviceToHost, s);
+    if (e == cudaSuccess) e = cudaStreamSynchronize(s);
+    return e == cudaSuccess ? PA_OK : cuda_fail(e, "status read");
+}
+
+const char* pa_status_string(pa_status status) {
+    switch (status) {
+        case PA_OK: return "PA_OK";
+        case PA_ERR_INVALID_ARGUMENT: return "PA_ERR_INVALID_ARGUMENT";
+        case PA_ERR_NOT_IMPLEMENTED: return "PA_ERR_NOT_IMPLEMENTED";
+        case PA_ERR_CUDA: return "PA_ERR_CUDA";
+    }
+    return "unknown pa_status";
+}
+
+const char* pa_last_error(void) { return g_last_error; }
+
+pa_status pa_trace_enable(int on) {
+    g_trace.on = on != 0;
+    return PA_OK;
+}
+
+int pa_trace_read(pa_trace_record* records, int max_records) {
+    int n = 0;
+    for (int i = 0; i < g_trace.n; ++i) {
+        float ms = -1.f;
+        if (cudaEventSynchronize(g_trace.ev1[i]) == cudaSuccess)
+            cudaEventElapsedTime(&ms, g_trace.ev0[i], g_trace.ev1[i]);
+        if (records != nullptr && n < max_records) {
+            records[n].kernel = g_trace.kernel[i];
+            records[n].ms = ms;
+            ++n;
+        }
+    }
+    g_trace.n = 0;
+    return n;
+}
+
+const char* pa_kernel_name(int32_t kernel) {
+    switch (kernel) {
+        case PA_KERNEL_SCATTER: return "scatter_kv";
+        case PA_KERNEL_SLOT_MAPPING: return "slot_mapping";
+        case PA_KERNEL_DECODE: return "decode_split_kv";
+        case PA_KERNEL_COMBINE: return "decode_combine";
+        case PA_KERNEL_PREFILL: return "prefill_tcgen05";
+    }
+    return "unknown";
+}
+
+}  // extern "C"

@@ -1,0 +1,564 @@
+// pa_decode.cu -- split-KV decode attention over the paged cache and the
+// log-sum-exp combine of the splits.
+//
+// Math: FlexAttention operator doc, "FlexAttention Computation" (Y =
+// softmax(Q K^T * scale) V, softmax in fp32) and "Grouped Query Attention
+// (GQA)" (query head h reads K/V head floor(h / group)); causal bound from
+// ONNX Runtime PR "[WebGPU] Initial PagedAttention implementation (1/n)",
+// "FlashAttention: optional seqlens_q input": row i of sequence b sees keys
+// [0, past_b + i], past_b = seqlens_kv[b] - q_len_b.
+//
+// Decode is bound by HBM: every K/V row of a sequence must be read once per
+// KV head, and there are only q_len * group query rows to multiply them by.
+// So the kernel is built around streaming pages:
+//   * one CTA per (split of the sequence's keys, KV head, sequence); the
+//     group * q_len query rows of that KV head share every page it loads;
+//   * a producer warp walks the block table and issues TMA tensor loads of
+//     32-key K and V tiles (one box per page and 64-element column block,
+//     128-byte swizzle) into a ring of shared-memory stages tracked by
+//     mbarriers;
+//   * consumer warps each own whole tiles (independent online softmax per
+//     warp, merged at the end), computing Q K^T and P V with mma.sync
+//     m16n8k16 (f16 in, f32 accumulate).  The tensor core is only a means to
+//     keep ALU work far below the memory time here, not the bound.
+// Splits are chunk-aligned in logical key order, so results do not depend on
+// which physical pages hold the keys.  A sequence with one split writes its
+// output directly; otherwise each split writes (O / l, m + log2 l) and the
+// combine kernel merges the splits in split order.
+#include <cuda_runtime.h>
+#include <math.h>
+
+#include "pa_common.cuh"
+#include "pa_internal.h"
+
+namespace pa {
+
+namespace {
+
+template <int HEAD, int MT>
+struct Cfg {
+    static constexpr int A = HEAD < 64 ? HEAD : 64;     // elements per swizzled row
+    static constexpr int RB = A * 2;                    // bytes per swizzled row
+    static constexpr int NA = HEAD / A;                 // column blocks
+    static constexpr int BN = kDecodeKeys;              // keys per stage
+    static constexpr int NST = 6;                       // stages
+    static constexpr int NCW = 4;                       // consumer warps
+    static constexpr int NG = NCW / MT;                 // tile groups (MT warps per group)
+    static constexpr int THREADS = 32 * (NCW + 1);
+    static constexpr int TILE_BYTES = BN * HEAD * 2;    // one tensor, one stage
+    static constexpr int STAGE_BYTES = 2 * TILE_BYTES;
+    static constexpr int RMAX = 16 * MT;
+    static constexpr int OST = HEAD + 8;                // merge scratch row stride (floats)
+    static constexpr int SMEM = NST * STAGE_BYTES + 1024 + 2 * NST * 8 + 2 * NG * RMAX * 4 +
+                                2 * RMAX * 4 + 16;
+    static_assert(NG * RMAX * OST * 4 <= NST * STAGE_BYTES, "merge scratch must fit the stages");
+};
+
+__device__ __forceinline__ uint32_t half2_mask(uint32_t v, bool lo_ok, bool hi_ok) {
+    return (lo_ok ? (v & 0xffffu) : 0u) | (hi_ok ? (v & 0xffff0000u) : 0u);
+}
+
+template <int HEAD, int MT>
+__global__ void __launch_bounds__(Cfg<HEAD, MT>::THREADS)
+decode_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_v,
+              const DecodeParams p) {
+    using C = Cfg<HEAD, MT>;
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t* smem = reinterpret_cast<uint8_t*>(
+        (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    uint8_t* stages = smem;
+    uint64_t* full = reinterpret_cast<uint64_t*>(smem + C::NST * C::STAGE_BYTES);
+    uint64_t* empty = full + C::NST;
+    float* red_m = reinterpret_cast<float*>(empty + C::NST);   // [NG][RMAX]
+    float* red_l = red_m + C::NG * C::RMAX;                     // [NG][RMAX]
+    float* row_l = red_l + C::NG * C::RMAX;                     // [RMAX]
+    float* row_m = row_l + C::RMAX;                             // [RMAX]
+    int* sflag = reinterpret_cast<int*>(row_m + C::RMAX);       // [0] bad seq, [1] abort, [2] issued
+
+    const int b = blockIdx.z, kvh = blockIdx.y, split = blockIdx.x;
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int g = p.group;
+    // Status bits of a sequence are reported once, by CTA (split 0, kv head 0).
+    const bool reporter = (split == 0 && kvh == 0 && threadIdx.x == 0);
+
+    SeqInfo s;
+    const bool ok = load_seq(p.cu_seqlens_q, p.seqlens_kv, b, p.batch, p.token_count, p.kv_cap,
+                             p.kv_hint, p.q_hint, nullptr, s);
+    if (!s.cu_ok) {
+        if (reporter) flag_status(p.status, PA_DEV_BAD_CU_SEQLENS);
+        return;
+    }
+    if (s.q_len > p.decode_max_q) {
+        // Prefill work, done by the prefill kernel -- unless the sequence breaks
+        // the q_len hint, in which case that kernel may not run at all: report
+        // it and zero its rows here.
+        if (!ok && p.q_hint > 0 && s.q_len > p.q_hint && split == 0) {
+            if (reporter)
+                load_seq(p.cu_seqlens_q, p.seqlens_kv, b, p.batch, p.token_count, p.kv_cap,
+                         p.kv_hint, p.q_hint, p.status, s);
+            for (int idx = threadIdx.x; idx < s.q_len * g * HEAD; idx += C::THREADS) {
+                const int r = idx / HEAD, d = idx % HEAD;
+                const long long o = ((long long)(s.q_start + r / g) * p.q_heads + kvh * g + r % g) * HEAD + d;
+                p.out[o] = __float2half_rn(0.f);
+            }
+        }
+        return;
+    }
+    if (s.q_len == 0) return;
+    const int T = ok ? s.kv_len : 0;
+    const int n_splits = ok ? (T + p.chunk - 1) / p.chunk : 1;
+    if (split >= n_splits) return;
+    const int R = s.q_len * g;
+
+    if (threadIdx.x == 0) {
+        if (reporter)
+            load_seq(p.cu_seqlens_q, p.seqlens_kv, b, p.batch, p.token_count, p.kv_cap,
+                     p.kv_hint, p.q_hint, p.status, s);
+        sflag[0] = ok ? 0 : 1;
+        sflag[1] = 0;
+        sflag[2] = 0;
+        for (int i = 0; i < C::NST; ++i) {
+            mbar_init(&full[i], 1);
+            mbar_init(&empty[i], MT);
+        }
+        fence_barrier_init();
+    }
+    __syncthreads();
+    if (ok && warp == 0) {
+        const int npages = (T + p.block_size - 1) / p.block_size;
+        const bool bok = warp_blocks_ok(p.block_table, b, p.max_blocks, npages, p.num_blocks,
+                                        (split == 0 && kvh == 0) ? p.status : nullptr);
+        if (!bok && lane == 0) sflag[0] = 1;
+    }
+    __syncthreads();
+    if (sflag[0]) {
+        // Invalid sequence: zero rows (split 0 only; the combine does the same).
+        if (split == 0) {
+            for (int idx = threadIdx.x; idx < R * HEAD; idx += C::THREADS) {
+                const int r = idx / HEAD, d = idx % HEAD;
+                const long long o = ((long long)(s.q_start + r / g) * p.q_heads + kvh * g + r % g) * HEAD + d;
+                p.out[o] = __float2half_rn(0.f);
+            }
+        }
+        return;
+    }
+
+    const int k_begin = split * p.chunk;
+    const int k_end = min(T, k_begin + p.chunk);
+    const int ntiles = (k_end - k_begin + C::BN - 1) / C::BN;
+    const int bs = p.block_size;
+    const int32_t* bt = p.block_table + (long long)b * p.max_blocks;
+
+    if (warp == C::NCW) {
+        // ------------------------------------------------------------ producer
+        if (lane == 0) {
+            tma_prefetch_desc(&tm_k);
+            tma_prefetch_desc(&tm_v);
+            const uint64_t pol = policy_evict_first();
+            for (int t = 0; t < ntiles; ++t) {
+                const int st = t % C::NST, u = t / C::NST;
+                if (u > 0 && !mbar_wait(&empty[st], (u - 1) & 1)) {
+                    flag_status(p.status, PA_DEV_TIMEOUT);
+                    atomicExch(&sflag[1], 1);
+                    break;
+                }
+                if (*(volatile int*)&sflag[1]) break;
+                sflag[2] = t + 1;
+                uint8_t* kdst = stages + st * C::STAGE_BYTES;
+                uint8_t* vdst = kdst + C::TILE_BYTES;
+                const int k0 = k_begin + t * C::BN;
+                if (bs >= C::BN) {
+                    const int blk = bt[k0 / bs];
+                    const int row = k0 % bs;
+                    mbar_arrive_expect_tx(&full[st], 2 * C::TILE_BYTES);
+#pragma unroll
+                    for (int c = 0; c < C::NA; ++c) {
+                        tma_load_4d_hint(kdst + c * C::BN * C::RB, &tm_k, &full[st], c * C::A, kvh, row, blk, pol);
+                        tma_load_4d_hint(vdst + c * C::BN * C::RB, &tm_v, &full[st], c * C::A, kvh, row, blk, pol);
+                    }
+                } else {
+                    // block_size 16: two pages per 32-key tile; skip a page past the end.
+                    const int npg = (k0 + bs < T) ? 2 : 1;
+                    mbar_arrive_expect_tx(&full[st], (uint32_t)(npg * bs * HEAD * 2 * 2));
+                    for (int pi = 0; pi < npg; ++pi) {
+                        const int blk = bt[k0 / bs + pi];
+#pragma unroll
+                        for (int c = 0; c < C::NA; ++c) {
+                            const int off = (c * C::BN + pi * bs) * C::RB;
+                            tma_load_4d_hint(kdst + off, &tm_k, &full[st], c * C::A, kvh, 0, blk, pol);
+                            tma_load_4d_hint(vdst + off, &tm_v, &full[st], c * C::A, kvh, 0, blk, pol);
+                        }
+                    }
+                }
+            }
+        }
+    } else {
+        // ------------------------------------------------------------ consumers
+        const int mt = warp % MT;          // which 16 query rows
+        const int grp = warp / MT;         // which tiles
+        const int quad = lane >> 2, qid = lane & 3;
+        // Rows held by this thread: r0 = mt*16 + quad, r1 = r0 + 8.
+        int rows[2] = {mt * 16 + quad, mt * 16 + quad + 8};
+        int lim[2];                        // last visible key (inclusive) per row
+#pragma unroll
+        for (int h = 0; h < 2; ++h) {
+            const int r = rows[h];
+            lim[h] = (r < R) ? (s.past + r / g) : (T - 1);
+        }
+        // Q fragments (A operand) straight from global memory.
+        uint32_t qf[HEAD / 16][4];
+        {
+            const __half* q0 = nullptr;
+            const __half* q1 = nullptr;
+            if (rows[0] < R)
+                q0 = p.query + ((long long)(s.q_start + rows[0] / g) * p.q_heads + kvh * g + rows[0] % g) * HEAD;
+            if (rows[1] < R)
+                q1 = p.query + ((long long)(s.q_start + rows[1] / g) * p.q_heads + kvh * g + rows[1] % g) * HEAD;
+#pragma unroll
+            for (int kk = 0; kk < HEAD / 16; ++kk) {
+                const int c = kk * 16 + 2 * qid;
+                qf[kk][0] = q0 ? *reinterpret_cast<const uint32_t*>(q0 + c) : 0u;
+                qf[kk][1] = q1 ? *reinterpret_cast<const uint32_t*>(q1 + c) : 0u;
+                qf[kk][2] = q0 ? *reinterpret_cast<const uint32_t*>(q0 + c + 8) : 0u;
+                qf[kk][3] = q1 ? *reinterpret_cast<const uint32_t*>(q1 + c + 8) : 0u;
+            }
+        }
+        float oacc[HEAD / 8][4];
+#pragma unroll
+        for (int i = 0; i < HEAD / 8; ++i)
+            oacc[i][0] = oacc[i][1] = oacc[i][2] = oacc[i][3] = 0.f;
+        float m_run[2] = {-INFINITY, -INFINITY};
+        float l_run[2] = {0.f, 0.f};
+
+        // ldmatrix lane roles: matrix mi = lane / 8, row rr = lane % 8.
+        const int mi = lane >> 3, rr = lane & 7;
+
+        for (int t = grp; t < ntiles; t += C::NG) {
+            const int st = t % C::NST, u = t / C::NST;
+            if (!mbar_wait_warp(&full[st], u & 1)) {
+                flag_status(p.status, PA_DEV_TIMEOUT);
+                atomicExch(&sflag[1], 1);
+                break;
+            }
+            const uint32_t kbase = smem_u32(stages + st * C::STAGE_BYTES);
+            const uint32_t vbase = kbase + C::TILE_BYTES;
+            const int k0 = k_begin + t * C::BN;
+
+            // S = Q K^T for this warp's 16 rows x 32 keys.
+            float sacc[4][4];
+#pragma unroll
+            for (int i = 0; i < 4; ++i) sacc[i][0] = sacc[i][1] = sacc[i][2] = sacc[i][3] = 0.f;
+#pragma unroll
+            for (int kk = 0; kk < HEAD / 16; ++kk) {
+#pragma unroll
+                for (int np = 0; np < 2; ++np) {
+                    const int key = np * 16 + (mi >> 1) * 8 + rr;
+                    const int chunk = kk * 2 + (mi & 1);          // 16-byte chunk along d
+                    const int c = (chunk * 8) / C::A, cc = chunk % (C::A / 8);
+                    const uint32_t off = (uint32_t)((c * C::BN + key) * C::RB + cc * 16);
+                    uint32_t b0, b1, b2, b3;
+                    ldsm_x4(kbase + swz<C::RB>(off), b0, b1, b2, b3);
+                    mma_16816(sacc[2 * np], qf[kk], b0, b1);
+                    mma_16816(sacc[2 * np + 1], qf[kk], b2, b3);
+                }
+            }
+            // Mask, scale to the log2 domain, online softmax.
+            float mx[2] = {-INFINITY, -INFINITY};
+#pragma unroll
+            for (int nt = 0; nt < 4; ++nt) {
+#pragma unroll
+                for (int e = 0; e < 4; ++e) {
+                    const int h = e >> 1;
+                    const int key = k0 + nt * 8 + 2 * qid + (e & 1);
+                    const bool vis = key < k_end && key <= lim[h];
+                    const float v = vis ? sacc[nt][e] * p.scale_log2 : -INFINITY;
+                    sacc[nt][e] = v;
+                    mx[h] = fmaxf(mx[h], v);
+                }
+            }
+            float alpha[2];
+#pragma unroll
+            for (int h = 0; h < 2; ++h) {
+                mx[h] = fmaxf(mx[h], __shfl_xor_sync(0xffffffffu, mx[h], 1));
+                mx[h] = fmaxf(mx[h], __shfl_xor_sync(0xffffffffu, mx[h], 2));
+                const float m_new = fmaxf(m_run[h], mx[h]);
+                const float base = (m_new == -INFINITY) ? 0.f : m_new;
+                alpha[h] = fast_exp2(m_run[h] - base);
+                m_run[h] = m_new;
+                mx[h] = base;
+            }
+            float psum[2] = {0.f, 0.f};
+#pragma unroll
+            for (int nt = 0; nt < 4; ++nt) {
+#pragma unroll
+                for (int e = 0; e < 4; ++e) {
+                    const float pe = fast_exp2(sacc[nt][e] - mx[e >> 1]);
+                    sacc[nt][e] = pe;
+                    psum[e >> 1] += pe;
+                }
+            }
+#pragma unroll
+            for (int h = 0; h < 2; ++h) l_run[h] = l_run[h] * alpha[h] + psum[h];
+#pragma unroll
+            for (int i = 0; i < HEAD / 8; ++i) {
+                oacc[i][0] *= alpha[0];
+                oacc[i][1] *= alpha[0];
+                oacc[i][2] *= alpha[1];
+                oacc[i][3] *= alpha[1];
+            }
+            // P as A fragments (two k16 steps over the 32 keys).
+            uint32_t pa[2][4];
+#pragma unroll
+            for (int j = 0; j < 2; ++j) {
+                pa[j][0] = pack_half2(sacc[2 * j][0], sacc[2 * j][1]);
+                pa[j][1] = pack_half2(sacc[2 * j][2], sacc[2 * j][3]);
+                pa[j][2] = pack_half2(sacc[2 * j + 1][0], sacc[2 * j + 1][1]);
+                pa[j][3] = pack_half2(sacc[2 * j + 1][2], sacc[2 * j + 1][3]);
+            }
+            // O += P V.  Rows of V past the sequence end may hold anything
+            // (NaN included): zero them in the fragments of the last tile.
+            const bool tail = (k0 + C::BN > k_end);
+#pragma unroll
+            for (int j = 0; j < 2; ++j) {
+                const int kv0 = k0 + j * 16 + 2 * qid;       // keys of b0 halves; +8 for b1
+#pragma unroll
+                for (int dp = 0; dp < HEAD / 16; ++dp) {
+                    const int key = j * 16 + (mi & 1) * 8 + rr;
+                    const int chunk = dp * 2 + (mi >> 1);
+                    const int c = (chunk * 8) / C::A, cc = chunk % (C::A / 8);
+                    const uint32_t off = (uint32_t)((c * C::BN + key) * C::RB + cc * 16);
+                    uint32_t b0, b1, b2, b3;
+                    ldsm_x4_t(vbase + swz<C::RB>(off), b0, b1, b2, b3);
+                    if (tail) {
+                        b0 = half2_mask(b0, kv0 < k_end, kv0 + 1 < k_end);
+                        b2 = half2_mask(b2, kv0 < k_end, kv0 + 1 < k_end);
+                        b1 = half2_mask(b1, kv0 + 8 < k_end, kv0 + 9 < k_end);
+                        b3 = half2_mask(b3, kv0 + 8 < k_end, kv0 + 9 < k_end);
+                    }
+                    mma_16816(oacc[2 * dp], pa[j], b0, b1);
+                    mma_16816(oacc[2 * dp + 1], pa[j], b2, b3);
+                }
+            }
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&empty[st]);
+        }
+
+        // ---------------------------------------------------- merge the groups
+        // Row sums over the quad (each thread summed only its own columns).
+#pragma unroll
+        for (int h = 0; h < 2; ++h) {
+            l_run[h] += __shfl_xor_sync(0xffffffffu, l_run[h], 1);
+            l_run[h] += __shfl_xor_sync(0xffffffffu, l_run[h], 2);
+        }
+        if (qid == 0) {
+#pragma unroll
+            for (int h = 0; h < 2; ++h) {
+                red_m[grp * C::RMAX + rows[h]] = m_run[h];
+                red_l[grp * C::RMAX + rows[h]] = l_run[h];
+            }
+        }
+        asm volatile("bar.sync 1, %0;" ::"r"(C::NCW * 32));
+        float* scr = reinterpret_cast<float*>(stages);     // [NG][RMAX][OST]
+#pragma unroll
+        for (int h = 0; h < 2; ++h) {
+            const int r = rows[h];
+            float M = -INFINITY;
+            for (int gg = 0; gg < C::NG; ++gg) M = fmaxf(M, red_m[gg * C::RMAX + r]);
+            const float base = (M == -INFINITY) ? 0.f : M;
+            const float f = fast_exp2(m_run[h] - base);
+            if (grp == 0 && qid == 0) {
+                float L = 0.f;
+                for (int gg = 0; gg < C::NG; ++gg)
+                    L += red_l[gg * C::RMAX + r] * fast_exp2(red_m[gg * C::RMAX + r] - base);
+                row_l[r] = L;
+                row_m[r] = M;
+            }
+            float* dst = scr + (grp * C::RMAX + r) * C::OST + 2 * qid;
+#pragma unroll
+            for (int i = 0; i < HEAD / 8; ++i) {
+                float2 v = make_float2(oacc[i][2 * h] * f, oacc[i][2 * h + 1] * f);
+                *reinterpret_cast<float2*>(dst + i * 8) = v;
+            }
+        }
+        asm volatile("bar.sync 1, %0;" ::"r"(C::NCW * 32));
+        // Final rows: sum the groups in order, normalise, write.
+        const bool direct = (n_splits == 1);
+        const long long pbase = (((long long)b * p.kv_heads + kvh) * p.max_splits + split) * p.rmax;
+        for (int idx = threadIdx.x; idx < R * (HEAD / 4); idx += C::NCW * 32) {
+            const int r = idx / (HEAD / 4), d4 = (idx % (HEAD / 4)) * 4;
+            float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+            for (int gg = 0; gg < C::NG; ++gg) {
+                const float4 v = *reinterpret_cast<const float4*>(scr + (gg * C::RMAX + r) * C::OST + d4);
+                acc.x += v.x; acc.y += v.y; acc.z += v.z; acc.w += v.w;
+            }
+            const float L = row_l[r];
+            const float inv = (L > 0.f) ? 1.f / L : 0.f;
+            acc.x *= inv; acc.y *= inv; acc.z *= inv; acc.w *= inv;
+            if (direct) {
+                const long long o = ((long long)(s.q_start + r / g) * p.q_heads + kvh * g + r % g) * HEAD + d4;
+                uint2 w;
+                w.x = pack_half2(acc.x, acc.y);
+                w.y = pack_half2(acc.z, acc.w);
+                *reinterpret_cast<uint2*>(p.out + o) = w;
+            } else {
+                *reinterpret_cast<float4*>(p.part_o + (pbase + r) * HEAD + d4) = acc;
+                if (d4 == 0)
+                    p.part_lse[pbase + r] = (L > 0.f) ? row_m[r] + __log2f(L) : -INFINITY;
+            }
+        }
+    }
+    // After an aborted wait (never expected), make sure no TMA load is still
+    // writing this CTA's shared memory before it exits.
+    __syncthreads();
+    if (threadIdx.x == 0 && sflag[1]) {
+        const int issued = sflag[2];
+        for (int t = issued - C::NST > 0 ? issued - C::NST : 0; t < issued; ++t)
+            mbar_wait(&full[t % C::NST], (t / C::NST) & 1);
+    }
+}
+
+// One CTA per (KV head, sequence): merge the splits of its q_len * group rows.
+template <int HEAD>
+__global__ void __launch_bounds__(128) combine_kernel(const DecodeParams p) {
+    extern __shared__ float wsm[];                        // [max_splits][rmax] then [rmax]
+    const int b = blockIdx.y, kvh = blockIdx.x;
+    const int g = p.group;
+    SeqInfo s;
+    const bool ok = load_seq(p.cu_seqlens_q, p.seqlens_kv, b, p.batch, p.token_count, p.kv_cap,
+                             p.kv_hint, p.q_hint, nullptr, s);
+    if (!s.cu_ok || s.q_len == 0 || s.q_len > p.decode_max_q) return;
+    const int R = s.q_len * g;
+    __shared__ int bad;
+    if (threadIdx.x == 0) bad = ok ? 0 : 1;
+    __syncthreads();
+    if (ok && threadIdx.x < 32) {
+        const int npages = (s.kv_len + p.block_size - 1) / p.block_size;
+        if (!warp_blocks_ok(p.block_table, b, p.max_blocks, npages, p.num_blocks, nullptr) &&
+            threadIdx.x == 0)
+            bad = 1;
+    }
+    __syncthreads();
+    const int n_splits = bad ? 1 : (s.kv_len + p.chunk - 1) / p.chunk;
+    if (!bad && n_splits == 1) return;                    // decode kernel wrote the rows
+    if (bad) {
+        for (int idx = threadIdx.x; idx < R * HEAD; idx += blockDim.x) {
+            const int r = idx / HEAD, d = idx % HEAD;
+            p.out[((long long)(s.q_start + r / g) * p.q_heads + kvh * g + r % g) * HEAD + d] =
+                __float2half_rn(0.f);
+        }
+        return;
+    }
+    const long long pbase = ((long long)b * p.kv_heads + kvh) * p.max_splits * p.rmax;
+    float* inv_l = wsm + p.max_splits * p.rmax;
+    for (int r = threadIdx.x; r < R; r += blockDim.x) {
+        float M = -INFINITY;
+        for (int sp = 0; sp < n_splits; ++sp) M = fmaxf(M, p.part_lse[pbase + (long long)sp * p.rmax + r]);
+        float L = 0.f;
+        for (int sp = 0; sp < n_splits; ++sp) {
+            const float w = fast_exp2(p.part_lse[pbase + (long long)sp * p.rmax + r] - M);
+            wsm[sp * p.rmax + r] = w;
+            L += w;
+        }
+        inv_l[r] = 1.f / L;
+    }
+    __syncthreads();
+    for (int idx = threadIdx.x; idx < R * (HEAD / 4); idx += blockDim.x) {
+        const int r = idx / (HEAD / 4), d4 = (idx % (HEAD / 4)) * 4;
+        float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+        for (int sp = 0; sp < n_splits; ++sp) {
+            const float w = wsm[sp * p.rmax + r];
+            const float4 v = *reinterpret_cast<const float4*>(
+                p.part_o + (pbase + (long long)sp * p.rmax + r) * HEAD + d4);
+            acc.x += w * v.x; acc.y += w * v.y; acc.z += w * v.z; acc.w += w * v.w;
+        }
+        const float il = inv_l[r];
+        const long long o = ((long long)(s.q_start + r / g) * p.q_heads + kvh * g + r % g) * HEAD + d4;
+        uint2 wv;
+        wv.x = pack_half2(acc.x * il, acc.y * il);
+        wv.y = pack_half2(acc.z * il, acc.w * il);
+        *reinterpret_cast<uint2*>(p.out + o) = wv;
+    }
+}
+
+template <int HEAD, int MT>
+cudaError_t launch_decode_t(const CUtensorMap& tm_k, const CUtensorMap& tm_v,
+                            const DecodeParams& p, cudaStream_t stream) {
+    using C = Cfg<HEAD, MT>;
+    auto kern = decode_kernel<HEAD, MT>;
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM);
+    if (e != cudaSuccess) return e;
+    dim3 grid(p.max_splits, p.kv_heads, p.batch);
+    kern<<<grid, C::THREADS, C::SMEM, stream>>>(tm_k, tm_v, p);
+    return cudaGetLastError();
+}
+
+}  // namespace
+
+DecodePlan plan_decode(const pa_dims& d, int num_sms) {
+    DecodePlan pl{};
+    const int g = d.q_heads / d.kv_heads;
+    int dq = kDecodeMaxQ;
+    if (32 / g < dq) dq = 32 / g;
+    if (d.max_seqlen_q_hint > 0 && d.max_seqlen_q_hint < dq) dq = d.max_seqlen_q_hint;
+    if (dq < 1) dq = 1;
+    pl.decode_max_q = dq;
+    pl.mtiles = (dq * g + 15) / 16;
+    long long max_kv = (long long)d.max_blocks_per_seq * d.block_size;
+    if (d.max_seqlen_kv_hint > 0 && d.max_seqlen_kv_hint < max_kv) max_kv = d.max_seqlen_kv_hint;
+    if (max_kv < 1) max_kv = 1;
+    // Aim for about eight waves of two CTAs per SM if every sequence were as
+    // long as the bound; chunks stay multiples of the key tile.
+    const long long units = (long long)d.batch * d.kv_heads;
+    long long chunk = (units * max_kv + (long long)num_sms * 16 - 1) / ((long long)num_sms * 16);
+    if (chunk < 256) chunk = 256;
+    if (chunk > 16384) chunk = 16384;
+    chunk = (chunk + kDecodeKeys - 1) / kDecodeKeys * kDecodeKeys;
+    pl.chunk = (int)chunk;
+    pl.max_splits = (int)((max_kv + chunk - 1) / chunk);
+    if (pl.max_splits > 1) {
+        const size_t rows = (size_t)d.batch * d.kv_heads * pl.max_splits * (16 * pl.mtiles);
+        pl.workspace_bytes = rows * (size_t)d.head_size * 4 + rows * 4;
+        pl.workspace_bytes = (pl.workspace_bytes + 255) / 256 * 256;
+    }
+    return pl;
+}
+
+cudaError_t launch_decode(const CUtensorMap& tm_k, const CUtensorMap& tm_v,
+                          const DecodeParams& p, int head_size, int mtiles, cudaStream_t stream) {
+#define PA_DECODE_CASE(H)                                                          \
+    case H:                                                                        \
+        return mtiles == 1 ? launch_decode_t<H, 1>(tm_k, tm_v, p, stream)          \
+                           : launch_decode_t<H, 2>(tm_k, tm_v, p, stream);
+    switch (head_size) {
+        PA_DECODE_CASE(16)
+        PA_DECODE_CASE(32)
+        PA_DECODE_CASE(64)
+        PA_DECODE_CASE(128)
+        default: return cudaErrorInvalidValue;
+    }
+#undef PA_DECODE_CASE
+}
+
+cudaError_t launch_combine(const DecodeParams& p, int head_size, cudaStream_t stream) {
+    dim3 grid(p.kv_heads, p.batch);
+    const size_t smem = ((size_t)p.max_splits + 1) * p.rmax * sizeof(float);
+#define PA_COMBINE_CASE(H)                                                             \
+    case H: {                                                                          \
+        cudaError_t e = cudaFuncSetAttribute(combine_kernel<H>,                        \
+                                             cudaFuncAttributeMaxDynamicSharedMemorySize, \
+                                             (int)smem);                               \
+        if (e != cudaSuccess) return e;                                                \
+        combine_kernel<H><<<grid, 128, smem, stream>>>(p);                             \
+        return cudaGetLastError();                                                     \
+    }
+    switch (head_size) {
+        PA_COMBINE_CASE(16)
+        PA_COMBINE_CASE(32)
+        PA_COMBINE_CASE(64)
+        PA_COMBINE_CASE(128)
+        default: return cudaErrorInvalidValue;
+    }
+#undef PA_COMBINE_CASE
+}
+
+}  // namespace pa

@@ -1,0 +1,98 @@
+// pa_internal.h -- host-side declarations shared by the library's .cu files.
+#pragma once
+
+#include <cuda.h>
+#include <cuda_fp16.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "pagedattn.h"
+
+namespace pa {
+
+// Everything the decode (split-KV) kernels need besides the tensor maps.
+struct DecodeParams {
+    const __half* query;
+    __half* out;
+    float* part_o;                // [batch, kv_heads, max_splits, rmax, head_size]
+    float* part_lse;              // [batch, kv_heads, max_splits, rmax] (log2 domain)
+    const int32_t* block_table;
+    const int32_t* cu_seqlens_q;
+    const int32_t* seqlens_kv;
+    int32_t* status;
+    long long token_count;
+    long long num_blocks;
+    int batch;
+    int q_heads;
+    int kv_heads;
+    int group;                    // q_heads / kv_heads
+    int block_size;
+    int max_blocks;
+    int kv_cap;                   // max_blocks_per_seq * block_size
+    int kv_hint;                  // caller bound on seqlens_kv (0 = none)
+    int q_hint;                   // caller bound on q_len (0 = none)
+    int decode_max_q;             // q_len cut-off of the decode path
+    int chunk;                    // keys per split (multiple of the key tile)
+    int max_splits;
+    int rmax;                     // row capacity per (sequence, kv head) = 16 * m-tiles
+    float scale_log2;             // scale * log2(e)
+};
+
+struct PrefillParams {
+    __half* out;
+    const int32_t* block_table;
+    const int32_t* cu_seqlens_q;
+    const int32_t* seqlens_kv;
+    int32_t* status;
+    long long token_count;
+    long long num_blocks;
+    int batch;
+    int q_heads;
+    int kv_heads;
+    int group;
+    int block_size;
+    int max_blocks;
+    int kv_cap;
+    int kv_hint;
+    int q_hint;
+    int decode_max_q;             // sequences with q_len <= this are not prefill work
+    int num_slots;                // q tiles the grid covers (upper bound)
+    float scale_log2;
+};
+
+struct DecodePlan {
+    int decode_max_q;
+    int mtiles;                   // 1 or 2 (16 query rows each)
+    int chunk;
+    int max_splits;
+    size_t workspace_bytes;
+};
+
+DecodePlan plan_decode(const pa_dims& d, int num_sms);
+
+cudaError_t launch_scatter(const void* key, const void* value, const int32_t* slot_mapping,
+                           void* key_cache, void* value_cache, const pa_dims& d,
+                           int32_t* status, cudaStream_t stream, int num_sms);
+
+cudaError_t launch_slot_mapping(const int32_t* block_table, const int32_t* cu,
+                                const int32_t* seqlens_kv, int32_t* slot_mapping,
+                                const pa_dims& d, int32_t* status, cudaStream_t stream);
+
+// Decode: split-KV partial attention, then (when any split count > 1) the
+// log-sum-exp combine.  Returns the CUDA error of the launches.
+cudaError_t launch_decode(const CUtensorMap& tm_k, const CUtensorMap& tm_v,
+                          const DecodeParams& p, int head_size, int mtiles, cudaStream_t stream);
+cudaError_t launch_combine(const DecodeParams& p, int head_size, cudaStream_t stream);
+
+cudaError_t launch_prefill(const CUtensorMap& tm_q, const CUtensorMap& tm_k,
+                           const CUtensorMap& tm_v, const PrefillParams& p, int head_size,
+                           cudaStream_t stream);
+
+// Key rows per decode stage; the cache tensor maps' box height is
+// min(block_size, kDecodeKeys) for decode and min(block_size, kPrefillKeys)
+// for prefill.
+constexpr int kDecodeKeys = 32;
+constexpr int kPrefillKeys = 128;
+constexpr int kPrefillRows = 128;
+
+}  // namespace pa

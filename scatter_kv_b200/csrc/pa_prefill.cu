@@ -1,0 +1,507 @@
+// pa_prefill.cu -- causal prefill / mixed-batch attention over the paged
+// cache on the sm_100a tensor cores (tcgen05 + tensor memory).
+//
+// Math: FlexAttention operator doc, "FlexAttention Computation" (Y =
+// softmax(Q K^T * scale) V with fp32 softmax) and "Grouped Query Attention
+// (GQA)"; causal bound from ONNX Runtime PR "[WebGPU] Initial PagedAttention
+// implementation (1/n)", "FlashAttention: optional seqlens_q input" (row i
+// of sequence b sees keys [0, seqlens_kv[b] - q_len_b + i]).
+//
+// One CTA computes a 128-row query tile of one KV head.  The rows are
+// (token, head) pairs: 128 / group consecutive tokens times the group query
+// heads that share the KV head, so every K/V page is loaded once for the
+// whole group.  There is no gathered or padded copy of the cache: the
+// producer warp walks the block table and TMA-loads 64-key K and V tiles
+// (one box per page and 64-element column block, 128-byte swizzle) straight
+// from their pages.
+//
+// Warp roles (192 threads):
+//   warps 0-3  softmax + epilogue; thread r owns query row r = TMEM lane r;
+//   warp 4     TMA producer (Q once, then K and V tiles, 2-stage rings);
+//   warp 5     TMEM allocator and single-thread tcgen05.mma issuer.
+// Per key tile j:  S_j = Q K_j^T  (M 128, N 64, fp32 in TMEM, two buffers)
+//                  softmax_j: row max / exp2 / row sum in registers, P_j
+//                  as f16 into shared memory (128-byte swizzled, K-major)
+//                  O += P_j V_j  (M 128, N head_size, fp32 in TMEM)
+// The MMA warp issues S_{j+1} before waiting for P_j, so the tensor core
+// works on the next scores while the softmax threads exponentiate.  O is
+// rescaled only when a row maximum grows by more than 2^8 (values of P
+// stay below 256, exact enough in f16 and fp32 sums), which after the first
+// tiles is rare.  Key tiles wholly above the causal diagonal are never
+// loaded; the diagonal tile is masked per element; rows of V past the end of
+// the sequence are zeroed in shared memory before the last P V product.
+// Two CTAs fit on an SM (112 KB shared memory, 256 TMEM columns each), so
+// one CTA's softmax overlaps the other's MMAs and loads.
+#include <cuda_runtime.h>
+#include <math.h>
+
+#include "pa_common.cuh"
+#include "pa_internal.h"
+
+namespace pa {
+
+namespace {
+
+template <int HEAD>
+struct PCfg {
+    static constexpr int BM = kPrefillRows;             // 128 query rows
+    static constexpr int BN = 64;                       // keys per tile
+    static constexpr int A = HEAD < 64 ? HEAD : 64;     // elements per swizzled row (Q, K, V)
+    static constexpr int RB = A * 2;
+    static constexpr int NA = HEAD / A;
+    static constexpr uint32_t LAYOUT = RB == 128 ? 2u : (RB == 64 ? 4u : 6u);
+    static constexpr int Q_BYTES = BM * HEAD * 2;
+    static constexpr int KV_BYTES = BN * HEAD * 2;
+    static constexpr int P_BYTES = BM * BN * 2;         // 128 rows x 64 keys, one 128-B atom column
+    static constexpr int NST = 2;
+    static constexpr int OFF_Q = 0;
+    static constexpr int OFF_K = OFF_Q + Q_BYTES;
+    static constexpr int OFF_V = OFF_K + NST * KV_BYTES;
+    static constexpr int OFF_P = OFF_V + NST * KV_BYTES;
+    static constexpr int OFF_BAR = OFF_P + P_BYTES;
+    // q, k_full/v_full/kv_empty per stage, s_full x2, s_free x2, p_full, pv_done, drain
+    static constexpr int NBAR = 1 + 3 * NST + 2 + 2 + 3;
+    static constexpr int SMEM = OFF_BAR + NBAR * 8 + 64;
+    static constexpr int THREADS = 192;
+    static constexpr uint32_t TMEM_COLS = 256;          // S0 (64) | S1 (64) | O (head_size)
+    static constexpr uint32_t COL_S0 = 0, COL_S1 = 64, COL_O = 128;
+};
+
+struct Work {
+    int b;          // sequence
+    int tile;       // query tile within the sequence
+};
+
+// Heavy-first order of the query tiles: slot k lists, for r = 0, 1, ..., the
+// sequences that have more than r tiles, taking tile (ntiles_b - 1 - r).
+// Later tiles see more keys, so the largest pieces of work start first.
+__device__ bool find_work(const PrefillParams& p, int slot, Work& w) {
+    const int lane = threadIdx.x & 31;
+    for (int r = 0;; ++r) {
+        int cnt = 0;
+        bool any = false;
+        for (int b0 = 0; b0 < p.batch; b0 += 32) {
+            const int b = b0 + lane;
+            int nt = 0;
+            if (b < p.batch) {
+                const int c0 = p.cu_seqlens_q[b], c1 = p.cu_seqlens_q[b + 1];
+                const int ql = c1 - c0;
+                if (ql > p.decode_max_q && c0 >= 0 && (long long)c1 <= p.token_count)
+                    nt = (ql * p.group + PCfg<128>::BM - 1) / PCfg<128>::BM;
+            }
+            const bool has = nt > r;
+            any |= nt > r;
+            const unsigned m = __ballot_sync(0xffffffffu, has);
+            const int n = __popc(m);
+            if (slot < cnt + n) {
+                // The (slot - cnt)-th set bit of m.
+                int want = slot - cnt;
+                unsigned mm = m;
+                for (int i = 0; i < want; ++i) mm &= mm - 1;
+                const int lb = __ffs(mm) - 1;
+                const int bsel = b0 + lb;
+                const int ntsel = __shfl_sync(0xffffffffu, nt, lb);
+                w.b = bsel;
+                w.tile = ntsel - 1 - r;
+                return true;
+            }
+            cnt += n;
+        }
+        if (!__any_sync(0xffffffffu, any)) return false;
+        slot -= cnt;
+    }
+}
+
+template <int HEAD>
+__global__ void __launch_bounds__(PCfg<HEAD>::THREADS, 2)
+prefill_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
+               const __grid_constant__ CUtensorMap tm_v, const PrefillParams p) {
+    using C = PCfg<HEAD>;
+    extern __shared__ __align__(1024) uint8_t smem[];
+    uint64_t* bars = reinterpret_cast<uint64_t*>(smem + C::OFF_BAR);
+    uint64_t* q_full = bars;
+    uint64_t* k_full = bars + 1;
+    uint64_t* v_full = k_full + C::NST;
+    uint64_t* kv_empty = v_full + C::NST;
+    uint64_t* s_full = kv_empty + C::NST;
+    uint64_t* s_free = s_full + 2;
+    uint64_t* p_full = s_free + 2;
+    uint64_t* pv_done = p_full + 1;
+    uint64_t* drain = pv_done + 1;
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + C::NBAR);
+    int* sh = reinterpret_cast<int*>(tmem_slot + 1);   // [0] b, [1] tile, [2] bad, [3] abort, [4] issued
+
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int kvh = blockIdx.x;
+    const int g = p.group;
+
+    if ((smem_u32(smem) & 1023u) != 0) {              // the swizzle needs 1024-B alignment
+        if (threadIdx.x == 0) flag_status(p.status, PA_DEV_TIMEOUT);
+        return;
+    }
+
+    if (warp == 0) {
+        Work w;
+        const bool has = find_work(p, blockIdx.y, w);
+        if (lane == 0) {
+            sh[0] = has ? w.b : -1;
+            sh[1] = has ? w.tile : 0;
+        }
+    }
+    __syncthreads();
+    const int b = sh[0];
+    if (b < 0) return;
+    const int tile = sh[1];
+
+    SeqInfo s;
+    const bool ok = load_seq(p.cu_seqlens_q, p.seqlens_kv, b, p.batch, p.token_count, p.kv_cap,
+                             p.kv_hint, p.q_hint, nullptr, s);
+    const int tok_per_tile = C::BM / g;
+    const int i0 = tile * tok_per_tile;                          // first token of the tile
+    const int rows_valid = min(C::BM, (s.q_len - i0) * g);
+    if (threadIdx.x == 0) {
+        if (tile == 0 && kvh == 0)
+            load_seq(p.cu_seqlens_q, p.seqlens_kv, b, p.batch, p.token_count, p.kv_cap,
+                     p.kv_hint, p.q_hint, p.status, s);
+        sh[2] = ok ? 0 : 1;
+        sh[3] = 0;
+        mbar_init(q_full, 1);
+        for (int i = 0; i < C::NST; ++i) {
+            mbar_init(&k_full[i], 1);
+            mbar_init(&v_full[i], 1);
+            mbar_init(&kv_empty[i], 1);
+        }
+        for (int i = 0; i < 2; ++i) {
+            mbar_init(&s_full[i], 1);
+            mbar_init(&s_free[i], 4);
+        }
+        mbar_init(p_full, 4);
+        mbar_init(pv_done, 1);
+        mbar_init(drain, 1);
+        sh[4] = 0;
+        fence_barrier_init();
+    }
+    __syncthreads();
+    const int T = s.kv_len;
+    if (ok && warp == 0) {
+        const int npages = (T + p.block_size - 1) / p.block_size;
+        if (!warp_blocks_ok(p.block_table, b, p.max_blocks, npages, p.num_blocks,
+                            (tile == 0 && kvh == 0) ? p.status : nullptr) && lane == 0)
+            sh[2] = 1;
+    }
+    __syncthreads();
+    if (sh[2]) {
+        for (int idx = threadIdx.x; idx < rows_valid * HEAD; idx += C::THREADS) {
+            const int r = idx / HEAD, d = idx % HEAD;
+            const long long o = ((long long)(s.q_start + i0 + r / g) * p.q_heads + kvh * g + r % g) * HEAD + d;
+            p.out[o] = __float2half_rn(0.f);
+        }
+        return;
+    }
+
+    // Keys this tile needs: [0, past + last token of the tile].
+    const int i_last = min(s.q_len, i0 + tok_per_tile) - 1;
+    const int n_keys = s.past + i_last + 1;
+    const int ntiles = (n_keys + C::BN - 1) / C::BN;
+
+    if (warp == 5) {
+        tmem_alloc(tmem_slot, C::TMEM_COLS);
+        tmem_relinquish();
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = *tmem_slot;
+
+    uint8_t* sQ = smem + C::OFF_Q;
+    uint8_t* sK = smem + C::OFF_K;
+    uint8_t* sV = smem + C::OFF_V;
+    uint8_t* sP = smem + C::OFF_P;
+    const int bs = p.block_size;
+    const int32_t* bt = p.block_table + (long long)b * p.max_blocks;
+
+    if (warp == 4) {
+        // ---------------------------------------------------------- producer
+        if (lane == 0) {
+            tma_prefetch_desc(&tm_q);
+            tma_prefetch_desc(&tm_k);
+            tma_prefetch_desc(&tm_v);
+            mbar_arrive_expect_tx(q_full, C::Q_BYTES);
+#pragma unroll
+            for (int c = 0; c < C::NA; ++c)
+                tma_load_3d(sQ + c * C::BM * C::RB, &tm_q, q_full, c * C::A, kvh * g, s.q_start + i0);
+            const int box = bs < C::BN ? bs : C::BN;
+            for (int j = 0; j < ntiles; ++j) {
+                const int st = j % C::NST, u = j / C::NST;
+                if (u > 0 && !mbar_wait(&kv_empty[st], (u - 1) & 1)) {
+                    flag_status(p.status, PA_DEV_TIMEOUT);
+                    atomicExch(&sh[3], 1);
+                    break;
+                }
+                if (*(volatile int*)&sh[3]) break;
+                sh[4] = j + 1;
+                const int k0 = j * C::BN;
+                // Pages (or the part of one page) covering [k0, k0 + BN) that start before T.
+                int npg = 1;
+                if (bs < C::BN) {
+                    npg = (min(k0 + C::BN, T) - k0 + bs - 1) / bs;
+                }
+                const uint32_t bytes = (uint32_t)(npg * box * HEAD * 2);
+                mbar_arrive_expect_tx(&k_full[st], bytes);
+                mbar_arrive_expect_tx(&v_full[st], bytes);
+                for (int pi = 0; pi < npg; ++pi) {
+                    const int key = k0 + pi * box;
+                    const int blk = bt[key / bs];
+                    const int row = key % bs;
+#pragma unroll
+                    for (int c = 0; c < C::NA; ++c) {
+                        const int off = (c * C::BN + pi * box) * C::RB;
+                        tma_load_4d(sK + st * C::KV_BYTES + off, &tm_k, &k_full[st], c * C::A, kvh, row, blk);
+                    }
+                }
+                for (int pi = 0; pi < npg; ++pi) {
+                    const int key = k0 + pi * box;
+                    const int blk = bt[key / bs];
+                    const int row = key % bs;
+#pragma unroll
+                    for (int c = 0; c < C::NA; ++c) {
+                        const int off = (c * C::BN + pi * box) * C::RB;
+                        tma_load_4d(sV + st * C::KV_BYTES + off, &tm_v, &v_full[st], c * C::A, kvh, row, blk);
+                    }
+                }
+            }
+        }
+    } else if (warp == 5) {
+        // ---------------------------------------------------------- MMA issuer
+        constexpr uint32_t idesc_s = umma_idesc_f16(C::BM, C::BN, false, false);
+        constexpr uint32_t idesc_o = umma_idesc_f16(C::BM, HEAD, false, true);
+        const uint32_t q_addr = smem_u32(sQ), k_addr = smem_u32(sK), v_addr = smem_u32(sV),
+                       p_addr = smem_u32(sP);
+        bool alive = mbar_wait_warp(q_full, 0);
+        auto issue_s = [&](int j) {
+            const int st = j % C::NST;
+            if (lane == 0) {
+#pragma unroll
+                for (int kk = 0; kk < HEAD / 16; ++kk) {
+                    const int c = (kk * 16) / C::A, w = (kk * 16) % C::A;
+                    const uint64_t da = umma_sdesc(q_addr + c * C::BM * C::RB + w * 2, 16, 8 * C::RB, C::LAYOUT);
+                    const uint64_t db = umma_sdesc(k_addr + st * C::KV_BYTES + c * C::BN * C::RB + w * 2, 16,
+                                                   8 * C::RB, C::LAYOUT);
+                    umma_f16(tmem + ((j & 1) ? C::COL_S1 : C::COL_S0), da, db, idesc_s, kk > 0 ? 1u : 0u);
+                }
+                umma_commit(&s_full[j & 1]);
+            }
+            __syncwarp();
+        };
+        auto issue_pv = [&](int j) -> bool {
+            const int st = j % C::NST;
+            if (!mbar_wait_warp(p_full, j & 1)) return false;
+            if (!mbar_wait_warp(&v_full[st], (j / C::NST) & 1)) return false;
+            tc_fence_after();
+            const int k0 = j * C::BN;
+            if (k0 + C::BN > T) {
+                // Zero V rows at or past the sequence end (stale or poisoned data).
+                const int r0 = T - k0 > 0 ? T - k0 : 0;
+                uint8_t* vst = sV + st * C::KV_BYTES;
+                for (int c = 0; c < C::NA; ++c)
+                    for (int idx = r0 * (C::RB / 16) + lane; idx < C::BN * (C::RB / 16); idx += 32)
+                        *reinterpret_cast<uint4*>(vst + c * C::BN * C::RB + idx * 16) = make_uint4(0, 0, 0, 0);
+                fence_proxy_async_smem();
+                __syncwarp();
+            }
+            if (lane == 0) {
+#pragma unroll
+                for (int kk = 0; kk < C::BN / 16; ++kk) {
+                    const uint64_t da = umma_sdesc(p_addr + kk * 32, 16, 1024, 2u);
+                    const uint64_t db = umma_sdesc(v_addr + st * C::KV_BYTES + kk * 16 * C::RB,
+                                                   C::BN * C::RB, 8 * C::RB, C::LAYOUT);
+                    umma_f16(tmem + C::COL_O, da, db, idesc_o, (j > 0 || kk > 0) ? 1u : 0u);
+                }
+                umma_commit(pv_done);
+                umma_commit(&kv_empty[st]);
+            }
+            __syncwarp();
+            return true;
+        };
+        for (int j = 0; alive && j < ntiles; ++j) {
+            const int st = j % C::NST;
+            if (!mbar_wait_warp(&k_full[st], (j / C::NST) & 1)) { alive = false; break; }
+            if (j >= 2 && !mbar_wait_warp(&s_free[j & 1], ((j - 2) >> 1) & 1)) { alive = false; break; }
+            tc_fence_after();
+            issue_s(j);
+            if (j >= 1 && !issue_pv(j - 1)) { alive = false; break; }
+        }
+        if (alive && ntiles > 0) alive = issue_pv(ntiles - 1);
+        if (!alive) {
+            if (lane == 0) {
+                flag_status(p.status, PA_DEV_TIMEOUT);
+                atomicExch(&sh[3], 1);
+                // Let every MMA already issued finish before the CTA moves on.
+                umma_commit(drain);
+                mbar_wait(drain, 0);
+            }
+            __syncwarp();
+        }
+    } else {
+        // ---------------------------------------------------------- softmax
+        const int r = threadIdx.x;                       // row == TMEM lane
+        const uint32_t lane_base = (uint32_t)(warp * 32) << 16;
+        const int tok = i0 + r / g;                      // token of this row within the sequence
+        const int lim = (r < rows_valid) ? s.past + tok : T - 1;   // last visible key
+        const int full_vis = s.past + i0;                // every row sees keys <= this
+        float m_used = -INFINITY, l = 0.f;
+        bool alive = true;
+        for (int j = 0; j < ntiles; ++j) {
+            if (!mbar_wait_warp(&s_full[j & 1], (j >> 1) & 1)) { alive = false; break; }
+            tc_fence_after();
+            uint32_t sv[C::BN];
+            const uint32_t scol = tmem + lane_base + ((j & 1) ? C::COL_S1 : C::COL_S0);
+            tmem_ld32(scol, sv);
+            tmem_ld32(scol + 32, sv + 32);
+            tmem_wait_ld();
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&s_free[j & 1]);
+            const int k0 = j * C::BN;
+            float x[C::BN];
+            float mx = -INFINITY;
+            if (k0 + C::BN - 1 <= full_vis) {
+#pragma unroll
+                for (int c = 0; c < C::BN; ++c) {
+                    x[c] = __uint_as_float(sv[c]) * p.scale_log2;
+                    mx = fmaxf(mx, x[c]);
+                }
+            } else {
+#pragma unroll
+                for (int c = 0; c < C::BN; ++c) {
+                    const bool vis = (k0 + c) <= lim;
+                    x[c] = vis ? __uint_as_float(sv[c]) * p.scale_log2 : -INFINITY;
+                    mx = fmaxf(mx, x[c]);
+                }
+            }
+            // Lazy rescale: move the exponent base only when the max grows by > 8.
+            if (mx > m_used + 8.f) {
+                const float alpha = (m_used == -INFINITY) ? 0.f : fast_exp2(m_used - mx);
+                l *= alpha;
+                if (j > 0) {
+                    if (!mbar_wait_warp(pv_done, (j - 1) & 1)) { alive = false; break; }
+                    tc_fence_after();
+                    const uint32_t ocol = tmem + lane_base + C::COL_O;
+#pragma unroll
+                    for (int c0 = 0; c0 < HEAD; c0 += 16) {
+                        uint32_t ov[16];
+                        tmem_ld16(ocol + c0, ov);
+                        tmem_wait_ld();
+#pragma unroll
+                        for (int c = 0; c < 16; ++c) ov[c] = __float_as_uint(__uint_as_float(ov[c]) * alpha);
+                        tmem_st16(ocol + c0, ov);
+                    }
+                    tmem_wait_st();
+                }
+                m_used = mx;
+            }
+            const float base = (m_used == -INFINITY) ? 0.f : m_used;
+            uint32_t pk[C::BN / 2];
+            float rs = 0.f;
+#pragma unroll
+            for (int c = 0; c < C::BN; c += 2) {
+                const float p0 = fast_exp2(x[c] - base);
+                const float p1 = fast_exp2(x[c + 1] - base);
+                rs += p0 + p1;
+                pk[c / 2] = pack_half2(p0, p1);
+            }
+            l += rs;
+            // P_j replaces P_{j-1}: wait until the previous P V product has read it.
+            if (j > 0) {
+                if (!mbar_wait_warp(pv_done, (j - 1) & 1)) { alive = false; break; }
+            }
+            // Row r of P: 64 f16 = 128 bytes = 8 16-byte chunks, 128-byte swizzle.
+#pragma unroll
+            for (int ch = 0; ch < 8; ++ch) {
+                const uint32_t off = swz<128>((uint32_t)(r * 128 + ch * 16));
+                *reinterpret_cast<uint4*>(sP + off) =
+                    make_uint4(pk[4 * ch], pk[4 * ch + 1], pk[4 * ch + 2], pk[4 * ch + 3]);
+            }
+            fence_proxy_async_smem();
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(p_full);
+        }
+        // Epilogue: O / l -> f16 rows of `out`.
+        if (alive && ntiles > 0 && mbar_wait_warp(pv_done, (ntiles - 1) & 1)) {
+            tc_fence_after();
+            const float inv = (l > 0.f) ? 1.f / l : 0.f;
+            const uint32_t ocol = tmem + lane_base + C::COL_O;
+            __half* orow = p.out + ((long long)(s.q_start + tok) * p.q_heads + kvh * g + r % g) * HEAD;
+#pragma unroll
+            for (int c0 = 0; c0 < HEAD; c0 += 16) {
+                uint32_t ov[16];
+                tmem_ld16(ocol + c0, ov);
+                tmem_wait_ld();
+                if (r < rows_valid) {
+                    uint4 w0, w1;
+                    w0.x = pack_half2(__uint_as_float(ov[0]) * inv, __uint_as_float(ov[1]) * inv);
+                    w0.y = pack_half2(__uint_as_float(ov[2]) * inv, __uint_as_float(ov[3]) * inv);
+                    w0.z = pack_half2(__uint_as_float(ov[4]) * inv, __uint_as_float(ov[5]) * inv);
+                    w0.w = pack_half2(__uint_as_float(ov[6]) * inv, __uint_as_float(ov[7]) * inv);
+                    w1.x = pack_half2(__uint_as_float(ov[8]) * inv, __uint_as_float(ov[9]) * inv);
+                    w1.y = pack_half2(__uint_as_float(ov[10]) * inv, __uint_as_float(ov[11]) * inv);
+                    w1.z = pack_half2(__uint_as_float(ov[12]) * inv, __uint_as_float(ov[13]) * inv);
+                    w1.w = pack_half2(__uint_as_float(ov[14]) * inv, __uint_as_float(ov[15]) * inv);
+                    *reinterpret_cast<uint4*>(orow + c0) = w0;
+                    *reinterpret_cast<uint4*>(orow + c0 + 8) = w1;
+                }
+            }
+        } else if (!alive) {
+            if (lane == 0) {
+                flag_status(p.status, PA_DEV_TIMEOUT);
+                atomicExch(&sh[3], 1);
+            }
+        }
+        tc_fence_before();
+    }
+
+    __syncthreads();
+    if (sh[3] && threadIdx.x == 0) {
+        // Aborted (never expected): let in-flight loads land before exit.
+        mbar_wait(q_full, 0);
+        const int issued = sh[4];
+        for (int t = issued - C::NST > 0 ? issued - C::NST : 0; t < issued; ++t) {
+            mbar_wait(&k_full[t % C::NST], (t / C::NST) & 1);
+            mbar_wait(&v_full[t % C::NST], (t / C::NST) & 1);
+        }
+    }
+    __syncthreads();
+    if (warp == 5) {
+        tc_fence_after();
+        tmem_dealloc(tmem, C::TMEM_COLS);
+    }
+}
+
+template <int HEAD>
+cudaError_t launch_prefill_t(const CUtensorMap& tm_q, const CUtensorMap& tm_k,
+                             const CUtensorMap& tm_v, const PrefillParams& p, cudaStream_t stream) {
+    using C = PCfg<HEAD>;
+    auto kern = prefill_kernel<HEAD>;
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM);
+    if (e != cudaSuccess) return e;
+    dim3 grid(p.kv_heads, p.num_slots);
+    kern<<<grid, C::THREADS, C::SMEM, stream>>>(tm_q, tm_k, tm_v, p);
+    return cudaGetLastError();
+}
+
+}  // namespace
+
+cudaError_t launch_prefill(const CUtensorMap& tm_q, const CUtensorMap& tm_k,
+                           const CUtensorMap& tm_v, const PrefillParams& p, int head_size,
+                           cudaStream_t stream) {
+    switch (head_size) {
+        case 16: return launch_prefill_t<16>(tm_q, tm_k, tm_v, p, stream);
+        case 32: return launch_prefill_t<32>(tm_q, tm_k, tm_v, p, stream);
+        case 64: return launch_prefill_t<64>(tm_q, tm_k, tm_v, p, stream);
+        case 128: return launch_prefill_t<128>(tm_q, tm_k, tm_v, p, stream);
+        default: return cudaErrorInvalidValue;
+    }
+}
+
+}  // namespace pa

@@ -1,0 +1,141 @@
+// pa_scatter.cu -- the K/V scatter into the block-table cache and the slot
+// mapping that feeds it.
+//
+// Scatter (ONNX Runtime PR "[WebGPU] Initial PagedAttention implementation
+// (1/n)", "Description": scatter K/V into the paged cache): token t's
+// [kv_heads, head_size] row of K (and of V) is copied to cache block
+// slot / block_size, row slot % block_size.  Both source and destination
+// rows are contiguous, so the copy is a run of 16-byte vectors; consecutive
+// threads take consecutive vectors of the same token, which keeps every warp
+// access fully coalesced on both sides.  Pure HBM traffic: 2 reads + 2
+// writes of token_count * kv_heads * head_size * 2 bytes.
+//
+// Slot mapping (same PR, review "Things I specifically checked": the token
+// -> sequence lookup is the first b with cu_seqlens_q[b+1] > t, skipping
+// zero-length sequences; past_len_b = seqlens_kv[b] - q_len_b).  One thread
+// per token, binary search over cu_seqlens_q.
+#include <cuda_runtime.h>
+
+#include "pa_common.cuh"
+#include "pa_internal.h"
+
+namespace pa {
+
+namespace {
+
+constexpr int kScatterThreads = 256;
+constexpr int kScatterUnroll = 4;
+
+__device__ __forceinline__ uint4 ld_stream(const uint4* p) {
+    uint4 v;
+    asm volatile("ld.global.nc.L1::no_allocate.v4.u32 {%0, %1, %2, %3}, [%4];"
+                 : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w) : "l"(p));
+    return v;
+}
+
+// Grid-stride over 16-byte vectors; each thread moves kScatterUnroll vectors
+// of K and of V per trip so several loads are in flight before the stores.
+__global__ void __launch_bounds__(kScatterThreads)
+scatter_kv_kernel(const uint4* __restrict__ key, const uint4* __restrict__ value,
+                  const int32_t* __restrict__ slot_mapping, uint4* __restrict__ key_cache,
+                  uint4* __restrict__ value_cache, long long token_count, int vec_per_token,
+                  long long num_slots, int32_t* status) {
+    const long long total = token_count * vec_per_token;
+    const long long stride = (long long)gridDim.x * kScatterThreads * kScatterUnroll;
+    for (long long base = (long long)blockIdx.x * kScatterThreads * kScatterUnroll + threadIdx.x;
+         base < total; base += stride) {
+        uint4 kv[kScatterUnroll], vv[kScatterUnroll];
+        long long dst[kScatterUnroll];
+#pragma unroll
+        for (int u = 0; u < kScatterUnroll; ++u) {
+            long long i = base + (long long)u * kScatterThreads;
+            dst[u] = -1;
+            if (i < total) {
+                long long t = i / vec_per_token;
+                int c = (int)(i - t * vec_per_token);
+                int slot = __ldg(slot_mapping + t);
+                if (slot >= 0) {
+                    if ((long long)slot < num_slots) {
+                        dst[u] = (long long)slot * vec_per_token + c;
+                        kv[u] = ld_stream(key + i);
+                        vv[u] = ld_stream(value + i);
+                    } else if (c == 0) {
+                        flag_status(status, PA_DEV_BAD_SLOT);
+                    }
+                }
+            }
+        }
+#pragma unroll
+        for (int u = 0; u < kScatterUnroll; ++u) {
+            if (dst[u] >= 0) {
+                key_cache[dst[u]] = kv[u];
+                value_cache[dst[u]] = vv[u];
+            }
+        }
+    }
+}
+
+__global__ void slot_mapping_kernel(const int32_t* __restrict__ block_table,
+                                    const int32_t* __restrict__ cu,
+                                    const int32_t* __restrict__ seqlens_kv,
+                                    int32_t* __restrict__ slot_mapping, int batch,
+                                    long long token_count, int max_blocks, int block_size,
+                                    long long num_blocks, int32_t* status) {
+    long long t = (long long)blockIdx.x * blockDim.x + threadIdx.x;
+    if (t >= token_count) return;
+    // First b with cu[b+1] > t.
+    int lo = 0, hi = batch;          // answer in [lo, hi)
+    while (lo < hi) {
+        int mid = (lo + hi) >> 1;
+        if ((long long)cu[mid + 1] > t) hi = mid; else lo = mid + 1;
+    }
+    int32_t slot = -1;
+    if (lo < batch) {
+        SeqInfo s;
+        if (load_seq(cu, seqlens_kv, lo, batch, token_count, max_blocks * block_size, 0, 0,
+                     status, s) &&
+            t >= s.q_start) {
+            long long p = (long long)s.past + (t - s.q_start);
+            int blk = block_table[(long long)lo * max_blocks + p / block_size];
+            if (blk < 0 || (long long)blk >= num_blocks) {
+                flag_status(status, PA_DEV_BAD_BLOCK);
+            } else {
+                slot = (int32_t)((long long)blk * block_size + p % block_size);
+            }
+        }
+    } else {
+        flag_status(status, PA_DEV_BAD_CU_SEQLENS);
+    }
+    slot_mapping[t] = slot;
+}
+
+}  // namespace
+
+cudaError_t launch_scatter(const void* key, const void* value, const int32_t* slot_mapping,
+                           void* key_cache, void* value_cache, const pa_dims& d,
+                           int32_t* status, cudaStream_t stream, int num_sms) {
+    const int vec_per_token = d.kv_heads * d.head_size * 2 / 16;
+    const long long total = d.token_count * vec_per_token;
+    long long blocks = (total + kScatterThreads * kScatterUnroll - 1) / (kScatterThreads * kScatterUnroll);
+    const long long cap = (long long)num_sms * 8;
+    if (blocks > cap) blocks = cap;
+    if (blocks < 1) blocks = 1;
+    scatter_kv_kernel<<<(unsigned)blocks, kScatterThreads, 0, stream>>>(
+        static_cast<const uint4*>(key), static_cast<const uint4*>(value), slot_mapping,
+        static_cast<uint4*>(key_cache), static_cast<uint4*>(value_cache), d.token_count,
+        vec_per_token, d.num_blocks * d.block_size, status);
+    return cudaGetLastError();
+}
+
+cudaError_t launch_slot_mapping(const int32_t* block_table, const int32_t* cu,
+                                const int32_t* seqlens_kv, int32_t* slot_mapping,
+                                const pa_dims& d, int32_t* status, cudaStream_t stream) {
+    const int threads = 256;
+    long long blocks = (d.token_count + threads - 1) / threads;
+    slot_mapping_kernel<<<(unsigned)blocks, threads, 0, stream>>>(
+        block_table, cu, seqlens_kv, slot_mapping, d.batch, d.token_count, d.max_blocks_per_seq,
+        d.block_size, d.num_blocks, status);
+    return cudaGetLastError();
+}
+
+}  // namespace pa

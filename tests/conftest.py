@@ -8,6 +8,21 @@ if ROOT not in sys.path:
     sys.path.insert(0, ROOT)
 
 
+def _build_library():
+    """Compile libpagedattn.so (nvcc cross-compiles without a GPU) before any
+    test imports the binding, which refuses to load without it."""
+    import importlib.util
+    path = os.path.join(ROOT, "scatter_kv_b200", "build.py")
+    spec = importlib.util.spec_from_file_location("_pa_build", path)
+    mod = importlib.util.module_from_spec(spec)
+    spec.loader.exec_module(mod)
+    mod.build()
+
+
+def pytest_sessionstart(session):
+    _build_library()
+
+
 def pytest_configure(config):
     config.addinivalue_line("markers", "gpu: needs a CUDA device (B200, sm_100a)")
     config.addinivalue_line("markers", "slow: long-running (full-size workloads)")

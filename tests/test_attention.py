@@ -1,0 +1,128 @@
+"""GPU parity of paged attention (decode split-KV path and tcgen05 prefill
+path) against the fp64 oracle, through the C ABI.  Tolerance: max-abs 4e-3
+and mean-abs 3e-4 on the f16 output (fp32 accumulation)."""
+import itertools
+
+import numpy as np
+import pytest
+
+import oracle
+import workloads
+from pa_harness import (assert_close, oracle_step, poison_unused, run_gpu, sample_rows)
+
+pytestmark = pytest.mark.gpu
+
+
+def _full_check(spec, hints=True, poison=True, seed=None):
+    x = workloads.generate(spec, seed=seed)
+    if poison:
+        poison_unused(spec, x)
+    got, _, status, slots = run_gpu(spec, x, hints=hints)
+    want, _, _, want_slots = oracle_step(spec, x)
+    assert status == 0
+    assert np.array_equal(slots, want_slots)
+    assert_close(got, want, what=spec.name)
+    return got, want
+
+
+def test_tiny_config():
+    _full_check(workloads.spec_tiny())
+
+
+# The shape matrix of the PagedAttention PR's parity suite ("Test coverage":
+# MHA and GQA, batch 1 and 2, new tokens 1/4/16, totals 32/64), at block sizes
+# 16 and 256 and head size 128.
+M1 = list(itertools.product([(4, 4), (8, 2)], [1, 2], [1, 4, 16], [32, 64], [16, 256]))
+
+
+@pytest.mark.parametrize("heads,batch,q_len,total,bs", M1)
+def test_shape_matrix(heads, batch, q_len, total, bs):
+    qh, kvh = heads
+    q = [q_len] * batch
+    past = [total - q_len] * batch
+    if batch == 2:                      # second sequence a little shorter: ragged ends
+        past[1] = max(0, past[1] - 7)
+    spec = workloads.custom(q, past, qh, kvh, 128, bs, seed=batch * 1000 + q_len * 10 + total)
+    _full_check(spec)
+
+
+@pytest.mark.parametrize("head_size", [16, 32, 64, 128])
+@pytest.mark.parametrize("q_lens,past", [
+    ([1, 3, 2], [40, 0, 129]),           # decode path, several splits of short sequences
+    ([9, 130, 64], [0, 17, 300]),        # prefill path: ragged query tiles and diagonals
+])
+def test_head_sizes(head_size, q_lens, past):
+    spec = workloads.custom(q_lens, past, 8, 2, head_size, 16, seed=head_size)
+    _full_check(spec)
+
+
+@pytest.mark.parametrize("qh,kvh,q_lens,past,bs", [
+    (16, 16, [129, 300], [0, 1000], 256),      # MHA, one row past a tile, long past
+    (32, 8, [37, 5, 200], [500, 3, 64], 16),   # GQA 4: 32 tokens per tile
+    (64, 8, [5, 77], [1000, 12], 32),          # GQA 8: 16 tokens per tile, bs 32
+    (32, 1, [2, 3, 40], [100, 0, 7], 64),      # GQA 32: decode cut-off 1, q_len 2 is prefill
+    (8, 4, [256], [0], 128),                   # exactly two tiles, no past
+])
+def test_prefill_shapes(qh, kvh, q_lens, past, bs):
+    spec = workloads.custom(q_lens, past, qh, kvh, 128, bs, seed=sum(q_lens))
+    _full_check(spec)
+
+
+def test_mixed_batch_with_empty_sequences():
+    q_lens = [1, 0, 200, 4, 0, 33, 1, 2, 3, 600]
+    past = [3000, 5, 100, 2000, 0, 0, 1, 7000, 12, 250]
+    spec = workloads.custom(q_lens, past, 32, 8, 128, 16, seed=77)
+    _full_check(spec)
+
+
+def test_without_hints():
+    spec = workloads.custom([1, 70, 3], [900, 40, 5000], 16, 4, 128, 16, seed=5)
+    _full_check(spec, hints=False)
+
+
+@pytest.mark.parametrize("q_lens,past,bs", [([1, 2, 4], [0, 0, 0], 16), ([50, 128], [0, 0], 256)])
+def test_first_row_of_fresh_sequence_is_v0(q_lens, past, bs):
+    spec = workloads.custom(q_lens, past, 8, 2, 128, bs, seed=3)
+    x = workloads.generate(spec)
+    got, _, status, _ = run_gpu(spec, x)
+    cu = np.concatenate([[0], np.cumsum(q_lens)])
+    for b in range(spec.batch):
+        for h in range(spec.q_heads):
+            v0 = x["value"][cu[b], h // (spec.q_heads // spec.kv_heads)]
+            assert np.array_equal(got[cu[b], h].view(np.uint16), v0.view(np.uint16))
+
+
+@pytest.mark.parametrize("cfg", [1, 3, 4])
+def test_deterministic_across_runs_and_page_permutations(cfg):
+    spec = workloads.CONFIGS[cfg]()
+    if cfg == 4:    # keep this one small: 2 sequences of the long-context shape
+        spec = workloads.custom(spec.q_lens[:2], spec.past[:2] // 8, spec.q_heads, spec.kv_heads,
+                                128, spec.block_size, seed=4)
+    x = workloads.generate(spec)
+    outs, _, _, _ = run_gpu(spec, x, repeat=2)
+    assert np.array_equal(outs[0].view(np.uint16), outs[1].view(np.uint16))
+    # Same logical contents under another placement of the pages.
+    rng = np.random.default_rng(11)
+    y = workloads.generate(spec, block_order=rng.permutation(spec.num_blocks))
+    for name in ("key_cache", "value_cache"):
+        y[name][:] = 0
+        for s in range(spec.batch):
+            for p in range(int(spec.pages_per_seq[s])):
+                y[name][y["block_table"][s, p]] = x[name][x["block_table"][s, p]]
+    for name in ("query", "key", "value"):
+        y[name] = x[name]
+    got2, _, _, _ = run_gpu(spec, y)
+    assert np.array_equal(outs[0].view(np.uint16), got2.view(np.uint16))
+
+
+@pytest.mark.parametrize("cfg", [1, 2, 3, 4])
+def test_full_size_config_sampled(cfg):
+    spec = workloads.CONFIGS[cfg]()
+    x = workloads.generate(spec)
+    got, _, status, slots = run_gpu(spec, x)
+    rows = sample_rows(spec, 96, seed=cfg)
+    want, _, _, want_slots = oracle_step(spec, x, rows=rows)
+    assert status == 0
+    assert np.array_equal(slots, want_slots)
+    assert_close(got[rows[:, 0], rows[:, 1]], want, what=spec.name)
+    assert np.isfinite(got.astype(np.float32)).all()
