@@ -145,6 +145,32 @@ pa_status pa_attention(const void* query, const void* key_cache, const void* val
                        void* workspace, size_t workspace_bytes, int32_t* dev_status,
                        void* stream);
 
+/* pa_attention_noalloc -- pa_attention for callers that cannot allocate
+ * device memory.  The pages describe no such variant; it exists for this
+ * library's users.  Some callers own no allocator: code embedded in a host
+ * runtime that hands out a fixed memory budget and no workspace hook, or a
+ * latency-critical path that must not call cudaMalloc (it can synchronise
+ * the device).  They still pass inputs and outputs exactly as for
+ * pa_attention; the split-KV scratch comes from a fixed array of 8 MiB
+ * compiled into the library, which every GPU that loads the library holds
+ * until the process exits.
+ *   Arguments: as for pa_attention, without workspace / workspace_bytes.
+ *   Limit: dims whose pa_attention_workspace_size() exceeds 8 MiB are
+ *          rejected with PA_ERR_INVALID_ARGUMENT (use pa_attention then).
+ *   Set-up: the first call on each device looks up the array's device
+ *          address (cudaGetSymbolAddress) with that device current; make that
+ *          first call before any stream capture.
+ *   Sharing: all calls on a device share the one array and it keeps the
+ *          last call's contents (none need clearing: every scratch value is
+ *          written before it is read within a call).  Calls whose kernels
+ *          overlap on the GPU -- other streams, other host threads -- race on
+ *          it; serialise them.
+ *   It allocates nothing: no cudaMalloc, cudaFree or allocating library call. */
+pa_status pa_attention_noalloc(const void* query, const void* key_cache, const void* value_cache,
+                               const int32_t* block_table, const int32_t* cu_seqlens_q,
+                               const int32_t* seqlens_kv, float scale, void* out,
+                               const pa_dims* dims, int32_t* dev_status, void* stream);
+
 /* pa_get_status -- synchronise `stream` and copy *dev_status to *host_code.
  * For tests and debugging; it blocks the host. */
 pa_status pa_get_status(const int32_t* dev_status, int32_t* host_code, void* stream);

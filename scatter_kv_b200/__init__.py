@@ -76,8 +76,11 @@ class PagedAttentionError(RuntimeError):
 EXPORTS = [
     "pa_scatter_kv", "pa_compute_slot_mapping", "pa_attention_workspace_size", "pa_attention",
     "pa_get_status", "pa_status_string", "pa_last_error", "pa_trace_enable", "pa_trace_read",
-    "pa_kernel_name",
+    "pa_kernel_name", "pa_attention_noalloc",
 ]
+
+# Bytes of the fixed scratch array behind pa_attention_noalloc.
+NOALLOC_SCRATCH_BYTES = 8 << 20
 
 
 def _load():
@@ -96,6 +99,8 @@ def _load():
     lib.pa_attention_workspace_size.restype = ctypes.c_int
     lib.pa_attention.argtypes = [P, P, P, P, P, P, ctypes.c_float, P, D, P, ctypes.c_size_t, P, P]
     lib.pa_attention.restype = ctypes.c_int
+    lib.pa_attention_noalloc.argtypes = [P, P, P, P, P, P, ctypes.c_float, P, D, P, P]
+    lib.pa_attention_noalloc.restype = ctypes.c_int
     lib.pa_get_status.argtypes = [P, I32P, P]
     lib.pa_get_status.restype = ctypes.c_int
     lib.pa_status_string.argtypes = [ctypes.c_int]
@@ -198,6 +203,19 @@ def pa_attention(query, key_cache, value_cache, block_table, cu_seqlens_q, seqle
                             _ptr(cu_seqlens_q), _ptr(seqlens_kv), float(scale), _ptr(out),
                             ctypes.byref(dims), _ptr(workspace), int(workspace_bytes),
                             _ptr(dev_status), _stream(stream)))
+
+
+def pa_attention_noalloc(query, key_cache, value_cache, block_table, cu_seqlens_q, seqlens_kv,
+                         scale, out, dims: pa_dims, dev_status=None, stream=None) -> None:
+    """pa_attention without a workspace argument, for callers that cannot
+    allocate device memory: the split-KV scratch is a fixed 8 MiB array inside
+    the library (dims needing more are rejected).  Calls that overlap on the
+    GPU share that array and race; the first call on a device looks up the
+    array's address and should come before any stream capture."""
+    _check(lib.pa_attention_noalloc(_ptr(query), _ptr(key_cache), _ptr(value_cache),
+                                    _ptr(block_table), _ptr(cu_seqlens_q), _ptr(seqlens_kv),
+                                    float(scale), _ptr(out), ctypes.byref(dims), _ptr(dev_status),
+                                    _stream(stream)))
 
 
 def pa_get_status(dev_status, stream=None) -> int:

@@ -363,6 +363,28 @@ pa_status pa_attention(const void* query, const void* key_cache, const void* val
     return PA_OK;
 }
 
+pa_status pa_attention_noalloc(const void* query, const void* key_cache, const void* value_cache,
+                               const int32_t* block_table, const int32_t* cu_seqlens_q,
+                               const int32_t* seqlens_kv, float scale, void* out,
+                               const pa_dims* dims, int32_t* dev_status, void* stream) {
+    g_last_error[0] = 0;
+    pa_status st = check_dims(dims);
+    if (st != PA_OK) return st;
+    const size_t need = pa::plan_decode(*dims, num_sms_of_current_device()).workspace_bytes;
+    if (need > pa::kNoAllocScratchBytes)
+        return fail(PA_ERR_INVALID_ARGUMENT,
+                    "these dims need %zu bytes of split-KV scratch, more than the %zu-byte fixed "
+                    "array of pa_attention_noalloc; call pa_attention with a workspace instead",
+                    need, pa::kNoAllocScratchBytes);
+    void* scratch = nullptr;
+    if (need > 0) {
+        cudaError_t e = pa::noalloc_scratch(&scratch);
+        if (e != cudaSuccess) return cuda_fail(e, "cudaGetSymbolAddress(noalloc scratch)");
+    }
+    return pa_attention(query, key_cache, value_cache, block_table, cu_seqlens_q, seqlens_kv, scale,
+                        out, dims, scratch, need, dev_status, stream);
+}
+
 pa_status pa_get_status(const int32_t* dev_status, int32_t* host_code, void* stream) {
     g_last_error[0] = 0;
     if (dev_status == nullptr || host_code == nullptr)

@@ -28,6 +28,8 @@
 #include <cuda_runtime.h>
 #include <math.h>
 
+#include <mutex>
+
 #include "pa_common.cuh"
 #include "pa_internal.h"
 
@@ -559,6 +561,37 @@ cudaError_t launch_combine(const DecodeParams& p, int head_size, cudaStream_t st
         default: return cudaErrorInvalidValue;
     }
 #undef PA_COMBINE_CASE
+}
+
+}  // namespace pa
+
+// ---------------------------------------------------------------------------
+// Fixed device scratch for pa_attention_noalloc: the split-KV partial results
+// live in this file-scope array instead of a caller-provided workspace.  The
+// array is part of the library image, so every GPU that loads the library
+// holds these bytes until the process exits.  In host code the symbol is
+// only a host-side stand-in; its device address comes from
+// cudaGetSymbolAddress, looked up once per device.
+static __device__ __align__(256) unsigned char pa_noalloc_scratch[pa::kNoAllocScratchBytes];
+
+namespace pa {
+
+cudaError_t noalloc_scratch(void** ptr) {
+    static std::mutex mu;
+    static void* addr[kMaxDevices] = {nullptr};
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return e;
+    if (dev < 0 || dev >= kMaxDevices) return cudaErrorInvalidDevice;
+    std::lock_guard<std::mutex> lock(mu);
+    if (addr[dev] == nullptr) {
+        void* p = nullptr;
+        e = cudaGetSymbolAddress(&p, pa_noalloc_scratch);
+        if (e != cudaSuccess) return e;
+        addr[dev] = p;
+    }
+    *ptr = addr[dev];
+    return cudaSuccess;
 }
 
 }  // namespace pa

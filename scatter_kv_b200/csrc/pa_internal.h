@@ -84,6 +84,12 @@ cudaError_t launch_decode(const CUtensorMap& tm_k, const CUtensorMap& tm_v,
                           const DecodeParams& p, int head_size, int mtiles, cudaStream_t stream);
 cudaError_t launch_combine(const DecodeParams& p, int head_size, cudaStream_t stream);
 
+// Size of the fixed scratch array behind pa_attention_noalloc, and the
+// lookup of its device address on the current device (once per device).
+constexpr size_t kNoAllocScratchBytes = size_t(8) << 20;
+constexpr int kMaxDevices = 64;
+cudaError_t noalloc_scratch(void** ptr);
+
 cudaError_t launch_prefill(const CUtensorMap& tm_q, const CUtensorMap& tm_k,
                            const CUtensorMap& tm_v, const PrefillParams& p, int head_size,
                            cudaStream_t stream);
