@@ -25,7 +25,6 @@ import json
 import math
 import os
 import re
-import subprocess
 import sys
 import threading
 import time
@@ -79,60 +78,75 @@ def load_peaks() -> dict:
 # ----------------------------------------------------------------- clocks
 
 class ClockSampler:
-    """nvidia-smi samples (every 200 ms) while the timed region runs."""
+    """SM clock and throttle reasons sampled through NVML (every ~1 ms) on
+    this rank's GPU while the timed region runs (read only: nothing is set)."""
 
-    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
-              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
-              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+    REASONS = {"hw_slowdown": "nvmlClocksEventReasonHwSlowdown",
+               "hw_thermal_slowdown": "nvmlClocksEventReasonHwThermalSlowdown",
+               "sw_thermal_slowdown": "nvmlClocksEventReasonSwThermalSlowdown",
+               "sw_power_cap": "nvmlClocksEventReasonSwPowerCap"}
 
-    def __init__(self, gpu_index: int):
-        self.gpu = gpu_index
-        self.proc = None
-        self.lines = []
+    def __init__(self, torch_device: int):
+        self.dev = torch_device
+        self.samples = []
+        self.max_mhz = None
+        self.stop_flag = threading.Event()
         self.thread = None
+        self.err = None
+
+    def _handle(self):
+        import pynvml
+        import torch
+        pynvml.nvmlInit()
+        props = torch.cuda.get_device_properties(self.dev)
+        bus = getattr(props, "pci_bus_id", None)
+        if bus is not None:
+            busid = "%08x:%02x:%02x.0" % (getattr(props, "pci_domain_id", 0), bus,
+                                          getattr(props, "pci_device_id", 0))
+            try:
+                return pynvml.nvmlDeviceGetHandleByPciBusId(busid.encode())
+            except Exception:
+                pass
+        vis = os.environ.get("CUDA_VISIBLE_DEVICES", "")
+        idx = self.dev
+        if vis and all(v.strip().isdigit() for v in vis.split(",")):
+            idx = int(vis.split(",")[self.dev])
+        return pynvml.nvmlDeviceGetHandleByIndex(idx)
 
     def start(self):
         try:
-            self.proc = subprocess.Popen(
-                ["nvidia-smi", "-i", str(self.gpu), f"--query-gpu={self.FIELDS}",
-                 "--format=csv,noheader,nounits", "-lms", "200"],
-                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
-        except OSError:
-            self.proc = None
+            import pynvml
+            h = self._handle()
+            self.max_mhz = float(pynvml.nvmlDeviceGetMaxClockInfo(h, pynvml.NVML_CLOCK_SM))
+            bits = {k: getattr(pynvml, v, 0) for k, v in self.REASONS.items()}
+        except Exception as e:  # NVML unavailable: report it, do not guess
+            self.err = f"nvml unavailable: {e}"
             return
-        self.thread = threading.Thread(target=self._read, daemon=True)
+
+        def run():
+            while not self.stop_flag.is_set():
+                try:
+                    mhz = pynvml.nvmlDeviceGetClockInfo(h, pynvml.NVML_CLOCK_SM)
+                    r = pynvml.nvmlDeviceGetCurrentClocksEventReasons(h)
+                    self.samples.append((float(mhz), [k for k, b in bits.items() if b and (r & b)]))
+                except Exception as e:
+                    self.err = str(e)
+                    return
+                time.sleep(0.001)
+        self.thread = threading.Thread(target=run, daemon=True)
         self.thread.start()
 
-    def _read(self):
-        for line in self.proc.stdout:
-            self.lines.append(line.strip())
-
     def stop(self) -> dict:
-        if self.proc is None:
-            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
-        time.sleep(0.25)
-        self.proc.terminate()
-        try:
-            self.proc.wait(timeout=5)
-        except subprocess.TimeoutExpired:
-            self.proc.kill()
-        sm, smax, reasons = [], [], set()
-        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
-        for ln in self.lines:
-            parts = [p.strip() for p in ln.split(",")]
-            if len(parts) < 9:
-                continue
-            try:
-                sm.append(float(parts[1]))
-                smax.append(float(parts[2]))
-            except ValueError:
-                continue
-            for n, v in zip(names, parts[5:9]):
-                if v.lower() == "active":
-                    reasons.add(n)
-        return {"sm_mhz": float(np.median(sm)) if sm else None,
-                "sm_max_mhz": max(smax) if smax else None,
-                "samples": len(sm), "reasons": sorted(reasons)}
+        self.stop_flag.set()
+        if self.thread is not None:
+            self.thread.join(timeout=5)
+        if not self.samples:
+            return {"sm_mhz": None, "sm_max_mhz": self.max_mhz, "samples": 0,
+                    "reasons": [self.err or "no samples"]}
+        mhz = [m for m, _ in self.samples]
+        reasons = sorted({r for _, rs in self.samples for r in rs})
+        return {"sm_mhz": float(np.median(mhz)), "sm_max_mhz": self.max_mhz,
+                "samples": len(mhz), "reasons": reasons}
 
 
 # ----------------------------------------------------------------- distributed
@@ -293,11 +307,17 @@ def run_gpu(args, spec, rank, world, local):
         if status != 0:
             raise RuntimeError(f"device status {status:#x} on the benchmark inputs")
 
-        # ---- device-timed region: K steps, L2 flushed between steps
+        # ---- the step as a CUDA graph (launch-bound small kernels replay
+        # without host gaps); tracing stays off during capture.
+        graph = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(graph, stream=stream):
+            step()
+        graph.replay()
+        stream.synchronize()
+
+        # ---- device-timed region: K graph replays, L2 flushed between steps
         ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
               for _ in range(args.steps)]
-        pa.pa_trace_read()
-        pa.pa_trace_enable(True)
         clocks = ClockSampler(local)
         clocks.start()
         barrier(world, dev)
@@ -305,15 +325,26 @@ def run_gpu(args, spec, rank, world, local):
         for k in range(args.steps):
             flush.fill_(k)
             ev[k][0].record(stream)
-            step()
+            graph.replay()
             ev[k][1].record(stream)
         torch.cuda.synchronize()
         barrier(world, dev)
         clk = clocks.stop()
-        pa.pa_trace_enable(False)
-        trace = pa.pa_trace_read()
         ms = sum(a.elapsed_time(b) for a, b in ev)
         ms = max_over_ranks(ms, world, dev)
+
+        # ---- per-kernel durations: K eager steps with the library's event
+        # tracing (one event pair around every launch), same flushes.
+        pa.pa_trace_read()
+        pa.pa_trace_enable(True)
+        barrier(world, dev)
+        torch.cuda.synchronize()
+        for k in range(args.steps):
+            flush.fill_(k)
+            step()
+        torch.cuda.synchronize()
+        pa.pa_trace_enable(False)
+        trace = pa.pa_trace_read()
 
         # ---- end-to-end through the public API with host buffers
         host = {k: torch.from_numpy(np.ascontiguousarray(x[k])).pin_memory()
@@ -399,6 +430,7 @@ def run_gpu(args, spec, rank, world, local):
             "e2e": {"value": e2e_value, "unit": unit, "h2d_bytes_per_step": h2d,
                     "d2h_bytes_per_step": d2h},
             "gpu_launches": launches,
+            "timing": "value: CUDA-graph replays of the step; kernels: eager traced steps",
             "kernels": {n: {"launches": len(v), "avg_ms": float(np.mean(v))} for n, v in per_kernel.items()},
             "algorithmic": {k: v for k, v in counts.items() if k != "decode"},
             "clocks": clk,
@@ -422,7 +454,7 @@ def x_with_scatter(x, spec):
 def main(argv=None):
     ap = argparse.ArgumentParser(description=__doc__.split("\n")[0])
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--steps", type=int, default=100)
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--workload", default="decode", choices=sorted(workloads.CONFIG_KEYS))

@@ -156,6 +156,7 @@ pa_status check_dims(const pa_dims* dp) {
     if (d.dtype != PA_DTYPE_F16) return fail(PA_ERR_INVALID_ARGUMENT, "unknown dtype %d", d.dtype);
     if (d.batch < 0 || d.token_count < 0)
         return fail(PA_ERR_INVALID_ARGUMENT, "negative batch or token_count");
+    if (d.batch > 65535) return fail(PA_ERR_NOT_IMPLEMENTED, "batch %d > 65535", d.batch);
     if (d.q_heads <= 0 || d.kv_heads <= 0 || d.q_heads % d.kv_heads != 0)
         return fail(PA_ERR_INVALID_ARGUMENT, "q_heads (%d) must be a positive multiple of kv_heads (%d)",
                     d.q_heads, d.kv_heads);
@@ -329,7 +330,8 @@ pa_status pa_attention(const void* query, const void* key_cache, const void* val
         const long long slots = (d.token_count * g + pa::kPrefillRows - 1) / pa::kPrefillRows +
                                 (longer < d.batch ? longer : d.batch);
         if (slots > 0) {
-            if (slots > 65535) return fail(PA_ERR_NOT_IMPLEMENTED, "too many query tiles (%lld)", slots);
+            if (slots * d.kv_heads >= (1ll << 31))
+                return fail(PA_ERR_NOT_IMPLEMENTED, "too many query tiles (%lld)", slots);
             CUtensorMap tq, tk, tv;
             const int rows = d.block_size < 64 ? d.block_size : 64;
             if ((st = make_query_map(&tq, query, d)) != PA_OK) return st;

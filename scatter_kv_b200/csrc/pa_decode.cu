@@ -77,7 +77,10 @@ decode_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ 
     float* row_m = row_l + C::RMAX;                             // [RMAX]
     int* sflag = reinterpret_cast<int*>(row_m + C::RMAX);       // [0] bad seq, [1] abort, [2] issued
 
-    const int b = blockIdx.z, kvh = blockIdx.y, split = blockIdx.x;
+    // Grid (kv_heads, splits, batch): the KV heads of one split are adjacent
+    // in launch order, so they stream the same pages (whose rows interleave
+    // all heads) at about the same time.
+    const int b = blockIdx.z, kvh = blockIdx.x, split = blockIdx.y;
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int g = p.group;
     // Status bits of a sequence are reported once, by CTA (split 0, kv head 0).
@@ -489,7 +492,7 @@ cudaError_t launch_decode_t(const CUtensorMap& tm_k, const CUtensorMap& tm_v,
     auto kern = decode_kernel<HEAD, MT>;
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM);
     if (e != cudaSuccess) return e;
-    dim3 grid(p.max_splits, p.kv_heads, p.batch);
+    dim3 grid(p.kv_heads, p.max_splits, p.batch);
     kern<<<grid, C::THREADS, C::SMEM, stream>>>(tm_k, tm_v, p);
     return cudaGetLastError();
 }
@@ -514,6 +517,7 @@ DecodePlan plan_decode(const pa_dims& d, int num_sms) {
     long long chunk = (units * max_kv + (long long)num_sms * 16 - 1) / ((long long)num_sms * 16);
     if (chunk < 256) chunk = 256;
     if (chunk > 16384) chunk = 16384;
+    if (chunk < (max_kv + 65534) / 65535) chunk = (max_kv + 65534) / 65535;   // grid.y limit
     chunk = (chunk + kDecodeKeys - 1) / kDecodeKeys * kDecodeKeys;
     pl.chunk = (int)chunk;
     pl.max_splits = (int)((max_kv + chunk - 1) / chunk);

@@ -17,21 +17,28 @@
 //
 // Warp roles (192 threads):
 //   warps 0-3  softmax + epilogue; thread r owns query row r = TMEM lane r;
-//   warp 4     TMA producer (Q once, then K and V tiles, 2-stage rings);
+//   warp 4     TMA producer (Q once; K tiles in a 3-stage ring, V tiles in a
+//              2-stage ring, K one tile ahead of V);
 //   warp 5     TMEM allocator and single-thread tcgen05.mma issuer.
-// Per key tile j:  S_j = Q K_j^T  (M 128, N 64, fp32 in TMEM, two buffers)
-//                  softmax_j: row max / exp2 / row sum in registers, P_j
-//                  as f16 into shared memory (128-byte swizzled, K-major)
-//                  O += P_j V_j  (M 128, N head_size, fp32 in TMEM)
-// The MMA warp issues S_{j+1} before waiting for P_j, so the tensor core
-// works on the next scores while the softmax threads exponentiate.  O is
-// rescaled only when a row maximum grows by more than 2^8 (values of P
-// stay below 256, exact enough in f16 and fp32 sums), which after the first
-// tiles is rare.  Key tiles wholly above the causal diagonal are never
-// loaded; the diagonal tile is masked per element; rows of V past the end of
-// the sequence are zeroed in shared memory before the last P V product.
-// Two CTAs fit on an SM (112 KB shared memory, 256 TMEM columns each), so
-// one CTA's softmax overlaps the other's MMAs and loads.
+// Per key tile j (TMEM: S/P buffers j % 2 at columns 0 / 64, O at 128):
+//   S_j = Q K_j^T        M 128, N 64, fp32 into buffer j % 2; K_j is released
+//                        as soon as this product is done;
+//   softmax_j            row max / exp2 / row sum in registers; P_j as f16
+//                        written back over S_j (32 columns, 2 per column);
+//   O += P_j V_j         A operand P_j straight from TMEM, M 128, N head_size.
+// The MMA warp issues S_{j+1} before waiting for P_j and S_{j+2} right after
+// P_j V_j (the tensor pipe runs a thread's MMAs in order, so S_{j+2} cannot
+// overwrite P_j before it is read): the softmax threads never wait for a P V
+// product except when a row maximum grows by more than 2^8 and O must be
+// rescaled (values of P stay below 256, exact enough in f16 and fp32 sums),
+// which after the first tiles is rare.  Key tiles wholly above the causal
+// diagonal are never loaded; the diagonal tile is masked per element; rows
+// of V past the end of the sequence are zeroed in shared memory before the
+// last P V product.  CTAs are ordered sequence-major, then KV head, then
+// query tile from the last (most keys) to the first, so the CTAs resident
+// at any time share few sequences' K/V and reuse them from L2.  Two CTAs fit
+// on an SM (112 KB shared memory, 256 TMEM columns each), so one CTA's
+// softmax overlaps the other's MMAs and loads.
 #include <cuda_runtime.h>
 #include <math.h>
 
@@ -52,64 +59,64 @@ struct PCfg {
     static constexpr uint32_t LAYOUT = RB == 128 ? 2u : (RB == 64 ? 4u : 6u);
     static constexpr int Q_BYTES = BM * HEAD * 2;
     static constexpr int KV_BYTES = BN * HEAD * 2;
-    static constexpr int P_BYTES = BM * BN * 2;         // 128 rows x 64 keys, one 128-B atom column
-    static constexpr int NST = 2;
+    static constexpr int NK = 3;                        // K stages
+    static constexpr int NV = 2;                        // V stages
     static constexpr int OFF_Q = 0;
     static constexpr int OFF_K = OFF_Q + Q_BYTES;
-    static constexpr int OFF_V = OFF_K + NST * KV_BYTES;
-    static constexpr int OFF_P = OFF_V + NST * KV_BYTES;
-    static constexpr int OFF_BAR = OFF_P + P_BYTES;
-    // q, k_full/v_full/kv_empty per stage, s_full x2, s_free x2, p_full, pv_done, drain
-    static constexpr int NBAR = 1 + 3 * NST + 2 + 2 + 3;
+    static constexpr int OFF_V = OFF_K + NK * KV_BYTES;
+    static constexpr int OFF_BAR = OFF_V + NV * KV_BYTES;
+    // q_full, k_full/k_empty x NK, v_full/v_empty x NV, s_full x2, p_full x2, pv_done,
+    // o_full, drain
+    static constexpr int NBAR = 1 + 2 * NK + 2 * NV + 2 + 2 + 3;
     static constexpr int SMEM = OFF_BAR + NBAR * 8 + 64;
     static constexpr int THREADS = 192;
-    static constexpr uint32_t TMEM_COLS = 256;          // S0 (64) | S1 (64) | O (head_size)
-    static constexpr uint32_t COL_S0 = 0, COL_S1 = 64, COL_O = 128;
+    static constexpr uint32_t TMEM_COLS = 256;          // S/P 0 (64) | S/P 1 (64) | O (head_size)
+    static constexpr uint32_t COL_O = 128;
 };
 
 struct Work {
     int b;          // sequence
+    int kvh;        // KV head
     int tile;       // query tile within the sequence
 };
 
-// Heavy-first order of the query tiles: slot k lists, for r = 0, 1, ..., the
-// sequences that have more than r tiles, taking tile (ntiles_b - 1 - r).
-// Later tiles see more keys, so the largest pieces of work start first.
-__device__ bool find_work(const PrefillParams& p, int slot, Work& w) {
+// CTA x -> (sequence, KV head, query tile): sequences in order, each with
+// its kv_heads x ntiles_b CTAs; within a KV head the tiles run from the last
+// (the most keys) to the first.  One warp, 32 sequences per step.
+__device__ bool find_work(const PrefillParams& p, long long slot, Work& w) {
     const int lane = threadIdx.x & 31;
-    for (int r = 0;; ++r) {
-        int cnt = 0;
-        bool any = false;
-        for (int b0 = 0; b0 < p.batch; b0 += 32) {
-            const int b = b0 + lane;
-            int nt = 0;
-            if (b < p.batch) {
-                const int c0 = p.cu_seqlens_q[b], c1 = p.cu_seqlens_q[b + 1];
-                const int ql = c1 - c0;
-                if (ql > p.decode_max_q && c0 >= 0 && (long long)c1 <= p.token_count)
-                    nt = (ql * p.group + PCfg<128>::BM - 1) / PCfg<128>::BM;
-            }
-            const bool has = nt > r;
-            any |= nt > r;
-            const unsigned m = __ballot_sync(0xffffffffu, has);
-            const int n = __popc(m);
-            if (slot < cnt + n) {
-                // The (slot - cnt)-th set bit of m.
-                int want = slot - cnt;
-                unsigned mm = m;
-                for (int i = 0; i < want; ++i) mm &= mm - 1;
-                const int lb = __ffs(mm) - 1;
-                const int bsel = b0 + lb;
-                const int ntsel = __shfl_sync(0xffffffffu, nt, lb);
-                w.b = bsel;
-                w.tile = ntsel - 1 - r;
-                return true;
-            }
-            cnt += n;
+    for (int b0 = 0; b0 < p.batch; b0 += 32) {
+        const int b = b0 + lane;
+        int nt = 0;
+        if (b < p.batch) {
+            const int c0 = p.cu_seqlens_q[b], c1 = p.cu_seqlens_q[b + 1];
+            const int ql = c1 - c0;
+            if (ql > p.decode_max_q && c0 >= 0 && (long long)c1 <= p.token_count)
+                nt = (ql * p.group + kPrefillRows - 1) / kPrefillRows;
         }
-        if (!__any_sync(0xffffffffu, any)) return false;
-        slot -= cnt;
+        const long long cnt = (long long)nt * p.kv_heads;
+        long long pre = cnt;                       // inclusive prefix over lanes
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+            const long long v = __shfl_up_sync(0xffffffffu, pre, o);
+            if (lane >= o) pre += v;
+        }
+        const long long total = __shfl_sync(0xffffffffu, pre, 31);
+        if (slot < total) {
+            const unsigned m = __ballot_sync(0xffffffffu, pre > slot);
+            const int lb = __ffs(m) - 1;
+            const long long pre_b = __shfl_sync(0xffffffffu, pre, lb);
+            const long long cnt_b = __shfl_sync(0xffffffffu, cnt, lb);
+            const int nt_b = __shfl_sync(0xffffffffu, nt, lb);
+            const long long local = slot - (pre_b - cnt_b);
+            w.b = b0 + lb;
+            w.kvh = (int)(local / nt_b);
+            w.tile = nt_b - 1 - (int)(local % nt_b);
+            return true;
+        }
+        slot -= total;
     }
+    return false;
 }
 
 template <int HEAD>
@@ -120,19 +127,20 @@ prefill_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
     extern __shared__ __align__(1024) uint8_t smem[];
     uint64_t* bars = reinterpret_cast<uint64_t*>(smem + C::OFF_BAR);
     uint64_t* q_full = bars;
-    uint64_t* k_full = bars + 1;
-    uint64_t* v_full = k_full + C::NST;
-    uint64_t* kv_empty = v_full + C::NST;
-    uint64_t* s_full = kv_empty + C::NST;
-    uint64_t* s_free = s_full + 2;
-    uint64_t* p_full = s_free + 2;
-    uint64_t* pv_done = p_full + 1;
-    uint64_t* drain = pv_done + 1;
+    uint64_t* k_full = q_full + 1;
+    uint64_t* k_empty = k_full + C::NK;
+    uint64_t* v_full = k_empty + C::NK;
+    uint64_t* v_empty = v_full + C::NV;
+    uint64_t* s_full = v_empty + C::NV;      // [2]
+    uint64_t* p_full = s_full + 2;           // [2]
+    uint64_t* pv_done = p_full + 2;
+    uint64_t* o_full = pv_done + 1;          // every MMA of the tile done (single use)
+    uint64_t* drain = o_full + 1;
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + C::NBAR);
-    int* sh = reinterpret_cast<int*>(tmem_slot + 1);   // [0] b, [1] tile, [2] bad, [3] abort, [4] issued
+    // [0] b, [1] tile, [2] bad, [3] abort, [4] K tiles issued, [5] V tiles issued, [6] kv head
+    int* sh = reinterpret_cast<int*>(tmem_slot + 1);
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const int kvh = blockIdx.x;
     const int g = p.group;
 
     if ((smem_u32(smem) & 1023u) != 0) {              // the swizzle needs 1024-B alignment
@@ -142,16 +150,18 @@ prefill_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
 
     if (warp == 0) {
         Work w;
-        const bool has = find_work(p, blockIdx.y, w);
+        const bool has = find_work(p, (long long)blockIdx.x, w);
         if (lane == 0) {
             sh[0] = has ? w.b : -1;
             sh[1] = has ? w.tile : 0;
+            sh[6] = has ? w.kvh : 0;
         }
     }
     __syncthreads();
     const int b = sh[0];
     if (b < 0) return;
     const int tile = sh[1];
+    const int kvh = sh[6];
 
     SeqInfo s;
     const bool ok = load_seq(p.cu_seqlens_q, p.seqlens_kv, b, p.batch, p.token_count, p.kv_cap,
@@ -165,20 +175,24 @@ prefill_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
                      p.kv_hint, p.q_hint, p.status, s);
         sh[2] = ok ? 0 : 1;
         sh[3] = 0;
+        sh[4] = 0;
+        sh[5] = 0;
         mbar_init(q_full, 1);
-        for (int i = 0; i < C::NST; ++i) {
+        for (int i = 0; i < C::NK; ++i) {
             mbar_init(&k_full[i], 1);
+            mbar_init(&k_empty[i], 1);
+        }
+        for (int i = 0; i < C::NV; ++i) {
             mbar_init(&v_full[i], 1);
-            mbar_init(&kv_empty[i], 1);
+            mbar_init(&v_empty[i], 1);
         }
         for (int i = 0; i < 2; ++i) {
             mbar_init(&s_full[i], 1);
-            mbar_init(&s_free[i], 4);
+            mbar_init(&p_full[i], 4);
         }
-        mbar_init(p_full, 4);
         mbar_init(pv_done, 1);
+        mbar_init(o_full, 1);
         mbar_init(drain, 1);
-        sh[4] = 0;
         fence_barrier_init();
     }
     __syncthreads();
@@ -216,7 +230,6 @@ prefill_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
     uint8_t* sQ = smem + C::OFF_Q;
     uint8_t* sK = smem + C::OFF_K;
     uint8_t* sV = smem + C::OFF_V;
-    uint8_t* sP = smem + C::OFF_P;
     const int bs = p.block_size;
     const int32_t* bt = p.block_table + (long long)b * p.max_blocks;
 
@@ -231,55 +244,51 @@ prefill_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
             for (int c = 0; c < C::NA; ++c)
                 tma_load_3d(sQ + c * C::BM * C::RB, &tm_q, q_full, c * C::A, kvh * g, s.q_start + i0);
             const int box = bs < C::BN ? bs : C::BN;
-            for (int j = 0; j < ntiles; ++j) {
-                const int st = j % C::NST, u = j / C::NST;
-                if (u > 0 && !mbar_wait(&kv_empty[st], (u - 1) & 1)) {
-                    flag_status(p.status, PA_DEV_TIMEOUT);
-                    atomicExch(&sh[3], 1);
-                    break;
-                }
-                if (*(volatile int*)&sh[3]) break;
-                sh[4] = j + 1;
+            // Load key tile j of K (which = 0) or V (which = 1) into `dst`.
+            auto load_tile = [&](int j, uint8_t* dst, const CUtensorMap* tm, uint64_t* bar) {
                 const int k0 = j * C::BN;
-                // Pages (or the part of one page) covering [k0, k0 + BN) that start before T.
-                int npg = 1;
-                if (bs < C::BN) {
-                    npg = (min(k0 + C::BN, T) - k0 + bs - 1) / bs;
-                }
-                const uint32_t bytes = (uint32_t)(npg * box * HEAD * 2);
-                mbar_arrive_expect_tx(&k_full[st], bytes);
-                mbar_arrive_expect_tx(&v_full[st], bytes);
+                const int npg = bs < C::BN ? (min(k0 + C::BN, T) - k0 + bs - 1) / bs : 1;
+                mbar_arrive_expect_tx(bar, (uint32_t)(npg * box * HEAD * 2));
                 for (int pi = 0; pi < npg; ++pi) {
                     const int key = k0 + pi * box;
                     const int blk = bt[key / bs];
                     const int row = key % bs;
 #pragma unroll
-                    for (int c = 0; c < C::NA; ++c) {
-                        const int off = (c * C::BN + pi * box) * C::RB;
-                        tma_load_4d(sK + st * C::KV_BYTES + off, &tm_k, &k_full[st], c * C::A, kvh, row, blk);
-                    }
+                    for (int c = 0; c < C::NA; ++c)
+                        tma_load_4d(dst + (c * C::BN + pi * box) * C::RB, tm, bar, c * C::A, kvh, row, blk);
                 }
-                for (int pi = 0; pi < npg; ++pi) {
-                    const int key = k0 + pi * box;
-                    const int blk = bt[key / bs];
-                    const int row = key % bs;
-#pragma unroll
-                    for (int c = 0; c < C::NA; ++c) {
-                        const int off = (c * C::BN + pi * box) * C::RB;
-                        tma_load_4d(sV + st * C::KV_BYTES + off, &tm_v, &v_full[st], c * C::A, kvh, row, blk);
-                    }
+            };
+            bool alive = true;
+            for (int j = 0; j <= ntiles && alive; ++j) {
+                if (j < ntiles) {
+                    const int st = j % C::NK, u = j / C::NK;
+                    if (u > 0 && !mbar_wait(&k_empty[st], (u - 1) & 1)) { alive = false; break; }
+                    if (*(volatile int*)&sh[3]) { alive = false; break; }
+                    sh[4] = j + 1;
+                    load_tile(j, sK + st * C::KV_BYTES, &tm_k, &k_full[st]);
                 }
+                if (j >= 1) {
+                    const int jv = j - 1;
+                    const int st = jv % C::NV, u = jv / C::NV;
+                    if (u > 0 && !mbar_wait(&v_empty[st], (u - 1) & 1)) { alive = false; break; }
+                    if (*(volatile int*)&sh[3]) { alive = false; break; }
+                    sh[5] = jv + 1;
+                    load_tile(jv, sV + st * C::KV_BYTES, &tm_v, &v_full[st]);
+                }
+            }
+            if (!alive) {
+                flag_status(p.status, PA_DEV_TIMEOUT);
+                atomicExch(&sh[3], 1);
             }
         }
     } else if (warp == 5) {
         // ---------------------------------------------------------- MMA issuer
         constexpr uint32_t idesc_s = umma_idesc_f16(C::BM, C::BN, false, false);
         constexpr uint32_t idesc_o = umma_idesc_f16(C::BM, HEAD, false, true);
-        const uint32_t q_addr = smem_u32(sQ), k_addr = smem_u32(sK), v_addr = smem_u32(sV),
-                       p_addr = smem_u32(sP);
+        const uint32_t q_addr = smem_u32(sQ), k_addr = smem_u32(sK), v_addr = smem_u32(sV);
         bool alive = mbar_wait_warp(q_full, 0);
         auto issue_s = [&](int j) {
-            const int st = j % C::NST;
+            const int st = j % C::NK;
             if (lane == 0) {
 #pragma unroll
                 for (int kk = 0; kk < HEAD / 16; ++kk) {
@@ -287,16 +296,17 @@ prefill_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
                     const uint64_t da = umma_sdesc(q_addr + c * C::BM * C::RB + w * 2, 16, 8 * C::RB, C::LAYOUT);
                     const uint64_t db = umma_sdesc(k_addr + st * C::KV_BYTES + c * C::BN * C::RB + w * 2, 16,
                                                    8 * C::RB, C::LAYOUT);
-                    umma_f16(tmem + ((j & 1) ? C::COL_S1 : C::COL_S0), da, db, idesc_s, kk > 0 ? 1u : 0u);
+                    umma_f16(tmem + (uint32_t)((j & 1) * C::BN), da, db, idesc_s, kk > 0 ? 1u : 0u);
                 }
                 umma_commit(&s_full[j & 1]);
+                umma_commit(&k_empty[st]);
             }
             __syncwarp();
         };
         auto issue_pv = [&](int j) -> bool {
-            const int st = j % C::NST;
-            if (!mbar_wait_warp(p_full, j & 1)) return false;
-            if (!mbar_wait_warp(&v_full[st], (j / C::NST) & 1)) return false;
+            const int st = j % C::NV;
+            if (!mbar_wait_warp(&p_full[j & 1], (j >> 1) & 1)) return false;
+            if (!mbar_wait_warp(&v_full[st], (j / C::NV) & 1)) return false;
             tc_fence_after();
             const int k0 = j * C::BN;
             if (k0 + C::BN > T) {
@@ -310,28 +320,29 @@ prefill_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
                 __syncwarp();
             }
             if (lane == 0) {
+                const uint32_t p_tmem = tmem + (uint32_t)((j & 1) * C::BN);
 #pragma unroll
                 for (int kk = 0; kk < C::BN / 16; ++kk) {
-                    const uint64_t da = umma_sdesc(p_addr + kk * 32, 16, 1024, 2u);
                     const uint64_t db = umma_sdesc(v_addr + st * C::KV_BYTES + kk * 16 * C::RB,
                                                    C::BN * C::RB, 8 * C::RB, C::LAYOUT);
-                    umma_f16(tmem + C::COL_O, da, db, idesc_o, (j > 0 || kk > 0) ? 1u : 0u);
+                    umma_f16_ts(tmem + C::COL_O, p_tmem + kk * 8, db, idesc_o, (j > 0 || kk > 0) ? 1u : 0u);
                 }
                 umma_commit(pv_done);
-                umma_commit(&kv_empty[st]);
+                umma_commit(&v_empty[st]);
             }
             __syncwarp();
             return true;
         };
         for (int j = 0; alive && j < ntiles; ++j) {
-            const int st = j % C::NST;
-            if (!mbar_wait_warp(&k_full[st], (j / C::NST) & 1)) { alive = false; break; }
-            if (j >= 2 && !mbar_wait_warp(&s_free[j & 1], ((j - 2) >> 1) & 1)) { alive = false; break; }
+            const int st = j % C::NK;
+            if (!mbar_wait_warp(&k_full[st], (j / C::NK) & 1)) { alive = false; break; }
             tc_fence_after();
             issue_s(j);
             if (j >= 1 && !issue_pv(j - 1)) { alive = false; break; }
         }
         if (alive && ntiles > 0) alive = issue_pv(ntiles - 1);
+        if (alive && lane == 0) umma_commit(o_full);
+        __syncwarp();
         if (!alive) {
             if (lane == 0) {
                 flag_status(p.status, PA_DEV_TIMEOUT);
@@ -355,35 +366,31 @@ prefill_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
             if (!mbar_wait_warp(&s_full[j & 1], (j >> 1) & 1)) { alive = false; break; }
             tc_fence_after();
             uint32_t sv[C::BN];
-            const uint32_t scol = tmem + lane_base + ((j & 1) ? C::COL_S1 : C::COL_S0);
+            const uint32_t scol = tmem + lane_base + (uint32_t)((j & 1) * C::BN);
             tmem_ld32(scol, sv);
             tmem_ld32(scol + 32, sv + 32);
             tmem_wait_ld();
-            tc_fence_before();
-            __syncwarp();
-            if (lane == 0) mbar_arrive(&s_free[j & 1]);
             const int k0 = j * C::BN;
-            float x[C::BN];
             float mx = -INFINITY;
             if (k0 + C::BN - 1 <= full_vis) {
 #pragma unroll
-                for (int c = 0; c < C::BN; ++c) {
-                    x[c] = __uint_as_float(sv[c]) * p.scale_log2;
-                    mx = fmaxf(mx, x[c]);
-                }
+                for (int c = 0; c < C::BN; ++c) mx = fmaxf(mx, __uint_as_float(sv[c]));
             } else {
 #pragma unroll
                 for (int c = 0; c < C::BN; ++c) {
                     const bool vis = (k0 + c) <= lim;
-                    x[c] = vis ? __uint_as_float(sv[c]) * p.scale_log2 : -INFINITY;
-                    mx = fmaxf(mx, x[c]);
+                    sv[c] = vis ? sv[c] : __float_as_uint(-INFINITY);
+                    mx = fmaxf(mx, __uint_as_float(sv[c]));
                 }
             }
+            mx *= p.scale_log2;
             // Lazy rescale: move the exponent base only when the max grows by > 8.
             if (mx > m_used + 8.f) {
                 const float alpha = (m_used == -INFINITY) ? 0.f : fast_exp2(m_used - mx);
                 l *= alpha;
                 if (j > 0) {
+                    // S_j's commit covered P_{j-2} V_{j-2}, so pv_done is at phase
+                    // j - 1 or j here and this parity wait means "P_{j-1} V_{j-1} done".
                     if (!mbar_wait_warp(pv_done, (j - 1) & 1)) { alive = false; break; }
                     tc_fence_after();
                     const uint32_t ocol = tmem + lane_base + C::COL_O;
@@ -396,7 +403,6 @@ prefill_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
                         for (int c = 0; c < 16; ++c) ov[c] = __float_as_uint(__uint_as_float(ov[c]) * alpha);
                         tmem_st16(ocol + c0, ov);
                     }
-                    tmem_wait_st();
                 }
                 m_used = mx;
             }
@@ -405,30 +411,21 @@ prefill_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
             float rs = 0.f;
 #pragma unroll
             for (int c = 0; c < C::BN; c += 2) {
-                const float p0 = fast_exp2(x[c] - base);
-                const float p1 = fast_exp2(x[c + 1] - base);
+                const float p0 = fast_exp2(fmaf(__uint_as_float(sv[c]), p.scale_log2, -base));
+                const float p1 = fast_exp2(fmaf(__uint_as_float(sv[c + 1]), p.scale_log2, -base));
                 rs += p0 + p1;
                 pk[c / 2] = pack_half2(p0, p1);
             }
             l += rs;
-            // P_j replaces P_{j-1}: wait until the previous P V product has read it.
-            if (j > 0) {
-                if (!mbar_wait_warp(pv_done, (j - 1) & 1)) { alive = false; break; }
-            }
-            // Row r of P: 64 f16 = 128 bytes = 8 16-byte chunks, 128-byte swizzle.
-#pragma unroll
-            for (int ch = 0; ch < 8; ++ch) {
-                const uint32_t off = swz<128>((uint32_t)(r * 128 + ch * 16));
-                *reinterpret_cast<uint4*>(sP + off) =
-                    make_uint4(pk[4 * ch], pk[4 * ch + 1], pk[4 * ch + 2], pk[4 * ch + 3]);
-            }
-            fence_proxy_async_smem();
+            // P_j over S_j: 64 f16 = 32 columns of this row's lane.
+            tmem_st32(scol, pk);
+            tmem_wait_st();
             tc_fence_before();
             __syncwarp();
-            if (lane == 0) mbar_arrive(p_full);
+            if (lane == 0) mbar_arrive(&p_full[j & 1]);
         }
         // Epilogue: O / l -> f16 rows of `out`.
-        if (alive && ntiles > 0 && mbar_wait_warp(pv_done, (ntiles - 1) & 1)) {
+        if (alive && ntiles > 0 && mbar_wait_warp(o_full, 0)) {
             tc_fence_after();
             const float inv = (l > 0.f) ? 1.f / l : 0.f;
             const uint32_t ocol = tmem + lane_base + C::COL_O;
@@ -465,11 +462,10 @@ prefill_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
     if (sh[3] && threadIdx.x == 0) {
         // Aborted (never expected): let in-flight loads land before exit.
         mbar_wait(q_full, 0);
-        const int issued = sh[4];
-        for (int t = issued - C::NST > 0 ? issued - C::NST : 0; t < issued; ++t) {
-            mbar_wait(&k_full[t % C::NST], (t / C::NST) & 1);
-            mbar_wait(&v_full[t % C::NST], (t / C::NST) & 1);
-        }
+        for (int t = sh[4] - C::NK > 0 ? sh[4] - C::NK : 0; t < sh[4]; ++t)
+            mbar_wait(&k_full[t % C::NK], (t / C::NK) & 1);
+        for (int t = sh[5] - C::NV > 0 ? sh[5] - C::NV : 0; t < sh[5]; ++t)
+            mbar_wait(&v_full[t % C::NV], (t / C::NV) & 1);
     }
     __syncthreads();
     if (warp == 5) {
@@ -485,8 +481,8 @@ cudaError_t launch_prefill_t(const CUtensorMap& tm_q, const CUtensorMap& tm_k,
     auto kern = prefill_kernel<HEAD>;
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM);
     if (e != cudaSuccess) return e;
-    dim3 grid(p.kv_heads, p.num_slots);
-    kern<<<grid, C::THREADS, C::SMEM, stream>>>(tm_q, tm_k, tm_v, p);
+    const long long ctas = (long long)p.num_slots * p.kv_heads;
+    kern<<<(unsigned)ctas, C::THREADS, C::SMEM, stream>>>(tm_q, tm_k, tm_v, p);
     return cudaGetLastError();
 }
 

@@ -126,3 +126,35 @@ def test_full_size_config_sampled(cfg):
     assert np.array_equal(slots, want_slots)
     assert_close(got[rows[:, 0], rows[:, 1]], want, what=spec.name)
     assert np.isfinite(got.astype(np.float32)).all()
+
+
+def test_step_replays_from_a_cuda_graph():
+    """The calls take no host sync, so a whole step can be captured in a CUDA
+    graph; replays give the eager result bit for bit."""
+    import torch
+    import scatter_kv_b200 as pa
+    from pa_harness import dims_for, to_dev
+    spec = workloads.custom([1, 3, 90, 1], [700, 2000, 30, 5], 16, 4, 128, 16, seed=8)
+    x = workloads.generate(spec)
+    dv = to_dev(x)
+    dims = dims_for(spec, x)
+    bufs = pa.allocate(dims)
+    scale = pa.default_scale(128)
+    s = torch.cuda.Stream()
+
+    def step():
+        pa.step(dv["query"], dv["key"], dv["value"], dv["key_cache"], dv["value_cache"],
+                dv["block_table"], dv["cu_seqlens_q"], dv["seqlens_kv"], scale, dims, bufs, s)
+
+    with torch.cuda.stream(s):
+        step()
+    torch.cuda.synchronize()
+    eager = bufs.out.clone()
+    graph = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(graph, stream=s):
+        step()
+    for _ in range(2):
+        bufs.out.fill_(float("nan"))
+        graph.replay()
+        torch.cuda.synchronize()
+        assert torch.equal(bufs.out.view(torch.int16), eager.view(torch.int16))
