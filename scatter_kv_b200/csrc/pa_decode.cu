@@ -15,8 +15,8 @@
 //     group * q_len query rows of that KV head share every page it loads;
 //   * a producer warp walks the block table and issues TMA tensor loads of
 //     32-key K and V tiles (one box per page and 64-element column block,
-//     128-byte swizzle) into a ring of shared-memory stages tracked by
-//     mbarriers;
+//     128-byte swizzle) into a ring of 4 shared-memory stages (64 KB for head
+//     size 128) tracked by mbarriers, each stage owned by one consumer group;
 //   * consumer warps each own whole tiles (independent online softmax per
 //     warp, merged at the end), computing Q K^T and P V with mma.sync
 //     m16n8k16 (f16 in, f32 accumulate).  The tensor core is only a means to
@@ -43,9 +43,15 @@ struct Cfg {
     static constexpr int RB = A * 2;                    // bytes per swizzled row
     static constexpr int NA = HEAD / A;                 // column blocks
     static constexpr int BN = kDecodeKeys;              // keys per stage
-    static constexpr int NST = 6;                       // stages
     static constexpr int NCW = 4;                       // consumer warps
     static constexpr int NG = NCW / MT;                 // tile groups (MT warps per group)
+    // Stages.  Tile t goes to stage t % NST and to group t % NG; NST must be
+    // a multiple of NG so that every stage is always consumed by the same
+    // group, which waits on it in order.  (An mbarrier parity wait only tells
+    // adjacent phases apart: a second group waiting two phases ahead would
+    // pass at once and read a stage whose previous tile is still in use.)
+    static constexpr int NST = 4;
+    static_assert(NST % NG == 0, "each stage must belong to one consumer group");
     static constexpr int THREADS = 32 * (NCW + 1);
     static constexpr int TILE_BYTES = BN * HEAD * 2;    // one tensor, one stage
     static constexpr int STAGE_BYTES = 2 * TILE_BYTES;
@@ -136,6 +142,8 @@ decode_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ 
         if (!bok && lane == 0) sflag[0] = 1;
     }
     __syncthreads();
+    if (split == 0 && kvh == 0 && threadIdx.x == 0 && p.seq_state != nullptr)
+        p.seq_state[b] = sflag[0] ? 0 : 1;          // read by the combine kernel
     if (sflag[0]) {
         // Invalid sequence: zero rows (split 0 only; the combine does the same).
         if (split == 0) {
@@ -422,67 +430,52 @@ decode_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ 
     }
 }
 
-// One CTA per (KV head, sequence): merge the splits of its q_len * group rows.
+// One warp per output row (row r of KV head kvh of sequence b): merge the
+// row's splits in split order, O = sum_s w_s O_s / sum_s w_s with
+// w_s = 2^(lse_s - max lse).  Lane i owns columns [4i, 4i + 4).
 template <int HEAD>
 __global__ void __launch_bounds__(128) combine_kernel(const DecodeParams p) {
-    extern __shared__ float wsm[];                        // [max_splits][rmax] then [rmax]
-    const int b = blockIdx.y, kvh = blockIdx.x;
+    const int b = blockIdx.z, kvh = blockIdx.y;
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int r = blockIdx.x * 4 + warp;
     const int g = p.group;
-    SeqInfo s;
-    const bool ok = load_seq(p.cu_seqlens_q, p.seqlens_kv, b, p.batch, p.token_count, p.kv_cap,
-                             p.kv_hint, p.q_hint, nullptr, s);
-    if (!s.cu_ok || s.q_len == 0 || s.q_len > p.decode_max_q) return;
-    const int R = s.q_len * g;
-    __shared__ int bad;
-    if (threadIdx.x == 0) bad = ok ? 0 : 1;
-    __syncthreads();
-    if (ok && threadIdx.x < 32) {
-        const int npages = (s.kv_len + p.block_size - 1) / p.block_size;
-        if (!warp_blocks_ok(p.block_table, b, p.max_blocks, npages, p.num_blocks, nullptr) &&
-            threadIdx.x == 0)
-            bad = 1;
-    }
-    __syncthreads();
-    const int n_splits = bad ? 1 : (s.kv_len + p.chunk - 1) / p.chunk;
-    if (!bad && n_splits == 1) return;                    // decode kernel wrote the rows
-    if (bad) {
-        for (int idx = threadIdx.x; idx < R * HEAD; idx += blockDim.x) {
-            const int r = idx / HEAD, d = idx % HEAD;
-            p.out[((long long)(s.q_start + r / g) * p.q_heads + kvh * g + r % g) * HEAD + d] =
-                __float2half_rn(0.f);
-        }
+    const int c0 = p.cu_seqlens_q[b], c1 = p.cu_seqlens_q[b + 1];
+    const int q_len = c1 - c0;
+    if (c0 < 0 || c1 < c0 || (long long)c1 > p.token_count) return;
+    if (q_len == 0 || q_len > p.decode_max_q || r >= q_len * g) return;
+    __half* orow = p.out + ((long long)(c0 + r / g) * p.q_heads + kvh * g + r % g) * HEAD;
+    const int state = p.seq_state[b];                 // written by the decode kernel
+    if (state != 1) {
+        // Invalid sequence: zero rows, like the decode kernel does for one split.
+        for (int d = lane; d < HEAD; d += 32) orow[d] = __float2half_rn(0.f);
         return;
     }
-    const long long pbase = ((long long)b * p.kv_heads + kvh) * p.max_splits * p.rmax;
-    float* inv_l = wsm + p.max_splits * p.rmax;
-    for (int r = threadIdx.x; r < R; r += blockDim.x) {
-        float M = -INFINITY;
-        for (int sp = 0; sp < n_splits; ++sp) M = fmaxf(M, p.part_lse[pbase + (long long)sp * p.rmax + r]);
-        float L = 0.f;
-        for (int sp = 0; sp < n_splits; ++sp) {
-            const float w = fast_exp2(p.part_lse[pbase + (long long)sp * p.rmax + r] - M);
-            wsm[sp * p.rmax + r] = w;
-            L += w;
-        }
-        inv_l[r] = 1.f / L;
+    const int n_splits = (p.seqlens_kv[b] + p.chunk - 1) / p.chunk;
+    if (n_splits == 1) return;                        // the decode kernel wrote the row
+    const long long base = ((long long)b * p.kv_heads + kvh) * p.max_splits * p.rmax + r;
+    const float* lse = p.part_lse + base;             // stride rmax per split
+    float M = -INFINITY;
+    for (int sp = lane; sp < n_splits; sp += 32) M = fmaxf(M, lse[(long long)sp * p.rmax]);
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, o));
+    float L = 0.f;
+    for (int sp = lane; sp < n_splits; sp += 32) L += fast_exp2(lse[(long long)sp * p.rmax] - M);
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) L += __shfl_xor_sync(0xffffffffu, L, o);
+    if (lane * 4 >= HEAD) return;
+    const float* po = p.part_o + base * HEAD + lane * 4;
+    float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll 4
+    for (int sp = 0; sp < n_splits; ++sp) {
+        const float w = fast_exp2(lse[(long long)sp * p.rmax] - M);
+        const float4 v = *reinterpret_cast<const float4*>(po + (long long)sp * p.rmax * HEAD);
+        acc.x += w * v.x; acc.y += w * v.y; acc.z += w * v.z; acc.w += w * v.w;
     }
-    __syncthreads();
-    for (int idx = threadIdx.x; idx < R * (HEAD / 4); idx += blockDim.x) {
-        const int r = idx / (HEAD / 4), d4 = (idx % (HEAD / 4)) * 4;
-        float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
-        for (int sp = 0; sp < n_splits; ++sp) {
-            const float w = wsm[sp * p.rmax + r];
-            const float4 v = *reinterpret_cast<const float4*>(
-                p.part_o + (pbase + (long long)sp * p.rmax + r) * HEAD + d4);
-            acc.x += w * v.x; acc.y += w * v.y; acc.z += w * v.z; acc.w += w * v.w;
-        }
-        const float il = inv_l[r];
-        const long long o = ((long long)(s.q_start + r / g) * p.q_heads + kvh * g + r % g) * HEAD + d4;
-        uint2 wv;
-        wv.x = pack_half2(acc.x * il, acc.y * il);
-        wv.y = pack_half2(acc.z * il, acc.w * il);
-        *reinterpret_cast<uint2*>(p.out + o) = wv;
-    }
+    const float il = 1.f / L;
+    uint2 wv;
+    wv.x = pack_half2(acc.x * il, acc.y * il);
+    wv.y = pack_half2(acc.z * il, acc.w * il);
+    *reinterpret_cast<uint2*>(orow + lane * 4) = wv;
 }
 
 template <int HEAD, int MT>
@@ -522,8 +515,9 @@ DecodePlan plan_decode(const pa_dims& d, int num_sms) {
     pl.chunk = (int)chunk;
     pl.max_splits = (int)((max_kv + chunk - 1) / chunk);
     if (pl.max_splits > 1) {
+        // [partial O: rows x head_size f32][partial lse: rows f32][state: batch i32]
         const size_t rows = (size_t)d.batch * d.kv_heads * pl.max_splits * (16 * pl.mtiles);
-        pl.workspace_bytes = rows * (size_t)d.head_size * 4 + rows * 4;
+        pl.workspace_bytes = rows * (size_t)d.head_size * 4 + rows * 4 + (size_t)d.batch * 4;
         pl.workspace_bytes = (pl.workspace_bytes + 255) / 256 * 256;
     }
     return pl;
@@ -546,25 +540,15 @@ cudaError_t launch_decode(const CUtensorMap& tm_k, const CUtensorMap& tm_v,
 }
 
 cudaError_t launch_combine(const DecodeParams& p, int head_size, cudaStream_t stream) {
-    dim3 grid(p.kv_heads, p.batch);
-    const size_t smem = ((size_t)p.max_splits + 1) * p.rmax * sizeof(float);
-#define PA_COMBINE_CASE(H)                                                             \
-    case H: {                                                                          \
-        cudaError_t e = cudaFuncSetAttribute(combine_kernel<H>,                        \
-                                             cudaFuncAttributeMaxDynamicSharedMemorySize, \
-                                             (int)smem);                               \
-        if (e != cudaSuccess) return e;                                                \
-        combine_kernel<H><<<grid, 128, smem, stream>>>(p);                             \
-        return cudaGetLastError();                                                     \
-    }
+    dim3 grid((p.rmax + 3) / 4, p.kv_heads, p.batch);
     switch (head_size) {
-        PA_COMBINE_CASE(16)
-        PA_COMBINE_CASE(32)
-        PA_COMBINE_CASE(64)
-        PA_COMBINE_CASE(128)
+        case 16: combine_kernel<16><<<grid, 128, 0, stream>>>(p); break;
+        case 32: combine_kernel<32><<<grid, 128, 0, stream>>>(p); break;
+        case 64: combine_kernel<64><<<grid, 128, 0, stream>>>(p); break;
+        case 128: combine_kernel<128><<<grid, 128, 0, stream>>>(p); break;
         default: return cudaErrorInvalidValue;
     }
-#undef PA_COMBINE_CASE
+    return cudaGetLastError();
 }
 
 }  // namespace pa
