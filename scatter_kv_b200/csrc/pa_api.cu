@@ -330,7 +330,7 @@ pa_status pa_attention(const void* query, const void* key_cache, const void* val
     // Prefill part: sequences with q_len > plan.decode_max_q.
     if (d.max_seqlen_q_hint == 0 || d.max_seqlen_q_hint > plan.decode_max_q) {
         const long long longer = d.token_count / (plan.decode_max_q + 1);
-        const long long slots = (d.token_count * g + pa::kPrefillRows - 1) / pa::kPrefillRows +
+        const long long slots = (d.token_count * g + pa::kPrefillCtaRows - 1) / pa::kPrefillCtaRows +
                                 (longer < d.batch ? longer : d.batch);
         if (slots > 0) {
             if (slots * d.kv_heads >= (1ll << 31))

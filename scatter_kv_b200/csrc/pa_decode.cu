@@ -57,8 +57,9 @@ struct Cfg {
     static constexpr int STAGE_BYTES = 2 * TILE_BYTES;
     static constexpr int RMAX = 16 * MT;
     static constexpr int OST = HEAD + 8;                // merge scratch row stride (floats)
+    static constexpr int MAX_IDS = 1056;                // block ids of one split (chunk <= 16384)
     static constexpr int SMEM = NST * STAGE_BYTES + 1024 + 2 * NST * 8 + 2 * NG * RMAX * 4 +
-                                2 * RMAX * 4 + 16;
+                                2 * RMAX * 4 + 16 + MAX_IDS * 4;
     static_assert(NG * RMAX * OST * 4 <= NST * STAGE_BYTES, "merge scratch must fit the stages");
 };
 
@@ -67,7 +68,7 @@ __device__ __forceinline__ uint32_t half2_mask(uint32_t v, bool lo_ok, bool hi_o
 }
 
 template <int HEAD, int MT>
-__global__ void __launch_bounds__(Cfg<HEAD, MT>::THREADS)
+__global__ void __launch_bounds__(Cfg<HEAD, MT>::THREADS, HEAD >= 128 ? 2 : 3)
 decode_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_v,
               const DecodeParams p) {
     using C = Cfg<HEAD, MT>;
@@ -82,6 +83,7 @@ decode_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ 
     float* row_l = red_l + C::NG * C::RMAX;                     // [RMAX]
     float* row_m = row_l + C::RMAX;                             // [RMAX]
     int* sflag = reinterpret_cast<int*>(row_m + C::RMAX);       // [0] bad seq, [1] abort, [2] issued
+    int* sids = sflag + 4;                                      // [MAX_IDS] block ids of the split
 
     // Grid (kv_heads, splits, batch): the KV heads of one split are adjacent
     // in launch order, so they stream the same pages (whose rows interleave
@@ -164,6 +166,16 @@ decode_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ 
 
     if (warp == C::NCW) {
         // ------------------------------------------------------------ producer
+        // The split's block ids, fetched once by the whole warp, so issuing a
+        // tile never waits on a dependent global load.
+        const int pg0 = k_begin / bs;
+        const int n_ids = (k_end - 1) / bs + 1 - pg0;
+        for (int i = lane; i < n_ids && i < C::MAX_IDS; i += 32) sids[i] = bt[pg0 + i];
+        __syncwarp();
+        auto block_of = [&](int page) {
+            const int i = page - pg0;
+            return i < C::MAX_IDS ? sids[i] : bt[page];
+        };
         if (lane == 0) {
             tma_prefetch_desc(&tm_k);
             tma_prefetch_desc(&tm_v);
@@ -181,7 +193,7 @@ decode_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ 
                 uint8_t* vdst = kdst + C::TILE_BYTES;
                 const int k0 = k_begin + t * C::BN;
                 if (bs >= C::BN) {
-                    const int blk = bt[k0 / bs];
+                    const int blk = block_of(k0 / bs);
                     const int row = k0 % bs;
                     mbar_arrive_expect_tx(&full[st], 2 * C::TILE_BYTES);
 #pragma unroll
@@ -194,7 +206,7 @@ decode_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ 
                     const int npg = (k0 + bs < T) ? 2 : 1;
                     mbar_arrive_expect_tx(&full[st], (uint32_t)(npg * bs * HEAD * 2 * 2));
                     for (int pi = 0; pi < npg; ++pi) {
-                        const int blk = bt[k0 / bs + pi];
+                        const int blk = block_of(k0 / bs + pi);
 #pragma unroll
                         for (int c = 0; c < C::NA; ++c) {
                             const int off = (c * C::BN + pi * bs) * C::RB;
@@ -484,6 +496,9 @@ cudaError_t launch_decode_t(const CUtensorMap& tm_k, const CUtensorMap& tm_v,
     using C = Cfg<HEAD, MT>;
     auto kern = decode_kernel<HEAD, MT>;
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM);
+    if (e != cudaSuccess) return e;
+    e = cudaFuncSetAttribute(kern, cudaFuncAttributePreferredSharedMemoryCarveout,
+                             cudaSharedmemCarveoutMaxShared);
     if (e != cudaSuccess) return e;
     dim3 grid(p.kv_heads, p.max_splits, p.batch);
     kern<<<grid, C::THREADS, C::SMEM, stream>>>(tm_k, tm_v, p);

@@ -57,7 +57,7 @@ struct PrefillParams {
     int kv_hint;
     int q_hint;
     int decode_max_q;             // sequences with q_len <= this are not prefill work
-    int num_slots;                // q tiles the grid covers (upper bound)
+    int num_slots;                // query-tile pairs the grid covers per KV head (upper bound)
     float scale_log2;
 };
 
@@ -100,6 +100,7 @@ cudaError_t launch_prefill(const CUtensorMap& tm_q, const CUtensorMap& tm_k,
 // for prefill.
 constexpr int kDecodeKeys = 32;
 constexpr int kPrefillKeys = 128;
-constexpr int kPrefillRows = 128;
+constexpr int kPrefillRows = 128;      // query rows per tensor-core tile
+constexpr int kPrefillCtaRows = 256;   // query rows per prefill CTA (two tiles)
 
 }  // namespace pa

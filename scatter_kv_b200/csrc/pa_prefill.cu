@@ -7,38 +7,40 @@
 // implementation (1/n)", "FlashAttention: optional seqlens_q input" (row i
 // of sequence b sees keys [0, seqlens_kv[b] - q_len_b + i]).
 //
-// One CTA computes a 128-row query tile of one KV head.  The rows are
-// (token, head) pairs: 128 / group consecutive tokens times the group query
-// heads that share the KV head, so every K/V page is loaded once for the
-// whole group.  There is no gathered or padded copy of the cache: the
-// producer warp walks the block table and TMA-loads 64-key K and V tiles
-// (one box per page and 64-element column block, 128-byte swizzle) straight
-// from their pages.
+// One CTA per SM computes two 128-row query tiles ("halves" a = 0, 1) of one
+// KV head.  Rows are (token, head) pairs: 128 / group consecutive tokens
+// times the group query heads that share the KV head, so every K/V page is
+// loaded once for 256 query rows.  There is no gathered or padded copy of
+// the cache: producer warps walk the block table and TMA-load 64-key K and V
+// tiles (one box per page and 64-element column block, 128-byte swizzle)
+// straight from their pages.
 //
-// Warp roles (192 threads):
-//   warps 0-3  softmax + epilogue; thread r owns query row r = TMEM lane r;
-//   warp 4     TMA producer (Q once; K tiles in a 3-stage ring, V tiles in a
-//              2-stage ring, K one tile ahead of V);
-//   warp 5     TMEM allocator and single-thread tcgen05.mma issuer.
-// Per key tile j (TMEM: S/P buffers j % 2 at columns 0 / 64, O at 128):
-//   S_j = Q K_j^T        M 128, N 64, fp32 into buffer j % 2; K_j is released
-//                        as soon as this product is done;
-//   softmax_j            row max / exp2 / row sum in registers; P_j as f16
-//                        written back over S_j (32 columns, 2 per column);
-//   O += P_j V_j         A operand P_j straight from TMEM, M 128, N head_size.
-// The MMA warp issues S_{j+1} before waiting for P_j and S_{j+2} right after
-// P_j V_j (the tensor pipe runs a thread's MMAs in order, so S_{j+2} cannot
-// overwrite P_j before it is read): the softmax threads never wait for a P V
-// product except when a row maximum grows by more than 2^8 and O must be
-// rescaled (values of P stay below 256, exact enough in f16 and fp32 sums),
-// which after the first tiles is rare.  Key tiles wholly above the causal
-// diagonal are never loaded; the diagonal tile is masked per element; rows
+// Warp roles (352 threads):
+//   warps 0-3   softmax + epilogue of half 0 (thread r = row r = TMEM lane r)
+//   warps 4-7   softmax + epilogue of half 1
+//   warp 8      TMA producer of Q (both halves) and of the K ring
+//   warp 9      TMA producer of the V ring
+//   warp 10     TMEM allocator and single-thread tcgen05.mma issuer
+// Tensor memory (512 columns): S/P of half a, two buffers of 64 columns at
+// a*128 + (j%2)*64; O of half a at 256 + a*128.
+// Per key tile j and half a:
+//   S_a,j = Q_a K_j^T     M 128, N 64, fp32; K_j is released once both
+//                          halves' products are done;
+//   softmax               row max / exp2 / row sum in registers; P as f16
+//                          written back over S (32 columns, 2 per column);
+//   O_a += P_a,j V_j      A operand straight from TMEM, M 128, N head_size.
+// The MMA warp issues S for tile j+1 before the P V products of tile j, and
+// the two halves' softmax warpgroups run independently, so the tensor core
+// always has one half's work while the other half exponentiates.  A thread's
+// MMAs run in order on the tensor pipe, so S_a,j+2 cannot overwrite P_a,j
+// before P_a,j V_j has read it.  O is rescaled only when a row maximum grows
+// by more than 2^8 (P stays below 256, exact enough in f16 and fp32 sums),
+// which after the first tiles is rare.  Key tiles wholly above a half's
+// causal diagonal are skipped; the diagonal tile is masked per element; rows
 // of V past the end of the sequence are zeroed in shared memory before the
-// last P V product.  CTAs are ordered sequence-major, then KV head, then
-// query tile from the last (most keys) to the first, so the CTAs resident
-// at any time share few sequences' K/V and reuse them from L2.  Two CTAs fit
-// on an SM (112 KB shared memory, 256 TMEM columns each), so one CTA's
-// softmax overlaps the other's MMAs and loads.
+// P V products that read them.  CTAs are ordered sequence-major, then KV
+// head, then tile pair from the last (most keys) to the first, so the CTAs
+// resident at any time share few sequences' K/V and reuse them from L2.
 #include <cuda_runtime.h>
 #include <math.h>
 
@@ -51,50 +53,57 @@ namespace {
 
 template <int HEAD>
 struct PCfg {
-    static constexpr int BM = kPrefillRows;             // 128 query rows
+    static constexpr int BM = kPrefillRows;             // 128 query rows per half
     static constexpr int BN = 64;                       // keys per tile
     static constexpr int A = HEAD < 64 ? HEAD : 64;     // elements per swizzled row (Q, K, V)
     static constexpr int RB = A * 2;
     static constexpr int NA = HEAD / A;
     static constexpr uint32_t LAYOUT = RB == 128 ? 2u : (RB == 64 ? 4u : 6u);
-    static constexpr int Q_BYTES = BM * HEAD * 2;
+    static constexpr int Q_BYTES = BM * HEAD * 2;       // one half
     static constexpr int KV_BYTES = BN * HEAD * 2;
-    static constexpr int NK = 3;                        // K stages
-    static constexpr int NV = 2;                        // V stages
+    // Stage counts: as deep as shared memory allows (the K and V loads of a
+    // tile are issued by separate warps and can each run that far ahead).
+    static constexpr int NK = HEAD >= 128 ? 5 : 8;
+    static constexpr int NV = HEAD >= 128 ? 4 : 8;
     static constexpr int OFF_Q = 0;
-    static constexpr int OFF_K = OFF_Q + Q_BYTES;
+    static constexpr int OFF_K = OFF_Q + 2 * Q_BYTES;
     static constexpr int OFF_V = OFF_K + NK * KV_BYTES;
     static constexpr int OFF_BAR = OFF_V + NV * KV_BYTES;
-    // q_full, k_full/k_empty x NK, v_full/v_empty x NV, s_full x2, p_full x2, pv_done,
-    // o_full, drain
-    static constexpr int NBAR = 1 + 2 * NK + 2 * NV + 2 + 2 + 3;
-    static constexpr int SMEM = OFF_BAR + NBAR * 8 + 64;
-    static constexpr int THREADS = 192;
-    static constexpr uint32_t TMEM_COLS = 256;          // S/P 0 (64) | S/P 1 (64) | O (head_size)
-    static constexpr uint32_t COL_O = 128;
+    // q_full, k_full/k_empty x NK, v_full/v_empty x NV, s_full[2][2], p_full[2][2],
+    // pv_done[2], o_full[2], drain
+    static constexpr int NBAR = 1 + 2 * NK + 2 * NV + 4 + 4 + 2 + 2 + 1;
+    // At least 120 KB, so that one CTA (which takes all 512 TMEM columns)
+    // runs per SM and no second CTA ever waits in tcgen05.alloc.
+    static constexpr int SMEM_USED = OFF_BAR + NBAR * 8 + 64;
+    static constexpr int SMEM = SMEM_USED > 120 * 1024 ? SMEM_USED : 120 * 1024;
+    static constexpr int THREADS = 352;
+    static constexpr int WARP_KLOAD = 8, WARP_VLOAD = 9, WARP_MMA = 10;
+    static constexpr uint32_t TMEM_COLS = 512;
+    static constexpr uint32_t COL_O = 256;
+    static_assert(SMEM <= 227 * 1024, "shared memory budget");
 };
 
 struct Work {
     int b;          // sequence
     int kvh;        // KV head
-    int tile;       // query tile within the sequence
+    int pair;       // pair of query tiles within the sequence
 };
 
-// CTA x -> (sequence, KV head, query tile): sequences in order, each with
-// its kv_heads x ntiles_b CTAs; within a KV head the tiles run from the last
+// CTA x -> (sequence, KV head, tile pair): sequences in order, each with its
+// kv_heads x npairs_b CTAs; within a KV head the pairs run from the last
 // (the most keys) to the first.  One warp, 32 sequences per step.
 __device__ bool find_work(const PrefillParams& p, long long slot, Work& w) {
     const int lane = threadIdx.x & 31;
     for (int b0 = 0; b0 < p.batch; b0 += 32) {
         const int b = b0 + lane;
-        int nt = 0;
+        int np = 0;
         if (b < p.batch) {
             const int c0 = p.cu_seqlens_q[b], c1 = p.cu_seqlens_q[b + 1];
             const int ql = c1 - c0;
             if (ql > p.decode_max_q && c0 >= 0 && (long long)c1 <= p.token_count)
-                nt = (ql * p.group + kPrefillRows - 1) / kPrefillRows;
+                np = (ql * p.group + kPrefillCtaRows - 1) / kPrefillCtaRows;
         }
-        const long long cnt = (long long)nt * p.kv_heads;
+        const long long cnt = (long long)np * p.kv_heads;
         long long pre = cnt;                       // inclusive prefix over lanes
 #pragma unroll
         for (int o = 1; o < 32; o <<= 1) {
@@ -107,11 +116,11 @@ __device__ bool find_work(const PrefillParams& p, long long slot, Work& w) {
             const int lb = __ffs(m) - 1;
             const long long pre_b = __shfl_sync(0xffffffffu, pre, lb);
             const long long cnt_b = __shfl_sync(0xffffffffu, cnt, lb);
-            const int nt_b = __shfl_sync(0xffffffffu, nt, lb);
+            const int np_b = __shfl_sync(0xffffffffu, np, lb);
             const long long local = slot - (pre_b - cnt_b);
             w.b = b0 + lb;
-            w.kvh = (int)(local / nt_b);
-            w.tile = nt_b - 1 - (int)(local % nt_b);
+            w.kvh = (int)(local / np_b);
+            w.pair = np_b - 1 - (int)(local % np_b);
             return true;
         }
         slot -= total;
@@ -120,7 +129,7 @@ __device__ bool find_work(const PrefillParams& p, long long slot, Work& w) {
 }
 
 template <int HEAD>
-__global__ void __launch_bounds__(PCfg<HEAD>::THREADS, 2)
+__global__ void __launch_bounds__(PCfg<HEAD>::THREADS, 1)
 prefill_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                const __grid_constant__ CUtensorMap tm_v, const PrefillParams p) {
     using C = PCfg<HEAD>;
@@ -131,13 +140,13 @@ prefill_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
     uint64_t* k_empty = k_full + C::NK;
     uint64_t* v_full = k_empty + C::NK;
     uint64_t* v_empty = v_full + C::NV;
-    uint64_t* s_full = v_empty + C::NV;      // [2]
-    uint64_t* p_full = s_full + 2;           // [2]
-    uint64_t* pv_done = p_full + 2;
-    uint64_t* o_full = pv_done + 1;          // every MMA of the tile done (single use)
-    uint64_t* drain = o_full + 1;
+    uint64_t* s_full = v_empty + C::NV;      // [half][buffer]
+    uint64_t* p_full = s_full + 4;           // [half][buffer]
+    uint64_t* pv_done = p_full + 4;          // [half]
+    uint64_t* o_full = pv_done + 2;          // [half], single use
+    uint64_t* drain = o_full + 2;
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + C::NBAR);
-    // [0] b, [1] tile, [2] bad, [3] abort, [4] K tiles issued, [5] V tiles issued, [6] kv head
+    // [0] b, [1] pair, [2] bad, [3] abort, [4] K tiles issued, [5] V tiles issued, [6] kv head
     int* sh = reinterpret_cast<int*>(tmem_slot + 1);
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -153,24 +162,34 @@ prefill_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
         const bool has = find_work(p, (long long)blockIdx.x, w);
         if (lane == 0) {
             sh[0] = has ? w.b : -1;
-            sh[1] = has ? w.tile : 0;
+            sh[1] = has ? w.pair : 0;
             sh[6] = has ? w.kvh : 0;
         }
     }
     __syncthreads();
     const int b = sh[0];
     if (b < 0) return;
-    const int tile = sh[1];
+    const int pair = sh[1];
     const int kvh = sh[6];
 
     SeqInfo s;
     const bool ok = load_seq(p.cu_seqlens_q, p.seqlens_kv, b, p.batch, p.token_count, p.kv_cap,
                              p.kv_hint, p.q_hint, nullptr, s);
-    const int tok_per_tile = C::BM / g;
-    const int i0 = tile * tok_per_tile;                          // first token of the tile
-    const int rows_valid = min(C::BM, (s.q_len - i0) * g);
+    const int tokp = C::BM / g;                                  // tokens per half
+    const int i0 = pair * 2 * tokp;                              // first token of half 0
+    // Rows and key tiles of each half (a half past the sequence end has none).
+    int rows_valid[2], ntiles_h[2];
+#pragma unroll
+    for (int a = 0; a < 2; ++a) {
+        const int ia = i0 + a * tokp;
+        rows_valid[a] = max(0, min(C::BM, (s.q_len - ia) * g));
+        const int last = min(s.q_len, ia + tokp) - 1;
+        ntiles_h[a] = rows_valid[a] > 0 ? (s.past + last + 1 + C::BN - 1) / C::BN : 0;
+    }
+    const int ntiles = max(ntiles_h[0], ntiles_h[1]);
+
     if (threadIdx.x == 0) {
-        if (tile == 0 && kvh == 0)
+        if (pair == 0 && kvh == 0)
             load_seq(p.cu_seqlens_q, p.seqlens_kv, b, p.batch, p.token_count, p.kv_cap,
                      p.kv_hint, p.q_hint, p.status, s);
         sh[2] = ok ? 0 : 1;
@@ -186,12 +205,14 @@ prefill_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
             mbar_init(&v_full[i], 1);
             mbar_init(&v_empty[i], 1);
         }
-        for (int i = 0; i < 2; ++i) {
+        for (int i = 0; i < 4; ++i) {
             mbar_init(&s_full[i], 1);
             mbar_init(&p_full[i], 4);
         }
-        mbar_init(pv_done, 1);
-        mbar_init(o_full, 1);
+        for (int i = 0; i < 2; ++i) {
+            mbar_init(&pv_done[i], 1);
+            mbar_init(&o_full[i], 1);
+        }
         mbar_init(drain, 1);
         fence_barrier_init();
     }
@@ -200,12 +221,13 @@ prefill_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
     if (ok && warp == 0) {
         const int npages = (T + p.block_size - 1) / p.block_size;
         if (!warp_blocks_ok(p.block_table, b, p.max_blocks, npages, p.num_blocks,
-                            (tile == 0 && kvh == 0) ? p.status : nullptr) && lane == 0)
+                            (pair == 0 && kvh == 0) ? p.status : nullptr) && lane == 0)
             sh[2] = 1;
     }
     __syncthreads();
     if (sh[2]) {
-        for (int idx = threadIdx.x; idx < rows_valid * HEAD; idx += C::THREADS) {
+        const int rows = rows_valid[0] + rows_valid[1];
+        for (int idx = threadIdx.x; idx < rows * HEAD; idx += C::THREADS) {
             const int r = idx / HEAD, d = idx % HEAD;
             const long long o = ((long long)(s.q_start + i0 + r / g) * p.q_heads + kvh * g + r % g) * HEAD + d;
             p.out[o] = __float2half_rn(0.f);
@@ -213,12 +235,7 @@ prefill_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
         return;
     }
 
-    // Keys this tile needs: [0, past + last token of the tile].
-    const int i_last = min(s.q_len, i0 + tok_per_tile) - 1;
-    const int n_keys = s.past + i_last + 1;
-    const int ntiles = (n_keys + C::BN - 1) / C::BN;
-
-    if (warp == 5) {
+    if (warp == C::WARP_MMA) {
         tmem_alloc(tmem_slot, C::TMEM_COLS);
         tmem_relinquish();
     }
@@ -232,80 +249,95 @@ prefill_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
     uint8_t* sV = smem + C::OFF_V;
     const int bs = p.block_size;
     const int32_t* bt = p.block_table + (long long)b * p.max_blocks;
+    const int box = bs < C::BN ? bs : C::BN;
 
-    if (warp == 4) {
-        // ---------------------------------------------------------- producer
+    // Key tile j of the cache map `tm` into `dst`: the pages (or the part of
+    // one page) covering [64 j, 64 j + 64) that start before T.
+    auto load_tile = [&](int j, uint8_t* dst, const CUtensorMap* tm, uint64_t* bar) {
+        const int k0 = j * C::BN;
+        const int npg = bs < C::BN ? (min(k0 + C::BN, T) - k0 + bs - 1) / bs : 1;
+        mbar_arrive_expect_tx(bar, (uint32_t)(npg * box * HEAD * 2));
+        for (int pi = 0; pi < npg; ++pi) {
+            const int key = k0 + pi * box;
+            const int blk = bt[key / bs];
+            const int row = key % bs;
+#pragma unroll
+            for (int c = 0; c < C::NA; ++c)
+                tma_load_4d(dst + (c * C::BN + pi * box) * C::RB, tm, bar, c * C::A, kvh, row, blk);
+        }
+    };
+
+    if (warp == C::WARP_KLOAD) {
+        // ---------------------------------------------------------- Q and K loads
         if (lane == 0) {
             tma_prefetch_desc(&tm_q);
             tma_prefetch_desc(&tm_k);
-            tma_prefetch_desc(&tm_v);
-            mbar_arrive_expect_tx(q_full, C::Q_BYTES);
+            mbar_arrive_expect_tx(q_full, 2 * C::Q_BYTES);
 #pragma unroll
-            for (int c = 0; c < C::NA; ++c)
-                tma_load_3d(sQ + c * C::BM * C::RB, &tm_q, q_full, c * C::A, kvh * g, s.q_start + i0);
-            const int box = bs < C::BN ? bs : C::BN;
-            // Load key tile j of K (which = 0) or V (which = 1) into `dst`.
-            auto load_tile = [&](int j, uint8_t* dst, const CUtensorMap* tm, uint64_t* bar) {
-                const int k0 = j * C::BN;
-                const int npg = bs < C::BN ? (min(k0 + C::BN, T) - k0 + bs - 1) / bs : 1;
-                mbar_arrive_expect_tx(bar, (uint32_t)(npg * box * HEAD * 2));
-                for (int pi = 0; pi < npg; ++pi) {
-                    const int key = k0 + pi * box;
-                    const int blk = bt[key / bs];
-                    const int row = key % bs;
+            for (int a = 0; a < 2; ++a)
 #pragma unroll
-                    for (int c = 0; c < C::NA; ++c)
-                        tma_load_4d(dst + (c * C::BN + pi * box) * C::RB, tm, bar, c * C::A, kvh, row, blk);
+                for (int c = 0; c < C::NA; ++c)
+                    tma_load_3d(sQ + a * C::Q_BYTES + c * C::BM * C::RB, &tm_q, q_full, c * C::A,
+                                kvh * g, s.q_start + i0 + a * tokp);
+            for (int j = 0; j < ntiles; ++j) {
+                const int st = j % C::NK, u = j / C::NK;
+                if (u > 0 && !mbar_wait(&k_empty[st], (u - 1) & 1)) {
+                    flag_status(p.status, PA_DEV_TIMEOUT);
+                    atomicExch(&sh[3], 1);
+                    break;
                 }
-            };
-            bool alive = true;
-            for (int j = 0; j <= ntiles && alive; ++j) {
-                if (j < ntiles) {
-                    const int st = j % C::NK, u = j / C::NK;
-                    if (u > 0 && !mbar_wait(&k_empty[st], (u - 1) & 1)) { alive = false; break; }
-                    if (*(volatile int*)&sh[3]) { alive = false; break; }
-                    sh[4] = j + 1;
-                    load_tile(j, sK + st * C::KV_BYTES, &tm_k, &k_full[st]);
-                }
-                if (j >= 1) {
-                    const int jv = j - 1;
-                    const int st = jv % C::NV, u = jv / C::NV;
-                    if (u > 0 && !mbar_wait(&v_empty[st], (u - 1) & 1)) { alive = false; break; }
-                    if (*(volatile int*)&sh[3]) { alive = false; break; }
-                    sh[5] = jv + 1;
-                    load_tile(jv, sV + st * C::KV_BYTES, &tm_v, &v_full[st]);
-                }
-            }
-            if (!alive) {
-                flag_status(p.status, PA_DEV_TIMEOUT);
-                atomicExch(&sh[3], 1);
+                if (*(volatile int*)&sh[3]) break;
+                sh[4] = j + 1;
+                load_tile(j, sK + st * C::KV_BYTES, &tm_k, &k_full[st]);
             }
         }
-    } else if (warp == 5) {
+    } else if (warp == C::WARP_VLOAD) {
+        // ---------------------------------------------------------- V loads
+        if (lane == 0) {
+            tma_prefetch_desc(&tm_v);
+            for (int j = 0; j < ntiles; ++j) {
+                const int st = j % C::NV, u = j / C::NV;
+                if (u > 0 && !mbar_wait(&v_empty[st], (u - 1) & 1)) {
+                    flag_status(p.status, PA_DEV_TIMEOUT);
+                    atomicExch(&sh[3], 1);
+                    break;
+                }
+                if (*(volatile int*)&sh[3]) break;
+                sh[5] = j + 1;
+                load_tile(j, sV + st * C::KV_BYTES, &tm_v, &v_full[st]);
+            }
+        }
+    } else if (warp == C::WARP_MMA) {
         // ---------------------------------------------------------- MMA issuer
         constexpr uint32_t idesc_s = umma_idesc_f16(C::BM, C::BN, false, false);
         constexpr uint32_t idesc_o = umma_idesc_f16(C::BM, HEAD, false, true);
-        const uint32_t q_addr = smem_u32(sQ), k_addr = smem_u32(sK), v_addr = smem_u32(sV);
+        // Descriptors of the stage / half bases; k-steps add byte offsets / 16
+        // to the start-address field (addresses stay below 256 KB).
+        const uint64_t dq0 = umma_sdesc(smem_u32(sQ), 16, 8 * C::RB, C::LAYOUT);
+        const uint64_t dk0 = umma_sdesc(smem_u32(sK), 16, 8 * C::RB, C::LAYOUT);
+        const uint64_t dv0 = umma_sdesc(smem_u32(sV), C::BN * C::RB, 8 * C::RB, C::LAYOUT);
         bool alive = mbar_wait_warp(q_full, 0);
         auto issue_s = [&](int j) {
             const int st = j % C::NK;
             if (lane == 0) {
 #pragma unroll
-                for (int kk = 0; kk < HEAD / 16; ++kk) {
-                    const int c = (kk * 16) / C::A, w = (kk * 16) % C::A;
-                    const uint64_t da = umma_sdesc(q_addr + c * C::BM * C::RB + w * 2, 16, 8 * C::RB, C::LAYOUT);
-                    const uint64_t db = umma_sdesc(k_addr + st * C::KV_BYTES + c * C::BN * C::RB + w * 2, 16,
-                                                   8 * C::RB, C::LAYOUT);
-                    umma_f16(tmem + (uint32_t)((j & 1) * C::BN), da, db, idesc_s, kk > 0 ? 1u : 0u);
+                for (int a = 0; a < 2; ++a) {
+                    if (j >= ntiles_h[a]) continue;
+#pragma unroll
+                    for (int kk = 0; kk < HEAD / 16; ++kk) {
+                        const int c = (kk * 16) / C::A, w = (kk * 16) % C::A;
+                        const uint64_t da = dq0 + (uint64_t)((a * C::Q_BYTES + c * C::BM * C::RB + w * 2) >> 4);
+                        const uint64_t db = dk0 + (uint64_t)((st * C::KV_BYTES + c * C::BN * C::RB + w * 2) >> 4);
+                        umma_f16(tmem + (uint32_t)(a * 128 + (j & 1) * C::BN), da, db, idesc_s, kk > 0 ? 1u : 0u);
+                    }
+                    umma_commit(&s_full[a * 2 + (j & 1)]);
                 }
-                umma_commit(&s_full[j & 1]);
                 umma_commit(&k_empty[st]);
             }
             __syncwarp();
         };
         auto issue_pv = [&](int j) -> bool {
             const int st = j % C::NV;
-            if (!mbar_wait_warp(&p_full[j & 1], (j >> 1) & 1)) return false;
             if (!mbar_wait_warp(&v_full[st], (j / C::NV) & 1)) return false;
             tc_fence_after();
             const int k0 = j * C::BN;
@@ -319,17 +351,25 @@ prefill_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
                 fence_proxy_async_smem();
                 __syncwarp();
             }
-            if (lane == 0) {
-                const uint32_t p_tmem = tmem + (uint32_t)((j & 1) * C::BN);
 #pragma unroll
-                for (int kk = 0; kk < C::BN / 16; ++kk) {
-                    const uint64_t db = umma_sdesc(v_addr + st * C::KV_BYTES + kk * 16 * C::RB,
-                                                   C::BN * C::RB, 8 * C::RB, C::LAYOUT);
-                    umma_f16_ts(tmem + C::COL_O, p_tmem + kk * 8, db, idesc_o, (j > 0 || kk > 0) ? 1u : 0u);
+            for (int a = 0; a < 2; ++a) {
+                if (j >= ntiles_h[a]) continue;
+                if (!mbar_wait_warp(&p_full[a * 2 + (j & 1)], (j >> 1) & 1)) return false;
+                tc_fence_after();
+                if (lane == 0) {
+                    const uint32_t p_tmem = tmem + (uint32_t)(a * 128 + (j & 1) * C::BN);
+#pragma unroll
+                    for (int kk = 0; kk < C::BN / 16; ++kk) {
+                        const uint64_t db = dv0 + (uint64_t)((st * C::KV_BYTES + kk * 16 * C::RB) >> 4);
+                        umma_f16_ts(tmem + C::COL_O + a * 128, p_tmem + kk * 8, db, idesc_o,
+                                    (j > 0 || kk > 0) ? 1u : 0u);
+                    }
+                    umma_commit(&pv_done[a]);
+                    if (j == ntiles_h[a] - 1) umma_commit(&o_full[a]);
                 }
-                umma_commit(pv_done);
-                umma_commit(&v_empty[st]);
+                __syncwarp();
             }
+            if (lane == 0) umma_commit(&v_empty[st]);
             __syncwarp();
             return true;
         };
@@ -341,8 +381,6 @@ prefill_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
             if (j >= 1 && !issue_pv(j - 1)) { alive = false; break; }
         }
         if (alive && ntiles > 0) alive = issue_pv(ntiles - 1);
-        if (alive && lane == 0) umma_commit(o_full);
-        __syncwarp();
         if (!alive) {
             if (lane == 0) {
                 flag_status(p.status, PA_DEV_TIMEOUT);
@@ -355,45 +393,51 @@ prefill_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
         }
     } else {
         // ---------------------------------------------------------- softmax
-        const int r = threadIdx.x;                       // row == TMEM lane
-        const uint32_t lane_base = (uint32_t)(warp * 32) << 16;
-        const int tok = i0 + r / g;                      // token of this row within the sequence
-        const int lim = (r < rows_valid) ? s.past + tok : T - 1;   // last visible key
-        const int full_vis = s.past + i0;                // every row sees keys <= this
+        const int a = warp >> 2;                         // half
+        const int r = threadIdx.x & 127;                 // row == TMEM lane
+        const uint32_t lane_base = (uint32_t)((warp & 3) * 32) << 16;
+        const int ia = i0 + a * tokp;                    // first token of this half
+        const int tok = ia + r / g;                      // token of this row within the sequence
+        const int my_rows = a ? rows_valid[1] : rows_valid[0];
+        const int lim = (r < my_rows) ? s.past + tok : T - 1;   // last visible key
+        const int full_vis = s.past + ia;                // every row of the half sees keys <= this
+        const int nt = a ? ntiles_h[1] : ntiles_h[0];
         float m_used = -INFINITY, l = 0.f;
         bool alive = true;
-        for (int j = 0; j < ntiles; ++j) {
-            if (!mbar_wait_warp(&s_full[j & 1], (j >> 1) & 1)) { alive = false; break; }
+        for (int j = 0; j < nt; ++j) {
+            const int buf = a * 2 + (j & 1);
+            if (!mbar_wait_warp(&s_full[buf], (j >> 1) & 1)) { alive = false; break; }
             tc_fence_after();
             uint32_t sv[C::BN];
-            const uint32_t scol = tmem + lane_base + (uint32_t)((j & 1) * C::BN);
+            const uint32_t scol = tmem + lane_base + (uint32_t)(a * 128 + (j & 1) * C::BN);
             tmem_ld32(scol, sv);
             tmem_ld32(scol + 32, sv + 32);
             tmem_wait_ld();
             const int k0 = j * C::BN;
-            float mx = -INFINITY;
-            if (k0 + C::BN - 1 <= full_vis) {
+            if (k0 + C::BN - 1 > full_vis) {
 #pragma unroll
-                for (int c = 0; c < C::BN; ++c) mx = fmaxf(mx, __uint_as_float(sv[c]));
-            } else {
-#pragma unroll
-                for (int c = 0; c < C::BN; ++c) {
-                    const bool vis = (k0 + c) <= lim;
-                    sv[c] = vis ? sv[c] : __float_as_uint(-INFINITY);
-                    mx = fmaxf(mx, __uint_as_float(sv[c]));
-                }
+                for (int c = 0; c < C::BN; ++c)
+                    sv[c] = (k0 + c) <= lim ? sv[c] : __float_as_uint(-INFINITY);
             }
+            // Row max as a tree (8 independent chains), not one 64-long chain.
+            float m8[8];
+#pragma unroll
+            for (int i = 0; i < 8; ++i) m8[i] = __uint_as_float(sv[i]);
+#pragma unroll
+            for (int c = 8; c < C::BN; ++c) m8[c & 7] = fmaxf(m8[c & 7], __uint_as_float(sv[c]));
+            float mx = fmaxf(fmaxf(fmaxf(m8[0], m8[1]), fmaxf(m8[2], m8[3])),
+                             fmaxf(fmaxf(m8[4], m8[5]), fmaxf(m8[6], m8[7])));
             mx *= p.scale_log2;
             // Lazy rescale: move the exponent base only when the max grows by > 8.
             if (mx > m_used + 8.f) {
                 const float alpha = (m_used == -INFINITY) ? 0.f : fast_exp2(m_used - mx);
                 l *= alpha;
                 if (j > 0) {
-                    // S_j's commit covered P_{j-2} V_{j-2}, so pv_done is at phase
-                    // j - 1 or j here and this parity wait means "P_{j-1} V_{j-1} done".
-                    if (!mbar_wait_warp(pv_done, (j - 1) & 1)) { alive = false; break; }
+                    // S_a,j's commit covered P_a,j-2 V_j-2, so pv_done[a] is at phase
+                    // j - 1 or j here and this parity wait means "P_a,j-1 V_j-1 done".
+                    if (!mbar_wait_warp(&pv_done[a], (j - 1) & 1)) { alive = false; break; }
                     tc_fence_after();
-                    const uint32_t ocol = tmem + lane_base + C::COL_O;
+                    const uint32_t ocol = tmem + lane_base + C::COL_O + a * 128;
 #pragma unroll
                     for (int c0 = 0; c0 < HEAD; c0 += 16) {
                         uint32_t ov[16];
@@ -408,34 +452,34 @@ prefill_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
             }
             const float base = (m_used == -INFINITY) ? 0.f : m_used;
             uint32_t pk[C::BN / 2];
-            float rs = 0.f;
+            float rs[4] = {0.f, 0.f, 0.f, 0.f};   // independent partial sums
 #pragma unroll
             for (int c = 0; c < C::BN; c += 2) {
                 const float p0 = fast_exp2(fmaf(__uint_as_float(sv[c]), p.scale_log2, -base));
                 const float p1 = fast_exp2(fmaf(__uint_as_float(sv[c + 1]), p.scale_log2, -base));
-                rs += p0 + p1;
+                rs[(c >> 1) & 3] += p0 + p1;
                 pk[c / 2] = pack_half2(p0, p1);
             }
-            l += rs;
-            // P_j over S_j: 64 f16 = 32 columns of this row's lane.
+            l += (rs[0] + rs[1]) + (rs[2] + rs[3]);
+            // P over S: 64 f16 = 32 columns of this row's lane.
             tmem_st32(scol, pk);
             tmem_wait_st();
             tc_fence_before();
             __syncwarp();
-            if (lane == 0) mbar_arrive(&p_full[j & 1]);
+            if (lane == 0) mbar_arrive(&p_full[buf]);
         }
         // Epilogue: O / l -> f16 rows of `out`.
-        if (alive && ntiles > 0 && mbar_wait_warp(o_full, 0)) {
+        if (alive && nt > 0 && mbar_wait_warp(&o_full[a], 0)) {
             tc_fence_after();
             const float inv = (l > 0.f) ? 1.f / l : 0.f;
-            const uint32_t ocol = tmem + lane_base + C::COL_O;
+            const uint32_t ocol = tmem + lane_base + C::COL_O + a * 128;
             __half* orow = p.out + ((long long)(s.q_start + tok) * p.q_heads + kvh * g + r % g) * HEAD;
 #pragma unroll
             for (int c0 = 0; c0 < HEAD; c0 += 16) {
                 uint32_t ov[16];
                 tmem_ld16(ocol + c0, ov);
                 tmem_wait_ld();
-                if (r < rows_valid) {
+                if (r < my_rows) {
                     uint4 w0, w1;
                     w0.x = pack_half2(__uint_as_float(ov[0]) * inv, __uint_as_float(ov[1]) * inv);
                     w0.y = pack_half2(__uint_as_float(ov[2]) * inv, __uint_as_float(ov[3]) * inv);
@@ -468,7 +512,7 @@ prefill_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
             mbar_wait(&v_full[t % C::NV], (t / C::NV) & 1);
     }
     __syncthreads();
-    if (warp == 5) {
+    if (warp == C::WARP_MMA) {
         tc_fence_after();
         tmem_dealloc(tmem, C::TMEM_COLS);
     }
