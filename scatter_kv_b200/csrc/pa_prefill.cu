@@ -15,12 +15,16 @@
 // tiles (one box per page and 64-element column block, 128-byte swizzle)
 // straight from their pages.
 //
-// Warp roles (352 threads):
+// Warp roles (384 threads):
 //   warps 0-3   softmax + epilogue of half 0 (thread r = row r = TMEM lane r)
 //   warps 4-7   softmax + epilogue of half 1
 //   warp 8      TMA producer of Q (both halves) and of the K ring
-//   warp 9      TMA producer of the V ring
-//   warp 10     TMEM allocator and single-thread tcgen05.mma issuer
+//   warp 9      TMA producer of the V ring (and zeroing of V rows past T)
+//   warp 10     TMEM allocator; one thread issues half 0's tcgen05.mma
+//   warp 11     one thread issues half 1's tcgen05.mma
+// tcgen05.mma holds its issuing thread until the tensor pipe accepts it, so
+// each half gets its own issuing thread: while one waits for its softmax,
+// the other keeps the tensor pipe fed.
 // Tensor memory (512 columns): S/P of half a, two buffers of 64 columns at
 // a*128 + (j%2)*64; O of half a at 256 + a*128.
 // Per key tile j and half a:
@@ -29,16 +33,17 @@
 //   softmax               row max / exp2 / row sum in registers; P as f16
 //                          written back over S (32 columns, 2 per column);
 //   O_a += P_a,j V_j      A operand straight from TMEM, M 128, N head_size.
-// The MMA warp issues S for tile j+1 before the P V products of tile j, and
-// the two halves' softmax warpgroups run independently, so the tensor core
-// always has one half's work while the other half exponentiates.  A thread's
-// MMAs run in order on the tensor pipe, so S_a,j+2 cannot overwrite P_a,j
-// before P_a,j V_j has read it.  O is rescaled only when a row maximum grows
+// Each MMA thread issues S for tile j+1 before the P V product of tile j,
+// and the two halves run independently, so the tensor core has one half's
+// work while the other half exponentiates.  A thread's MMAs run in order on
+// the tensor pipe, so S_a,j+2 cannot overwrite P_a,j before P_a,j V_j has
+// read it.  O is rescaled only when a row maximum grows
 // by more than 2^8 (P stays below 256, exact enough in f16 and fp32 sums),
 // which after the first tiles is rare.  Key tiles wholly above a half's
 // causal diagonal are skipped; the diagonal tile is masked per element; rows
-// of V past the end of the sequence are zeroed in shared memory before the
-// P V products that read them.  CTAs are ordered sequence-major, then KV
+// of V past the end of the sequence are zeroed in shared memory (by the V
+// producer, before it marks the tile ready) so that 0 * garbage never
+// reaches the P V products.  CTAs are ordered sequence-major, then KV
 // head, then tile pair from the last (most keys) to the first, so the CTAs
 // resident at any time share few sequences' K/V and reuse them from L2.
 #include <cuda_runtime.h>
@@ -70,14 +75,14 @@ struct PCfg {
     static constexpr int OFF_V = OFF_K + NK * KV_BYTES;
     static constexpr int OFF_BAR = OFF_V + NV * KV_BYTES;
     // q_full, k_full/k_empty x NK, v_full/v_empty x NV, s_full[2][2], p_full[2][2],
-    // pv_done[2], o_full[2], drain
-    static constexpr int NBAR = 1 + 2 * NK + 2 * NV + 4 + 4 + 2 + 2 + 1;
+    // pv_done[2], o_full[2], drain[2], v_tail
+    static constexpr int NBAR = 1 + 2 * NK + 2 * NV + 4 + 4 + 2 + 2 + 2 + 1;
     // At least 120 KB, so that one CTA (which takes all 512 TMEM columns)
     // runs per SM and no second CTA ever waits in tcgen05.alloc.
     static constexpr int SMEM_USED = OFF_BAR + NBAR * 8 + 64;
     static constexpr int SMEM = SMEM_USED > 120 * 1024 ? SMEM_USED : 120 * 1024;
-    static constexpr int THREADS = 352;
-    static constexpr int WARP_KLOAD = 8, WARP_VLOAD = 9, WARP_MMA = 10;
+    static constexpr int THREADS = 384;
+    static constexpr int WARP_KLOAD = 8, WARP_VLOAD = 9, WARP_MMA = 10;   // MMA warps 10, 11
     static constexpr uint32_t TMEM_COLS = 512;
     static constexpr uint32_t COL_O = 256;
     static_assert(SMEM <= 227 * 1024, "shared memory budget");
@@ -144,7 +149,8 @@ prefill_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
     uint64_t* p_full = s_full + 4;           // [half][buffer]
     uint64_t* pv_done = p_full + 4;          // [half]
     uint64_t* o_full = pv_done + 2;          // [half], single use
-    uint64_t* drain = o_full + 2;
+    uint64_t* drain = o_full + 2;            // [half]
+    uint64_t* v_tail = drain + 2;            // TMA of the last V tile (zeroed before release)
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + C::NBAR);
     // [0] b, [1] pair, [2] bad, [3] abort, [4] K tiles issued, [5] V tiles issued, [6] kv head
     int* sh = reinterpret_cast<int*>(tmem_slot + 1);
@@ -199,11 +205,11 @@ prefill_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
         mbar_init(q_full, 1);
         for (int i = 0; i < C::NK; ++i) {
             mbar_init(&k_full[i], 1);
-            mbar_init(&k_empty[i], 1);
+            mbar_init(&k_empty[i], 2);               // one arrival per half
         }
         for (int i = 0; i < C::NV; ++i) {
             mbar_init(&v_full[i], 1);
-            mbar_init(&v_empty[i], 1);
+            mbar_init(&v_empty[i], 2);               // one arrival per half
         }
         for (int i = 0; i < 4; ++i) {
             mbar_init(&s_full[i], 1);
@@ -212,8 +218,9 @@ prefill_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
         for (int i = 0; i < 2; ++i) {
             mbar_init(&pv_done[i], 1);
             mbar_init(&o_full[i], 1);
+            mbar_init(&drain[i], 1);
         }
-        mbar_init(drain, 1);
+        mbar_init(v_tail, 1);
         fence_barrier_init();
     }
     __syncthreads();
@@ -304,93 +311,100 @@ prefill_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
                 }
                 if (*(volatile int*)&sh[3]) break;
                 sh[5] = j + 1;
-                load_tile(j, sV + st * C::KV_BYTES, &tm_v, &v_full[st]);
+                uint8_t* vst = sV + st * C::KV_BYTES;
+                const int k0 = j * C::BN;
+                if (k0 + C::BN <= T) {
+                    load_tile(j, vst, &tm_v, &v_full[st]);
+                } else {
+                    // Last tile: rows at or past T hold stale or poisoned data.  Land
+                    // the tile, zero those rows, then release it to the MMA threads.
+                    load_tile(j, vst, &tm_v, v_tail);
+                    if (!mbar_wait(v_tail, 0)) {
+                        flag_status(p.status, PA_DEV_TIMEOUT);
+                        atomicExch(&sh[3], 1);
+                        break;
+                    }
+                    const int r0 = T - k0 > 0 ? T - k0 : 0;
+                    for (int c = 0; c < C::NA; ++c)
+                        for (int idx = r0 * (C::RB / 16); idx < C::BN * (C::RB / 16); ++idx)
+                            *reinterpret_cast<uint4*>(vst + c * C::BN * C::RB + idx * 16) = make_uint4(0, 0, 0, 0);
+                    fence_proxy_async_smem();
+                    mbar_arrive(&v_full[st]);
+                }
             }
         }
-    } else if (warp == C::WARP_MMA) {
-        // ---------------------------------------------------------- MMA issuer
-        constexpr uint32_t idesc_s = umma_idesc_f16(C::BM, C::BN, false, false);
-        constexpr uint32_t idesc_o = umma_idesc_f16(C::BM, HEAD, false, true);
-        // Descriptors of the stage / half bases; k-steps add byte offsets / 16
-        // to the start-address field (addresses stay below 256 KB).
-        const uint64_t dq0 = umma_sdesc(smem_u32(sQ), 16, 8 * C::RB, C::LAYOUT);
-        const uint64_t dk0 = umma_sdesc(smem_u32(sK), 16, 8 * C::RB, C::LAYOUT);
-        const uint64_t dv0 = umma_sdesc(smem_u32(sV), C::BN * C::RB, 8 * C::RB, C::LAYOUT);
-        bool alive = mbar_wait_warp(q_full, 0);
-        auto issue_s = [&](int j) {
-            const int st = j % C::NK;
-            if (lane == 0) {
-#pragma unroll
-                for (int a = 0; a < 2; ++a) {
-                    if (j >= ntiles_h[a]) continue;
+    } else if (warp >= C::WARP_MMA) {
+        // ---------------------------------------------------------- MMA issuers
+        // Lane 0 of warp 10 + a issues every tcgen05.mma of half a: waits,
+        // descriptor arithmetic, issue.  Past its own last key tile it still
+        // takes part in the K / V ring (waits for the tile, releases the stage)
+        // so that both halves release every stage.
+        const int a = warp - C::WARP_MMA;
+        const int nta = a ? ntiles_h[1] : ntiles_h[0];
+        if (lane == 0) {
+            constexpr uint32_t idesc_s = umma_idesc_f16(C::BM, C::BN, false, false);
+            constexpr uint32_t idesc_o = umma_idesc_f16(C::BM, HEAD, false, true);
+            // Descriptors of the stage / half bases; k-steps add byte offsets / 16
+            // to the start-address field (addresses stay below 256 KB).
+            const uint64_t dq0 = umma_sdesc(smem_u32(sQ + a * C::Q_BYTES), 16, 8 * C::RB, C::LAYOUT);
+            const uint64_t dk0 = umma_sdesc(smem_u32(sK), 16, 8 * C::RB, C::LAYOUT);
+            const uint64_t dv0 = umma_sdesc(smem_u32(sV), C::BN * C::RB, 8 * C::RB, C::LAYOUT);
+            const uint32_t s_col = tmem + (uint32_t)(a * 128);
+            const uint32_t o_col = tmem + C::COL_O + (uint32_t)(a * 128);
+            bool alive = mbar_wait(q_full, 0);
+            auto issue_s = [&](int j) -> bool {
+                const int st = j % C::NK;
+                if (!mbar_wait(&k_full[st], (j / C::NK) & 1)) return false;
+                if (j < nta) {
+                    tc_fence_after();
 #pragma unroll
                     for (int kk = 0; kk < HEAD / 16; ++kk) {
                         const int c = (kk * 16) / C::A, w = (kk * 16) % C::A;
-                        const uint64_t da = dq0 + (uint64_t)((a * C::Q_BYTES + c * C::BM * C::RB + w * 2) >> 4);
+                        const uint64_t da = dq0 + (uint64_t)((c * C::BM * C::RB + w * 2) >> 4);
                         const uint64_t db = dk0 + (uint64_t)((st * C::KV_BYTES + c * C::BN * C::RB + w * 2) >> 4);
-                        umma_f16(tmem + (uint32_t)(a * 128 + (j & 1) * C::BN), da, db, idesc_s, kk > 0 ? 1u : 0u);
+                        umma_f16(s_col + (uint32_t)((j & 1) * C::BN), da, db, idesc_s, kk > 0 ? 1u : 0u);
                     }
                     umma_commit(&s_full[a * 2 + (j & 1)]);
+                    umma_commit(&k_empty[st]);
+                } else {
+                    mbar_arrive(&k_empty[st]);
                 }
-                umma_commit(&k_empty[st]);
-            }
-            __syncwarp();
-        };
-        auto issue_pv = [&](int j) -> bool {
-            const int st = j % C::NV;
-            if (!mbar_wait_warp(&v_full[st], (j / C::NV) & 1)) return false;
-            tc_fence_after();
-            const int k0 = j * C::BN;
-            if (k0 + C::BN > T) {
-                // Zero V rows at or past the sequence end (stale or poisoned data).
-                const int r0 = T - k0 > 0 ? T - k0 : 0;
-                uint8_t* vst = sV + st * C::KV_BYTES;
-                for (int c = 0; c < C::NA; ++c)
-                    for (int idx = r0 * (C::RB / 16) + lane; idx < C::BN * (C::RB / 16); idx += 32)
-                        *reinterpret_cast<uint4*>(vst + c * C::BN * C::RB + idx * 16) = make_uint4(0, 0, 0, 0);
-                fence_proxy_async_smem();
-                __syncwarp();
-            }
-#pragma unroll
-            for (int a = 0; a < 2; ++a) {
-                if (j >= ntiles_h[a]) continue;
-                if (!mbar_wait_warp(&p_full[a * 2 + (j & 1)], (j >> 1) & 1)) return false;
-                tc_fence_after();
-                if (lane == 0) {
-                    const uint32_t p_tmem = tmem + (uint32_t)(a * 128 + (j & 1) * C::BN);
+                return true;
+            };
+            auto issue_pv = [&](int j) -> bool {
+                const int st = j % C::NV;
+                if (!mbar_wait(&v_full[st], (j / C::NV) & 1)) return false;
+                if (j < nta) {
+                    if (!mbar_wait(&p_full[a * 2 + (j & 1)], (j >> 1) & 1)) return false;
+                    tc_fence_after();
+                    const uint32_t p_tmem = s_col + (uint32_t)((j & 1) * C::BN);
 #pragma unroll
                     for (int kk = 0; kk < C::BN / 16; ++kk) {
                         const uint64_t db = dv0 + (uint64_t)((st * C::KV_BYTES + kk * 16 * C::RB) >> 4);
-                        umma_f16_ts(tmem + C::COL_O + a * 128, p_tmem + kk * 8, db, idesc_o,
-                                    (j > 0 || kk > 0) ? 1u : 0u);
+                        umma_f16_ts(o_col, p_tmem + kk * 8, db, idesc_o, (j > 0 || kk > 0) ? 1u : 0u);
                     }
                     umma_commit(&pv_done[a]);
-                    if (j == ntiles_h[a] - 1) umma_commit(&o_full[a]);
+                    if (j == nta - 1) umma_commit(&o_full[a]);
+                    umma_commit(&v_empty[st]);
+                } else {
+                    mbar_arrive(&v_empty[st]);
                 }
-                __syncwarp();
+                return true;
+            };
+            for (int j = 0; alive && j < ntiles; ++j) {
+                if (!issue_s(j)) { alive = false; break; }
+                if (j >= 1 && !issue_pv(j - 1)) { alive = false; break; }
             }
-            if (lane == 0) umma_commit(&v_empty[st]);
-            __syncwarp();
-            return true;
-        };
-        for (int j = 0; alive && j < ntiles; ++j) {
-            const int st = j % C::NK;
-            if (!mbar_wait_warp(&k_full[st], (j / C::NK) & 1)) { alive = false; break; }
-            tc_fence_after();
-            issue_s(j);
-            if (j >= 1 && !issue_pv(j - 1)) { alive = false; break; }
-        }
-        if (alive && ntiles > 0) alive = issue_pv(ntiles - 1);
-        if (!alive) {
-            if (lane == 0) {
+            if (alive && ntiles > 0) alive = issue_pv(ntiles - 1);
+            if (!alive) {
                 flag_status(p.status, PA_DEV_TIMEOUT);
                 atomicExch(&sh[3], 1);
                 // Let every MMA already issued finish before the CTA moves on.
-                umma_commit(drain);
-                mbar_wait(drain, 0);
+                umma_commit(&drain[a]);
+                mbar_wait(&drain[a], 0);
             }
-            __syncwarp();
         }
+        __syncwarp();
     } else {
         // ---------------------------------------------------------- softmax
         const int a = warp >> 2;                         // half
