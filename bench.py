@@ -252,9 +252,10 @@ def run_reference(args, spec, rank, world):
     slots = oracle.slot_mapping(x["block_table"], x["cu_seqlens_q"], x["seqlens_kv"],
                                 spec.block_size)
     oracle.scatter_kv(x["key"], x["value"], slots, x["key_cache"], x["value_cache"])
-    per_step = max(2.0, min(15.0, 150.0 / max(1, args.steps + args.warmup)))
+    # Each step is a bounded sample sized so the whole run takes about two minutes.
+    per_step = max(0.5, min(15.0, 120.0 / max(1, args.steps + args.warmup)))
     for w in range(args.warmup):
-        time_oracle(spec, x, min(per_step, 2.0), seed=1000 + w)
+        time_oracle(spec, x, per_step, seed=1000 + w)
     vals, secs, samples = [], [], []
     for k in range(args.steps):
         v, dt, sample, cores = time_oracle(spec, x, per_step, seed=k)
