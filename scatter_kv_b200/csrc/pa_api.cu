@@ -292,9 +292,6 @@ pa_status pa_attention(const void* query, const void* key_cache, const void* val
         p.part_o = static_cast<float*>(workspace);
         p.part_lse = plan.workspace_bytes ? static_cast<float*>(workspace) + rows_total * d.head_size
                                           : nullptr;
-        p.seq_state = plan.workspace_bytes
-                          ? reinterpret_cast<int32_t*>(p.part_lse + rows_total)
-                          : nullptr;
         p.block_table = block_table;
         p.cu_seqlens_q = cu_seqlens_q;
         p.seqlens_kv = seqlens_kv;

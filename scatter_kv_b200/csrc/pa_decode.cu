@@ -59,7 +59,7 @@ struct Cfg {
     static constexpr int OST = HEAD + 8;                // merge scratch row stride (floats)
     static constexpr int MAX_IDS = 1056;                // block ids of one split (chunk <= 16384)
     static constexpr int SMEM = NST * STAGE_BYTES + 1024 + 2 * NST * 8 + 2 * NG * RMAX * 4 +
-                                2 * RMAX * 4 + 16 + MAX_IDS * 4;
+                                2 * RMAX * 4 + 16 + MAX_IDS * 4 + 32;
     static_assert(NG * RMAX * OST * 4 <= NST * STAGE_BYTES, "merge scratch must fit the stages");
 };
 
@@ -82,8 +82,9 @@ decode_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ 
     float* red_l = red_m + C::NG * C::RMAX;                     // [NG][RMAX]
     float* row_l = red_l + C::NG * C::RMAX;                     // [RMAX]
     float* row_m = row_l + C::RMAX;                             // [RMAX]
-    int* sflag = reinterpret_cast<int*>(row_m + C::RMAX);       // [0] bad seq, [1] abort, [2] issued
+    int* sflag = reinterpret_cast<int*>(row_m + C::RMAX);       // [0] bad split, [1] abort, [2] issued
     int* sids = sflag + 4;                                      // [MAX_IDS] block ids of the split
+    uint64_t* verdict = reinterpret_cast<uint64_t*>(sids + C::MAX_IDS + 4);   // 8-B aligned
 
     // Grid (kv_heads, splits, batch): the KV heads of one split are adjacent
     // in launch order, so they stream the same pages (whose rows interleave
@@ -118,36 +119,12 @@ decode_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ 
         return;
     }
     if (s.q_len == 0) return;
-    const int T = ok ? s.kv_len : 0;
-    const int n_splits = ok ? (T + p.chunk - 1) / p.chunk : 1;
-    if (split >= n_splits) return;
     const int R = s.q_len * g;
-
-    if (threadIdx.x == 0) {
+    if (!ok) {
+        // Invalid metadata: zero rows (split 0 only).
         if (reporter)
             load_seq(p.cu_seqlens_q, p.seqlens_kv, b, p.batch, p.token_count, p.kv_cap,
                      p.kv_hint, p.q_hint, p.status, s);
-        sflag[0] = ok ? 0 : 1;
-        sflag[1] = 0;
-        sflag[2] = 0;
-        for (int i = 0; i < C::NST; ++i) {
-            mbar_init(&full[i], 1);
-            mbar_init(&empty[i], MT);
-        }
-        fence_barrier_init();
-    }
-    __syncthreads();
-    if (ok && warp == 0) {
-        const int npages = (T + p.block_size - 1) / p.block_size;
-        const bool bok = warp_blocks_ok(p.block_table, b, p.max_blocks, npages, p.num_blocks,
-                                        (split == 0 && kvh == 0) ? p.status : nullptr);
-        if (!bok && lane == 0) sflag[0] = 1;
-    }
-    __syncthreads();
-    if (split == 0 && kvh == 0 && threadIdx.x == 0 && p.seq_state != nullptr)
-        p.seq_state[b] = sflag[0] ? 0 : 1;          // read by the combine kernel
-    if (sflag[0]) {
-        // Invalid sequence: zero rows (split 0 only; the combine does the same).
         if (split == 0) {
             for (int idx = threadIdx.x; idx < R * HEAD; idx += C::THREADS) {
                 const int r = idx / HEAD, d = idx % HEAD;
@@ -157,6 +134,22 @@ decode_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ 
         }
         return;
     }
+    const int T = s.kv_len;
+    const int n_splits = (T + p.chunk - 1) / p.chunk;
+    if (split >= n_splits) return;
+
+    if (threadIdx.x == 0) {
+        sflag[0] = 0;
+        sflag[1] = 0;
+        sflag[2] = 0;
+        for (int i = 0; i < C::NST; ++i) {
+            mbar_init(&full[i], 1);
+            mbar_init(&empty[i], MT);
+        }
+        mbar_init(verdict, 1);
+        fence_barrier_init();
+    }
+    __syncthreads();
 
     const int k_begin = split * p.chunk;
     const int k_end = min(T, k_begin + p.chunk);
@@ -168,15 +161,28 @@ decode_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ 
         // ------------------------------------------------------------ producer
         // The split's block ids, fetched once by the whole warp, so issuing a
         // tile never waits on a dependent global load.
+        // They are range-checked here, and only here: the consumers wait for
+        // this verdict instead of re-reading the block table.
         const int pg0 = k_begin / bs;
         const int n_ids = (k_end - 1) / bs + 1 - pg0;
-        for (int i = lane; i < n_ids && i < C::MAX_IDS; i += 32) sids[i] = bt[pg0 + i];
+        bool bad = false;
+        for (int i = lane; i < n_ids; i += 32) {
+            const int id = bt[pg0 + i];
+            bad |= (id < 0 || (long long)id >= p.num_blocks);
+            if (i < C::MAX_IDS) sids[i] = id;
+        }
+        bad = __any_sync(0xffffffffu, bad);
         __syncwarp();
+        if (lane == 0) {
+            if (bad) flag_status(p.status, PA_DEV_BAD_BLOCK);
+            sflag[0] = bad ? 1 : 0;
+            mbar_arrive(verdict);
+        }
         auto block_of = [&](int page) {
             const int i = page - pg0;
             return i < C::MAX_IDS ? sids[i] : bt[page];
         };
-        if (lane == 0) {
+        if (lane == 0 && !bad) {
             tma_prefetch_desc(&tm_k);
             tma_prefetch_desc(&tm_v);
             const uint64_t pol = policy_evict_first();
@@ -248,6 +254,15 @@ decode_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ 
                 qf[kk][3] = q1 ? *reinterpret_cast<const uint32_t*>(q1 + c + 8) : 0u;
             }
         }
+        const long long pbase = (((long long)b * p.kv_heads + kvh) * p.max_splits + split) * p.rmax;
+        // The producer's verdict on this split's block ids.
+        bool split_bad = true;
+        if (mbar_wait_warp(verdict, 0)) {
+            split_bad = *(volatile int*)&sflag[0] != 0;
+        } else {
+            flag_status(p.status, PA_DEV_TIMEOUT);
+            atomicExch(&sflag[1], 1);
+        }
         float oacc[HEAD / 8][4];
 #pragma unroll
         for (int i = 0; i < HEAD / 8; ++i)
@@ -258,7 +273,10 @@ decode_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ 
         // ldmatrix lane roles: matrix mi = lane / 8, row rr = lane % 8.
         const int mi = lane >> 3, rr = lane & 7;
 
-        for (int t = grp; t < ntiles; t += C::NG) {
+        // A split with a bad block id runs no tile: its rows come out as zero
+        // when the sequence has one split; otherwise it writes an lse of +inf,
+        // on which the combine zeroes the sequence's rows.
+        for (int t = split_bad ? ntiles : grp; t < ntiles; t += C::NG) {
             const int st = t % C::NST, u = t / C::NST;
             if (!mbar_wait_warp(&full[st], u & 1)) {
                 flag_status(p.status, PA_DEV_TIMEOUT);
@@ -408,7 +426,6 @@ decode_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ 
         asm volatile("bar.sync 1, %0;" ::"r"(C::NCW * 32));
         // Final rows: sum the groups in order, normalise, write.
         const bool direct = (n_splits == 1);
-        const long long pbase = (((long long)b * p.kv_heads + kvh) * p.max_splits + split) * p.rmax;
         for (int idx = threadIdx.x; idx < R * (HEAD / 4); idx += C::NCW * 32) {
             const int r = idx / (HEAD / 4), d4 = (idx % (HEAD / 4)) * 4;
             float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
@@ -428,7 +445,8 @@ decode_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ 
             } else {
                 *reinterpret_cast<float4*>(p.part_o + (pbase + r) * HEAD + d4) = acc;
                 if (d4 == 0)
-                    p.part_lse[pbase + r] = (L > 0.f) ? row_m[r] + __log2f(L) : -INFINITY;
+                    p.part_lse[pbase + r] = split_bad ? INFINITY
+                                          : (L > 0.f) ? row_m[r] + __log2f(L) : -INFINITY;
             }
         }
     }
@@ -451,25 +469,26 @@ __global__ void __launch_bounds__(128) combine_kernel(const DecodeParams p) {
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int r = blockIdx.x * 4 + warp;
     const int g = p.group;
-    const int c0 = p.cu_seqlens_q[b], c1 = p.cu_seqlens_q[b + 1];
-    const int q_len = c1 - c0;
-    if (c0 < 0 || c1 < c0 || (long long)c1 > p.token_count) return;
-    if (q_len == 0 || q_len > p.decode_max_q || r >= q_len * g) return;
-    __half* orow = p.out + ((long long)(c0 + r / g) * p.q_heads + kvh * g + r % g) * HEAD;
-    const int state = p.seq_state[b];                 // written by the decode kernel
-    if (state != 1) {
-        // Invalid sequence: zero rows, like the decode kernel does for one split.
-        for (int d = lane; d < HEAD; d += 32) orow[d] = __float2half_rn(0.f);
+    SeqInfo s;
+    // Invalid metadata: the decode kernel has zeroed the rows already.
+    if (!load_seq(p.cu_seqlens_q, p.seqlens_kv, b, p.batch, p.token_count, p.kv_cap, p.kv_hint,
+                  p.q_hint, nullptr, s))
         return;
-    }
-    const int n_splits = (p.seqlens_kv[b] + p.chunk - 1) / p.chunk;
+    if (s.q_len == 0 || s.q_len > p.decode_max_q || r >= s.q_len * g) return;
+    const int n_splits = (s.kv_len + p.chunk - 1) / p.chunk;
     if (n_splits == 1) return;                        // the decode kernel wrote the row
+    __half* orow = p.out + ((long long)(s.q_start + r / g) * p.q_heads + kvh * g + r % g) * HEAD;
     const long long base = ((long long)b * p.kv_heads + kvh) * p.max_splits * p.rmax + r;
     const float* lse = p.part_lse + base;             // stride rmax per split
     float M = -INFINITY;
     for (int sp = lane; sp < n_splits; sp += 32) M = fmaxf(M, lse[(long long)sp * p.rmax]);
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, o));
+    if (M == INFINITY) {
+        // Some split found a bad block id: the sequence gets zero rows.
+        for (int d = lane; d < HEAD; d += 32) orow[d] = __float2half_rn(0.f);
+        return;
+    }
     float L = 0.f;
     for (int sp = lane; sp < n_splits; sp += 32) L += fast_exp2(lse[(long long)sp * p.rmax] - M);
 #pragma unroll
@@ -530,9 +549,9 @@ DecodePlan plan_decode(const pa_dims& d, int num_sms) {
     pl.chunk = (int)chunk;
     pl.max_splits = (int)((max_kv + chunk - 1) / chunk);
     if (pl.max_splits > 1) {
-        // [partial O: rows x head_size f32][partial lse: rows f32][state: batch i32]
+        // [partial O: rows x head_size f32][partial lse: rows f32]
         const size_t rows = (size_t)d.batch * d.kv_heads * pl.max_splits * (16 * pl.mtiles);
-        pl.workspace_bytes = rows * (size_t)d.head_size * 4 + rows * 4 + (size_t)d.batch * 4;
+        pl.workspace_bytes = rows * (size_t)d.head_size * 4 + rows * 4;
         pl.workspace_bytes = (pl.workspace_bytes + 255) / 256 * 256;
     }
     return pl;

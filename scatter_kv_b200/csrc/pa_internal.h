@@ -16,7 +16,6 @@ struct DecodeParams {
     __half* out;
     float* part_o;                // [batch, kv_heads, max_splits, rmax, head_size]
     float* part_lse;              // [batch, kv_heads, max_splits, rmax] (log2 domain)
-    int32_t* seq_state;           // [batch]: 1 valid decode sequence, 0 invalid (split runs only)
     const int32_t* block_table;
     const int32_t* cu_seqlens_q;
     const int32_t* seqlens_kv;

@@ -32,13 +32,30 @@ def _check(spec, x, bad_seq, bit, hints=True, want_x=None):
             assert_close(got[_rows(spec, b)], want[_rows(spec, b)], what=f"seq {b}")
 
 
+@pytest.mark.parametrize("where", ["first", "last"])
 @pytest.mark.parametrize("bad_seq", [0, 1, 2, 3])
-def test_out_of_range_block_id(bad_seq):
+def test_out_of_range_block_id(bad_seq, where):
+    # "last" puts the bad id in the sequence's last page, which for sequence 2
+    # belongs to its last split rather than the first.
     spec = _spec()
     x = workloads.generate(spec)
     ref = {k: v.copy() for k, v in x.items()}
-    x["block_table"][bad_seq, 0] = spec.num_blocks + 5
+    page = 0 if where == "first" else (int(spec.seqlens_kv[bad_seq]) - 1) // spec.block_size
+    x["block_table"][bad_seq, page] = spec.num_blocks + 5 if where == "first" else -1
     _check(spec, x, bad_seq, pa.PA_DEV_BAD_BLOCK, want_x=ref)
+
+
+def test_bad_id_past_sequence_end_ignored():
+    # Block-table entries past a sequence's last page are never read.
+    spec = _spec()
+    x = workloads.generate(spec)
+    for b in range(spec.batch):
+        npages = int(spec.pages_per_seq[b])
+        x["block_table"][b, npages:] = -7
+    got, _, status, _ = run_gpu(spec, x)
+    assert status == 0, f"status {status:#x}"
+    want, _, _, _ = oracle_step(spec, x)
+    assert_close(got, want)
 
 
 @pytest.mark.parametrize("bad_seq", [0, 1])
