@@ -333,7 +333,7 @@ pa_status pa_attention(const void* query, const void* key_cache, const void* val
             if (slots * d.kv_heads >= (1ll << 31))
                 return fail(PA_ERR_NOT_IMPLEMENTED, "too many query tiles (%lld)", slots);
             CUtensorMap tq, tk, tv;
-            const int rows = d.block_size < 64 ? d.block_size : 64;
+            const int rows = d.block_size < pa::kPrefillKeys ? d.block_size : pa::kPrefillKeys;
             if ((st = make_query_map(&tq, query, d)) != PA_OK) return st;
             if ((st = make_cache_map(&tk, key_cache, d, rows)) != PA_OK) return st;
             if ((st = make_cache_map(&tv, value_cache, d, rows)) != PA_OK) return st;

@@ -101,5 +101,6 @@ constexpr int kDecodeKeys = 32;
 constexpr int kPrefillKeys = 128;
 constexpr int kPrefillRows = 128;      // query rows per tensor-core tile
 constexpr int kPrefillCtaRows = 256;   // query rows per prefill CTA (two tiles)
+constexpr int kPrefillLaunchRegs = 168; // registers per thread of the 384-thread prefill CTA
 
 }  // namespace pa

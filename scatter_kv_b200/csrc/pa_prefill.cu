@@ -11,41 +11,49 @@
 // KV head.  Rows are (token, head) pairs: 128 / group consecutive tokens
 // times the group query heads that share the KV head, so every K/V page is
 // loaded once for 256 query rows.  There is no gathered or padded copy of
-// the cache: producer warps walk the block table and TMA-load 64-key K and V
-// tiles (one box per page and 64-element column block, 128-byte swizzle)
-// straight from their pages.
+// the cache: the producer warp walks the block table and TMA-loads 128-key K
+// and V tiles (one box per page and 64-element column block, 128-byte
+// swizzle) straight from their pages into one ring of shared-memory stages,
+// in the order K_0, V_0, K_1, V_1, ...
 //
-// Warp roles (384 threads):
+// Warp roles (384 threads, three warpgroups):
 //   warps 0-3   softmax + epilogue of half 0 (thread r = row r = TMEM lane r)
 //   warps 4-7   softmax + epilogue of half 1
-//   warp 8      TMA producer of Q (both halves) and of the K ring
-//   warp 9      TMA producer of the V ring (and zeroing of V rows past T)
-//   warp 10     TMEM allocator; one thread issues half 0's tcgen05.mma
-//   warp 11     one thread issues half 1's tcgen05.mma
-// tcgen05.mma holds its issuing thread until the tensor pipe accepts it, so
-// each half gets its own issuing thread: while one waits for its softmax,
-// the other keeps the tensor pipe fed.
-// Tensor memory (512 columns): S/P of half a, two buffers of 64 columns at
-// a*128 + (j%2)*64; O of half a at 256 + a*128.
+//   warps 8, 10, 11  TMA producers (Q of both halves, then the K/V ring;
+//               each ring item's boxes are dealt out over the three warps,
+//               since one issuing warp gets through only a few boxes per
+//               microsecond and small pages make many boxes)
+//   warp 9      TMEM allocator; one thread issues every tcgen05.mma
+// The third warpgroup hands registers to the softmax warpgroups
+// (setmaxnreg): a softmax thread holds its whole 128-key row of S.
+// Tensor memory (512 columns): S/P of half a at a*128 (128 columns); O of
+// half a at 256 + a*128.
 // Per key tile j and half a:
-//   S_a,j = Q_a K_j^T     M 128, N 64, fp32; K_j is released once both
-//                          halves' products are done;
-//   softmax               row max / exp2 / row sum in registers; P as f16
-//                          written back over S (32 columns, 2 per column);
-//   O_a += P_a,j V_j      A operand straight from TMEM, M 128, N head_size.
-// Each MMA thread issues S for tile j+1 before the P V product of tile j,
-// and the two halves run independently, so the tensor core has one half's
-// work while the other half exponentiates.  A thread's MMAs run in order on
-// the tensor pipe, so S_a,j+2 cannot overwrite P_a,j before P_a,j V_j has
-// read it.  O is rescaled only when a row maximum grows
-// by more than 2^8 (P stays below 256, exact enough in f16 and fp32 sums),
-// which after the first tiles is rare.  Key tiles wholly above a half's
-// causal diagonal are skipped; the diagonal tile is masked per element; rows
-// of V past the end of the sequence are zeroed in shared memory (by the V
-// producer, before it marks the tile ready) so that 0 * garbage never
-// reaches the P V products.  CTAs are ordered sequence-major, then KV
-// head, then tile pair from the last (most keys) to the first, so the CTAs
-// resident at any time share few sequences' K/V and reuse them from L2.
+//   S_a = Q_a K_j^T        M 128, N 128, K head_size (fp32 in TMEM)
+//   (softmax: row max, exp2, row sum; P as f16 written over S)
+//   O_a += P_a V_j         A operand read from TMEM, M 128, N head_size.
+// One thread issues every product, in the order
+//   S_0,0  S_1,0 | P_0,0 V_0  S_0,1 | P_1,0 V_0  S_1,1 | P_0,1 V_1  S_0,2 | ...
+// so each half's softmax of tile j runs while the tensor pipe works through
+// the other half's group (its P V and next S, 2 x 8 N = 128 instructions),
+// and the two halves' exponentials take turns on the MUFU units by
+// construction.  MMAs of one thread run in order, so S_a of tile j+1 cannot
+// overwrite P_a (which lives in S_a's columns) before P_a V_j has read it,
+// and the commit that signals "S_a of tile j+1 is ready" also covers P_a V_j.
+// exp2 runs on the MUFU unit.  A polynomial exp2 on the FMA pipe
+// (exp2_poly) can take a share of the columns (kPolyEvery); measured on
+// B200 with head size 128 it only adds instructions to a softmax whose cost
+// is set by instruction issue, not by MUFU throughput, so it is off.
+// O is rescaled only when some row maximum of a warp grows by more than 2^8
+// (P stays below 256, exact enough in f16 and fp32 sums), which after the
+// first tiles is rare; the decision is warp-uniform because tcgen05.ld/st
+// are warp-collective.  Key tiles wholly above a half's causal diagonal are
+// skipped; the diagonal tile is masked per element; rows of V past the end
+// of the sequence are zeroed in shared memory (by the producer, before it
+// marks the tile ready) so that 0 * garbage never reaches the P V products.
+// CTAs are ordered sequence-major, then KV head, then tile pair from the
+// last (most keys) to the first, so the CTAs resident at any time share few
+// sequences' K/V and reuse them from L2.
 #include <cuda_runtime.h>
 #include <math.h>
 
@@ -59,34 +67,49 @@ namespace {
 template <int HEAD>
 struct PCfg {
     static constexpr int BM = kPrefillRows;             // 128 query rows per half
-    static constexpr int BN = 64;                       // keys per tile
+    static constexpr int BN = kPrefillKeys;             // 128 keys per tile
     static constexpr int A = HEAD < 64 ? HEAD : 64;     // elements per swizzled row (Q, K, V)
     static constexpr int RB = A * 2;
     static constexpr int NA = HEAD / A;
     static constexpr uint32_t LAYOUT = RB == 128 ? 2u : (RB == 64 ? 4u : 6u);
     static constexpr int Q_BYTES = BM * HEAD * 2;       // one half
-    static constexpr int KV_BYTES = BN * HEAD * 2;
-    // Stage counts: as deep as shared memory allows (the K and V loads of a
-    // tile are issued by separate warps and can each run that far ahead).
-    static constexpr int NK = HEAD >= 128 ? 5 : 8;
-    static constexpr int NV = HEAD >= 128 ? 4 : 8;
+    static constexpr int KV_BYTES = BN * HEAD * 2;      // one K or V tile
+    // Ring stages: as many as shared memory holds, at most 8.
+    static constexpr int NS_FIT = (226 * 1024 - 2 * Q_BYTES) / KV_BYTES;
+    static constexpr int NS = NS_FIT < 8 ? NS_FIT : 8;
     static constexpr int OFF_Q = 0;
-    static constexpr int OFF_K = OFF_Q + 2 * Q_BYTES;
-    static constexpr int OFF_V = OFF_K + NK * KV_BYTES;
-    static constexpr int OFF_BAR = OFF_V + NV * KV_BYTES;
-    // q_full, k_full/k_empty x NK, v_full/v_empty x NV, s_full[2][2], p_full[2][2],
-    // pv_done[2], o_full[2], drain[2], v_tail
-    static constexpr int NBAR = 1 + 2 * NK + 2 * NV + 4 + 4 + 2 + 2 + 2 + 1;
+    static constexpr int OFF_RING = OFF_Q + 2 * Q_BYTES;
+    static constexpr int OFF_BAR = OFF_RING + NS * KV_BYTES;
+    // q_full, full/empty x NS, s_full[2], p_full[2], o_full[2], drain, v_tail
+    static constexpr int NBAR = 1 + 2 * NS + 2 + 2 + 2 + 1 + 1;
     // At least 120 KB, so that one CTA (which takes all 512 TMEM columns)
     // runs per SM and no second CTA ever waits in tcgen05.alloc.
     static constexpr int SMEM_USED = OFF_BAR + NBAR * 8 + 64;
     static constexpr int SMEM = SMEM_USED > 120 * 1024 ? SMEM_USED : 120 * 1024;
     static constexpr int THREADS = 384;
-    static constexpr int WARP_KLOAD = 8, WARP_VLOAD = 9, WARP_MMA = 10;   // MMA warps 10, 11
+    static constexpr int WARP_MMA = 9;            // producers: warps 8, 10, 11
+    static constexpr int NPROD = 3;
+    // Register split: launched with kLaunchRegs per thread; the softmax
+    // warpgroups raise theirs to REGS_SOFTMAX, the third lowers to REGS_OTHER.
+    // The shares must add up to exactly the launch's registers.
+    static constexpr int REGS_SOFTMAX = 208, REGS_OTHER = 88;
+    static_assert(128 * (2 * REGS_SOFTMAX + REGS_OTHER) == THREADS * kPrefillLaunchRegs,
+                  "register split must equal the launch budget");
     static constexpr uint32_t TMEM_COLS = 512;
     static constexpr uint32_t COL_O = 256;
+    static_assert(NS >= 2, "the ring needs at least two stages");
     static_assert(SMEM <= 227 * 1024, "shared memory budget");
+    static_assert(HEAD <= 128, "O of both halves must fit beside S in 512 TMEM columns");
 };
+
+template <int N>
+__device__ __forceinline__ void regs_inc() {
+    asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(N));
+}
+template <int N>
+__device__ __forceinline__ void regs_dec() {
+    asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(N));
+}
 
 struct Work {
     int b;          // sequence
@@ -133,6 +156,36 @@ __device__ bool find_work(const PrefillParams& p, long long slot, Work& w) {
     return false;
 }
 
+// 2^x on the FMA pipe, for x <= 8 (x = -inf gives a value below 2^-124,
+// which rounds to 0 in f16).  Range reduction in the style of Cody and
+// Waite: x = n + f with n = round(x) (the 1.5 * 2^23 shifter leaves n in the
+// low mantissa bits) and f in [-1/2, 1/2]; 2^f by a degree-3 polynomial with
+// constant term exactly 1, coefficients fitted here by iteratively
+// reweighted least squares (Lawson) for minimum maximum relative error on
+// [-1/2, 1/2]; 2^n is added to the exponent field.  Maximum relative error
+// about 1.2e-4, under half an f16 ulp (P is rounded to f16 right after).
+__device__ __forceinline__ float exp2_poly(float x) {
+    x = fmaxf(x, -125.f);                          // keeps the exponent field >= 1
+    const float shifter = 12582912.f;              // 1.5 * 2^23
+    const float t = x + shifter;
+    const float f = x - (t - shifter);
+    float p = fmaf(0.05541787f, f, 0.24221125f);
+    p = fmaf(p, f, 0.69319951f);
+    p = fmaf(p, f, 1.0f);
+    return __uint_as_float(__float_as_uint(p) + (__float_as_uint(t) << 23));
+}
+
+// Columns c with (c % kPolyEvery) == kPolyEvery - 1 take exp2_poly
+// (kPolyEvery 0: none).
+#ifndef PA_POLY_EVERY
+#define PA_POLY_EVERY 0
+#endif
+constexpr int kPolyEvery = PA_POLY_EVERY;
+__device__ __forceinline__ bool poly_col(int c) {
+    return kPolyEvery > 0 && (c % (kPolyEvery > 0 ? kPolyEvery : 1)) == kPolyEvery - 1;
+}
+
+
 template <int HEAD>
 __global__ void __launch_bounds__(PCfg<HEAD>::THREADS, 1)
 prefill_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
@@ -141,18 +194,15 @@ prefill_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
     extern __shared__ __align__(1024) uint8_t smem[];
     uint64_t* bars = reinterpret_cast<uint64_t*>(smem + C::OFF_BAR);
     uint64_t* q_full = bars;
-    uint64_t* k_full = q_full + 1;
-    uint64_t* k_empty = k_full + C::NK;
-    uint64_t* v_full = k_empty + C::NK;
-    uint64_t* v_empty = v_full + C::NV;
-    uint64_t* s_full = v_empty + C::NV;      // [half][buffer]
-    uint64_t* p_full = s_full + 4;           // [half][buffer]
-    uint64_t* pv_done = p_full + 4;          // [half]
-    uint64_t* o_full = pv_done + 2;          // [half], single use
-    uint64_t* drain = o_full + 2;            // [half]
-    uint64_t* v_tail = drain + 2;            // TMA of the last V tile (zeroed before release)
+    uint64_t* full = q_full + 1;             // [NS] ring stage loaded
+    uint64_t* empty = full + C::NS;          // [NS] ring stage released (MMAs reading it done)
+    uint64_t* s_full = empty + C::NS;        // [half] S ready (and the previous P V done)
+    uint64_t* p_full = s_full + 2;           // [half] P written (4 warps)
+    uint64_t* o_full = p_full + 2;           // [half] last P V done, single use
+    uint64_t* drain = o_full + 2;            // every MMA issued so far is done (abort path)
+    uint64_t* v_tail = drain + 1;            // TMA of the last V tile (zeroed before release)
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + C::NBAR);
-    // [0] b, [1] pair, [2] bad, [3] abort, [4] K tiles issued, [5] V tiles issued, [6] kv head
+    // [0] b, [1] pair, [2] bad, [3] abort, [4] ring items issued, [6] kv head
     int* sh = reinterpret_cast<int*>(tmem_slot + 1);
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -201,25 +251,17 @@ prefill_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
         sh[2] = ok ? 0 : 1;
         sh[3] = 0;
         sh[4] = 0;
-        sh[5] = 0;
         mbar_init(q_full, 1);
-        for (int i = 0; i < C::NK; ++i) {
-            mbar_init(&k_full[i], 1);
-            mbar_init(&k_empty[i], 2);               // one arrival per half
-        }
-        for (int i = 0; i < C::NV; ++i) {
-            mbar_init(&v_full[i], 1);
-            mbar_init(&v_empty[i], 2);               // one arrival per half
-        }
-        for (int i = 0; i < 4; ++i) {
-            mbar_init(&s_full[i], 1);
-            mbar_init(&p_full[i], 4);
+        for (int i = 0; i < C::NS; ++i) {
+            mbar_init(&full[i], C::NPROD);           // one arrival per producer warp
+            mbar_init(&empty[i], 1);
         }
         for (int i = 0; i < 2; ++i) {
-            mbar_init(&pv_done[i], 1);
+            mbar_init(&s_full[i], 1);
+            mbar_init(&p_full[i], 4);
             mbar_init(&o_full[i], 1);
-            mbar_init(&drain[i], 1);
         }
+        mbar_init(drain, 1);
         mbar_init(v_tail, 1);
         fence_barrier_init();
     }
@@ -252,33 +294,23 @@ prefill_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
     const uint32_t tmem = *tmem_slot;
 
     uint8_t* sQ = smem + C::OFF_Q;
-    uint8_t* sK = smem + C::OFF_K;
-    uint8_t* sV = smem + C::OFF_V;
+    uint8_t* ring = smem + C::OFF_RING;
     const int bs = p.block_size;
     const int32_t* bt = p.block_table + (long long)b * p.max_blocks;
     const int box = bs < C::BN ? bs : C::BN;
 
-    // Key tile j of the cache map `tm` into `dst`: the pages (or the part of
-    // one page) covering [64 j, 64 j + 64) that start before T.
-    auto load_tile = [&](int j, uint8_t* dst, const CUtensorMap* tm, uint64_t* bar) {
-        const int k0 = j * C::BN;
-        const int npg = bs < C::BN ? (min(k0 + C::BN, T) - k0 + bs - 1) / bs : 1;
-        mbar_arrive_expect_tx(bar, (uint32_t)(npg * box * HEAD * 2));
-        for (int pi = 0; pi < npg; ++pi) {
-            const int key = k0 + pi * box;
-            const int blk = bt[key / bs];
-            const int row = key % bs;
-#pragma unroll
-            for (int c = 0; c < C::NA; ++c)
-                tma_load_4d(dst + (c * C::BN + pi * box) * C::RB, tm, bar, c * C::A, kvh, row, blk);
-        }
-    };
-
-    if (warp == C::WARP_KLOAD) {
-        // ---------------------------------------------------------- Q and K loads
-        if (lane == 0) {
+    if (warp == 8 || warp >= 10) {
+        // -------------------------------------------------------------- producers
+        regs_dec<C::REGS_OTHER>();
+        const int pw = warp == 8 ? 0 : warp - 9;       // producer index 0, 1, 2
+        // Ring item u: K_{u/2} (u even) or V_{u/2} (u odd), in stage u % NS.
+        // Key tile j covers keys [128 j, 128 j + 128): the pages (or the part of
+        // one page) holding them, up to the last page that starts before T.
+        // Box b = page * NA + column block goes to producer b % NPROD.
+        if (pw == 0 && lane == 0) {
             tma_prefetch_desc(&tm_q);
             tma_prefetch_desc(&tm_k);
+            tma_prefetch_desc(&tm_v);
             mbar_arrive_expect_tx(q_full, 2 * C::Q_BYTES);
 #pragma unroll
             for (int a = 0; a < 2; ++a)
@@ -286,127 +318,168 @@ prefill_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
                 for (int c = 0; c < C::NA; ++c)
                     tma_load_3d(sQ + a * C::Q_BYTES + c * C::BM * C::RB, &tm_q, q_full, c * C::A,
                                 kvh * g, s.q_start + i0 + a * tokp);
-            for (int j = 0; j < ntiles; ++j) {
-                const int st = j % C::NK, u = j / C::NK;
-                if (u > 0 && !mbar_wait(&k_empty[st], (u - 1) & 1)) {
-                    flag_status(p.status, PA_DEV_TIMEOUT);
-                    atomicExch(&sh[3], 1);
-                    break;
-                }
-                if (*(volatile int*)&sh[3]) break;
-                sh[4] = j + 1;
-                load_tile(j, sK + st * C::KV_BYTES, &tm_k, &k_full[st]);
-            }
         }
-    } else if (warp == C::WARP_VLOAD) {
-        // ---------------------------------------------------------- V loads
-        if (lane == 0) {
-            tma_prefetch_desc(&tm_v);
-            for (int j = 0; j < ntiles; ++j) {
-                const int st = j % C::NV, u = j / C::NV;
-                if (u > 0 && !mbar_wait(&v_empty[st], (u - 1) & 1)) {
+        // Block ids of the sequence, 32 pages at a time in registers (lane i
+        // holds page win_base + i); the next window is fetched a whole window
+        // ahead, so issuing a tile never waits on a block-table load.
+        const int npages = (T + bs - 1) / bs;
+        int win_base = 0;
+        int win_id = lane < npages ? bt[lane] : 0;
+        int nxt_id = 32 + lane < npages ? bt[32 + lane] : 0;
+        auto page_id = [&](int page) -> int {          // warp-uniform, pages ascending
+            while (page >= win_base + 32) {
+                win_base += 32;
+                win_id = nxt_id;
+                nxt_id = win_base + 32 + lane < npages ? bt[win_base + 32 + lane] : 0;
+            }
+            return __shfl_sync(0xffffffffu, win_id, page - win_base);
+        };
+        for (int u = 0; u < 2 * ntiles; ++u) {
+            const int st = u % C::NS;
+            const int j = u >> 1;
+            const bool is_v = (u & 1) != 0;
+            const int k0 = j * C::BN;
+            // The last V tile (rows past T to be zeroed) is producer 0's alone.
+            const bool tail = is_v && (k0 + C::BN > T);
+            if (tail && pw != 0) continue;
+            bool go = true;
+            if (lane == 0 && u >= C::NS) go = mbar_wait(&empty[st], ((u / C::NS) - 1) & 1);
+            go = __shfl_sync(0xffffffffu, go, 0);
+            if (!go) {
+                if (lane == 0) {
                     flag_status(p.status, PA_DEV_TIMEOUT);
                     atomicExch(&sh[3], 1);
-                    break;
                 }
-                if (*(volatile int*)&sh[3]) break;
-                sh[5] = j + 1;
-                uint8_t* vst = sV + st * C::KV_BYTES;
-                const int k0 = j * C::BN;
-                if (k0 + C::BN <= T) {
-                    load_tile(j, vst, &tm_v, &v_full[st]);
-                } else {
-                    // Last tile: rows at or past T hold stale or poisoned data.  Land
-                    // the tile, zero those rows, then release it to the MMA threads.
-                    load_tile(j, vst, &tm_v, v_tail);
-                    if (!mbar_wait(v_tail, 0)) {
+                break;
+            }
+            if (__shfl_sync(0xffffffffu, *(volatile int*)&sh[3], 0)) break;
+            uint8_t* dst = ring + st * C::KV_BYTES;
+            const int npg = bs < C::BN ? (min(k0 + C::BN, T) - k0 + bs - 1) / bs : 1;
+            const int nbox = npg * C::NA;
+            const int mine = tail ? nbox : (nbox - pw + C::NPROD - 1) / C::NPROD;
+            uint64_t* bar = tail ? v_tail : &full[st];
+            if (lane == 0) {
+                if (pw == 0) sh[4] = u + 1;
+                mbar_arrive_expect_tx(bar, (uint32_t)(mine * box * C::RB));
+            }
+            const CUtensorMap* tm = is_v ? &tm_v : &tm_k;
+            for (int pi = 0; pi < npg; ++pi) {
+                const int key = k0 + pi * box;
+                const int blk = page_id(key / bs);
+                const int row = key % bs;
+                if (lane == 0) {
+#pragma unroll
+                    for (int c = 0; c < C::NA; ++c)
+                        if (tail || (pi * C::NA + c) % C::NPROD == pw)
+                            tma_load_4d(dst + (c * C::BN + pi * box) * C::RB, tm, bar, c * C::A, kvh, row, blk);
+                }
+            }
+            if (tail) {
+                // Last V tile: rows at or past T hold stale or poisoned data.  Land
+                // the tile, zero those rows, then release it to the MMA thread
+                // (arriving for all producers).
+                if (!mbar_wait_warp(v_tail, 0)) {
+                    if (lane == 0) {
                         flag_status(p.status, PA_DEV_TIMEOUT);
                         atomicExch(&sh[3], 1);
-                        break;
                     }
-                    const int r0 = T - k0 > 0 ? T - k0 : 0;
-                    for (int c = 0; c < C::NA; ++c)
-                        for (int idx = r0 * (C::RB / 16); idx < C::BN * (C::RB / 16); ++idx)
-                            *reinterpret_cast<uint4*>(vst + c * C::BN * C::RB + idx * 16) = make_uint4(0, 0, 0, 0);
-                    fence_proxy_async_smem();
-                    mbar_arrive(&v_full[st]);
+                    break;
                 }
+                const int r0 = T - k0 > 0 ? T - k0 : 0;
+                constexpr int CH = C::RB / 16;                 // 16-byte chunks per row
+                for (int c = 0; c < C::NA; ++c)
+                    for (int idx = r0 * CH + lane; idx < C::BN * CH; idx += 32)
+                        *reinterpret_cast<uint4*>(dst + c * C::BN * C::RB + idx * 16) = make_uint4(0, 0, 0, 0);
+                fence_proxy_async_smem();
+                __syncwarp();
+                if (lane == 0) mbar_arrive_cnt(&full[st], C::NPROD);
             }
         }
-    } else if (warp >= C::WARP_MMA) {
-        // ---------------------------------------------------------- MMA issuers
-        // Lane 0 of warp 10 + a issues every tcgen05.mma of half a: waits,
-        // descriptor arithmetic, issue.  Past its own last key tile it still
-        // takes part in the K / V ring (waits for the tile, releases the stage)
-        // so that both halves release every stage.
-        const int a = warp - C::WARP_MMA;
-        const int nta = a ? ntiles_h[1] : ntiles_h[0];
+    } else if (warp == C::WARP_MMA) {
+        // -------------------------------------------------------------- MMA issuer
+        regs_dec<C::REGS_OTHER>();
         if (lane == 0) {
             constexpr uint32_t idesc_s = umma_idesc_f16(C::BM, C::BN, false, false);
             constexpr uint32_t idesc_o = umma_idesc_f16(C::BM, HEAD, false, true);
-            // Descriptors of the stage / half bases; k-steps add byte offsets / 16
-            // to the start-address field (addresses stay below 256 KB).
-            const uint64_t dq0 = umma_sdesc(smem_u32(sQ + a * C::Q_BYTES), 16, 8 * C::RB, C::LAYOUT);
-            const uint64_t dk0 = umma_sdesc(smem_u32(sK), 16, 8 * C::RB, C::LAYOUT);
-            const uint64_t dv0 = umma_sdesc(smem_u32(sV), C::BN * C::RB, 8 * C::RB, C::LAYOUT);
-            const uint32_t s_col = tmem + (uint32_t)(a * 128);
-            const uint32_t o_col = tmem + C::COL_O + (uint32_t)(a * 128);
-            bool alive = mbar_wait(q_full, 0);
-            auto issue_s = [&](int j) -> bool {
-                const int st = j % C::NK;
-                if (!mbar_wait(&k_full[st], (j / C::NK) & 1)) return false;
-                if (j < nta) {
-                    tc_fence_after();
+            // Descriptors of the bases; k-steps add byte offsets / 16 to the
+            // start-address field (addresses stay below 256 KB).
+            const uint64_t dq0 = umma_sdesc(smem_u32(sQ), 16, 8 * C::RB, C::LAYOUT);
+            const uint64_t dk0 = umma_sdesc(smem_u32(ring), 16, 8 * C::RB, C::LAYOUT);
+            const uint64_t dv0 = umma_sdesc(smem_u32(ring), C::BN * C::RB, 8 * C::RB, C::LAYOUT);
+            // S_a = Q_a K_j^T, K_j in ring stage sk.
+            auto issue_s = [&](int a, int sk) {
+                const uint32_t s_col = tmem + (uint32_t)(a * 128);
 #pragma unroll
-                    for (int kk = 0; kk < HEAD / 16; ++kk) {
-                        const int c = (kk * 16) / C::A, w = (kk * 16) % C::A;
-                        const uint64_t da = dq0 + (uint64_t)((c * C::BM * C::RB + w * 2) >> 4);
-                        const uint64_t db = dk0 + (uint64_t)((st * C::KV_BYTES + c * C::BN * C::RB + w * 2) >> 4);
-                        umma_f16(s_col + (uint32_t)((j & 1) * C::BN), da, db, idesc_s, kk > 0 ? 1u : 0u);
-                    }
-                    umma_commit(&s_full[a * 2 + (j & 1)]);
-                    umma_commit(&k_empty[st]);
-                } else {
-                    mbar_arrive(&k_empty[st]);
+                for (int kk = 0; kk < HEAD / 16; ++kk) {
+                    const int c = (kk * 16) / C::A, w = (kk * 16) % C::A;
+                    const uint64_t da = dq0 + (uint64_t)((a * C::Q_BYTES + c * C::BM * C::RB + w * 2) >> 4);
+                    const uint64_t db = dk0 + (uint64_t)((sk * C::KV_BYTES + c * C::BN * C::RB + w * 2) >> 4);
+                    umma_f16(s_col, da, db, idesc_s, kk > 0 ? 1u : 0u);
                 }
-                return true;
+                umma_commit(&s_full[a]);
             };
-            auto issue_pv = [&](int j) -> bool {
-                const int st = j % C::NV;
-                if (!mbar_wait(&v_full[st], (j / C::NV) & 1)) return false;
-                if (j < nta) {
-                    if (!mbar_wait(&p_full[a * 2 + (j & 1)], (j >> 1) & 1)) return false;
-                    tc_fence_after();
-                    const uint32_t p_tmem = s_col + (uint32_t)((j & 1) * C::BN);
+            // O_a += P_a V_j, V_j in ring stage sv, P_a over S_a's columns.
+            auto issue_pv = [&](int a, int sv, bool first) {
+                const uint32_t p_col = tmem + (uint32_t)(a * 128);
+                const uint32_t o_col = tmem + C::COL_O + (uint32_t)(a * 128);
 #pragma unroll
-                    for (int kk = 0; kk < C::BN / 16; ++kk) {
-                        const uint64_t db = dv0 + (uint64_t)((st * C::KV_BYTES + kk * 16 * C::RB) >> 4);
-                        umma_f16_ts(o_col, p_tmem + kk * 8, db, idesc_o, (j > 0 || kk > 0) ? 1u : 0u);
-                    }
-                    umma_commit(&pv_done[a]);
-                    if (j == nta - 1) umma_commit(&o_full[a]);
-                    umma_commit(&v_empty[st]);
-                } else {
-                    mbar_arrive(&v_empty[st]);
+                for (int kk = 0; kk < C::BN / 16; ++kk) {
+                    const uint64_t db = dv0 + (uint64_t)((sv * C::KV_BYTES + kk * 16 * C::RB) >> 4);
+                    umma_f16_ts(o_col, p_col + kk * 8, db, idesc_o, (!first || kk > 0) ? 1u : 0u);
                 }
-                return true;
             };
-            for (int j = 0; alive && j < ntiles; ++j) {
-                if (!issue_s(j)) { alive = false; break; }
-                if (j >= 1 && !issue_pv(j - 1)) { alive = false; break; }
+            const int nt0 = ntiles_h[0], nt1 = ntiles_h[1];
+            bool alive = mbar_wait(q_full, 0) && (ntiles == 0 || mbar_wait(&full[0], 0));
+            if (alive && ntiles > 0) {
+                tc_fence_after();
+                if (nt0 > 0) issue_s(0, 0);
+                if (nt1 > 0) issue_s(1, 0);
+                umma_commit(&empty[0]);                  // K_0 read by both S products
             }
-            if (alive && ntiles > 0) alive = issue_pv(ntiles - 1);
+            for (int j = 0; alive && j < ntiles; ++j) {
+                const int uv = 2 * j + 1, sv = uv % C::NS;
+                const int uk = 2 * j + 2, sk = uk % C::NS;      // K_{j+1}
+                const bool more = j + 1 < ntiles;
+                // Both ring items of this step first (loaded tiles ago, as a rule), so
+                // that the two products of a group issue back to back.
+                if (!mbar_wait(&full[sv], (uv / C::NS) & 1)) { alive = false; break; }
+                if (more && !mbar_wait(&full[sk], (uk / C::NS) & 1)) { alive = false; break; }
+                // Half 0 group: P_0,j V_j, then S_0,j+1.
+                if (j < nt0) {
+                    if (!mbar_wait(&p_full[0], j & 1)) { alive = false; break; }
+                    tc_fence_after();
+                    issue_pv(0, sv, j == 0);
+                    if (j == nt0 - 1) umma_commit(&o_full[0]);
+                }
+                if (more && j + 1 < nt0) {
+                    tc_fence_after();
+                    issue_s(0, sk);
+                }
+                // Half 1 group: P_1,j V_j, then S_1,j+1.
+                if (j < nt1) {
+                    if (!mbar_wait(&p_full[1], j & 1)) { alive = false; break; }
+                    tc_fence_after();
+                    issue_pv(1, sv, j == 0);
+                    if (j == nt1 - 1) umma_commit(&o_full[1]);
+                }
+                umma_commit(&empty[sv]);                 // V_j read by both P V products
+                if (more) {
+                    if (j + 1 < nt1) issue_s(1, sk);
+                    umma_commit(&empty[sk]);             // K_{j+1} read by both S products
+                }
+            }
             if (!alive) {
                 flag_status(p.status, PA_DEV_TIMEOUT);
                 atomicExch(&sh[3], 1);
                 // Let every MMA already issued finish before the CTA moves on.
-                umma_commit(&drain[a]);
-                mbar_wait(&drain[a], 0);
+                umma_commit(drain);
+                mbar_wait(drain, 0);
             }
         }
         __syncwarp();
     } else {
-        // ---------------------------------------------------------- softmax
+        // -------------------------------------------------------------- softmax
+        regs_inc<C::REGS_SOFTMAX>();
         const int a = warp >> 2;                         // half
         const int r = threadIdx.x & 127;                 // row == TMEM lane
         const uint32_t lane_base = (uint32_t)((warp & 3) * 32) << 16;
@@ -416,16 +489,16 @@ prefill_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
         const int lim = (r < my_rows) ? s.past + tok : T - 1;   // last visible key
         const int full_vis = s.past + ia;                // every row of the half sees keys <= this
         const int nt = a ? ntiles_h[1] : ntiles_h[0];
+        const uint32_t scol = tmem + lane_base + (uint32_t)(a * 128);
+        const uint32_t ocol = tmem + lane_base + C::COL_O + (uint32_t)(a * 128);
         float m_used = -INFINITY, l = 0.f;
         bool alive = true;
         for (int j = 0; j < nt; ++j) {
-            const int buf = a * 2 + (j & 1);
-            if (!mbar_wait_warp(&s_full[buf], (j >> 1) & 1)) { alive = false; break; }
+            if (!mbar_wait_warp(&s_full[a], j & 1)) { alive = false; break; }
             tc_fence_after();
             uint32_t sv[C::BN];
-            const uint32_t scol = tmem + lane_base + (uint32_t)(a * 128 + (j & 1) * C::BN);
-            tmem_ld32(scol, sv);
-            tmem_ld32(scol + 32, sv + 32);
+#pragma unroll
+            for (int c = 0; c < C::BN; c += 32) tmem_ld32(scol + c, sv + c);
             tmem_wait_ld();
             const int k0 = j * C::BN;
             if (k0 + C::BN - 1 > full_vis) {
@@ -433,25 +506,28 @@ prefill_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
                 for (int c = 0; c < C::BN; ++c)
                     sv[c] = (k0 + c) <= lim ? sv[c] : __float_as_uint(-INFINITY);
             }
-            // Row max as a tree (8 independent chains), not one 64-long chain.
+            // Row max: 8 independent chains of three-input maxima.
             float m8[8];
 #pragma unroll
-            for (int i = 0; i < 8; ++i) m8[i] = __uint_as_float(sv[i]);
+            for (int i = 0; i < 8; ++i) m8[i] = fmaxf(__uint_as_float(sv[i]), __uint_as_float(sv[8 + i]));
 #pragma unroll
-            for (int c = 8; c < C::BN; ++c) m8[c & 7] = fmaxf(m8[c & 7], __uint_as_float(sv[c]));
-            float mx = fmaxf(fmaxf(fmaxf(m8[0], m8[1]), fmaxf(m8[2], m8[3])),
-                             fmaxf(fmaxf(m8[4], m8[5]), fmaxf(m8[6], m8[7])));
-            mx *= p.scale_log2;
-            // Lazy rescale: move the exponent base only when the max grows by > 8.
-            if (mx > m_used + 8.f) {
-                const float alpha = (m_used == -INFINITY) ? 0.f : fast_exp2(m_used - mx);
+            for (int c = 16; c < C::BN; c += 16)
+#pragma unroll
+                for (int i = 0; i < 8; ++i)
+                    m8[i] = fmax3(m8[i], __uint_as_float(sv[c + i]), __uint_as_float(sv[c + 8 + i]));
+            const float mx = p.scale_log2 *
+                fmax3(fmax3(m8[0], m8[1], m8[2]), fmax3(m8[3], m8[4], m8[5]), fmaxf(m8[6], m8[7]));
+            // Lazy rescale: a row moves its exponent base only when its max grows
+            // by more than 8; the warp rescales O when any of its rows does.
+            const bool grow = mx > m_used + 8.f;
+            if (__any_sync(0xffffffffu, grow)) {
+                const float m_new = grow ? mx : m_used;
+                const float alpha = grow ? ((m_used == -INFINITY) ? 0.f : fast_exp2(m_used - m_new)) : 1.f;
                 l *= alpha;
+                m_used = m_new;
                 if (j > 0) {
-                    // S_a,j's commit covered P_a,j-2 V_j-2, so pv_done[a] is at phase
-                    // j - 1 or j here and this parity wait means "P_a,j-1 V_j-1 done".
-                    if (!mbar_wait_warp(&pv_done[a], (j - 1) & 1)) { alive = false; break; }
-                    tc_fence_after();
-                    const uint32_t ocol = tmem + lane_base + C::COL_O + a * 128;
+                    // s_full's commit for this tile also covered P_a V_{j-1}: O is
+                    // final up to tile j-1 and no MMA writes it until P_a is ready.
 #pragma unroll
                     for (int c0 = 0; c0 < HEAD; c0 += 16) {
                         uint32_t ov[16];
@@ -462,31 +538,35 @@ prefill_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
                         tmem_st16(ocol + c0, ov);
                     }
                 }
-                m_used = mx;
             }
             const float base = (m_used == -INFINITY) ? 0.f : m_used;
-            uint32_t pk[C::BN / 2];
             float rs[4] = {0.f, 0.f, 0.f, 0.f};   // independent partial sums
+            // P over S, 64 keys at a time: 64 f16 = 32 columns of this row's
+            // lane, over S columns already read into registers.
 #pragma unroll
-            for (int c = 0; c < C::BN; c += 2) {
-                const float p0 = fast_exp2(fmaf(__uint_as_float(sv[c]), p.scale_log2, -base));
-                const float p1 = fast_exp2(fmaf(__uint_as_float(sv[c + 1]), p.scale_log2, -base));
-                rs[(c >> 1) & 3] += p0 + p1;
-                pk[c / 2] = pack_half2(p0, p1);
+            for (int h = 0; h < C::BN; h += 64) {
+                uint32_t pk[32];
+#pragma unroll
+                for (int c = h; c < h + 64; c += 2) {
+                    const float x0 = fmaf(__uint_as_float(sv[c]), p.scale_log2, -base);
+                    const float x1 = fmaf(__uint_as_float(sv[c + 1]), p.scale_log2, -base);
+                    const float p0 = poly_col(c) ? exp2_poly(x0) : fast_exp2(x0);
+                    const float p1 = poly_col(c + 1) ? exp2_poly(x1) : fast_exp2(x1);
+                    rs[(c >> 1) & 3] += p0 + p1;
+                    pk[(c - h) / 2] = pack_half2(p0, p1);
+                }
+                tmem_st32(scol + h / 2, pk);
             }
             l += (rs[0] + rs[1]) + (rs[2] + rs[3]);
-            // P over S: 64 f16 = 32 columns of this row's lane.
-            tmem_st32(scol, pk);
             tmem_wait_st();
             tc_fence_before();
             __syncwarp();
-            if (lane == 0) mbar_arrive(&p_full[buf]);
+            if (lane == 0) mbar_arrive(&p_full[a]);
         }
         // Epilogue: O / l -> f16 rows of `out`.
         if (alive && nt > 0 && mbar_wait_warp(&o_full[a], 0)) {
             tc_fence_after();
             const float inv = (l > 0.f) ? 1.f / l : 0.f;
-            const uint32_t ocol = tmem + lane_base + C::COL_O + a * 128;
             __half* orow = p.out + ((long long)(s.q_start + tok) * p.q_heads + kvh * g + r % g) * HEAD;
 #pragma unroll
             for (int c0 = 0; c0 < HEAD; c0 += 16) {
@@ -520,10 +600,12 @@ prefill_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
     if (sh[3] && threadIdx.x == 0) {
         // Aborted (never expected): let in-flight loads land before exit.
         mbar_wait(q_full, 0);
-        for (int t = sh[4] - C::NK > 0 ? sh[4] - C::NK : 0; t < sh[4]; ++t)
-            mbar_wait(&k_full[t % C::NK], (t / C::NK) & 1);
-        for (int t = sh[5] - C::NV > 0 ? sh[5] - C::NV : 0; t < sh[5]; ++t)
-            mbar_wait(&v_full[t % C::NV], (t / C::NV) & 1);
+        const int issued = sh[4];
+        for (int u = issued - C::NS > 0 ? issued - C::NS : 0; u < issued; ++u) {
+            const bool tail = (u & 1) && ((u >> 1) * C::BN + C::BN > T);
+            if (tail) mbar_wait(v_tail, 0);
+            else mbar_wait(&full[u % C::NS], (u / C::NS) & 1);
+        }
     }
     __syncthreads();
     if (warp == C::WARP_MMA) {
@@ -537,7 +619,13 @@ cudaError_t launch_prefill_t(const CUtensorMap& tm_q, const CUtensorMap& tm_k,
                              const CUtensorMap& tm_v, const PrefillParams& p, cudaStream_t stream) {
     using C = PCfg<HEAD>;
     auto kern = prefill_kernel<HEAD>;
-    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM);
+    // The register split inside the kernel assumes this launch budget; with
+    // any other, setmaxnreg.inc could wait for registers that never come.
+    cudaFuncAttributes fa;
+    cudaError_t e = cudaFuncGetAttributes(&fa, kern);
+    if (e != cudaSuccess) return e;
+    if (fa.numRegs != kPrefillLaunchRegs) return cudaErrorInvalidKernelImage;
+    e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM);
     if (e != cudaSuccess) return e;
     const long long ctas = (long long)p.num_slots * p.kv_heads;
     kern<<<(unsigned)ctas, C::THREADS, C::SMEM, stream>>>(tm_q, tm_k, tm_v, p);
