@@ -287,6 +287,8 @@ pa_status pa_attention(const void* query, const void* key_cache, const void* val
         if ((st = make_cache_map(&tv, value_cache, d, rows)) != PA_OK) return st;
         pa::DecodeParams p{};
         p.query = static_cast<const __half*>(query);
+        p.key_cache = static_cast<const __half*>(key_cache);
+        p.value_cache = static_cast<const __half*>(value_cache);
         p.out = static_cast<__half*>(out);
         const size_t rows_total = (size_t)d.batch * d.kv_heads * plan.max_splits * (16 * plan.mtiles);
         p.part_o = static_cast<float*>(workspace);
@@ -339,6 +341,8 @@ pa_status pa_attention(const void* query, const void* key_cache, const void* val
             if ((st = make_cache_map(&tv, value_cache, d, rows)) != PA_OK) return st;
             pa::PrefillParams p{};
             p.out = static_cast<__half*>(out);
+            p.key_cache = static_cast<const __half*>(key_cache);
+            p.value_cache = static_cast<const __half*>(value_cache);
             p.block_table = block_table;
             p.cu_seqlens_q = cu_seqlens_q;
             p.seqlens_kv = seqlens_kv;

@@ -13,10 +13,15 @@
 // So the kernel is built around streaming pages:
 //   * one CTA per (split of the sequence's keys, KV head, sequence); the
 //     group * q_len query rows of that KV head share every page it loads;
-//   * a producer warp walks the block table and issues TMA tensor loads of
-//     32-key K and V tiles (one box per page and 64-element column block,
-//     128-byte swizzle) into a ring of 4 shared-memory stages (64 KB for head
-//     size 128) tracked by mbarriers, each stage owned by one consumer group;
+//   * producer warps walk the block table and fill a ring of 4 shared-memory
+//     stages (64 KB for head size 128) with 32-key K and V tiles, tracked by
+//     mbarriers, each stage owned by one consumer group.  Pages of 32 keys
+//     or more: one warp issues TMA tensor loads (one box per page and
+//     64-element column block, 128-byte swizzle).  Smaller pages: a TMA box
+//     per 16-row page is too little work per box -- the SM's TMA unit then
+//     caps the stream well below HBM bandwidth -- so two warps copy the rows
+//     16 bytes per thread (cp.async), each chunk placed where the 128-byte
+//     swizzle would put it;
 //   * consumer warps each own whole tiles (independent online softmax per
 //     warp, merged at the end), computing Q K^T and P V with mma.sync
 //     m16n8k16 (f16 in, f32 accumulate).  The tensor core is only a means to
@@ -37,7 +42,7 @@ namespace pa {
 
 namespace {
 
-template <int HEAD, int MT>
+template <int HEAD, int MT, bool CPA>
 struct Cfg {
     static constexpr int A = HEAD < 64 ? HEAD : 64;     // elements per swizzled row
     static constexpr int RB = A * 2;                    // bytes per swizzled row
@@ -52,7 +57,9 @@ struct Cfg {
     // pass at once and read a stage whose previous tile is still in use.)
     static constexpr int NST = 4;
     static_assert(NST % NG == 0, "each stage must belong to one consumer group");
-    static constexpr int THREADS = 32 * (NCW + 1);
+    static constexpr int NPW = CPA ? 2 : 1;             // producer warps
+    static constexpr int THREADS = 32 * (NCW + NPW);
+    static constexpr int CPR = HEAD * 2 / 16;           // 16-byte chunks per cache row
     static constexpr int TILE_BYTES = BN * HEAD * 2;    // one tensor, one stage
     static constexpr int STAGE_BYTES = 2 * TILE_BYTES;
     static constexpr int RMAX = 16 * MT;
@@ -67,11 +74,11 @@ __device__ __forceinline__ uint32_t half2_mask(uint32_t v, bool lo_ok, bool hi_o
     return (lo_ok ? (v & 0xffffu) : 0u) | (hi_ok ? (v & 0xffff0000u) : 0u);
 }
 
-template <int HEAD, int MT>
-__global__ void __launch_bounds__(Cfg<HEAD, MT>::THREADS, HEAD >= 128 ? 2 : 3)
+template <int HEAD, int MT, bool CPA>
+__global__ void __launch_bounds__(Cfg<HEAD, MT, CPA>::THREADS, HEAD >= 128 ? 2 : 3)
 decode_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_v,
               const DecodeParams p) {
-    using C = Cfg<HEAD, MT>;
+    using C = Cfg<HEAD, MT, CPA>;
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>(
         (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -143,7 +150,7 @@ decode_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ 
         sflag[1] = 0;
         sflag[2] = 0;
         for (int i = 0; i < C::NST; ++i) {
-            mbar_init(&full[i], 1);
+            mbar_init(&full[i], CPA ? C::NPW * 32 : 1);   // cp.async: one arrival per producer thread
             mbar_init(&empty[i], MT);
         }
         mbar_init(verdict, 1);
@@ -157,32 +164,85 @@ decode_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ 
     const int bs = p.block_size;
     const int32_t* bt = p.block_table + (long long)b * p.max_blocks;
 
-    if (warp == C::NCW) {
-        // ------------------------------------------------------------ producer
-        // The split's block ids, fetched once by the whole warp, so issuing a
-        // tile never waits on a dependent global load.
-        // They are range-checked here, and only here: the consumers wait for
-        // this verdict instead of re-reading the block table.
+    if (warp >= C::NCW) {
+        // ------------------------------------------------------------ producers
+        const int pw = warp - C::NCW;
+        // The split's block ids, fetched once by the first producer warp, so
+        // issuing a tile never waits on a dependent global load.  They are
+        // range-checked here, and only here: everyone else waits for this
+        // verdict instead of re-reading the block table.
         const int pg0 = k_begin / bs;
         const int n_ids = (k_end - 1) / bs + 1 - pg0;
         bool bad = false;
-        for (int i = lane; i < n_ids; i += 32) {
-            const int id = bt[pg0 + i];
-            bad |= (id < 0 || (long long)id >= p.num_blocks);
-            if (i < C::MAX_IDS) sids[i] = id;
-        }
-        bad = __any_sync(0xffffffffu, bad);
-        __syncwarp();
-        if (lane == 0) {
-            if (bad) flag_status(p.status, PA_DEV_BAD_BLOCK);
-            sflag[0] = bad ? 1 : 0;
-            mbar_arrive(verdict);
+        if (pw == 0) {
+            for (int i = lane; i < n_ids; i += 32) {
+                const int id = bt[pg0 + i];
+                bad |= (id < 0 || (long long)id >= p.num_blocks);
+                if (i < C::MAX_IDS) sids[i] = id;
+            }
+            bad = __any_sync(0xffffffffu, bad);
+            __syncwarp();
+            if (lane == 0) {
+                if (bad) flag_status(p.status, PA_DEV_BAD_BLOCK);
+                sflag[0] = bad ? 1 : 0;
+                mbar_arrive(verdict);
+            }
+        } else {
+            bad = !mbar_wait_warp(verdict, 0) || *(volatile int*)&sflag[0] != 0;
         }
         auto block_of = [&](int page) {
             const int i = page - pg0;
             return i < C::MAX_IDS ? sids[i] : bt[page];
         };
-        if (lane == 0 && !bad) {
+        if (CPA && !bad) {
+            // 16-key pages (the only size that takes this path): a 32-key tile
+            // is exactly pages k0/16 and k0/16 + 1.  Producer thread q copies
+            // the 16-byte chunk q % CPR of rows q / CPR + i * RPI (a fixed
+            // column per thread); rows at or past the split's end are not read
+            // (their block-table entries are not pages of this sequence).  Each
+            // thread arrives on the stage's mbarrier once its copies have landed.
+            constexpr int RPI = C::NPW * 32 / C::CPR;         // rows per pass of all producers
+            static_assert(C::BN * C::CPR % (C::NPW * 32) == 0, "chunks must split evenly");
+            const int q0 = pw * 32 + lane;
+            const int r0 = q0 / C::CPR, jc = q0 % C::CPR;
+            const int c = (jc * 8) / C::A, jj = jc % (C::A / 8);
+            const char* kc = reinterpret_cast<const char*>(p.key_cache);
+            const char* vc = reinterpret_cast<const char*>(p.value_cache);
+            const long long row_bytes = (long long)p.kv_heads * HEAD * 2;
+            const long long colb = (long long)kvh * HEAD * 2 + jc * 16;
+            for (int t = 0; t < ntiles; ++t) {
+                const int st = t % C::NST, u = t / C::NST;
+                bool go = true;
+                if (lane == 0 && u > 0) go = mbar_wait(&empty[st], (u - 1) & 1);
+                go = __shfl_sync(0xffffffffu, go, 0);
+                if (!go) {
+                    if (lane == 0) {
+                        flag_status(p.status, PA_DEV_TIMEOUT);
+                        atomicExch(&sflag[1], 1);
+                    }
+                    break;
+                }
+                if (__shfl_sync(0xffffffffu, *(volatile int*)&sflag[1], 0)) break;
+                const uint32_t kdst = smem_u32(stages + st * C::STAGE_BYTES);
+                const uint32_t vdst = kdst + C::TILE_BYTES;
+                const int k0 = k_begin + t * C::BN;
+                const int blk0 = block_of(k0 >> 4);
+                const int blk1 = (k0 + 16 < k_end) ? block_of((k0 >> 4) + 1) : 0;
+#pragma unroll
+                for (int i = 0; i < C::BN / RPI; ++i) {
+                    const int r = r0 + i * RPI;
+                    if (k0 + r < k_end) {
+                        const int blk = (r >> 4) ? blk1 : blk0;
+                        const long long goff = (long long)(blk * 16 + (r & 15)) * row_bytes + colb;
+                        const uint32_t soff = swz<C::RB>((uint32_t)((c * C::BN + r) * C::RB + jj * 16));
+                        cp_async16(kdst + soff, kc + goff);
+                        cp_async16(vdst + soff, vc + goff);
+                    }
+                }
+                cp_async_arrive(&full[st]);
+            }
+            cp_async_wait_all();
+        } else if (!CPA && pw == 0 && lane == 0 && !bad) {
             tma_prefetch_desc(&tm_k);
             tma_prefetch_desc(&tm_v);
             const uint64_t pol = policy_evict_first();
@@ -198,28 +258,14 @@ decode_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ 
                 uint8_t* kdst = stages + st * C::STAGE_BYTES;
                 uint8_t* vdst = kdst + C::TILE_BYTES;
                 const int k0 = k_begin + t * C::BN;
-                if (bs >= C::BN) {
-                    const int blk = block_of(k0 / bs);
-                    const int row = k0 % bs;
-                    mbar_arrive_expect_tx(&full[st], 2 * C::TILE_BYTES);
+                // Pages of at least BN keys (smaller ones take the cp.async path).
+                const int blk = block_of(k0 / bs);
+                const int row = k0 % bs;
+                mbar_arrive_expect_tx(&full[st], 2 * C::TILE_BYTES);
 #pragma unroll
-                    for (int c = 0; c < C::NA; ++c) {
-                        tma_load_4d_hint(kdst + c * C::BN * C::RB, &tm_k, &full[st], c * C::A, kvh, row, blk, pol);
-                        tma_load_4d_hint(vdst + c * C::BN * C::RB, &tm_v, &full[st], c * C::A, kvh, row, blk, pol);
-                    }
-                } else {
-                    // block_size 16: two pages per 32-key tile; skip a page past the end.
-                    const int npg = (k0 + bs < T) ? 2 : 1;
-                    mbar_arrive_expect_tx(&full[st], (uint32_t)(npg * bs * HEAD * 2 * 2));
-                    for (int pi = 0; pi < npg; ++pi) {
-                        const int blk = block_of(k0 / bs + pi);
-#pragma unroll
-                        for (int c = 0; c < C::NA; ++c) {
-                            const int off = (c * C::BN + pi * bs) * C::RB;
-                            tma_load_4d_hint(kdst + off, &tm_k, &full[st], c * C::A, kvh, 0, blk, pol);
-                            tma_load_4d_hint(vdst + off, &tm_v, &full[st], c * C::A, kvh, 0, blk, pol);
-                        }
-                    }
+                for (int c = 0; c < C::NA; ++c) {
+                    tma_load_4d_hint(kdst + c * C::BN * C::RB, &tm_k, &full[st], c * C::A, kvh, row, blk, pol);
+                    tma_load_4d_hint(vdst + c * C::BN * C::RB, &tm_v, &full[st], c * C::A, kvh, row, blk, pol);
                 }
             }
         }
@@ -509,11 +555,11 @@ __global__ void __launch_bounds__(128) combine_kernel(const DecodeParams p) {
     *reinterpret_cast<uint2*>(orow + lane * 4) = wv;
 }
 
-template <int HEAD, int MT>
+template <int HEAD, int MT, bool CPA>
 cudaError_t launch_decode_t(const CUtensorMap& tm_k, const CUtensorMap& tm_v,
                             const DecodeParams& p, cudaStream_t stream) {
-    using C = Cfg<HEAD, MT>;
-    auto kern = decode_kernel<HEAD, MT>;
+    using C = Cfg<HEAD, MT, CPA>;
+    auto kern = decode_kernel<HEAD, MT, CPA>;
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM);
     if (e != cudaSuccess) return e;
     e = cudaFuncSetAttribute(kern, cudaFuncAttributePreferredSharedMemoryCarveout,
@@ -559,10 +605,14 @@ DecodePlan plan_decode(const pa_dims& d, int num_sms) {
 
 cudaError_t launch_decode(const CUtensorMap& tm_k, const CUtensorMap& tm_v,
                           const DecodeParams& p, int head_size, int mtiles, cudaStream_t stream) {
-#define PA_DECODE_CASE(H)                                                          \
-    case H:                                                                        \
-        return mtiles == 1 ? launch_decode_t<H, 1>(tm_k, tm_v, p, stream)          \
-                           : launch_decode_t<H, 2>(tm_k, tm_v, p, stream);
+    const bool cpa = p.block_size < kDecodeKeys;
+#define PA_DECODE_CASE(H)                                                                      \
+    case H:                                                                                    \
+        if (cpa)                                                                               \
+            return mtiles == 1 ? launch_decode_t<H, 1, true>(tm_k, tm_v, p, stream)            \
+                               : launch_decode_t<H, 2, true>(tm_k, tm_v, p, stream);           \
+        return mtiles == 1 ? launch_decode_t<H, 1, false>(tm_k, tm_v, p, stream)               \
+                           : launch_decode_t<H, 2, false>(tm_k, tm_v, p, stream);
     switch (head_size) {
         PA_DECODE_CASE(16)
         PA_DECODE_CASE(32)

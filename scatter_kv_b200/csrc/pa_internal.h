@@ -13,6 +13,8 @@ namespace pa {
 // Everything the decode (split-KV) kernels need besides the tensor maps.
 struct DecodeParams {
     const __half* query;
+    const __half* key_cache;      // [num_blocks, block_size, kv_heads, head_size]
+    const __half* value_cache;
     __half* out;
     float* part_o;                // [batch, kv_heads, max_splits, rmax, head_size]
     float* part_lse;              // [batch, kv_heads, max_splits, rmax] (log2 domain)
@@ -40,6 +42,8 @@ struct DecodeParams {
 
 struct PrefillParams {
     __half* out;
+    const __half* key_cache;      // [num_blocks, block_size, kv_heads, head_size]
+    const __half* value_cache;
     const int32_t* block_table;
     const int32_t* cu_seqlens_q;
     const int32_t* seqlens_kv;

@@ -19,10 +19,13 @@
 // Warp roles (384 threads, three warpgroups):
 //   warps 0-3   softmax + epilogue of half 0 (thread r = row r = TMEM lane r)
 //   warps 4-7   softmax + epilogue of half 1
-//   warps 8, 10, 11  TMA producers (Q of both halves, then the K/V ring;
-//               each ring item's boxes are dealt out over the three warps,
-//               since one issuing warp gets through only a few boxes per
-//               microsecond and small pages make many boxes)
+//   warps 8, 10, 11  producers: Q of both halves by TMA, then the K/V ring.
+//               Pages of 128 keys or more: TMA boxes, dealt out over the
+//               three warps.  Smaller pages: 16-byte cp.async copies by all
+//               96 producer threads, each chunk placed where the 128-byte
+//               swizzle would put it -- a TMA box per small page is too
+//               little work per box, and the SM's TMA unit then caps the
+//               stream far below what the tensor cores consume.
 //   warp 9      TMEM allocator; one thread issues every tcgen05.mma
 // The third warpgroup hands registers to the softmax warpgroups
 // (setmaxnreg): a softmax thread holds its whole 128-key row of S.
@@ -64,7 +67,7 @@ namespace pa {
 
 namespace {
 
-template <int HEAD>
+template <int HEAD, bool CPA>
 struct PCfg {
     static constexpr int BM = kPrefillRows;             // 128 query rows per half
     static constexpr int BN = kPrefillKeys;             // 128 keys per tile
@@ -89,6 +92,8 @@ struct PCfg {
     static constexpr int THREADS = 384;
     static constexpr int WARP_MMA = 9;            // producers: warps 8, 10, 11
     static constexpr int NPROD = 3;
+    static constexpr int CPR = HEAD * 2 / 16;           // 16-byte chunks per cache row
+    static constexpr int RPI = NPROD * 32 / CPR;        // rows per pass of all producer threads
     // Register split: launched with kLaunchRegs per thread; the softmax
     // warpgroups raise theirs to REGS_SOFTMAX, the third lowers to REGS_OTHER.
     // The shares must add up to exactly the launch's registers.
@@ -186,11 +191,11 @@ __device__ __forceinline__ bool poly_col(int c) {
 }
 
 
-template <int HEAD>
-__global__ void __launch_bounds__(PCfg<HEAD>::THREADS, 1)
+template <int HEAD, bool CPA>
+__global__ void __launch_bounds__(PCfg<HEAD, CPA>::THREADS, 1)
 prefill_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                const __grid_constant__ CUtensorMap tm_v, const PrefillParams p) {
-    using C = PCfg<HEAD>;
+    using C = PCfg<HEAD, CPA>;
     extern __shared__ __align__(1024) uint8_t smem[];
     uint64_t* bars = reinterpret_cast<uint64_t*>(smem + C::OFF_BAR);
     uint64_t* q_full = bars;
@@ -253,7 +258,7 @@ prefill_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
         sh[4] = 0;
         mbar_init(q_full, 1);
         for (int i = 0; i < C::NS; ++i) {
-            mbar_init(&full[i], C::NPROD);           // one arrival per producer warp
+            mbar_init(&full[i], CPA ? C::NPROD * 32 : C::NPROD);   // per producer thread / warp
             mbar_init(&empty[i], 1);
         }
         for (int i = 0; i < 2; ++i) {
@@ -334,14 +339,29 @@ prefill_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
             }
             return __shfl_sync(0xffffffffu, win_id, page - win_base);
         };
+        // cp.async path: producer thread q = pw * 32 + lane copies chunk q % CPR
+        // of rows q / CPR + i * RPI (a fixed column per thread).
+        const int qt = pw * 32 + lane;
+        const int r0 = qt / C::CPR, jc = qt % C::CPR;
+        const int cb = (jc * 8) / C::A, jj = jc % (C::A / 8);
+        const int lbs = 31 - __clz(bs);
+        const long long row_bytes = (long long)p.kv_heads * HEAD * 2;
+        const long long colb = (long long)kvh * HEAD * 2 + jc * 16;
+        int tile_ids = 0;
+        int next_ids = 0;
+        if (CPA) {
+            const int np0 = (min(C::BN, T) + bs - 1) / bs;
+            next_ids = lane < np0 ? bt[lane] : 0;          // becomes tile 0's ids at u = 0
+        }
         for (int u = 0; u < 2 * ntiles; ++u) {
             const int st = u % C::NS;
             const int j = u >> 1;
             const bool is_v = (u & 1) != 0;
             const int k0 = j * C::BN;
-            // The last V tile (rows past T to be zeroed) is producer 0's alone.
+            // The last V tile (rows past T to be zeroed) is producer 0's alone
+            // on the TMA path.
             const bool tail = is_v && (k0 + C::BN > T);
-            if (tail && pw != 0) continue;
+            if (!CPA && tail && pw != 0) continue;
             bool go = true;
             if (lane == 0 && u >= C::NS) go = mbar_wait(&empty[st], ((u / C::NS) - 1) & 1);
             go = __shfl_sync(0xffffffffu, go, 0);
@@ -355,6 +375,44 @@ prefill_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
             if (__shfl_sync(0xffffffffu, *(volatile int*)&sh[3], 0)) break;
             uint8_t* dst = ring + st * C::KV_BYTES;
             const int npg = bs < C::BN ? (min(k0 + C::BN, T) - k0 + bs - 1) / bs : 1;
+            if (CPA) {
+                // Block ids of this tile's pages: lane l holds page k0 / bs + l
+                // (K and V share them; loaded one tile ahead).
+                if (!is_v) {
+                    tile_ids = next_ids;
+                    const int kn = k0 + C::BN;
+                    const int npn = kn < T ? (min(kn + C::BN, T) - kn + bs - 1) / bs : 0;
+                    next_ids = lane < npn ? bt[(kn >> lbs) + lane] : 0;
+                }
+                const char* cache = reinterpret_cast<const char*>(is_v ? p.value_cache : p.key_cache);
+                const uint32_t sdst = smem_u32(dst);
+#pragma unroll 2
+                for (int i = 0; i < (C::BN + C::RPI - 1) / C::RPI; ++i) {
+                    const int r = r0 + i * C::RPI;
+                    const int key = k0 + r;
+                    const int blk = __shfl_sync(0xffffffffu, tile_ids, r < C::BN ? (r >> lbs) : 0);
+                    if (r < C::BN) {
+                        const uint32_t soff = swz<C::RB>((uint32_t)((cb * C::BN + r) * C::RB + jj * 16));
+                        if (key < T) {
+                            const long long row = ((long long)blk << lbs) + (key & (bs - 1));
+                            cp_async16(sdst + soff, cache + row * row_bytes + colb);
+                        } else if (is_v) {
+                            // V rows past the end: zero, so 0 * garbage never meets P V.
+                            *reinterpret_cast<uint4*>(dst + soff) = make_uint4(0, 0, 0, 0);
+                        }
+                    }
+                }
+                if (tail) {
+                    // Zero stores are generic-proxy writes: land the copies, make
+                    // both visible to the tensor core, then arrive.
+                    cp_async_wait_all();
+                    fence_proxy_async_smem();
+                    mbar_arrive(&full[st]);
+                } else {
+                    cp_async_arrive(&full[st]);
+                }
+                continue;
+            }
             const int nbox = npg * C::NA;
             const int mine = tail ? nbox : (nbox - pw + C::NPROD - 1) / C::NPROD;
             uint64_t* bar = tail ? v_tail : &full[st];
@@ -395,6 +453,7 @@ prefill_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
                 if (lane == 0) mbar_arrive_cnt(&full[st], C::NPROD);
             }
         }
+        if (CPA) cp_async_wait_all();
     } else if (warp == C::WARP_MMA) {
         // -------------------------------------------------------------- MMA issuer
         regs_dec<C::REGS_OTHER>();
@@ -614,11 +673,11 @@ prefill_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
     }
 }
 
-template <int HEAD>
+template <int HEAD, bool CPA>
 cudaError_t launch_prefill_t(const CUtensorMap& tm_q, const CUtensorMap& tm_k,
                              const CUtensorMap& tm_v, const PrefillParams& p, cudaStream_t stream) {
-    using C = PCfg<HEAD>;
-    auto kern = prefill_kernel<HEAD>;
+    using C = PCfg<HEAD, CPA>;
+    auto kern = prefill_kernel<HEAD, CPA>;
     // The register split inside the kernel assumes this launch budget; with
     // any other, setmaxnreg.inc could wait for registers that never come.
     cudaFuncAttributes fa;
@@ -637,13 +696,19 @@ cudaError_t launch_prefill_t(const CUtensorMap& tm_q, const CUtensorMap& tm_k,
 cudaError_t launch_prefill(const CUtensorMap& tm_q, const CUtensorMap& tm_k,
                            const CUtensorMap& tm_v, const PrefillParams& p, int head_size,
                            cudaStream_t stream) {
+    const bool cpa = p.block_size < kPrefillKeys;
+#define PA_PREFILL_CASE(H)                                                               \
+    case H:                                                                              \
+        return cpa ? launch_prefill_t<H, true>(tm_q, tm_k, tm_v, p, stream)              \
+                   : launch_prefill_t<H, false>(tm_q, tm_k, tm_v, p, stream);
     switch (head_size) {
-        case 16: return launch_prefill_t<16>(tm_q, tm_k, tm_v, p, stream);
-        case 32: return launch_prefill_t<32>(tm_q, tm_k, tm_v, p, stream);
-        case 64: return launch_prefill_t<64>(tm_q, tm_k, tm_v, p, stream);
-        case 128: return launch_prefill_t<128>(tm_q, tm_k, tm_v, p, stream);
+        PA_PREFILL_CASE(16)
+        PA_PREFILL_CASE(32)
+        PA_PREFILL_CASE(64)
+        PA_PREFILL_CASE(128)
         default: return cudaErrorInvalidValue;
     }
+#undef PA_PREFILL_CASE
 }
 
 }  // namespace pa
