@@ -515,6 +515,11 @@ __global__ void __launch_bounds__(128) combine_kernel(const DecodeParams p) {
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int r = blockIdx.x * 4 + warp;
     const int g = p.group;
+    const long long base = ((long long)b * p.kv_heads + kvh) * p.max_splits * p.rmax + r;
+    const float* lse = p.part_lse + base;             // stride rmax per split
+    // Lane sp's split lse, fetched together with the metadata (it does not
+    // depend on it; splits past the sequence's count are ignored below).
+    const float lse_l = lane < p.max_splits ? lse[(long long)lane * p.rmax] : -INFINITY;
     SeqInfo s;
     // Invalid metadata: the decode kernel has zeroed the rows already.
     if (!load_seq(p.cu_seqlens_q, p.seqlens_kv, b, p.batch, p.token_count, p.kv_cap, p.kv_hint,
@@ -524,10 +529,9 @@ __global__ void __launch_bounds__(128) combine_kernel(const DecodeParams p) {
     const int n_splits = (s.kv_len + p.chunk - 1) / p.chunk;
     if (n_splits == 1) return;                        // the decode kernel wrote the row
     __half* orow = p.out + ((long long)(s.q_start + r / g) * p.q_heads + kvh * g + r % g) * HEAD;
-    const long long base = ((long long)b * p.kv_heads + kvh) * p.max_splits * p.rmax + r;
-    const float* lse = p.part_lse + base;             // stride rmax per split
     float M = -INFINITY;
-    for (int sp = lane; sp < n_splits; sp += 32) M = fmaxf(M, lse[(long long)sp * p.rmax]);
+    for (int sp = lane; sp < n_splits; sp += 32)
+        M = fmaxf(M, sp < 32 ? lse_l : lse[(long long)sp * p.rmax]);
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, o));
     if (M == INFINITY) {
@@ -535,19 +539,26 @@ __global__ void __launch_bounds__(128) combine_kernel(const DecodeParams p) {
         for (int d = lane; d < HEAD; d += 32) orow[d] = __float2half_rn(0.f);
         return;
     }
-    float L = 0.f;
-    for (int sp = lane; sp < n_splits; sp += 32) L += fast_exp2(lse[(long long)sp * p.rmax] - M);
+    // Split weights 2^(lse_s - M), lane sp holding split sp's (splits beyond 32
+    // read theirs directly).
+    const float w_l = (lane < n_splits) ? fast_exp2(lse_l - M) : 0.f;
+    float L = w_l;
+    for (int sp = lane + 32; sp < n_splits; sp += 32) L += fast_exp2(lse[(long long)sp * p.rmax] - M);
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) L += __shfl_xor_sync(0xffffffffu, L, o);
-    if (lane * 4 >= HEAD) return;
     const float* po = p.part_o + base * HEAD + lane * 4;
     float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+    const bool active = lane * 4 < HEAD;
 #pragma unroll 4
     for (int sp = 0; sp < n_splits; ++sp) {
-        const float w = fast_exp2(lse[(long long)sp * p.rmax] - M);
-        const float4 v = *reinterpret_cast<const float4*>(po + (long long)sp * p.rmax * HEAD);
-        acc.x += w * v.x; acc.y += w * v.y; acc.z += w * v.z; acc.w += w * v.w;
+        const float w = sp < 32 ? __shfl_sync(0xffffffffu, w_l, sp)
+                                : fast_exp2(lse[(long long)sp * p.rmax] - M);
+        if (active) {
+            const float4 v = *reinterpret_cast<const float4*>(po + (long long)sp * p.rmax * HEAD);
+            acc.x += w * v.x; acc.y += w * v.y; acc.z += w * v.z; acc.w += w * v.w;
+        }
     }
+    if (!active) return;
     const float il = 1.f / L;
     uint2 wv;
     wv.x = pack_half2(acc.x * il, acc.y * il);

@@ -13,7 +13,9 @@
 // Slot mapping (same PR, review "Things I specifically checked": the token
 // -> sequence lookup is the first b with cu_seqlens_q[b+1] > t, skipping
 // zero-length sequences; past_len_b = seqlens_kv[b] - q_len_b).  One thread
-// per token, binary search over cu_seqlens_q.
+// per token, binary search over cu_seqlens_q, which each block first stages
+// in shared memory with one coalesced load (the search would otherwise be a
+// chain of dependent global loads).
 #include <cuda_runtime.h>
 
 #include "pa_common.cuh"
@@ -51,14 +53,16 @@ scatter_kv_kernel(const uint4* __restrict__ key, const uint4* __restrict__ value
             long long i = base + (long long)u * kScatterThreads;
             dst[u] = -1;
             if (i < total) {
+                // The K/V loads do not depend on the slot: issue them first, so
+                // that their latency and the slot's overlap.
+                kv[u] = ld_stream(key + i);
+                vv[u] = ld_stream(value + i);
                 long long t = i / vec_per_token;
                 int c = (int)(i - t * vec_per_token);
                 int slot = __ldg(slot_mapping + t);
                 if (slot >= 0) {
                     if ((long long)slot < num_slots) {
                         dst[u] = (long long)slot * vec_per_token + c;
-                        kv[u] = ld_stream(key + i);
-                        vv[u] = ld_stream(value + i);
                     } else if (c == 0) {
                         flag_status(status, PA_DEV_BAD_SLOT);
                     }
@@ -75,19 +79,26 @@ scatter_kv_kernel(const uint4* __restrict__ key, const uint4* __restrict__ value
     }
 }
 
-__global__ void slot_mapping_kernel(const int32_t* __restrict__ block_table,
-                                    const int32_t* __restrict__ cu,
-                                    const int32_t* __restrict__ seqlens_kv,
-                                    int32_t* __restrict__ slot_mapping, int batch,
-                                    long long token_count, int max_blocks, int block_size,
-                                    long long num_blocks, int32_t* status) {
+constexpr int kSlotThreads = 256;
+constexpr int kSlotMaxStaged = 8192;     // cu_seqlens_q entries staged in shared memory
+
+__global__ void __launch_bounds__(kSlotThreads)
+slot_mapping_kernel(const int32_t* __restrict__ block_table, const int32_t* __restrict__ cu,
+                    const int32_t* __restrict__ seqlens_kv, int32_t* __restrict__ slot_mapping,
+                    int batch, long long token_count, int max_blocks, int block_size,
+                    long long num_blocks, int32_t* status) {
+    extern __shared__ int32_t s_cu[];    // cu_seqlens_q[1 .. batch] (when batch <= kSlotMaxStaged)
+    const bool staged = batch <= kSlotMaxStaged;
+    if (staged)
+        for (int i = threadIdx.x; i < batch; i += kSlotThreads) s_cu[i] = cu[i + 1];
+    __syncthreads();
     long long t = (long long)blockIdx.x * blockDim.x + threadIdx.x;
     if (t >= token_count) return;
     // First b with cu[b+1] > t.
     int lo = 0, hi = batch;          // answer in [lo, hi)
     while (lo < hi) {
         int mid = (lo + hi) >> 1;
-        if ((long long)cu[mid + 1] > t) hi = mid; else lo = mid + 1;
+        if ((long long)(staged ? s_cu[mid] : cu[mid + 1]) > t) hi = mid; else lo = mid + 1;
     }
     int32_t slot = -1;
     if (lo < batch) {
@@ -130,9 +141,10 @@ cudaError_t launch_scatter(const void* key, const void* value, const int32_t* sl
 cudaError_t launch_slot_mapping(const int32_t* block_table, const int32_t* cu,
                                 const int32_t* seqlens_kv, int32_t* slot_mapping,
                                 const pa_dims& d, int32_t* status, cudaStream_t stream) {
-    const int threads = 256;
+    const int threads = kSlotThreads;
     long long blocks = (d.token_count + threads - 1) / threads;
-    slot_mapping_kernel<<<(unsigned)blocks, threads, 0, stream>>>(
+    const size_t smem = d.batch <= kSlotMaxStaged ? (size_t)d.batch * 4 : 0;
+    slot_mapping_kernel<<<(unsigned)blocks, threads, smem, stream>>>(
         block_table, cu, seqlens_kv, slot_mapping, d.batch, d.token_count, d.max_blocks_per_seq,
         d.block_size, d.num_blocks, status);
     return cudaGetLastError();
