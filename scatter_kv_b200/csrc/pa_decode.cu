@@ -21,7 +21,10 @@
 //     per 16-row page is too little work per box -- the SM's TMA unit then
 //     caps the stream well below HBM bandwidth -- so two warps copy the rows
 //     16 bytes per thread (cp.async), each chunk placed where the 128-byte
-//     swizzle would put it;
+//     swizzle would put it.  That path runs three CTAs per SM (the producer
+//     warpgroup hands its registers to the consumers through setmaxnreg), so
+//     that the SM keeps enough bytes in flight while one of its CTAs is in
+//     its start-up or final merge;
 //   * consumer warps each own whole tiles (independent online softmax per
 //     warp, merged at the end), computing Q K^T and P V with mma.sync
 //     m16n8k16 (f16 in, f32 accumulate).  The tensor core is only a means to
@@ -42,6 +45,17 @@ namespace pa {
 
 namespace {
 
+// cp.async path: three 256-thread CTAs per SM are launched with
+// kDecodeLaunchRegs registers per thread; the consumer warpgroup raises its
+// share to kDecRegsCons, the producer warpgroup lowers its to kDecRegsProd.
+// The shares add up to exactly the launch's registers (the host checks the
+// built kernel's count before launching: with fewer, setmaxnreg.inc could
+// wait for registers that never come).
+constexpr int kDecodeLaunchRegs = 80;
+constexpr int kDecRegsCons = 136, kDecRegsProd = 24;
+static_assert(128 * (kDecRegsCons + kDecRegsProd) == 256 * kDecodeLaunchRegs,
+              "register split must equal the launch budget");
+
 template <int HEAD, int MT, bool CPA>
 struct Cfg {
     static constexpr int A = HEAD < 64 ? HEAD : 64;     // elements per swizzled row
@@ -57,7 +71,7 @@ struct Cfg {
     // pass at once and read a stage whose previous tile is still in use.)
     static constexpr int NST = 4;
     static_assert(NST % NG == 0, "each stage must belong to one consumer group");
-    static constexpr int NPW = CPA ? 2 : 1;             // producer warps
+    static constexpr int NPW = CPA ? 4 : 1;             // producer warps (cp.async: a warpgroup)
     static constexpr int THREADS = 32 * (NCW + NPW);
     static constexpr int CPR = HEAD * 2 / 16;           // 16-byte chunks per cache row
     static constexpr int TILE_BYTES = BN * HEAD * 2;    // one tensor, one stage
@@ -75,7 +89,7 @@ __device__ __forceinline__ uint32_t half2_mask(uint32_t v, bool lo_ok, bool hi_o
 }
 
 template <int HEAD, int MT, bool CPA>
-__global__ void __launch_bounds__(Cfg<HEAD, MT, CPA>::THREADS, HEAD >= 128 ? 2 : 3)
+__global__ void __launch_bounds__(Cfg<HEAD, MT, CPA>::THREADS, (HEAD >= 128 && !CPA) ? 2 : 3)
 decode_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_v,
               const DecodeParams p) {
     using C = Cfg<HEAD, MT, CPA>;
@@ -166,6 +180,7 @@ decode_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ 
 
     if (warp >= C::NCW) {
         // ------------------------------------------------------------ producers
+        if (CPA) asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(kDecRegsProd));
         const int pw = warp - C::NCW;
         // The split's block ids, fetched once by the first producer warp, so
         // issuing a tile never waits on a dependent global load.  They are
@@ -202,7 +217,7 @@ decode_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ 
             // (their block-table entries are not pages of this sequence).  Each
             // thread arrives on the stage's mbarrier once its copies have landed.
             constexpr int RPI = C::NPW * 32 / C::CPR;         // rows per pass of all producers
-            static_assert(C::BN * C::CPR % (C::NPW * 32) == 0, "chunks must split evenly");
+            static_assert((C::NPW * 32) % C::CPR == 0, "a fixed column per producer thread");
             const int q0 = pw * 32 + lane;
             const int r0 = q0 / C::CPR, jc = q0 % C::CPR;
             const int c = (jc * 8) / C::A, jj = jc % (C::A / 8);
@@ -229,9 +244,9 @@ decode_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ 
                 const int blk0 = block_of(k0 >> 4);
                 const int blk1 = (k0 + 16 < k_end) ? block_of((k0 >> 4) + 1) : 0;
 #pragma unroll
-                for (int i = 0; i < C::BN / RPI; ++i) {
+                for (int i = 0; i < (C::BN + RPI - 1) / RPI; ++i) {
                     const int r = r0 + i * RPI;
-                    if (k0 + r < k_end) {
+                    if (r < C::BN && k0 + r < k_end) {
                         const int blk = (r >> 4) ? blk1 : blk0;
                         const long long goff = (long long)(blk * 16 + (r & 15)) * row_bytes + colb;
                         const uint32_t soff = swz<C::RB>((uint32_t)((c * C::BN + r) * C::RB + jj * 16));
@@ -271,6 +286,7 @@ decode_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ 
         }
     } else {
         // ------------------------------------------------------------ consumers
+        if (CPA) asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(kDecRegsCons));
         const int mt = warp % MT;          // which 16 query rows
         const int grp = warp / MT;         // which tiles
         const int quad = lane >> 2, qid = lane & 3;
@@ -571,7 +587,14 @@ cudaError_t launch_decode_t(const CUtensorMap& tm_k, const CUtensorMap& tm_v,
                             const DecodeParams& p, cudaStream_t stream) {
     using C = Cfg<HEAD, MT, CPA>;
     auto kern = decode_kernel<HEAD, MT, CPA>;
-    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM);
+    cudaError_t e;
+    if (CPA) {
+        cudaFuncAttributes fa;
+        e = cudaFuncGetAttributes(&fa, kern);
+        if (e != cudaSuccess) return e;
+        if (fa.numRegs != kDecodeLaunchRegs) return cudaErrorInvalidKernelImage;
+    }
+    e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM);
     if (e != cudaSuccess) return e;
     e = cudaFuncSetAttribute(kern, cudaFuncAttributePreferredSharedMemoryCarveout,
                              cudaSharedmemCarveoutMaxShared);
