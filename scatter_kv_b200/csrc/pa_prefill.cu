@@ -599,7 +599,11 @@ prefill_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
                 }
             }
             const float base = (m_used == -INFINITY) ? 0.f : m_used;
-            float rs[4] = {0.f, 0.f, 0.f, 0.f};   // independent partial sums
+            // Column pairs run on the packed f32x2 pipe: x = s * scale - base and
+            // the row sums (two independent pair accumulators).
+            const uint64_t scale2 = f2_pack(p.scale_log2, p.scale_log2);
+            const uint64_t nbase2 = f2_pack(-base, -base);
+            uint64_t rs2[2] = {f2_pack(0.f, 0.f), f2_pack(0.f, 0.f)};
             // P over S, 64 keys at a time: 64 f16 = 32 columns of this row's
             // lane, over S columns already read into registers.
 #pragma unroll
@@ -607,16 +611,23 @@ prefill_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
                 uint32_t pk[32];
 #pragma unroll
                 for (int c = h; c < h + 64; c += 2) {
-                    const float x0 = fmaf(__uint_as_float(sv[c]), p.scale_log2, -base);
-                    const float x1 = fmaf(__uint_as_float(sv[c + 1]), p.scale_log2, -base);
+                    const uint64_t x2 = f2_fma(f2_pack(__uint_as_float(sv[c]), __uint_as_float(sv[c + 1])),
+                                               scale2, nbase2);
+                    float x0, x1;
+                    f2_unpack(x2, x0, x1);
                     const float p0 = poly_col(c) ? exp2_poly(x0) : fast_exp2(x0);
                     const float p1 = poly_col(c + 1) ? exp2_poly(x1) : fast_exp2(x1);
-                    rs[(c >> 1) & 3] += p0 + p1;
+                    rs2[(c >> 1) & 1] = f2_add(rs2[(c >> 1) & 1], f2_pack(p0, p1));
                     pk[(c - h) / 2] = pack_half2(p0, p1);
                 }
                 tmem_st32(scol + h / 2, pk);
             }
-            l += (rs[0] + rs[1]) + (rs[2] + rs[3]);
+            {
+                float a0, a1, b0, b1;
+                f2_unpack(rs2[0], a0, a1);
+                f2_unpack(rs2[1], b0, b1);
+                l += (a0 + a1) + (b0 + b1);
+            }
             tmem_wait_st();
             tc_fence_before();
             __syncwarp();
