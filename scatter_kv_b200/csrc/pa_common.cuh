@@ -90,12 +90,30 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity) {
     }
 }
 
+// The same wait with its polls in a rolled loop: a few instructions of code
+// instead of 64 unrolled polls at every call site, for kernels whose hot loop
+// would otherwise not fit the instruction cache.
+__device__ __forceinline__ bool mbar_wait_lean(uint64_t* bar, uint32_t parity) {
+    if (mbar_try_wait(bar, parity)) return true;
+    unsigned long long t0 = globaltimer();
+    while (true) {
+#pragma unroll 1
+        for (int i = 0; i < 64; ++i)
+            if (mbar_try_wait(bar, parity)) return true;
+        if (globaltimer() - t0 > kWaitLimitNs) return false;
+    }
+}
+
 // Warp-uniform variant: every lane waits, and all lanes agree on the result
 // (warp-collective instructions may follow).  All lanes poll: on B200 a
 // whole warp suspended in try_wait resumes sooner after the phase completes
 // than a warp whose lane 0 polls alone (measured in this kernel set).
 __device__ __forceinline__ bool mbar_wait_warp(uint64_t* bar, uint32_t parity) {
     const bool ok = mbar_wait(bar, parity);
+    return __all_sync(0xffffffffu, ok);
+}
+__device__ __forceinline__ bool mbar_wait_warp_lean(uint64_t* bar, uint32_t parity) {
+    const bool ok = mbar_wait_lean(bar, parity);
     return __all_sync(0xffffffffu, ok);
 }
 

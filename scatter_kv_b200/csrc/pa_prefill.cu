@@ -191,6 +191,19 @@ __device__ __forceinline__ bool poly_col(int c) {
 }
 
 
+// Bounded waits of the kernel.  With TMA producers the kernel's hot loop only
+// fits the SM's instruction cache with rolled polling loops (unrolled ones
+// cost about 6% of the kernel's time there); the cp.async path measures
+// faster with the unrolled polls.
+template <bool LEAN>
+__device__ __forceinline__ bool pwait(uint64_t* bar, uint32_t parity) {
+    return LEAN ? mbar_wait_lean(bar, parity) : mbar_wait(bar, parity);
+}
+template <bool LEAN>
+__device__ __forceinline__ bool pwait_warp(uint64_t* bar, uint32_t parity) {
+    return LEAN ? mbar_wait_warp_lean(bar, parity) : mbar_wait_warp(bar, parity);
+}
+
 template <int HEAD, bool CPA>
 __global__ void __launch_bounds__(PCfg<HEAD, CPA>::THREADS, 1)
 prefill_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
@@ -363,7 +376,7 @@ prefill_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
             const bool tail = is_v && (k0 + C::BN > T);
             if (!CPA && tail && pw != 0) continue;
             bool go = true;
-            if (lane == 0 && u >= C::NS) go = mbar_wait(&empty[st], ((u / C::NS) - 1) & 1);
+            if (lane == 0 && u >= C::NS) go = pwait<!CPA>(&empty[st], ((u / C::NS) - 1) & 1);
             go = __shfl_sync(0xffffffffu, go, 0);
             if (!go) {
                 if (lane == 0) {
@@ -436,7 +449,7 @@ prefill_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
                 // Last V tile: rows at or past T hold stale or poisoned data.  Land
                 // the tile, zero those rows, then release it to the MMA thread
                 // (arriving for all producers).
-                if (!mbar_wait_warp(v_tail, 0)) {
+                if (!pwait_warp<!CPA>(v_tail, 0)) {
                     if (lane == 0) {
                         flag_status(p.status, PA_DEV_TIMEOUT);
                         atomicExch(&sh[3], 1);
@@ -488,7 +501,7 @@ prefill_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
                 }
             };
             const int nt0 = ntiles_h[0], nt1 = ntiles_h[1];
-            bool alive = mbar_wait(q_full, 0) && (ntiles == 0 || mbar_wait(&full[0], 0));
+            bool alive = pwait<!CPA>(q_full, 0) && (ntiles == 0 || pwait<!CPA>(&full[0], 0));
             if (alive && ntiles > 0) {
                 tc_fence_after();
                 if (nt0 > 0) issue_s(0, 0);
@@ -501,11 +514,11 @@ prefill_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
                 const bool more = j + 1 < ntiles;
                 // Both ring items of this step first (loaded tiles ago, as a rule), so
                 // that the two products of a group issue back to back.
-                if (!mbar_wait(&full[sv], (uv / C::NS) & 1)) { alive = false; break; }
-                if (more && !mbar_wait(&full[sk], (uk / C::NS) & 1)) { alive = false; break; }
+                if (!pwait<!CPA>(&full[sv], (uv / C::NS) & 1)) { alive = false; break; }
+                if (more && !pwait<!CPA>(&full[sk], (uk / C::NS) & 1)) { alive = false; break; }
                 // Half 0 group: P_0,j V_j, then S_0,j+1.
                 if (j < nt0) {
-                    if (!mbar_wait(&p_full[0], j & 1)) { alive = false; break; }
+                    if (!pwait<!CPA>(&p_full[0], j & 1)) { alive = false; break; }
                     tc_fence_after();
                     issue_pv(0, sv, j == 0);
                     if (j == nt0 - 1) umma_commit(&o_full[0]);
@@ -516,7 +529,7 @@ prefill_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
                 }
                 // Half 1 group: P_1,j V_j, then S_1,j+1.
                 if (j < nt1) {
-                    if (!mbar_wait(&p_full[1], j & 1)) { alive = false; break; }
+                    if (!pwait<!CPA>(&p_full[1], j & 1)) { alive = false; break; }
                     tc_fence_after();
                     issue_pv(1, sv, j == 0);
                     if (j == nt1 - 1) umma_commit(&o_full[1]);
@@ -532,7 +545,7 @@ prefill_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
                 atomicExch(&sh[3], 1);
                 // Let every MMA already issued finish before the CTA moves on.
                 umma_commit(drain);
-                mbar_wait(drain, 0);
+                pwait<!CPA>(drain, 0);
             }
         }
         __syncwarp();
@@ -553,7 +566,7 @@ prefill_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
         float m_used = -INFINITY, l = 0.f;
         bool alive = true;
         for (int j = 0; j < nt; ++j) {
-            if (!mbar_wait_warp(&s_full[a], j & 1)) { alive = false; break; }
+            if (!pwait_warp<!CPA>(&s_full[a], j & 1)) { alive = false; break; }
             tc_fence_after();
             uint32_t sv[C::BN];
 #pragma unroll
@@ -634,7 +647,7 @@ prefill_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
             if (lane == 0) mbar_arrive(&p_full[a]);
         }
         // Epilogue: O / l -> f16 rows of `out`.
-        if (alive && nt > 0 && mbar_wait_warp(&o_full[a], 0)) {
+        if (alive && nt > 0 && pwait_warp<!CPA>(&o_full[a], 0)) {
             tc_fence_after();
             const float inv = (l > 0.f) ? 1.f / l : 0.f;
             __half* orow = p.out + ((long long)(s.q_start + tok) * p.q_heads + kvh * g + r % g) * HEAD;
@@ -669,12 +682,12 @@ prefill_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
     __syncthreads();
     if (sh[3] && threadIdx.x == 0) {
         // Aborted (never expected): let in-flight loads land before exit.
-        mbar_wait(q_full, 0);
+        pwait<!CPA>(q_full, 0);
         const int issued = sh[4];
         for (int u = issued - C::NS > 0 ? issued - C::NS : 0; u < issued; ++u) {
             const bool tail = (u & 1) && ((u >> 1) * C::BN + C::BN > T);
-            if (tail) mbar_wait(v_tail, 0);
-            else mbar_wait(&full[u % C::NS], (u / C::NS) & 1);
+            if (tail) pwait<!CPA>(v_tail, 0);
+            else pwait<!CPA>(&full[u % C::NS], (u / C::NS) & 1);
         }
     }
     __syncthreads();
