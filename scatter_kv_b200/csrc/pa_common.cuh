@@ -403,11 +403,11 @@ struct SeqInfo {
 // false when the sequence is invalid; with a non-null `status` also ORs the
 // matching PA_DEV_* bits into it.  kv_cap = max_blocks_per_seq * block_size;
 // kv_hint / q_hint are the caller's optional bounds (0 = none).
-__device__ __forceinline__ bool load_seq(const int32_t* cu, const int32_t* seqlens_kv, int b,
-                                         int batch, long long token_count, int kv_cap,
-                                         int kv_hint, int q_hint, int32_t* status, SeqInfo& s) {
-    const int c0 = cu[b], c1 = cu[b + 1];
-    const int kv = seqlens_kv[b];
+// Sequence b's geometry from its offsets c0 = cu_seqlens_q[b], c1 =
+// cu_seqlens_q[b + 1] and kv = seqlens_kv[b], with the same checks as load_seq.
+__device__ __forceinline__ bool seq_info(int c0, int c1, int kv, int b, int batch,
+                                         long long token_count, int kv_cap, int kv_hint,
+                                         int q_hint, int32_t* status, SeqInfo& s) {
     s.q_start = c0;
     s.q_len = c1 - c0;
     s.kv_len = kv;
@@ -424,6 +424,13 @@ __device__ __forceinline__ bool load_seq(const int32_t* cu, const int32_t* seqle
         bits |= PA_DEV_HINT_EXCEEDED;
     if (bits) flag_status(status, bits);
     return bits == 0;
+}
+
+__device__ __forceinline__ bool load_seq(const int32_t* cu, const int32_t* seqlens_kv, int b,
+                                         int batch, long long token_count, int kv_cap,
+                                         int kv_hint, int q_hint, int32_t* status, SeqInfo& s) {
+    return seq_info(cu[b], cu[b + 1], seqlens_kv[b], b, batch, token_count, kv_cap, kv_hint,
+                    q_hint, status, s);
 }
 
 // Warp-cooperative check that every block id sequence `b` uses is in range.

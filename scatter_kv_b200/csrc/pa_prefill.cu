@@ -120,6 +120,8 @@ struct Work {
     int b;          // sequence
     int kvh;        // KV head
     int pair;       // pair of query tiles within the sequence
+    int c0, c1;     // cu_seqlens_q[b], cu_seqlens_q[b + 1]
+    int kv;         // seqlens_kv[b]
 };
 
 // CTA x -> (sequence, KV head, tile pair), longest work first: rank r
@@ -128,20 +130,28 @@ struct Work {
 // then every rank-1 pair, and so on.  The light pairs of all sequences fill
 // the end of the grid, so SMs finish close together; measured 4-6% faster
 // than a sequence-major order, whose last CTAs included heavy pairs.  One
-// warp, 32 sequences per step.
+// warp, 32 sequences per step; the first 32 sequences' lengths are read once
+// (one round trip for the usual batch), later ones once per rank.
 __device__ bool find_work(const PrefillParams& p, long long slot, Work& w) {
     const int lane = threadIdx.x & 31;
+    auto lengths = [&](int b, int& c0, int& c1, int& kv, int& np) {
+        c0 = c1 = kv = np = 0;
+        if (b < p.batch) {
+            c0 = p.cu_seqlens_q[b];
+            c1 = p.cu_seqlens_q[b + 1];
+            kv = p.seqlens_kv[b];
+            const int ql = c1 - c0;
+            if (ql > p.decode_max_q && c0 >= 0 && (long long)c1 <= p.token_count)
+                np = (ql * p.group + kPrefillCtaRows - 1) / kPrefillCtaRows;
+        }
+    };
+    int c0f, c1f, kvf, npf;
+    lengths(lane, c0f, c1f, kvf, npf);
     for (int r = 0;; ++r) {
         bool more = false;                        // some sequence has a pair of rank >= r
         for (int b0 = 0; b0 < p.batch; b0 += 32) {
-            const int b = b0 + lane;
-            int np = 0;
-            if (b < p.batch) {
-                const int c0 = p.cu_seqlens_q[b], c1 = p.cu_seqlens_q[b + 1];
-                const int ql = c1 - c0;
-                if (ql > p.decode_max_q && c0 >= 0 && (long long)c1 <= p.token_count)
-                    np = (ql * p.group + kPrefillCtaRows - 1) / kPrefillCtaRows;
-            }
+            int c0 = c0f, c1 = c1f, kv = kvf, np = npf;
+            if (b0 > 0) lengths(b0 + lane, c0, c1, kv, np);
             const unsigned m = __ballot_sync(0xffffffffu, np > r);
             more = more || m != 0u;
             const long long total = (long long)__popc(m) * p.kv_heads;
@@ -154,6 +164,9 @@ __device__ bool find_work(const PrefillParams& p, long long slot, Work& w) {
                 w.b = b0 + lb;
                 w.kvh = (int)(slot % p.kv_heads);
                 w.pair = __shfl_sync(0xffffffffu, np, lb) - 1 - r;
+                w.c0 = __shfl_sync(0xffffffffu, c0, lb);
+                w.c1 = __shfl_sync(0xffffffffu, c1, lb);
+                w.kv = __shfl_sync(0xffffffffu, kv, lb);
                 return true;
             }
             slot -= total;
@@ -232,25 +245,86 @@ prefill_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
         return;
     }
 
+    // Setup with its memory round trips overlapped.  The MMA warp allocates
+    // tensor memory while warp 0 finds the work item (one round trip for the
+    // item and the sequence's lengths); Q's TMA starts as soon as the item is
+    // known (its tensor map bounds every coordinate) and streams while warp 0
+    // checks the block table.
+    const int tokp = C::BM / g;                                  // tokens per half
+    if (warp == C::WARP_MMA) {
+        tmem_alloc(tmem_slot, C::TMEM_COLS);
+        tmem_relinquish();
+    }
     if (warp == 0) {
+        if (lane == 0) {
+            sh[3] = 0;
+            sh[4] = 0;
+            mbar_init(q_full, 1);
+            for (int i = 0; i < C::NS; ++i) {
+                mbar_init(&full[i], CPA ? C::NPROD * 32 : C::NPROD);   // per producer thread / warp
+                mbar_init(&empty[i], 1);
+            }
+            for (int i = 0; i < 2; ++i) {
+                mbar_init(&s_full[i], 1);
+                mbar_init(&p_full[i], 4);
+                mbar_init(&o_full[i], 1);
+            }
+            mbar_init(drain, 1);
+            mbar_init(v_tail, 1);
+            fence_barrier_init();
+            tma_prefetch_desc(&tm_q);
+            tma_prefetch_desc(&tm_k);
+            tma_prefetch_desc(&tm_v);
+        }
+        __syncwarp();
         Work w;
         const bool has = find_work(p, (long long)blockIdx.x, w);
+        // sh[2]: 0 valid, 1 invalid, 2 invalid with Q's TMA in flight.
+        int bad = 1;
+        SeqInfo si{};
+        if (has) {
+            // The sequence's first CTA reports its errors.
+            const bool first = w.pair == 0 && w.kvh == 0;
+            bool ok = seq_info(w.c0, w.c1, w.kv, w.b, p.batch, p.token_count, p.kv_cap, p.kv_hint,
+                               p.q_hint, (first && lane == 0) ? p.status : nullptr, si);
+            if (ok) {
+                if (lane == 0) {
+                    mbar_arrive_expect_tx(q_full, 2 * C::Q_BYTES);
+#pragma unroll
+                    for (int a = 0; a < 2; ++a)
+#pragma unroll
+                        for (int c = 0; c < C::NA; ++c)
+                            tma_load_3d(smem + C::OFF_Q + a * C::Q_BYTES + c * C::BM * C::RB, &tm_q,
+                                        q_full, c * C::A, w.kvh * g, si.q_start + (w.pair * 2 + a) * tokp);
+                }
+                const int npages = (si.kv_len + p.block_size - 1) / p.block_size;
+                ok = warp_blocks_ok(p.block_table, w.b, p.max_blocks, npages, p.num_blocks,
+                                    first ? p.status : nullptr);
+                bad = ok ? 0 : 2;
+            }
+        }
         if (lane == 0) {
             sh[0] = has ? w.b : -1;
             sh[1] = has ? w.pair : 0;
             sh[6] = has ? w.kvh : 0;
+            sh[2] = bad;
+            sh[7] = si.q_start;
+            sh[8] = si.q_len;
+            sh[9] = si.kv_len;
         }
     }
+    tc_fence_before();
     __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = *tmem_slot;
     const int b = sh[0];
-    if (b < 0) return;
     const int pair = sh[1];
     const int kvh = sh[6];
-
     SeqInfo s;
-    const bool ok = load_seq(p.cu_seqlens_q, p.seqlens_kv, b, p.batch, p.token_count, p.kv_cap,
-                             p.kv_hint, p.q_hint, nullptr, s);
-    const int tokp = C::BM / g;                                  // tokens per half
+    s.q_start = sh[7];
+    s.q_len = sh[8];
+    s.kv_len = sh[9];
+    s.past = s.kv_len - s.q_len;
     const int i0 = pair * 2 * tokp;                              // first token of half 0
     // Rows and key tiles of each half (a half past the sequence end has none).
     int rows_valid[2], ntiles_h[2];
@@ -262,55 +336,22 @@ prefill_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
         ntiles_h[a] = rows_valid[a] > 0 ? (s.past + last + 1 + C::BN - 1) / C::BN : 0;
     }
     const int ntiles = max(ntiles_h[0], ntiles_h[1]);
-
-    if (threadIdx.x == 0) {
-        if (pair == 0 && kvh == 0)
-            load_seq(p.cu_seqlens_q, p.seqlens_kv, b, p.batch, p.token_count, p.kv_cap,
-                     p.kv_hint, p.q_hint, p.status, s);
-        sh[2] = ok ? 0 : 1;
-        sh[3] = 0;
-        sh[4] = 0;
-        mbar_init(q_full, 1);
-        for (int i = 0; i < C::NS; ++i) {
-            mbar_init(&full[i], CPA ? C::NPROD * 32 : C::NPROD);   // per producer thread / warp
-            mbar_init(&empty[i], 1);
-        }
-        for (int i = 0; i < 2; ++i) {
-            mbar_init(&s_full[i], 1);
-            mbar_init(&p_full[i], 4);
-            mbar_init(&o_full[i], 1);
-        }
-        mbar_init(drain, 1);
-        mbar_init(v_tail, 1);
-        fence_barrier_init();
-    }
-    __syncthreads();
     const int T = s.kv_len;
-    if (ok && warp == 0) {
-        const int npages = (T + p.block_size - 1) / p.block_size;
-        if (!warp_blocks_ok(p.block_table, b, p.max_blocks, npages, p.num_blocks,
-                            (pair == 0 && kvh == 0) ? p.status : nullptr) && lane == 0)
-            sh[2] = 1;
-    }
-    __syncthreads();
-    if (sh[2]) {
-        const int rows = rows_valid[0] + rows_valid[1];
-        for (int idx = threadIdx.x; idx < rows * HEAD; idx += C::THREADS) {
-            const int r = idx / HEAD, d = idx % HEAD;
-            const long long o = ((long long)(s.q_start + i0 + r / g) * p.q_heads + kvh * g + r % g) * HEAD + d;
-            p.out[o] = __float2half_rn(0.f);
+    if (b < 0 || sh[2] != 0) {
+        if (b >= 0) {
+            // Invalid sequence or block table: its rows of `out` are zero.
+            const int rows = rows_valid[0] + rows_valid[1];
+            for (int idx = threadIdx.x; idx < rows * HEAD; idx += C::THREADS) {
+                const int r = idx / HEAD, d = idx % HEAD;
+                const long long o = ((long long)(s.q_start + i0 + r / g) * p.q_heads + kvh * g + r % g) * HEAD + d;
+                p.out[o] = __float2half_rn(0.f);
+            }
+            // Q's copy lands before the CTA's shared memory is released.
+            if (sh[2] == 2 && threadIdx.x == 0) pwait<!CPA>(q_full, 0);
         }
+        if (warp == C::WARP_MMA) tmem_dealloc(tmem, C::TMEM_COLS);
         return;
     }
-
-    if (warp == C::WARP_MMA) {
-        tmem_alloc(tmem_slot, C::TMEM_COLS);
-        tmem_relinquish();
-    }
-    tc_fence_before();
-    __syncthreads();
-    tc_fence_after();
-    const uint32_t tmem = *tmem_slot;
 
     uint8_t* sQ = smem + C::OFF_Q;
     uint8_t* ring = smem + C::OFF_RING;
@@ -326,18 +367,6 @@ prefill_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
         // Key tile j covers keys [128 j, 128 j + 128): the pages (or the part of
         // one page) holding them, up to the last page that starts before T.
         // Box b = page * NA + column block goes to producer b % NPROD.
-        if (pw == 0 && lane == 0) {
-            tma_prefetch_desc(&tm_q);
-            tma_prefetch_desc(&tm_k);
-            tma_prefetch_desc(&tm_v);
-            mbar_arrive_expect_tx(q_full, 2 * C::Q_BYTES);
-#pragma unroll
-            for (int a = 0; a < 2; ++a)
-#pragma unroll
-                for (int c = 0; c < C::NA; ++c)
-                    tma_load_3d(sQ + a * C::Q_BYTES + c * C::BM * C::RB, &tm_q, q_full, c * C::A,
-                                kvh * g, s.q_start + i0 + a * tokp);
-        }
         // Block ids of the sequence, 32 pages at a time in registers (lane i
         // holds page win_base + i); the next window is fetched a whole window
         // ahead, so issuing a tile never waits on a block-table load.
