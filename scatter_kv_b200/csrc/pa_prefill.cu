@@ -297,9 +297,30 @@ prefill_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
                             tma_load_3d(smem + C::OFF_Q + a * C::Q_BYTES + c * C::BM * C::RB, &tm_q,
                                         q_full, c * C::A, w.kvh * g, si.q_start + (w.pair * 2 + a) * tokp);
                 }
+                // Block-table check (the row's ids in range), keeping page 0's id.
                 const int npages = (si.kv_len + p.block_size - 1) / p.block_size;
-                ok = warp_blocks_ok(p.block_table, w.b, p.max_blocks, npages, p.num_blocks,
-                                    first ? p.status : nullptr);
+                const int32_t* row = p.block_table + (long long)w.b * p.max_blocks;
+                bool badid = false;
+                int id0 = 0;
+                for (int pg = lane; pg < npages; pg += 32) {
+                    const int id = row[pg];
+                    if (pg == 0) id0 = id;
+                    badid |= id < 0 || (long long)id >= p.num_blocks;
+                }
+                ok = !__any_sync(0xffffffffu, badid);
+                if (!ok && first && lane == 0) flag_status(p.status, PA_DEV_BAD_BLOCK);
+                if (!CPA && ok && lane == 0) {
+                    // TMA path: key tile 0 (ring item 0, one page of at least 128
+                    // rows) is issued here too, with the arrivals of every producer;
+                    // the producers start at ring item 1.
+                    mbar_arrive_expect_tx(&full[0], (uint32_t)C::KV_BYTES);
+#pragma unroll
+                    for (int c = 0; c < C::NA; ++c)
+                        tma_load_4d(smem + C::OFF_RING + c * C::BN * C::RB, &tm_k, &full[0], c * C::A,
+                                    w.kvh, 0, id0);
+                    if (C::NPROD > 1) mbar_arrive_cnt(&full[0], C::NPROD - 1);
+                    sh[4] = 1;                           // ring items issued (abort drain)
+                }
                 bad = ok ? 0 : 2;
             }
         }
@@ -396,7 +417,7 @@ prefill_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
             const int np0 = (min(C::BN, T) + bs - 1) / bs;
             next_ids = lane < np0 ? bt[lane] : 0;          // becomes tile 0's ids at u = 0
         }
-        for (int u = 0; u < 2 * ntiles; ++u) {
+        for (int u = CPA ? 0 : 1; u < 2 * ntiles; ++u) {
             const int st = u % C::NS;
             const int j = u >> 1;
             const bool is_v = (u & 1) != 0;
@@ -681,23 +702,26 @@ prefill_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
             tc_fence_after();
             const float inv = (l > 0.f) ? 1.f / l : 0.f;
             __half* orow = p.out + ((long long)(s.q_start + tok) * p.q_heads + kvh * g + r % g) * HEAD;
+            // O in EPB-column batches, one round trip to tensor memory each: the
+            // whole row on the TMA path; 16 columns on the cp.async path, which
+            // measured faster with them.
+            constexpr int EPB = CPA ? 16 : HEAD;
 #pragma unroll
-            for (int c0 = 0; c0 < HEAD; c0 += 16) {
-                uint32_t ov[16];
-                tmem_ld16(ocol + c0, ov);
+            for (int h0 = 0; h0 < HEAD; h0 += EPB) {
+                uint32_t ov[EPB];
+#pragma unroll
+                for (int c0 = 0; c0 < EPB; c0 += 16) tmem_ld16(ocol + h0 + c0, ov + c0);
                 tmem_wait_ld();
                 if (r < my_rows) {
-                    uint4 w0, w1;
-                    w0.x = pack_half2(__uint_as_float(ov[0]) * inv, __uint_as_float(ov[1]) * inv);
-                    w0.y = pack_half2(__uint_as_float(ov[2]) * inv, __uint_as_float(ov[3]) * inv);
-                    w0.z = pack_half2(__uint_as_float(ov[4]) * inv, __uint_as_float(ov[5]) * inv);
-                    w0.w = pack_half2(__uint_as_float(ov[6]) * inv, __uint_as_float(ov[7]) * inv);
-                    w1.x = pack_half2(__uint_as_float(ov[8]) * inv, __uint_as_float(ov[9]) * inv);
-                    w1.y = pack_half2(__uint_as_float(ov[10]) * inv, __uint_as_float(ov[11]) * inv);
-                    w1.z = pack_half2(__uint_as_float(ov[12]) * inv, __uint_as_float(ov[13]) * inv);
-                    w1.w = pack_half2(__uint_as_float(ov[14]) * inv, __uint_as_float(ov[15]) * inv);
-                    *reinterpret_cast<uint4*>(orow + c0) = w0;
-                    *reinterpret_cast<uint4*>(orow + c0 + 8) = w1;
+#pragma unroll
+                    for (int c0 = 0; c0 < EPB; c0 += 8) {
+                        uint4 w0;
+                        w0.x = pack_half2(__uint_as_float(ov[c0]) * inv, __uint_as_float(ov[c0 + 1]) * inv);
+                        w0.y = pack_half2(__uint_as_float(ov[c0 + 2]) * inv, __uint_as_float(ov[c0 + 3]) * inv);
+                        w0.z = pack_half2(__uint_as_float(ov[c0 + 4]) * inv, __uint_as_float(ov[c0 + 5]) * inv);
+                        w0.w = pack_half2(__uint_as_float(ov[c0 + 6]) * inv, __uint_as_float(ov[c0 + 7]) * inv);
+                        *reinterpret_cast<uint4*>(orow + h0 + c0) = w0;
+                    }
                 }
             }
         } else if (!alive) {
