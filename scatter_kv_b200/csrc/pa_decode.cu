@@ -73,6 +73,9 @@ struct Cfg {
     static_assert(NST % NG == 0, "each stage must belong to one consumer group");
     static constexpr int NPW = CPA ? 4 : 1;             // producer warps (cp.async: a warpgroup)
     static constexpr int THREADS = 32 * (NCW + NPW);
+    // setmaxnreg (cp.async path) acts on whole warpgroups: consumers are one,
+    // the producer warps another.
+    static_assert(!CPA || (NCW == 4 && NPW == 4), "register split needs two whole warpgroups");
     static constexpr int CPR = HEAD * 2 / 16;           // 16-byte chunks per cache row
     static constexpr int TILE_BYTES = BN * HEAD * 2;    // one tensor, one stage
     static constexpr int STAGE_BYTES = 2 * TILE_BYTES;

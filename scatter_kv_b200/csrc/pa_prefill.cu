@@ -90,6 +90,9 @@ struct PCfg {
     static constexpr int SMEM_USED = OFF_BAR + NBAR * 8 + 64;
     static constexpr int SMEM = SMEM_USED > 120 * 1024 ? SMEM_USED : 120 * 1024;
     static constexpr int THREADS = 384;
+    // setmaxnreg acts on whole warpgroups (warps 4k .. 4k + 3, all executing
+    // the same instruction); a CTA with a partial warpgroup hung in it.
+    static_assert(THREADS % 128 == 0, "the register split needs whole warpgroups");
     static constexpr int WARP_MMA = 9;            // producers: warps 8, 10, 11
     static constexpr int NPROD = 3;
     static constexpr int CPR = HEAD * 2 / 16;           // 16-byte chunks per cache row
