@@ -219,11 +219,24 @@ def time_oracle(spec: workloads.Spec, x: dict, target_s: float, seed: int = 0):
 
 # ----------------------------------------------------------------- profiles
 
+_CODE_TOKENS = re.compile(r'"(?:\\.|[^"\\\n])*"|\'(?:\\.|[^\'\\\n])*\'|//[^\n]*|/\*.*?\*/', re.S)
+
+
+def _strip_comments(src: str) -> str:
+    """C/C++/CUDA source without its comments (string and character literals
+    kept), with blank-line runs and trailing blanks removed."""
+    code = _CODE_TOKENS.sub(lambda m: "" if m.group(0).startswith("/") else m.group(0), src)
+    lines = [ln.rstrip() for ln in code.splitlines()]
+    return "\n".join(ln for ln in lines if ln)
+
+
 def kernel_source_hash() -> str:
+    """Hash of the kernel sources' code: a profile taken on them stays valid
+    through comment-only edits, and any code change invalidates it."""
     h = hashlib.sha256()
     for name in sorted(os.listdir(os.path.join(ROOT, "scatter_kv_b200", "csrc"))):
-        with open(os.path.join(ROOT, "scatter_kv_b200", "csrc", name), "rb") as f:
-            h.update(name.encode() + f.read())
+        with open(os.path.join(ROOT, "scatter_kv_b200", "csrc", name), encoding="utf-8") as f:
+            h.update(name.encode() + _strip_comments(f.read()).encode())
     return h.hexdigest()[:16]
 
 

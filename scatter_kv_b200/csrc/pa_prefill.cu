@@ -19,7 +19,7 @@
 // Warp roles (384 threads, three warpgroups):
 //   warps 0-3   softmax + epilogue of half 0 (thread r = row r = TMEM lane r)
 //   warps 4-7   softmax + epilogue of half 1
-//   warps 8, 10, 11  producers: Q of both halves by TMA, then the K/V ring.
+//   warps 8, 10, 11  producers of the K/V ring (warp 0 issues Q's TMA first).
 //               Pages of 128 keys or more: TMA boxes, dealt out over the
 //               three warps.  Smaller pages: 16-byte cp.async copies by all
 //               96 producer threads, each chunk placed where the 128-byte
@@ -54,9 +54,9 @@
 // skipped; the diagonal tile is masked per element; rows of V past the end
 // of the sequence are zeroed in shared memory (by the producer, before it
 // marks the tile ready) so that 0 * garbage never reaches the P V products.
-// CTAs are ordered sequence-major, then KV head, then tile pair from the
-// last (most keys) to the first, so the CTAs resident at any time share few
-// sequences' K/V and reuse them from L2.
+// CTAs run longest work first (find_work): every sequence's last tile pair,
+// then every second-to-last, and so on, so SMs finish close together; the
+// set-up overlaps its metadata round trips with Q's and key tile 0's TMA.
 #include <cuda_runtime.h>
 #include <math.h>
 
