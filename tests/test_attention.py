@@ -68,6 +68,19 @@ def test_prefill_shapes(qh, kvh, q_lens, past, bs):
     _full_check(spec)
 
 
+@pytest.mark.parametrize("bs", [16, 256])
+def test_more_than_32_prefill_sequences(bs):
+    # The prefill CTAs take their work in longest-work-first order across
+    # 32-sequence chunks; 70 sequences of ragged lengths (decode ones among
+    # them) make the ranks span three chunks.
+    rng = np.random.Generator(np.random.PCG64(70))
+    q_lens = rng.integers(1, 160, size=70)
+    q_lens[::7] = 1
+    past = rng.integers(0, 160, size=70)
+    spec = workloads.custom(q_lens, past, 8, 2, 128, bs, seed=70 + bs)
+    _full_check(spec)
+
+
 def test_mixed_batch_with_empty_sequences():
     q_lens = [1, 0, 200, 4, 0, 33, 1, 2, 3, 600]
     past = [3000, 5, 100, 2000, 0, 0, 1, 7000, 12, 250]
