@@ -70,10 +70,23 @@ double oracle_half_to_double(uint16_t h)
     return sign ? -v : v;
 }
 
+/* Every binary16 pattern's value, filled from oracle_half_to_double before
+ * the first attention call: a table lookup returns exactly what the function
+ * would, only faster (the attention loops decode each element many times). */
+static double half_table[65536];
+static int half_table_ready = 0;
+
+static void fill_half_table(void)
+{
+    if (half_table_ready) return;
+    for (int i = 0; i < 65536; ++i) half_table[i] = oracle_half_to_double((uint16_t)i);
+    half_table_ready = 1;
+}
+
 static double load(const void *base, int64_t idx, int dtype)
 {
     if (dtype == ORACLE_F64) return ((const double *)base)[idx];
-    return oracle_half_to_double(((const uint16_t *)base)[idx]);
+    return half_table[((const uint16_t *)base)[idx]];
 }
 
 /* Scatter new K/V tokens into the paged caches.
@@ -193,6 +206,7 @@ void oracle_attention(const void *query, const void *key_cache, const void *valu
                       double *scratch, int64_t max_keys, double *out)
 {
     if (rows == NULL) nrows = token_count * q_heads;
+    fill_half_table();
 #pragma omp parallel
     {
         int tid = 0;
