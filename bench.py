@@ -43,26 +43,46 @@ L2_BYTES = 126 * 1024 * 1024
 
 # ----------------------------------------------------------------- work counts
 
+def decode_cutoff(spec: workloads.Spec) -> int:
+    """q_len up to which the library takes the split-KV decode path (its rule:
+    at most 4 query tokens and at most 32 query rows per KV head)."""
+    g = spec.q_heads // spec.kv_heads
+    return max(1, min(4, 32 // g))
+
+
 def algorithmic_counts(spec: workloads.Spec) -> dict:
     """Bytes and FLOPs the method must move / compute for one step.
 
     attention bytes: every K/V row of a sequence read once per KV head, plus
     Q read and O written; FLOPs: 4 * q_heads * d per visible (query, key)
-    pair, causal; scatter bytes: new K/V read and written, slots read."""
+    pair, causal; scatter bytes: new K/V read and written, slots read.  The
+    decode_* and prefill_* entries split the same counts between the
+    sequences each kernel serves."""
     T = spec.seqlens_kv.astype(np.int64)
+    ql = spec.q_lens.astype(np.int64)
+    past = spec.past.astype(np.int64)
     d, kvh, qh = spec.head_size, spec.kv_heads, spec.q_heads
-    kv_bytes = int((T * kvh * d * 2 * 2).sum())
-    q_bytes = spec.token_count * qh * d * 2
-    o_bytes = q_bytes
-    flops = 0
-    for ql, past in zip(spec.q_lens.astype(np.int64), spec.past.astype(np.int64)):
-        # sum over i < ql of (past + i + 1) visible keys
-        flops += 4 * qh * d * int(ql * past + ql * (ql + 1) // 2)
+    kv_seq = T * kvh * d * 2 * 2
+    q_seq = ql * qh * d * 2
+    # sum over i < q_len of (past + i + 1) visible keys
+    flops_seq = 4 * qh * d * (ql * past + ql * (ql + 1) // 2)
+    dec = (ql > 0) & (ql <= decode_cutoff(spec))
+    pre = ql > decode_cutoff(spec)
     scatter_bytes = 4 * spec.token_count * kvh * d * 2 + 4 * spec.token_count
-    is_decode = bool(spec.q_lens.max() <= 4)
-    return dict(kv_bytes=kv_bytes, q_bytes=q_bytes, o_bytes=o_bytes, flops=flops,
+    kv_bytes, q_bytes = int(kv_seq.sum()), int(q_seq.sum())
+    return dict(kv_bytes=kv_bytes, q_bytes=q_bytes, o_bytes=q_bytes, flops=int(flops_seq.sum()),
                 scatter_bytes=scatter_bytes,
-                step_bytes=kv_bytes + q_bytes + o_bytes + scatter_bytes, decode=is_decode)
+                step_bytes=kv_bytes + 2 * q_bytes + scatter_bytes,
+                decode_bytes=int(kv_seq[dec].sum() + q_seq[dec].sum()),
+                prefill_flops=int(flops_seq[pre].sum()),
+                prefill_bytes=int(kv_seq[pre].sum() + 2 * q_seq[pre].sum()),
+                decode=bool(spec.q_lens.max() <= decode_cutoff(spec)))
+
+
+# Datasheet figures, reported beside the measured ones: HBM3e bandwidth of an
+# HGX B200 and its dense 16-bit tensor-core rate.
+NOMINAL_HBM_GBS = 7700.0
+NOMINAL_TFLOPS = 2250.0
 
 
 def load_peaks() -> dict:
@@ -197,7 +217,7 @@ def time_oracle(spec: workloads.Spec, x: dict, target_s: float, seed: int = 0):
     cu = np.concatenate([[0], np.cumsum(spec.q_lens)])
     g = spec.q_heads // spec.kv_heads
     scale = 1.0 / math.sqrt(spec.head_size)
-    done_bytes, done_units, rows_done = 0, 0, 0
+    done_bytes, done_flops, done_units, rows_done = 0, 0, 0, 0
     t0 = time.perf_counter()
     i = 0
     while i < len(order) and time.perf_counter() - t0 < target_s:
@@ -209,12 +229,15 @@ def time_oracle(spec: workloads.Spec, x: dict, target_s: float, seed: int = 0):
                          x["cu_seqlens_q"], x["seqlens_kv"], scale, rows=rows)
         T = int(spec.seqlens_kv[b])
         done_bytes += T * spec.head_size * 2 * 2 + 2 * rows.shape[0] * spec.head_size * 2
+        q, p = int(spec.q_lens[b]), int(spec.past[b])
+        done_flops += 4 * g * spec.head_size * (q * p + q * (q + 1) // 2)
         done_units += 1
         rows_done += rows.shape[0]
     dt = time.perf_counter() - t0
     sample = (f"{done_units} of {len(units)} (sequence, KV head) units, {rows_done} output rows, "
               f"fp64 oracle attention, {dt:.1f} s")
-    return done_bytes / dt / 1e9, dt, sample, oracle.max_threads()
+    return dict(gbs=done_bytes / dt / 1e9, tflops=done_flops / dt / 1e12, seconds=dt,
+                sample=sample, cores=oracle.max_threads())
 
 
 # ----------------------------------------------------------------- profiles
@@ -256,6 +279,20 @@ def profiled_traffic(kernel: str, workload: str):
 
 # ----------------------------------------------------------------- main arms
 
+def unit_of(spec: workloads.Spec) -> str:
+    """Decode-only batches are judged on bytes moved, the others on FLOPs."""
+    return "GB/s" if algorithmic_counts(spec)["decode"] else "TFLOP/s"
+
+
+def config_of(spec: workloads.Spec, world: int = 1) -> dict:
+    return {"workload": spec.name, "batch": spec.batch, "tokens": spec.token_count,
+            "q_heads": spec.q_heads, "kv_heads": spec.kv_heads, "head_size": spec.head_size,
+            "block_size": spec.block_size, "num_blocks": spec.num_blocks, "seed": spec.seed,
+            "l2": "flushed between steps, outside the timed events: 252 MB written, then "
+                  "252 MB read so no dirty line is left to write back",
+            "parallelism": f"replicas x{world}"}
+
+
 def run_reference(args, spec, rank, world):
     if rank != 0:
         return
@@ -265,36 +302,56 @@ def run_reference(args, spec, rank, world):
     slots = oracle.slot_mapping(x["block_table"], x["cu_seqlens_q"], x["seqlens_kv"],
                                 spec.block_size)
     oracle.scatter_kv(x["key"], x["value"], slots, x["key_cache"], x["value_cache"])
+    unit = unit_of(spec)
+    key = "gbs" if unit == "GB/s" else "tflops"
     # Each step is a bounded sample sized so the whole run takes about two minutes.
     per_step = max(0.5, min(15.0, 120.0 / max(1, args.steps + args.warmup)))
     for w in range(args.warmup):
         time_oracle(spec, x, per_step, seed=1000 + w)
-    vals, secs, samples = [], [], []
-    for k in range(args.steps):
-        v, dt, sample, cores = time_oracle(spec, x, per_step, seed=k)
-        vals.append(v)
-        secs.append(dt)
-        samples.append(sample)
-    value = float(np.median(vals))
+    runs = [time_oracle(spec, x, per_step, seed=k) for k in range(args.steps)]
+    value = float(np.median([r[key] for r in runs]))
     line = {
-        "impl": "reference", "metric": METRIC, "value": value, "unit": "GB/s",
+        "impl": "reference", "metric": METRIC, "value": value, "unit": unit,
         "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
-        "ms_per_step": float(np.mean(secs)) * 1e3, "higher_is_better": True,
-        "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-        "config": {"workload": spec.name, "l2": "n/a (host)"},
-        "cpu_baseline": {"value": value, "unit": "GB/s", "cores": cores, "kind": "oracle",
-                         "sample": samples[-1]},
-        "e2e": {"value": value, "unit": "GB/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+        "ms_per_step": float(np.mean([r["seconds"] for r in runs])) * 1e3,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+        "data": "synthetic", "config": config_of(spec, world),
+        "cpu_baseline": {"value": value, "unit": unit, "cores": runs[-1]["cores"],
+                         "kind": "oracle", "sample": runs[-1]["sample"]},
+        "e2e": {"value": value, "unit": unit, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
     }
     print(json.dumps(line), flush=True)
 
 
-def run_gpu(args, spec, rank, world, local):
+def kernel_roofline(name: str, avg_ms: float, counts: dict, peaks: dict, workload: str) -> dict:
+    """Roofline record of one kernel: algorithmic work of one launch over its
+    average launch time, against the measured peak (and the nominal one)."""
+    if name == "prefill_tcgen05":
+        achieved = counts["prefill_flops"] / (avg_ms * 1e-3) / 1e12
+        rec = {"bound": "tensor", "achieved": achieved, "peak": peaks["tflops"], "unit": "TFLOP/s",
+               "frac": achieved / peaks["tflops"], "frac_nominal": achieved / NOMINAL_TFLOPS,
+               "peak_source": f"{peaks['source']} bf16 burst (fp16 same rate)",
+               "work": f"{counts['prefill_flops']} FLOP per launch (causal, prefill sequences)"}
+    else:
+        alg = counts["scatter_bytes"] if name == "scatter_kv" else counts["decode_bytes"]
+        achieved = alg / (avg_ms * 1e-3) / 1e9
+        rec = {"bound": "hbm", "achieved": achieved, "peak": peaks["hbm_gbs"], "unit": "GB/s",
+               "frac": achieved / peaks["hbm_gbs"], "frac_nominal": achieved / NOMINAL_HBM_GBS,
+               "peak_source": f"{peaks['source']} copy bandwidth",
+               "work": f"{alg} bytes per launch"}
+    rec["traffic"] = profiled_traffic(name, workload)
+    rec["kernel"] = name
+    rec["kernel_ms"] = avg_ms
+    return rec
+
+
+def measure_workload(args, spec, wl_key, world, dev, steps, e2e=True, cpu=True):
+    """Time one workload: CUDA-graph replays of the whole step (value),
+    traced eager steps (per-kernel times), and optionally the end-to-end step
+    through the public API with host buffers."""
     import torch
     import scatter_kv_b200 as pa
 
-    torch.cuda.set_device(local)
-    dev = torch.device("cuda", local)
     counts = algorithmic_counts(spec)
     peaks = load_peaks()
     x = workloads.generate(spec)
@@ -303,9 +360,10 @@ def run_gpu(args, spec, rank, world, local):
                         kv_heads=spec.kv_heads, head_size=spec.head_size,
                         num_blocks=spec.num_blocks, block_size=spec.block_size,
                         max_blocks_per_seq=x["block_table"].shape[1],
-                        max_seqlen_q=int(spec.q_lens.max()), max_seqlen_kv=int(spec.seqlens_kv.max()))
+                        max_seqlen_q=int(spec.q_lens.max()), max_seqlen_kv=int(spec.seqlens_kv.max()),
+                        min_seqlen_q=int(spec.q_lens[spec.q_lens > 0].min()))
     bufs = pa.allocate(dims, device=dev)
-    scale = pa.default_scale(spec.head_size)
+    scale = 0.0                     # the library's default, 1 / sqrt(head_size)
     stream = torch.cuda.Stream(device=dev)
     flush = torch.empty(2 * L2_BYTES // 4, dtype=torch.int32, device=dev)
     scrub = torch.zeros(2 * L2_BYTES // 4, dtype=torch.int32, device=dev)
@@ -322,13 +380,14 @@ def run_gpu(args, spec, rank, world, local):
         pa.step(d["query"], d["key"], d["value"], d["key_cache"], d["value_cache"],
                 d["block_table"], d["cu_seqlens_q"], d["seqlens_kv"], scale, dims, bufs, stream)
 
+    rec = {}
     with torch.cuda.stream(stream):
         for _ in range(max(3, args.warmup)):
             step()
         stream.synchronize()
         status = int(bufs.status[0].item())
         if status != 0:
-            raise RuntimeError(f"device status {status:#x} on the benchmark inputs")
+            raise RuntimeError(f"device status {status:#x} on the {spec.name} inputs")
 
         # ---- the step as a CUDA graph (launch-bound small kernels replay
         # without host gaps); tracing stays off during capture.
@@ -340,21 +399,20 @@ def run_gpu(args, spec, rank, world, local):
 
         # ---- device-timed region: K graph replays, L2 flushed between steps
         ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
-              for _ in range(args.steps)]
-        clocks = ClockSampler(local)
+              for _ in range(steps)]
+        clocks = ClockSampler(dev.index)
         clocks.start()
         barrier(world, dev)
         torch.cuda.synchronize()
-        for k in range(args.steps):
+        for k in range(steps):
             flush_l2(k)
             ev[k][0].record(stream)
             graph.replay()
             ev[k][1].record(stream)
         torch.cuda.synchronize()
         barrier(world, dev)
-        clk = clocks.stop()
-        ms = sum(a.elapsed_time(b) for a, b in ev)
-        ms = max_over_ranks(ms, world, dev)
+        rec["clocks"] = clocks.stop()
+        ms = max_over_ranks(sum(a.elapsed_time(b) for a, b in ev), world, dev)
 
         # ---- per-kernel durations: K eager steps with the library's event
         # tracing (one event pair around every launch), same flushes.
@@ -362,7 +420,7 @@ def run_gpu(args, spec, rank, world, local):
         pa.pa_trace_enable(True)
         barrier(world, dev)
         torch.cuda.synchronize()
-        for k in range(args.steps):
+        for k in range(steps):
             flush_l2(k)
             step()
         torch.cuda.synchronize()
@@ -370,96 +428,104 @@ def run_gpu(args, spec, rank, world, local):
         trace = pa.pa_trace_read()
 
         # ---- end-to-end through the public API with host buffers
-        host = {k: torch.from_numpy(np.ascontiguousarray(x[k])).pin_memory()
-                for k in ("query", "key", "value", "block_table", "cu_seqlens_q", "seqlens_kv")}
-        out_host = torch.empty(bufs.out.shape, dtype=bufs.out.dtype).pin_memory()
-        h2d = sum(t.numel() * t.element_size() for t in host.values())
-        d2h = out_host.numel() * out_host.element_size()
-        ev2 = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
-               for _ in range(args.steps)]
-        barrier(world, dev)
-        torch.cuda.synchronize()
-        for k in range(args.steps):
-            flush_l2(k)
-            ev2[k][0].record(stream)
-            for name, t in host.items():
-                d[name].copy_(t, non_blocking=True)
-            step()
-            out_host.copy_(bufs.out, non_blocking=True)
-            ev2[k][1].record(stream)
-        torch.cuda.synchronize()
-        barrier(world, dev)
-        ms_e2e = max_over_ranks(sum(a.elapsed_time(b) for a, b in ev2), world, dev)
+        ms_e2e, h2d, d2h = None, 0, 0
+        if e2e:
+            host = {k: torch.from_numpy(np.ascontiguousarray(x[k])).pin_memory()
+                    for k in ("query", "key", "value", "block_table", "cu_seqlens_q", "seqlens_kv")}
+            out_host = torch.empty(bufs.out.shape, dtype=bufs.out.dtype).pin_memory()
+            h2d = sum(t.numel() * t.element_size() for t in host.values())
+            d2h = out_host.numel() * out_host.element_size()
+            ev2 = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+                   for _ in range(steps)]
+            barrier(world, dev)
+            torch.cuda.synchronize()
+            for k in range(steps):
+                flush_l2(k)
+                ev2[k][0].record(stream)
+                for name, t in host.items():
+                    d[name].copy_(t, non_blocking=True)
+                step()
+                out_host.copy_(bufs.out, non_blocking=True)
+                ev2[k][1].record(stream)
+            torch.cuda.synchronize()
+            barrier(world, dev)
+            ms_e2e = max_over_ranks(sum(a.elapsed_time(b) for a, b in ev2), world, dev)
 
-    # ---- roofline of the dominant kernel (from the live trace)
     per_kernel = {}
     for name, t in trace:
         per_kernel.setdefault(name, []).append(t)
-    launches = sum(len(v) for v in per_kernel.values())
     total_k = sum(sum(v) for v in per_kernel.values())
     dominant = max(per_kernel, key=lambda n: sum(per_kernel[n]))
-    avg_ms = float(np.mean(per_kernel[dominant]))
-    wl_key = args.workload
-    if dominant == "prefill_tcgen05":
-        achieved = counts["flops"] / (avg_ms * 1e-3) / 1e12
-        roof = {"bound": "tensor", "achieved": achieved, "peak": peaks["tflops"], "unit": "TFLOP/s",
-                "frac": achieved / peaks["tflops"],
-                "traffic": profiled_traffic(dominant, wl_key),
-                "kernel": dominant, "peak_source": f"{peaks['source']} bf16 burst (fp16 same rate)"}
-    else:
-        alg = counts["kv_bytes"] + counts["q_bytes"]
-        if dominant == "scatter_kv":
-            alg = counts["scatter_bytes"]
-        achieved = alg / (avg_ms * 1e-3) / 1e9
-        roof = {"bound": "hbm", "achieved": achieved, "peak": peaks["hbm_gbs"], "unit": "GB/s",
-                "frac": achieved / peaks["hbm_gbs"],
-                "traffic": profiled_traffic(dominant, wl_key),
-                "kernel": dominant, "peak_source": f"{peaks['source']} copy bandwidth"}
-    roof["kernel_ms"] = avg_ms
+    roof = kernel_roofline(dominant, float(np.mean(per_kernel[dominant])), counts, peaks, wl_key)
     roof["share_of_kernel_time"] = sum(per_kernel[dominant]) / total_k if total_k else None
 
-    if counts["decode"]:
-        unit, value = "GB/s", counts["step_bytes"] * world / (ms / args.steps * 1e-3) / 1e9
-        e2e_value = counts["step_bytes"] * world / (ms_e2e / args.steps * 1e-3) / 1e9
-    else:
-        unit, value = "TFLOP/s", counts["flops"] * world / (ms / args.steps * 1e-3) / 1e12
-        e2e_value = counts["flops"] * world / (ms_e2e / args.steps * 1e-3) / 1e12
+    step_s = ms / steps * 1e-3
+    unit = unit_of(spec)
+    per_sec = (lambda sec: counts["step_bytes"] * world / sec / 1e9) if unit == "GB/s" else \
+        (lambda sec: counts["flops"] * world / sec / 1e12)
+    # The step's own roofline: the slower of its FLOPs at the tensor peak and
+    # its bytes (attention K/V + Q + O, and the scatter's) at HBM bandwidth.
+    flop_us = counts["flops"] / (peaks["tflops"] * 1e12) * 1e6
+    byte_us = counts["step_bytes"] / (peaks["hbm_gbs"] * 1e9) * 1e6
+    rec.update({
+        "value": per_sec(step_s), "unit": unit, "ms_per_step": ms / steps,
+        "tokens_per_s": spec.token_count * world / step_s,
+        "roofline": roof,
+        "step_roofline": {"flop_us": flop_us, "byte_us": byte_us,
+                          "bound": "tensor" if flop_us > byte_us else "hbm",
+                          "frac": max(flop_us, byte_us) / (step_s * 1e6),
+                          "frac_nominal": max(counts["flops"] / (NOMINAL_TFLOPS * 1e12),
+                                              counts["step_bytes"] / (NOMINAL_HBM_GBS * 1e9))
+                          / step_s},
+        "gpu_launches": sum(len(v) for v in per_kernel.values()),
+        "kernels": {n: {"launches": len(v), "avg_ms": float(np.mean(v))}
+                    for n, v in per_kernel.items()},
+        "algorithmic": {k: v for k, v in counts.items() if k != "decode"},
+        "config": config_of(spec, world),
+    })
+    if e2e:
+        rec["e2e"] = {"value": per_sec(ms_e2e / steps * 1e-3), "unit": unit,
+                      "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h}
+    if cpu and world == 1 and not args.no_cpu_baseline:
+        r = time_oracle(spec, x_with_scatter(x, spec), args.cpu_seconds)
+        rec["cpu_baseline"] = {"value": r["gbs"] if unit == "GB/s" else r["tflops"], "unit": unit,
+                               "cores": r["cores"], "kind": "oracle", "sample": r["sample"]}
+    del d, bufs, flush, scrub, graph
+    torch.cuda.empty_cache()
+    return rec
 
-    line = None
-    if rank == 0:
-        cpu = None
-        if world == 1 and not args.no_cpu_baseline:
-            import oracle  # noqa: F401
-            gbs, dt, sample, cores = time_oracle(spec, x_with_scatter(x, spec), args.cpu_seconds)
-            if counts["decode"]:
-                cpu = {"value": gbs, "unit": "GB/s", "cores": cores, "kind": "oracle", "sample": sample}
-            else:
-                # Same sample expressed in the step's unit: FLOPs of the rows run per second.
-                cpu = {"value": gbs * counts["flops"] / max(1, counts["kv_bytes"] + 2 * counts["q_bytes"]) / 1e3,
-                       "unit": "TFLOP/s", "cores": cores, "kind": "oracle",
-                       "sample": sample + " (rate scaled by the workload's FLOP/byte ratio)"}
-        line = {
-            "metric": METRIC, "value": value, "unit": unit, "n_gpus": world, "steps": args.steps,
-            "warmup": args.warmup, "ms_per_step": ms / args.steps, "higher_is_better": True,
-            "scaling": "weak", "vs_baseline": None, "dtype": "f16", "data": "synthetic",
-            "config": {"workload": spec.name, "batch": spec.batch, "tokens": spec.token_count,
-                       "q_heads": spec.q_heads, "kv_heads": spec.kv_heads,
-                       "head_size": spec.head_size, "block_size": spec.block_size,
-                       "num_blocks": spec.num_blocks, "seed": spec.seed,
-                       "l2": "flushed between steps, outside the timed events: 252 MB written, then "
-                             "252 MB read so no dirty line is left to write back",
-                       "parallelism": f"replicas x{world}"},
-            "roofline": roof,
-            "cpu_baseline": cpu,
-            "e2e": {"value": e2e_value, "unit": unit, "h2d_bytes_per_step": h2d,
-                    "d2h_bytes_per_step": d2h},
-            "gpu_launches": launches,
-            "timing": "value: CUDA-graph replays of the step; kernels: eager traced steps",
-            "kernels": {n: {"launches": len(v), "avg_ms": float(np.mean(v))} for n, v in per_kernel.items()},
-            "algorithmic": {k: v for k, v in counts.items() if k != "decode"},
-            "clocks": clk,
-        }
-        print(json.dumps(line), flush=True)
+
+def run_gpu(args, spec, rank, world, local):
+    import torch
+
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    main = measure_workload(args, spec, args.workload, world, dev, args.steps)
+    # The other full-size workloads, measured in the same process and reported
+    # in the same line (each with its own clocks, roofline and CPU baseline).
+    others = {}
+    if not args.only:
+        for key in ("prefill", "mixed", "long_decode", "decode"):
+            if key == args.workload:
+                continue
+            o = workloads.CONFIGS[workloads.CONFIG_KEYS[key]]()
+            others[key] = measure_workload(args, o, key, world, dev, max(10, args.steps // 2),
+                                           e2e=True)
+    if rank != 0:
+        return None
+    line = {
+        "metric": METRIC, "value": main["value"], "unit": main["unit"], "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": main["ms_per_step"],
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f16",
+        "data": "synthetic", "config": main["config"], "roofline": main["roofline"],
+        "step_roofline": main["step_roofline"], "cpu_baseline": main.get("cpu_baseline"),
+        "e2e": main["e2e"], "gpu_launches": main["gpu_launches"],
+        "timing": "value: CUDA-graph replays of the step; kernels: eager traced steps",
+        "kernels": main["kernels"], "algorithmic": main["algorithmic"],
+        "tokens_per_s": main["tokens_per_s"], "clocks": main["clocks"],
+        "workloads": others,
+    }
+    print(json.dumps(line), flush=True)
     return line
 
 
@@ -484,6 +550,8 @@ def main(argv=None):
     ap.add_argument("--workload", default="decode", choices=sorted(workloads.CONFIG_KEYS))
     ap.add_argument("--cpu-seconds", type=float, default=10.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--only", action="store_true",
+                    help="measure only --workload (default: every full-size workload)")
     args = ap.parse_args(argv)
     if args.warmup < 3 and args.impl == "ours":
         args.warmup = 3

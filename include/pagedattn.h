@@ -73,7 +73,12 @@ enum {
  * The hints are optional upper bounds (0 = unknown): max_seqlen_q_hint
  * bounds every q_len_b, max_seqlen_kv_hint every seqlens_kv[b].  They size
  * grids and workspace; a sequence that exceeds a hint is treated as invalid
- * (PA_DEV_HINT_EXCEEDED, zero output rows). */
+ * (PA_DEV_HINT_EXCEEDED, zero output rows).
+ * min_seqlen_q_hint (0 = unknown) is a lower bound on the q_len_b of the
+ * non-empty sequences.  It only routes work: when it exceeds the decode
+ * cut-off, pa_attention launches no decode kernels and every sequence goes
+ * through the prefill kernel, which computes any q_len_b correctly -- so a
+ * wrong lower bound costs speed, never correctness. */
 typedef struct {
     int32_t batch;
     int64_t token_count;
@@ -86,6 +91,7 @@ typedef struct {
     int32_t max_seqlen_q_hint;
     int32_t max_seqlen_kv_hint;
     int32_t dtype;                 /* pa_dtype */
+    int32_t min_seqlen_q_hint;
 } pa_dims;
 
 /* pa_scatter_kv -- write the new tokens' keys and values into the paged caches.
@@ -158,8 +164,9 @@ pa_status pa_attention(const void* query, const void* key_cache, const void* val
  *   Limit: dims whose pa_attention_workspace_size() exceeds 8 MiB are
  *          rejected with PA_ERR_INVALID_ARGUMENT (use pa_attention then).
  *   Set-up: the first call on each device looks up the array's device
- *          address (cudaGetSymbolAddress) with that device current; make that
- *          first call before any stream capture.
+ *          address (cudaGetSymbolAddress) with that device current, and so
+ *          does the first call after the device's context changes (a device
+ *          reset); make such a first call before any stream capture.
  *   Sharing: all calls on a device share the one array and it keeps the
  *          last call's contents (none need clearing: every scratch value is
  *          written before it is read within a call).  Calls whose kernels

@@ -16,7 +16,6 @@ Calls:
 from __future__ import annotations
 
 import ctypes
-import math
 import os
 from dataclasses import dataclass
 
@@ -60,6 +59,7 @@ class pa_dims(ctypes.Structure):
         ("max_seqlen_q_hint", ctypes.c_int32),
         ("max_seqlen_kv_hint", ctypes.c_int32),
         ("dtype", ctypes.c_int32),
+        ("min_seqlen_q_hint", ctypes.c_int32),
     ]
 
 
@@ -149,7 +149,7 @@ def _stream(stream):
 def make_dims(query=None, key_cache=None, block_table=None, cu_seqlens_q=None, *, batch=None,
               token_count=None, q_heads=None, kv_heads=None, head_size=None, num_blocks=None,
               block_size=None, max_blocks_per_seq=None, max_seqlen_q=0, max_seqlen_kv=0,
-              dtype=PA_DTYPE_F16) -> pa_dims:
+              min_seqlen_q=0, dtype=PA_DTYPE_F16) -> pa_dims:
     """pa_dims from tensor shapes (query [T, qh, d], cache [nb, bs, kvh, d],
     block table [B, maxblk], cu_seqlens_q [B + 1]); keywords override."""
     d = pa_dims()
@@ -169,6 +169,7 @@ def make_dims(query=None, key_cache=None, block_table=None, cu_seqlens_q=None, *
             setattr(d, name, int(val))
     d.max_seqlen_q_hint = int(max_seqlen_q)
     d.max_seqlen_kv_hint = int(max_seqlen_kv)
+    d.min_seqlen_q_hint = int(min_seqlen_q)
     d.dtype = int(dtype)
     return d
 
@@ -233,10 +234,6 @@ def pa_trace_read():
     buf = (pa_trace_record * PA_TRACE_CAPACITY)()
     n = lib.pa_trace_read(buf, PA_TRACE_CAPACITY)
     return [(lib.pa_kernel_name(buf[i].kernel).decode(), float(buf[i].ms)) for i in range(n)]
-
-
-def default_scale(head_size: int) -> float:
-    return 1.0 / math.sqrt(head_size)
 
 
 @dataclass

@@ -178,7 +178,7 @@ pa_status check_dims(const pa_dims* dp) {
         return fail(PA_ERR_INVALID_ARGUMENT, "max_blocks_per_seq * block_size must be < 2^31");
     if (d.token_count >= (1ll << 31))
         return fail(PA_ERR_INVALID_ARGUMENT, "token_count must be < 2^31");
-    if (d.max_seqlen_q_hint < 0 || d.max_seqlen_kv_hint < 0)
+    if (d.max_seqlen_q_hint < 0 || d.max_seqlen_kv_hint < 0 || d.min_seqlen_q_hint < 0)
         return fail(PA_ERR_INVALID_ARGUMENT, "negative hint");
     return PA_OK;
 }
@@ -279,8 +279,12 @@ pa_status pa_attention(const void* query, const void* key_cache, const void* val
     const int kv_cap = d.max_blocks_per_seq * d.block_size;
     cudaStream_t s = static_cast<cudaStream_t>(stream);
 
-    // Decode (split-KV) part: sequences with q_len <= plan.decode_max_q.
-    {
+    // Decode (split-KV) part: sequences with q_len <= plan.decode_max_q.  A
+    // lower bound on q_len above the cut-off sends every sequence to the
+    // prefill kernel instead (it handles any q_len), and no decode runs.
+    const bool run_decode = d.min_seqlen_q_hint <= plan.decode_max_q;
+    const int prefill_min_q = run_decode ? plan.decode_max_q : 0;   // prefill takes q_len > this
+    if (run_decode) {
         CUtensorMap tk, tv;
         const int rows = d.block_size < pa::kDecodeKeys ? d.block_size : pa::kDecodeKeys;
         if ((st = make_cache_map(&tk, key_cache, d, rows)) != PA_OK) return st;
@@ -326,9 +330,9 @@ pa_status pa_attention(const void* query, const void* key_cache, const void* val
         }
     }
 
-    // Prefill part: sequences with q_len > plan.decode_max_q.
-    if (d.max_seqlen_q_hint == 0 || d.max_seqlen_q_hint > plan.decode_max_q) {
-        const long long longer = d.token_count / (plan.decode_max_q + 1);
+    // Prefill part: sequences with q_len > prefill_min_q.
+    if (d.max_seqlen_q_hint == 0 || d.max_seqlen_q_hint > prefill_min_q) {
+        const long long longer = d.token_count / (prefill_min_q + 1);
         const long long slots = (d.token_count * g + pa::kPrefillCtaRows - 1) / pa::kPrefillCtaRows +
                                 (longer < d.batch ? longer : d.batch);
         if (slots > 0) {
@@ -358,7 +362,7 @@ pa_status pa_attention(const void* query, const void* key_cache, const void* val
             p.kv_cap = kv_cap;
             p.kv_hint = d.max_seqlen_kv_hint;
             p.q_hint = d.max_seqlen_q_hint;
-            p.decode_max_q = plan.decode_max_q;
+            p.decode_max_q = prefill_min_q;
             p.num_slots = (int)slots;
             p.scale_log2 = scale_log2;
             TraceScope tr(PA_KERNEL_PREFILL, s);

@@ -680,24 +680,53 @@ cudaError_t launch_combine(const DecodeParams& p, int head_size, cudaStream_t st
 // array is part of the library image, so every GPU that loads the library
 // holds these bytes until the process exits.  In host code the symbol is
 // only a host-side stand-in; its device address comes from
-// cudaGetSymbolAddress, looked up once per device.
+// cudaGetSymbolAddress, looked up with the device current.  The address is
+// kept per device together with the CUDA context it was found in: after a
+// device reset the context (and the module image holding the array) is new,
+// so a cached address whose context no longer matches is looked up again.
 static __device__ __align__(256) unsigned char pa_noalloc_scratch[pa::kNoAllocScratchBytes];
 
 namespace pa {
 
+namespace {
+typedef CUresult (*CtxGetCurrentFn)(CUcontext*);
+
+CtxGetCurrentFn ctx_get_current_fn() {
+    static CtxGetCurrentFn fn = nullptr;
+    static std::once_flag once;
+    std::call_once(once, [] {
+        void* p = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuCtxGetCurrent", &p, cudaEnableDefault, &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<CtxGetCurrentFn>(p);
+    });
+    return fn;
+}
+}  // namespace
+
 cudaError_t noalloc_scratch(void** ptr) {
     static std::mutex mu;
     static void* addr[kMaxDevices] = {nullptr};
+    static CUcontext ctx_of[kMaxDevices] = {nullptr};
     int dev = 0;
     cudaError_t e = cudaGetDevice(&dev);
     if (e != cudaSuccess) return e;
     if (dev < 0 || dev >= kMaxDevices) return cudaErrorInvalidDevice;
+    CtxGetCurrentFn get_ctx = ctx_get_current_fn();
+    if (get_ctx == nullptr) return cudaErrorDeviceUninitialized;
+    CUcontext ctx = nullptr;
+    if (get_ctx(&ctx) != CUDA_SUCCESS) ctx = nullptr;
     std::lock_guard<std::mutex> lock(mu);
-    if (addr[dev] == nullptr) {
+    if (ctx == nullptr || addr[dev] == nullptr || ctx_of[dev] != ctx) {
+        // The lookup also makes the device's primary context current on this
+        // thread when none is yet; the context is read again after it.
         void* p = nullptr;
         e = cudaGetSymbolAddress(&p, pa_noalloc_scratch);
         if (e != cudaSuccess) return e;
+        if (get_ctx(&ctx) != CUDA_SUCCESS || ctx == nullptr) return cudaErrorDeviceUninitialized;
         addr[dev] = p;
+        ctx_of[dev] = ctx;
     }
     *ptr = addr[dev];
     return cudaSuccess;

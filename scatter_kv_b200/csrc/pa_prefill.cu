@@ -43,10 +43,7 @@
 // construction.  MMAs of one thread run in order, so S_a of tile j+1 cannot
 // overwrite P_a (which lives in S_a's columns) before P_a V_j has read it,
 // and the commit that signals "S_a of tile j+1 is ready" also covers P_a V_j.
-// exp2 runs on the MUFU unit.  A polynomial exp2 on the FMA pipe
-// (exp2_poly) can take a share of the columns (kPolyEvery); measured on
-// B200 with head size 128 it only adds instructions to a softmax whose cost
-// is set by instruction issue, not by MUFU throughput, so it is off.
+// exp2 runs on the MUFU unit.
 // O is rescaled only when some row maximum of a warp grows by more than 2^8
 // (P stays below 256, exact enough in f16 and fp32 sums), which after the
 // first tiles is rare; the decision is warp-uniform because tcgen05.ld/st
@@ -177,36 +174,6 @@ __device__ bool find_work(const PrefillParams& p, long long slot, Work& w) {
         if (!more) return false;
     }
 }
-
-// 2^x on the FMA pipe, for x <= 8 (x = -inf gives a value below 2^-124,
-// which rounds to 0 in f16).  Range reduction in the style of Cody and
-// Waite: x = n + f with n = round(x) (the 1.5 * 2^23 shifter leaves n in the
-// low mantissa bits) and f in [-1/2, 1/2]; 2^f by a degree-3 polynomial with
-// constant term exactly 1, coefficients fitted here by iteratively
-// reweighted least squares (Lawson) for minimum maximum relative error on
-// [-1/2, 1/2]; 2^n is added to the exponent field.  Maximum relative error
-// about 1.2e-4, under half an f16 ulp (P is rounded to f16 right after).
-__device__ __forceinline__ float exp2_poly(float x) {
-    x = fmaxf(x, -125.f);                          // keeps the exponent field >= 1
-    const float shifter = 12582912.f;              // 1.5 * 2^23
-    const float t = x + shifter;
-    const float f = x - (t - shifter);
-    float p = fmaf(0.05541787f, f, 0.24221125f);
-    p = fmaf(p, f, 0.69319951f);
-    p = fmaf(p, f, 1.0f);
-    return __uint_as_float(__float_as_uint(p) + (__float_as_uint(t) << 23));
-}
-
-// Columns c with (c % kPolyEvery) == kPolyEvery - 1 take exp2_poly
-// (kPolyEvery 0: none).
-#ifndef PA_POLY_EVERY
-#define PA_POLY_EVERY 0
-#endif
-constexpr int kPolyEvery = PA_POLY_EVERY;
-__device__ __forceinline__ bool poly_col(int c) {
-    return kPolyEvery > 0 && (c % (kPolyEvery > 0 ? kPolyEvery : 1)) == kPolyEvery - 1;
-}
-
 
 // Bounded waits of the kernel.  With TMA producers the kernel's hot loop only
 // fits the SM's instruction cache with rolled polling loops (unrolled ones
@@ -682,8 +649,8 @@ prefill_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
                                                scale2, nbase2);
                     float x0, x1;
                     f2_unpack(x2, x0, x1);
-                    const float p0 = poly_col(c) ? exp2_poly(x0) : fast_exp2(x0);
-                    const float p1 = poly_col(c + 1) ? exp2_poly(x1) : fast_exp2(x1);
+                    const float p0 = fast_exp2(x0);
+                    const float p1 = fast_exp2(x1);
                     rs2[(c >> 1) & 1] = f2_add(rs2[(c >> 1) & 1], f2_pack(p0, p1));
                     pk[(c - h) / 2] = pack_half2(p0, p1);
                 }

@@ -37,7 +37,7 @@ def run_gpu(spec: workloads.Spec, x: dict, hints: bool = True, scale: float | No
     dv = to_dev(x)
     dims = dims_for(spec, x, hints)
     bufs = pa.allocate(dims)
-    sc = pa.default_scale(spec.head_size) if scale is None else scale
+    sc = 0.0 if scale is None else scale    # 0: the library's 1 / sqrt(head_size)
     outs = []
     for _ in range(repeat):
         pa.step(dv["query"], dv["key"], dv["value"], dv["key_cache"], dv["value_cache"],

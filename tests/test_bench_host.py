@@ -29,3 +29,20 @@ def test_source_hash_ignores_comments_but_not_code(tmp_path, monkeypatch):
     (csrc / "k.cu").write_text("__global__ void k(int* p) { p[0] = 1; }\n")
     (csrc / "k2.cuh").write_text("#define X 1\n")
     assert bench.kernel_source_hash() != h0
+
+
+def test_algorithmic_counts_split_between_kernels():
+    import workloads
+    # GQA 4 (decode cut-off 4): two decode sequences, one prefill chunk.
+    spec = workloads.custom([1, 4, 10], [100, 20, 5], 8, 2, 16, 16)
+    c = bench.algorithmic_counts(spec)
+    kv = lambda t: t * 2 * 16 * 2 * 2          # K and V rows of 2 KV heads, f16
+    q = lambda n: n * 8 * 16 * 2                # query (or output) rows of 8 heads
+    assert c["kv_bytes"] == kv(101) + kv(24) + kv(15)
+    assert c["decode_bytes"] == kv(101) + kv(24) + q(1) + q(4)
+    assert c["prefill_bytes"] == kv(15) + 2 * q(10)
+    # visible keys: 101 for the first sequence; 21..24; 6..15
+    assert c["flops"] == 4 * 8 * 16 * (101 + sum(range(21, 25)) + sum(range(6, 16)))
+    assert c["prefill_flops"] == 4 * 8 * 16 * sum(range(6, 16))
+    assert not c["decode"] and bench.unit_of(spec) == "TFLOP/s"
+    assert bench.unit_of(workloads.custom([1, 3], [9, 9], 8, 2, 16, 16)) == "GB/s"
