@@ -27,6 +27,7 @@ _lib = None
 
 F16 = 0
 F64 = 1
+BF16 = 2
 
 
 def build(force: bool = False) -> str:
@@ -47,6 +48,8 @@ def _load():
         i32, i64 = ctypes.c_int32, ctypes.c_int64
         lib.oracle_half_to_double.argtypes = [ctypes.c_uint16]
         lib.oracle_half_to_double.restype = ctypes.c_double
+        lib.oracle_bf16_to_double.argtypes = [ctypes.c_uint16]
+        lib.oracle_bf16_to_double.restype = ctypes.c_double
         lib.oracle_scatter_kv.argtypes = [P, P, P, P, P, i64, ctypes.c_int, ctypes.c_int,
                                           ctypes.c_int, ctypes.c_int]
         lib.oracle_slot_mapping.argtypes = [P, P, P, ctypes.c_int, ctypes.c_int, ctypes.c_int,
@@ -55,8 +58,11 @@ def _load():
         lib.oracle_kv_slots.restype = i64
         lib.oracle_attention.argtypes = [P, P, P, P, P, P, ctypes.c_int, i64, ctypes.c_int,
                                          ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_int,
-                                         ctypes.c_double, ctypes.c_int, ctypes.c_int, P, i64,
-                                         P, i64, P]
+                                         ctypes.c_double, ctypes.c_double, ctypes.c_int,
+                                         ctypes.c_int, ctypes.c_int, P, i64, P, i64, P]
+        lib.oracle_token_positions.argtypes = [P, P, ctypes.c_int, i64, P]
+        lib.oracle_rotary.argtypes = [P, i64, ctypes.c_int, ctypes.c_int, i64, P, P, P,
+                                      ctypes.c_int, ctypes.c_int, ctypes.c_int, P]
         lib.oracle_max_threads.restype = ctypes.c_int
         _lib = lib
     return _lib
@@ -77,6 +83,22 @@ def max_threads() -> int:
 
 def half_to_double(bits: int) -> float:
     return float(_load().oracle_half_to_double(int(bits) & 0xFFFF))
+
+
+def bf16_to_double(bits: int) -> float:
+    return float(_load().oracle_bf16_to_double(int(bits) & 0xFFFF))
+
+
+def _elem_type(a: np.ndarray, bf16: bool) -> int:
+    if bf16:
+        if a.dtype != np.uint16:
+            raise TypeError("bfloat16 arrays are passed as uint16 bit patterns")
+        return BF16
+    if a.dtype == np.float16:
+        return F16
+    if a.dtype == np.float64:
+        return F64
+    raise TypeError("oracle takes float16, float64 or (bf16=True) uint16 arrays")
 
 
 def scatter_kv(key, value, slot_mapping, key_cache, value_cache) -> None:
@@ -116,21 +138,20 @@ def kv_slots(block_table, seqlens_kv, block_size: int) -> np.ndarray:
 
 
 def attention(query, key_cache, value_cache, block_table, cu_seqlens_q, seqlens_kv,
-              scale: float, causal: bool = True, rows=None) -> np.ndarray:
+              scale: float, causal: bool = True, rows=None, softcap: float = 0.0,
+              window: int = -1, bf16: bool = False) -> np.ndarray:
     """fp64 paged attention.
 
     query [token_count, q_heads, head_size]; caches [num_blocks, block_size,
-    kv_heads, head_size]; all float16 or all float64.  ``rows``: optional
-    int64 [n, 2] array of (token, q_head) pairs to compute; the result is
-    then [n, head_size], else [token_count, q_heads, head_size] (float64).
+    kv_heads, head_size]; all float16, all float64, or (bf16=True) all
+    bfloat16 bit patterns held as uint16.  ``rows``: optional int64 [n, 2]
+    array of (token, q_head) pairs to compute; the result is then
+    [n, head_size], else [token_count, q_heads, head_size] (float64).
+    ``softcap`` > 0 caps the scaled scores at c * tanh(s / c); ``window`` >= 0
+    lets query position P see only keys [P - window, P].
     """
     lib = _load()
-    if query.dtype == np.float16:
-        dtype = F16
-    elif query.dtype == np.float64:
-        dtype = F64
-    else:
-        raise TypeError("oracle takes float16 or float64 arrays")
+    dtype = _elem_type(query, bf16)
     assert key_cache.dtype == value_cache.dtype == query.dtype
     q = _c(query, query.dtype)
     kc = key_cache if key_cache.flags.c_contiguous else np.ascontiguousarray(key_cache)
@@ -154,6 +175,40 @@ def attention(query, key_cache, value_cache, block_table, cu_seqlens_q, seqlens_
     if nrows:
         lib.oracle_attention(_ptr(q), _ptr(kc), _ptr(vc), _ptr(bt), _ptr(cu), _ptr(skv), len(skv),
                              token_count, q_heads, kv_heads, head_size, bs, bt.shape[1],
-                             float(scale), 1 if causal else 0, dtype, rows_p, nrows,
-                             _ptr(scratch), max_keys, _ptr(out))
+                             float(scale), float(softcap), int(window), 1 if causal else 0, dtype,
+                             rows_p, nrows, _ptr(scratch), max_keys, _ptr(out))
+    return out
+
+
+def token_positions(cu_seqlens_q, seqlens_kv) -> np.ndarray:
+    """Position past_len_b + i of every packed token (int64 [token_count])."""
+    lib = _load()
+    cu = _c(cu_seqlens_q, np.int32)
+    skv = _c(seqlens_kv, np.int32)
+    out = np.empty(int(cu[-1]), dtype=np.int64)
+    lib.oracle_token_positions(_ptr(cu), _ptr(skv), len(skv), out.size, _ptr(out))
+    return out
+
+
+def rotary(x, positions, cos_cache, sin_cache, rotary_dim: int, interleaved: bool,
+           bf16: bool = False) -> np.ndarray:
+    """Rotary embedding of x [token_count, heads, head_size] (any row stride
+    over tokens; heads contiguous) at the given positions; cos/sin caches
+    [max_position, rotary_dim / 2] of x's element type.  Returns float64."""
+    lib = _load()
+    dtype = _elem_type(x, bf16)
+    assert cos_cache.dtype == sin_cache.dtype == x.dtype
+    T, H, d = x.shape
+    assert x.strides[2] == x.itemsize and x.strides[1] == d * x.itemsize
+    assert rotary_dim % 2 == 0 and 0 <= rotary_dim <= d
+    assert cos_cache.shape[1] == rotary_dim // 2 and cos_cache.shape == sin_cache.shape
+    pos = _c(positions, np.int64)
+    assert pos.size == T and (T == 0 or (pos.min() >= 0 and pos.max() < cos_cache.shape[0]))
+    cc = _c(cos_cache, cos_cache.dtype)
+    sc = _c(sin_cache, sin_cache.dtype)
+    out = np.empty((T, H, d), dtype=np.float64)
+    if T:
+        base = x.ctypes.data_as(ctypes.c_void_p)
+        lib.oracle_rotary(base, T, H, d, x.strides[0] // x.itemsize, _ptr(pos), _ptr(cc), _ptr(sc),
+                          rotary_dim, 1 if interleaved else 0, dtype, _ptr(out))
     return out

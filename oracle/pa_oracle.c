@@ -35,9 +35,29 @@
  *    specifically checked"): the sequence of packed token t is the first b
  *    with cu_seqlens_q[b+1] > t, which skips zero-length sequences.
  *
- * Arithmetic: every floating-point value is taken to fp64 exactly (binary16
- * and binary32 are subsets of binary64) and all sums run in increasing key
- * order, so the result does not depend on where pages sit in the pool.
+ *  - Score modifiers (FlexAttention doc, "FlexAttention Computation": the
+ *    scores are scaled first, then score_mod runs, then the softmax; the
+ *    "Modifier Subgraphs" section adds that masking is a score_mod writing
+ *    -inf).  The PagedAttention PR ("Description") names the two it leaves
+ *    for later, softcap and local_window_size, without defining them; the
+ *    readings taken here are the usual ones: softcap c > 0 replaces a scaled
+ *    score s by c * tanh(s / c); a local window w >= 0 keeps, for query
+ *    position P = past_len_b + i, only the keys j with P - w <= j <= P (the
+ *    w keys before the query and its own), masking the rest.
+ *
+ *  - Rotary embedding (the same PR's "split packed QKV" and "rotary"
+ *    programs; its review checks "interleaved/split pairing + sign + h >=
+ *    rotary_dim pass-through").  Token i of sequence b sits at position
+ *    past_len_b + i.  With cos/sin caches [max_position, rotary_dim / 2] and
+ *    pair index m < rotary_dim / 2, the pair (x1, x2) -- elements (m,
+ *    m + rotary_dim/2) in split pairing, (2m, 2m+1) in interleaved pairing --
+ *    becomes (x1 cos - x2 sin, x2 cos + x1 sin), a rotation by the pair's
+ *    angle; elements at or past rotary_dim pass through unchanged.
+ *
+ * Arithmetic: every floating-point value is taken to fp64 exactly (binary16,
+ * bfloat16 and binary32 are subsets of binary64) and all sums run in
+ * increasing key order, so the result does not depend on where pages sit in
+ * the pool.
  * Scores use fp64 throughout; the maximum is subtracted before exp() as the
  * textbook softmax does (it changes nothing in exact arithmetic).
  *
@@ -51,6 +71,7 @@
 
 #define ORACLE_F16 0
 #define ORACLE_F64 1
+#define ORACLE_BF16 2
 
 /* IEEE 754 binary16 -> binary64, written from the format's definition:
  * 1 sign bit, 5 exponent bits (bias 15), 10 fraction bits. */
@@ -70,22 +91,45 @@ double oracle_half_to_double(uint16_t h)
     return sign ? -v : v;
 }
 
+/* bfloat16 -> binary64, from the format's definition: the upper half of a
+ * binary32, i.e. 1 sign bit, 8 exponent bits (bias 127), 7 fraction bits. */
+double oracle_bf16_to_double(uint16_t h)
+{
+    int sign = (h >> 15) & 1;
+    int e = (h >> 7) & 0xff;
+    int f = h & 0x7f;
+    double v;
+    if (e == 0) {
+        v = ldexp((double)f, -133);              /* zero / subnormal: f * 2^-7 * 2^-126 */
+    } else if (e == 255) {
+        v = (f == 0) ? INFINITY : NAN;
+    } else {
+        v = ldexp((double)(128 + f), e - 134);   /* (1 + f/128) * 2^(e-127) */
+    }
+    return sign ? -v : v;
+}
+
 /* Every binary16 pattern's value, filled from oracle_half_to_double before
  * the first attention call: a table lookup returns exactly what the function
  * would, only faster (the attention loops decode each element many times). */
 static double half_table[65536];
+static double bf16_table[65536];
 static int half_table_ready = 0;
 
 static void fill_half_table(void)
 {
     if (half_table_ready) return;
-    for (int i = 0; i < 65536; ++i) half_table[i] = oracle_half_to_double((uint16_t)i);
+    for (int i = 0; i < 65536; ++i) {
+        half_table[i] = oracle_half_to_double((uint16_t)i);
+        bf16_table[i] = oracle_bf16_to_double((uint16_t)i);
+    }
     half_table_ready = 1;
 }
 
 static double load(const void *base, int64_t idx, int dtype)
 {
     if (dtype == ORACLE_F64) return ((const double *)base)[idx];
+    if (dtype == ORACLE_BF16) return bf16_table[((const uint16_t *)base)[idx]];
     return half_table[((const uint16_t *)base)[idx]];
 }
 
@@ -156,32 +200,36 @@ static void attention_row(const void *query, const void *key_cache, const void *
                           const int32_t *block_table, const int32_t *cu_seqlens_q,
                           const int32_t *seqlens_kv, int batch, int q_heads, int kv_heads,
                           int head_size, int block_size, int max_blocks_per_seq, double scale,
-                          int causal, int dtype, int64_t t, int h, double *scores, double *y)
+                          double softcap, int window, int causal, int dtype, int64_t t, int h,
+                          double *scores, double *y)
 {
     int b = seq_of_token(cu_seqlens_q, batch, t);
     int64_t q_len = cu_seqlens_q[b + 1] - cu_seqlens_q[b];
     int64_t total = seqlens_kv[b];
     int64_t past = total - q_len;
     int64_t i = t - cu_seqlens_q[b];
-    int64_t nkeys = causal ? past + i + 1 : total;       /* keys [0, nkeys) */
+    int64_t nkeys = causal ? past + i + 1 : total;       /* keys [first, nkeys) */
+    int64_t first = 0;
+    if (window >= 0 && past + i - window > 0) first = past + i - window;
     int group = q_heads / kv_heads;
     int kvh = h / group;
     int64_t qbase = (t * q_heads + h) * (int64_t)head_size;
 
     double m = -INFINITY;
-    for (int64_t j = 0; j < nkeys; ++j) {
+    for (int64_t j = first; j < nkeys; ++j) {
         int64_t block = block_table[(int64_t)b * max_blocks_per_seq + j / block_size];
         int64_t kbase = ((block * block_size + j % block_size) * kv_heads + kvh) * (int64_t)head_size;
         double s = 0.0;
         for (int d = 0; d < head_size; ++d)
             s += load(query, qbase + d, dtype) * load(key_cache, kbase + d, dtype);
         s *= scale;
+        if (softcap > 0.0) s = softcap * tanh(s / softcap);
         scores[j] = s;
         if (s > m) m = s;
     }
     double denom = 0.0;
     for (int d = 0; d < head_size; ++d) y[d] = 0.0;
-    for (int64_t j = 0; j < nkeys; ++j) {
+    for (int64_t j = first; j < nkeys; ++j) {
         double p = exp(scores[j] - m);
         denom += p;
         int64_t block = block_table[(int64_t)b * max_blocks_per_seq + j / block_size];
@@ -197,13 +245,17 @@ static void attention_row(const void *query, const void *key_cache, const void *
  * as int64 [nrows, 2]; rows == NULL means every (token, head) in order.
  * out: [nrows, head_size] doubles.  scratch: max_keys doubles per thread
  * (callers pass max_keys >= the longest sequence).  causal = 0 attends to all
- * seqlens_kv[b] keys (only used for the FlexAttention worked examples). */
+ * seqlens_kv[b] keys (only used for the FlexAttention worked examples).
+ * softcap > 0 caps the scaled scores (c * tanh(s / c)); window >= 0 limits
+ * each query to its window (both as in the file header); 0 and -1 turn them
+ * off. */
 void oracle_attention(const void *query, const void *key_cache, const void *value_cache,
                       const int32_t *block_table, const int32_t *cu_seqlens_q,
                       const int32_t *seqlens_kv, int batch, int64_t token_count, int q_heads,
                       int kv_heads, int head_size, int block_size, int max_blocks_per_seq,
-                      double scale, int causal, int dtype, const int64_t *rows, int64_t nrows,
-                      double *scratch, int64_t max_keys, double *out)
+                      double scale, double softcap, int window, int causal, int dtype,
+                      const int64_t *rows, int64_t nrows, double *scratch, int64_t max_keys,
+                      double *out)
 {
     if (rows == NULL) nrows = token_count * q_heads;
     fill_half_table();
@@ -221,7 +273,50 @@ void oracle_attention(const void *query, const void *key_cache, const void *valu
             int h = rows ? (int)rows[2 * r + 1] : (int)(r % q_heads);
             attention_row(query, key_cache, value_cache, block_table, cu_seqlens_q, seqlens_kv,
                           batch, q_heads, kv_heads, head_size, block_size, max_blocks_per_seq,
-                          scale, causal, dtype, t, h, scores, out + r * head_size);
+                          scale, softcap, window, causal, dtype, t, h, scores,
+                          out + r * head_size);
+        }
+    }
+}
+
+/* Position of every packed token: token t of sequence b (local index i)
+ * sits at past_len_b + i, past_len_b = seqlens_kv[b] - q_len_b. */
+void oracle_token_positions(const int32_t *cu_seqlens_q, const int32_t *seqlens_kv, int batch,
+                            int64_t token_count, int64_t *positions)
+{
+    for (int64_t t = 0; t < token_count; ++t) {
+        int b = seq_of_token(cu_seqlens_q, batch, t);
+        int64_t q_len = cu_seqlens_q[b + 1] - cu_seqlens_q[b];
+        positions[t] = seqlens_kv[b] - q_len + (t - cu_seqlens_q[b]);
+    }
+}
+
+/* Rotary embedding of `heads` head vectors per token (file header).
+ * x: token t's head h starts at element t * row_stride + h * head_size;
+ * cos_cache / sin_cache: [max_position, rotary_dim / 2]; all three of
+ * element type dtype.  out: [token_count, heads, head_size] doubles. */
+void oracle_rotary(const void *x, int64_t token_count, int heads, int head_size,
+                   int64_t row_stride, const int64_t *positions, const void *cos_cache,
+                   const void *sin_cache, int rotary_dim, int interleaved, int dtype, double *out)
+{
+    fill_half_table();
+    int half = rotary_dim / 2;
+    for (int64_t t = 0; t < token_count; ++t) {
+        int64_t pos = positions[t];
+        for (int h = 0; h < heads; ++h) {
+            int64_t src = t * row_stride + (int64_t)h * head_size;
+            double *y = out + (t * heads + h) * (int64_t)head_size;
+            for (int e = rotary_dim; e < head_size; ++e) y[e] = load(x, src + e, dtype);
+            for (int m = 0; m < half; ++m) {
+                int e1 = interleaved ? 2 * m : m;
+                int e2 = interleaved ? 2 * m + 1 : m + half;
+                double x1 = load(x, src + e1, dtype);
+                double x2 = load(x, src + e2, dtype);
+                double c = load(cos_cache, pos * half + m, dtype);
+                double sn = load(sin_cache, pos * half + m, dtype);
+                y[e1] = x1 * c - x2 * sn;
+                y[e2] = x2 * c + x1 * sn;
+            }
         }
     }
 }
