@@ -62,8 +62,9 @@ enum {
     PA_DEV_BAD_BLOCK      = 1 << 3,  /* a block_table entry in use is outside [0, num_blocks) */
     PA_DEV_BAD_SLOT       = 1 << 4,  /* a slot_mapping entry >= num_blocks * block_size */
     PA_DEV_TIMEOUT        = 1 << 5,  /* a bounded in-kernel wait gave up (never expected) */
-    PA_DEV_HINT_EXCEEDED  = 1 << 6   /* a sequence is longer than max_seqlen_q_hint or
+    PA_DEV_HINT_EXCEEDED  = 1 << 6,  /* a sequence is longer than max_seqlen_q_hint or
                                         max_seqlen_kv_hint */
+    PA_DEV_BAD_POSITION   = 1 << 7   /* a token's position is past the rotary caches' rows */
 };
 
 /* Problem dimensions, all host-known.  token_count = cu_seqlens_q[batch].
@@ -123,6 +124,54 @@ pa_status pa_scatter_kv(const void* key, const void* value, const int32_t* slot_
 pa_status pa_compute_slot_mapping(const int32_t* block_table, const int32_t* cu_seqlens_q,
                                   const int32_t* seqlens_kv, int32_t* slot_mapping,
                                   const pa_dims* dims, int32_t* dev_status, void* stream);
+
+/* Rotary embedding parameters of pa_split_qkv_rotary_scatter. */
+typedef struct {
+    int32_t rotary_dim;            /* rotated leading elements of each head, a multiple of 16 in
+                                      [0, head_size]; 0 = no rotation (split and scatter only) */
+    int32_t interleaved;           /* 1: pairs (2m, 2m + 1); 0: pairs (m, m + rotary_dim / 2) */
+    int64_t max_position;          /* rows of cos_cache and sin_cache */
+} pa_rotary;
+
+/* pa_split_qkv_rotary_scatter -- the new tokens' Q, K and V, from one packed
+ * QKV projection or from three tensors, in one pass: rotary embedding of Q
+ * and K, Q written out, K and V scattered into the paged caches.
+ * PR "[WebGPU] Initial PagedAttention implementation (1/n)": Copilot's file
+ * summary ("split packed QKV", "rotary", "scatter K/V into the paged cache")
+ * and the review's "Things I specifically checked" (rotary interleaved /
+ * split pairing, sign, pass-through for h >= rotary_dim; scatter block
+ * addressing).
+ *   query, key, value: token t's heads start at query + t * q_token_stride
+ *          (q_heads heads of head_size contiguous elements) and at key / value
+ *          + t * kv_token_stride (kv_heads heads each).  A packed QKV tensor
+ *          [token_count, q_heads + 2 kv_heads, head_size] passes
+ *          query = qkv, key = qkv + q_heads * head_size, value = key +
+ *          kv_heads * head_size, both strides (q_heads + 2 kv_heads) *
+ *          head_size.  Strides are in elements, multiples of 8; 0 = dense.
+ *          Element type: dims->dtype (f16 or bf16), read only.
+ *   cos_cache, sin_cache: [max_position, rotary_dim / 2], dims->dtype; may be
+ *          NULL when rotary is NULL or rotary_dim is 0.
+ *   Token t of sequence b (local index i) is at position p = seqlens_kv[b] -
+ *   q_len_b + i.  Each pair (x1, x2) of a Q or K head becomes (x1 cos - x2
+ *   sin, x2 cos + x1 sin) with cos / sin = cache[p][m] for pair index m;
+ *   elements from rotary_dim on are copied.  fp32 arithmetic, rounded to
+ *   nearest-even.
+ *   query_out: [token_count, q_heads, head_size] (rotated Q), written.
+ *   key_cache, value_cache: as for pa_scatter_kv; rotated K and V land in
+ *          slot block_table[b][p / block_size] * block_size + p % block_size.
+ *   slot_mapping: optional [token_count] int32 output of those slots (-1
+ *          for a token with invalid metadata); may be NULL.
+ * A token whose sequence fails the device checks, or whose position is not
+ * below max_position (PA_DEV_BAD_POSITION), gets zero query_out rows and no
+ * cache write.  token_count == 0 is a valid no-op. */
+pa_status pa_split_qkv_rotary_scatter(const void* query, const void* key, const void* value,
+                                      int64_t q_token_stride, int64_t kv_token_stride,
+                                      const void* cos_cache, const void* sin_cache,
+                                      const pa_rotary* rotary, const int32_t* block_table,
+                                      const int32_t* cu_seqlens_q, const int32_t* seqlens_kv,
+                                      void* query_out, void* key_cache, void* value_cache,
+                                      int32_t* slot_mapping, const pa_dims* dims,
+                                      int32_t* dev_status, void* stream);
 
 /* pa_attention_workspace_size -- device workspace bytes pa_attention needs for
  * these dims (split-KV partial results of the decode path).  *bytes may be 0. */
@@ -206,7 +255,8 @@ enum {
     PA_KERNEL_DECODE = 2,
     PA_KERNEL_COMBINE = 3,
     PA_KERNEL_PREFILL = 4,
-    PA_KERNEL_COUNT = 5
+    PA_KERNEL_QKV_ROTARY = 5,
+    PA_KERNEL_COUNT = 6
 };
 
 pa_status pa_trace_enable(int on);

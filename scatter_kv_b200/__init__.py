@@ -37,12 +37,14 @@ PA_DEV_BAD_BLOCK = 1 << 3
 PA_DEV_BAD_SLOT = 1 << 4
 PA_DEV_TIMEOUT = 1 << 5
 PA_DEV_HINT_EXCEEDED = 1 << 6
+PA_DEV_BAD_POSITION = 1 << 7
 
 PA_KERNEL_SCATTER = 0
 PA_KERNEL_SLOT_MAPPING = 1
 PA_KERNEL_DECODE = 2
 PA_KERNEL_COMBINE = 3
 PA_KERNEL_PREFILL = 4
+PA_KERNEL_QKV_ROTARY = 5
 PA_TRACE_CAPACITY = 4096
 
 
@@ -63,6 +65,14 @@ class pa_dims(ctypes.Structure):
     ]
 
 
+class pa_rotary(ctypes.Structure):
+    _fields_ = [
+        ("rotary_dim", ctypes.c_int32),
+        ("interleaved", ctypes.c_int32),
+        ("max_position", ctypes.c_int64),
+    ]
+
+
 class pa_trace_record(ctypes.Structure):
     _fields_ = [("kernel", ctypes.c_int32), ("ms", ctypes.c_float)]
 
@@ -76,7 +86,7 @@ class PagedAttentionError(RuntimeError):
 EXPORTS = [
     "pa_scatter_kv", "pa_compute_slot_mapping", "pa_attention_workspace_size", "pa_attention",
     "pa_get_status", "pa_status_string", "pa_last_error", "pa_trace_enable", "pa_trace_read",
-    "pa_kernel_name", "pa_attention_noalloc",
+    "pa_kernel_name", "pa_attention_noalloc", "pa_split_qkv_rotary_scatter",
 ]
 
 # Bytes of the fixed scratch array behind pa_attention_noalloc.
@@ -101,6 +111,10 @@ def _load():
     lib.pa_attention.restype = ctypes.c_int
     lib.pa_attention_noalloc.argtypes = [P, P, P, P, P, P, ctypes.c_float, P, D, P, P]
     lib.pa_attention_noalloc.restype = ctypes.c_int
+    lib.pa_split_qkv_rotary_scatter.argtypes = [P, P, P, ctypes.c_int64, ctypes.c_int64, P, P,
+                                                ctypes.POINTER(pa_rotary), P, P, P, P, P, P, P,
+                                                D, P, P]
+    lib.pa_split_qkv_rotary_scatter.restype = ctypes.c_int
     lib.pa_get_status.argtypes = [P, I32P, P]
     lib.pa_get_status.restype = ctypes.c_int
     lib.pa_status_string.argtypes = [ctypes.c_int]
@@ -217,6 +231,32 @@ def pa_attention_noalloc(query, key_cache, value_cache, block_table, cu_seqlens_
                                     _ptr(block_table), _ptr(cu_seqlens_q), _ptr(seqlens_kv),
                                     float(scale), _ptr(out), ctypes.byref(dims), _ptr(dev_status),
                                     _stream(stream)))
+
+
+def pa_split_qkv_rotary_scatter(query, key, value, q_token_stride, kv_token_stride, cos_cache,
+                                sin_cache, rotary: pa_rotary, block_table, cu_seqlens_q,
+                                seqlens_kv, query_out, key_cache, value_cache, slot_mapping,
+                                dims: pa_dims, dev_status=None, stream=None) -> None:
+    """query / key / value: tensors or raw device addresses (ints), with the
+    token strides in elements (0 = dense)."""
+    _check(lib.pa_split_qkv_rotary_scatter(
+        _ptr(query), _ptr(key), _ptr(value), int(q_token_stride), int(kv_token_stride),
+        _ptr(cos_cache), _ptr(sin_cache), ctypes.byref(rotary) if rotary is not None else None,
+        _ptr(block_table), _ptr(cu_seqlens_q), _ptr(seqlens_kv), _ptr(query_out), _ptr(key_cache),
+        _ptr(value_cache), _ptr(slot_mapping), ctypes.byref(dims), _ptr(dev_status),
+        _stream(stream)))
+
+
+def packed_qkv_views(qkv, dims: pa_dims):
+    """(query, key, value, stride) addresses of a packed QKV tensor
+    [token_count, q_heads + 2 kv_heads, head_size] for
+    pa_split_qkv_rotary_scatter."""
+    esz = qkv.element_size()
+    base = qkv.data_ptr()
+    hd = dims.head_size
+    stride = (dims.q_heads + 2 * dims.kv_heads) * hd
+    return (base, base + dims.q_heads * hd * esz,
+            base + (dims.q_heads + dims.kv_heads) * hd * esz, stride)
 
 
 def pa_get_status(dev_status, stream=None) -> int:

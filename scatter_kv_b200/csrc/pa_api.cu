@@ -151,9 +151,8 @@ struct TraceScope {
 pa_status check_dims(const pa_dims* dp) {
     if (dp == nullptr) return fail(PA_ERR_INVALID_ARGUMENT, "dims is NULL");
     const pa_dims& d = *dp;
-    if (d.dtype == PA_DTYPE_BF16)
-        return fail(PA_ERR_NOT_IMPLEMENTED, "bfloat16 is not implemented (f16 only)");
-    if (d.dtype != PA_DTYPE_F16) return fail(PA_ERR_INVALID_ARGUMENT, "unknown dtype %d", d.dtype);
+    if (d.dtype != PA_DTYPE_F16 && d.dtype != PA_DTYPE_BF16)
+        return fail(PA_ERR_INVALID_ARGUMENT, "unknown dtype %d", d.dtype);
     if (d.batch < 0 || d.token_count < 0)
         return fail(PA_ERR_INVALID_ARGUMENT, "negative batch or token_count");
     if (d.batch > 65535) return fail(PA_ERR_NOT_IMPLEMENTED, "batch %d > 65535", d.batch);
@@ -256,6 +255,8 @@ pa_status pa_attention(const void* query, const void* key_cache, const void* val
     pa_status st = check_dims(dims);
     if (st != PA_OK) return st;
     const pa_dims& d = *dims;
+    if (d.dtype == PA_DTYPE_BF16)
+        return fail(PA_ERR_NOT_IMPLEMENTED, "bfloat16 attention is not implemented (f16 only)");
     if (d.token_count == 0) return PA_OK;
     if (d.batch == 0) return fail(PA_ERR_INVALID_ARGUMENT, "token_count > 0 with batch 0");
     if (!(scale >= 0.f) || isinf(scale))
@@ -395,6 +396,82 @@ pa_status pa_attention_noalloc(const void* query, const void* key_cache, const v
                         out, dims, scratch, need, dev_status, stream);
 }
 
+pa_status pa_split_qkv_rotary_scatter(const void* query, const void* key, const void* value,
+                                      int64_t q_token_stride, int64_t kv_token_stride,
+                                      const void* cos_cache, const void* sin_cache,
+                                      const pa_rotary* rotary, const int32_t* block_table,
+                                      const int32_t* cu_seqlens_q, const int32_t* seqlens_kv,
+                                      void* query_out, void* key_cache, void* value_cache,
+                                      int32_t* slot_mapping, const pa_dims* dims,
+                                      int32_t* dev_status, void* stream) {
+    g_last_error[0] = 0;
+    pa_status st = check_dims(dims);
+    if (st != PA_OK) return st;
+    const pa_dims& d = *dims;
+    const int rd = rotary ? rotary->rotary_dim : 0;
+    if (rd < 0 || rd > d.head_size || rd % 2 != 0)
+        return fail(PA_ERR_INVALID_ARGUMENT, "rotary_dim %d must be even and in [0, head_size]", rd);
+    if (rd % 16 != 0)
+        return fail(PA_ERR_NOT_IMPLEMENTED, "rotary_dim %d: only multiples of 16", rd);
+    if (rd > 0 && rotary->max_position <= 0)
+        return fail(PA_ERR_INVALID_ARGUMENT, "max_position must be positive with rotary_dim > 0");
+    if (d.token_count == 0) return PA_OK;
+    if (d.batch == 0) return fail(PA_ERR_INVALID_ARGUMENT, "token_count > 0 with batch 0");
+    const long long qs = q_token_stride ? q_token_stride : (long long)d.q_heads * d.head_size;
+    const long long ks = kv_token_stride ? kv_token_stride : (long long)d.kv_heads * d.head_size;
+    if (qs < (long long)d.q_heads * d.head_size || ks < (long long)d.kv_heads * d.head_size ||
+        qs % 8 != 0 || ks % 8 != 0)
+        return fail(PA_ERR_INVALID_ARGUMENT,
+                    "token strides (%lld, %lld) must cover the heads and be multiples of 8 elements",
+                    qs, ks);
+    PA_REQUIRE_PTR(query);
+    PA_REQUIRE_PTR(key);
+    PA_REQUIRE_PTR(value);
+    PA_REQUIRE_PTR(query_out);
+    PA_REQUIRE_PTR(key_cache);
+    PA_REQUIRE_PTR(value_cache);
+    PA_REQUIRE_IPTR(block_table);
+    PA_REQUIRE_IPTR(cu_seqlens_q);
+    PA_REQUIRE_IPTR(seqlens_kv);
+    if (slot_mapping != nullptr) PA_REQUIRE_IPTR(slot_mapping);
+    if (rd > 0) {
+        PA_REQUIRE_PTR(cos_cache);
+        PA_REQUIRE_PTR(sin_cache);
+    }
+    pa::QkvParams p{};
+    p.q_src = static_cast<const uint16_t*>(query);
+    p.k_src = static_cast<const uint16_t*>(key);
+    p.v_src = static_cast<const uint16_t*>(value);
+    p.q_stride = qs;
+    p.kv_stride = ks;
+    p.cos = static_cast<const uint16_t*>(cos_cache);
+    p.sin = static_cast<const uint16_t*>(sin_cache);
+    p.rotary_dim = rd;
+    p.interleaved = (rotary && rotary->interleaved) ? 1 : 0;
+    p.max_position = rd > 0 ? rotary->max_position : 0;
+    p.block_table = block_table;
+    p.cu_seqlens_q = cu_seqlens_q;
+    p.seqlens_kv = seqlens_kv;
+    p.query_out = static_cast<uint16_t*>(query_out);
+    p.key_cache = static_cast<uint16_t*>(key_cache);
+    p.value_cache = static_cast<uint16_t*>(value_cache);
+    p.slot_out = slot_mapping;
+    p.status = dev_status;
+    p.token_count = d.token_count;
+    p.num_blocks = d.num_blocks;
+    p.batch = d.batch;
+    p.q_heads = d.q_heads;
+    p.kv_heads = d.kv_heads;
+    p.head_size = d.head_size;
+    p.block_size = d.block_size;
+    p.max_blocks = d.max_blocks_per_seq;
+    p.kv_cap = d.max_blocks_per_seq * d.block_size;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    TraceScope tr(PA_KERNEL_QKV_ROTARY, s);
+    cudaError_t e = pa::launch_qkv_rotary_scatter(p, d.dtype == PA_DTYPE_BF16, s);
+    return e == cudaSuccess ? PA_OK : cuda_fail(e, "split-QKV rotary scatter launch");
+}
+
 pa_status pa_get_status(const int32_t* dev_status, int32_t* host_code, void* stream) {
     g_last_error[0] = 0;
     if (dev_status == nullptr || host_code == nullptr)
@@ -445,6 +522,7 @@ const char* pa_kernel_name(int32_t kernel) {
         case PA_KERNEL_DECODE: return "decode_split_kv";
         case PA_KERNEL_COMBINE: return "decode_combine";
         case PA_KERNEL_PREFILL: return "prefill_tcgen05";
+        case PA_KERNEL_QKV_ROTARY: return "qkv_rotary_scatter";
     }
     return "unknown";
 }

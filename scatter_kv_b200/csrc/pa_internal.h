@@ -64,6 +64,40 @@ struct PrefillParams {
     float scale_log2;
 };
 
+// The fused split-QKV + rotary + scatter pass (16-bit elements held as
+// uint16_t; the kernel reads them as f16 or bf16).
+struct QkvParams {
+    const uint16_t* q_src;        // token t's Q heads start at q_src + t * q_stride
+    const uint16_t* k_src;        // token t's K heads start at k_src + t * kv_stride
+    const uint16_t* v_src;        // token t's V heads start at v_src + t * kv_stride
+    long long q_stride;
+    long long kv_stride;
+    const uint16_t* cos;          // [max_position, rotary_dim / 2] (unused when rotary_dim == 0)
+    const uint16_t* sin;
+    int rotary_dim;               // 0: no rotation
+    int interleaved;
+    long long max_position;
+    const int32_t* block_table;
+    const int32_t* cu_seqlens_q;
+    const int32_t* seqlens_kv;
+    uint16_t* query_out;          // [token_count, q_heads, head_size]
+    uint16_t* key_cache;          // [num_blocks, block_size, kv_heads, head_size]
+    uint16_t* value_cache;
+    int32_t* slot_out;            // [token_count] or NULL
+    int32_t* status;
+    long long token_count;
+    long long num_blocks;
+    int batch;
+    int q_heads;
+    int kv_heads;
+    int head_size;
+    int block_size;
+    int max_blocks;
+    int kv_cap;
+};
+
+cudaError_t launch_qkv_rotary_scatter(const QkvParams& p, bool bf16, cudaStream_t stream);
+
 struct DecodePlan {
     int decode_max_q;
     int mtiles;                   // 1 or 2 (16 query rows each)

@@ -67,12 +67,46 @@ def test_dims_rejected_before_launch(pa, kw, status):
     assert e.value.status == status
 
 
-def test_bf16_is_not_implemented(pa):
+def test_bf16_attention_is_not_implemented(pa):
     d = _dims(pa, dtype=pa.PA_DTYPE_BF16)
     with pytest.raises(pa.PagedAttentionError) as e:
-        pa.pa_scatter_kv(FAKE, FAKE, FAKE, FAKE, FAKE, d, None, 0)
+        pa.pa_attention(FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, 0.0, FAKE, d, FAKE, 1 << 30, None, 0)
     assert e.value.status == pa.PA_ERR_NOT_IMPLEMENTED
     assert "bfloat16" in str(e.value)
+
+
+def _rotary(pa, rd, inter=0, maxpos=64):
+    r = pa.pa_rotary()
+    r.rotary_dim, r.interleaved, r.max_position = rd, inter, maxpos
+    return r
+
+
+@pytest.mark.parametrize("rd,maxpos,qs,status,text", [
+    (15, 64, 0, 1, "rotary_dim"),        # odd
+    (136, 64, 0, 1, "rotary_dim"),       # beyond head_size
+    (24, 64, 0, 2, "multiples of 16"),   # even, valid per the pages, not built
+    (64, 0, 0, 1, "max_position"),
+    (64, 64, 8 * 128 - 8, 1, "strides"),  # stride shorter than the query heads
+    (64, 64, 8 * 128 + 4, 1, "strides"),  # not a multiple of 8 elements
+])
+def test_split_qkv_rotary_rejects_bad_arguments(pa, rd, maxpos, qs, status, text):
+    d = _dims(pa)
+    with pytest.raises(pa.PagedAttentionError) as e:
+        pa.pa_split_qkv_rotary_scatter(FAKE, FAKE, FAKE, qs, 0, FAKE, FAKE, _rotary(pa, rd, 0, maxpos),
+                                       FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, None, d, None, 0)
+    assert e.value.status == status
+    assert text in str(e.value)
+
+
+def test_split_qkv_rotary_needs_caches_only_with_rotation(pa):
+    d = _dims(pa)
+    with pytest.raises(pa.PagedAttentionError) as e:
+        pa.pa_split_qkv_rotary_scatter(FAKE, FAKE, FAKE, 0, 0, None, FAKE, _rotary(pa, 64), FAKE,
+                                       FAKE, FAKE, FAKE, FAKE, FAKE, None, d, None, 0)
+    assert "cos_cache" in str(e.value)
+    # token_count 0: nothing to do, nothing read.
+    pa.pa_split_qkv_rotary_scatter(None, None, None, 0, 0, None, None, None, None, None, None,
+                                   None, None, None, None, _dims(pa, token_count=0), None, 0)
 
 
 def test_null_and_misaligned_pointers(pa):
