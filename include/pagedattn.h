@@ -93,6 +93,11 @@ typedef struct {
     int32_t max_seqlen_kv_hint;
     int32_t dtype;                 /* pa_dtype */
     int32_t min_seqlen_q_hint;
+    float softcap;                 /* > 0: each scaled score s becomes softcap * tanh(s / softcap)
+                                      before the softmax; 0 = off */
+    int32_t local_window;          /* 1: local window on; 0 = off */
+    int32_t local_window_size;     /* with local_window: the query at position P sees only keys
+                                      [P - local_window_size, P]; >= 0 */
 } pa_dims;
 
 /* pa_scatter_kv -- write the new tokens' keys and values into the paged caches.

@@ -62,6 +62,9 @@ class pa_dims(ctypes.Structure):
         ("max_seqlen_kv_hint", ctypes.c_int32),
         ("dtype", ctypes.c_int32),
         ("min_seqlen_q_hint", ctypes.c_int32),
+        ("softcap", ctypes.c_float),
+        ("local_window", ctypes.c_int32),
+        ("local_window_size", ctypes.c_int32),
     ]
 
 
@@ -163,9 +166,11 @@ def _stream(stream):
 def make_dims(query=None, key_cache=None, block_table=None, cu_seqlens_q=None, *, batch=None,
               token_count=None, q_heads=None, kv_heads=None, head_size=None, num_blocks=None,
               block_size=None, max_blocks_per_seq=None, max_seqlen_q=0, max_seqlen_kv=0,
-              min_seqlen_q=0, dtype=PA_DTYPE_F16) -> pa_dims:
+              min_seqlen_q=0, dtype=PA_DTYPE_F16, softcap=0.0, window=None) -> pa_dims:
     """pa_dims from tensor shapes (query [T, qh, d], cache [nb, bs, kvh, d],
-    block table [B, maxblk], cu_seqlens_q [B + 1]); keywords override."""
+    block table [B, maxblk], cu_seqlens_q [B + 1]); keywords override.
+    ``softcap`` > 0 caps the scaled scores; ``window`` = w (an int >= 0) lets
+    the query at position P see only keys [P - w, P] (None: no window)."""
     d = pa_dims()
     if query is not None:
         d.token_count, d.q_heads, d.head_size = query.shape
@@ -185,6 +190,9 @@ def make_dims(query=None, key_cache=None, block_table=None, cu_seqlens_q=None, *
     d.max_seqlen_kv_hint = int(max_seqlen_kv)
     d.min_seqlen_q_hint = int(min_seqlen_q)
     d.dtype = int(dtype)
+    d.softcap = float(softcap)
+    d.local_window = 0 if window is None else 1
+    d.local_window_size = 0 if window is None else int(window)
     return d
 
 
@@ -291,7 +299,8 @@ def allocate(dims: pa_dims, device="cuda", out=None):
     import torch
     nbytes = pa_attention_workspace_size(dims)
     if out is None:
-        out = torch.empty((dims.token_count, dims.q_heads, dims.head_size), dtype=torch.float16,
+        out = torch.empty((dims.token_count, dims.q_heads, dims.head_size),
+                          dtype=torch.bfloat16 if dims.dtype == PA_DTYPE_BF16 else torch.float16,
                           device=device)
     ws = torch.empty(max(nbytes, 16), dtype=torch.uint8, device=device)
     status = torch.zeros(4, dtype=torch.int32, device=device)

@@ -70,46 +70,54 @@ EncodeTiledFn encode_fn() {
     return fn;
 }
 
-CUtensorMapSwizzle swizzle_for(int head_size) {
-    const int row_bytes = (head_size < 64 ? head_size : 64) * 2;
+CUtensorMapSwizzle swizzle_for(int head) {
+    const int row_bytes = (head < 64 ? head : 64) * 2;
     return row_bytes == 128 ? CU_TENSOR_MAP_SWIZZLE_128B
          : row_bytes == 64  ? CU_TENSOR_MAP_SWIZZLE_64B
                             : CU_TENSOR_MAP_SWIZZLE_32B;
 }
 
+CUtensorMapDataType tma_type(const pa_dims& d) {
+    return d.dtype == PA_DTYPE_BF16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT16;
+}
+
 // Cache [num_blocks, block_size, kv_heads, head_size] seen as the 4-D tensor
 // (head_size, kv_heads, block_size, num_blocks); a box is `rows` rows of one
-// KV head of one page, 64 (or head_size, if smaller) elements wide.
+// KV head of one page, 64 (or the padded head size, if smaller) elements
+// wide.  Columns of a box past head_size are filled with zeros.
 pa_status make_cache_map(CUtensorMap* m, const void* base, const pa_dims& d, int rows) {
     EncodeTiledFn fn = encode_fn();
     if (!fn) return fail(PA_ERR_CUDA, "cuTensorMapEncodeTiled entry point unavailable");
-    const int A = d.head_size < 64 ? d.head_size : 64;
+    const int head = pa::padded_head(d.head_size);
+    const int A = head < 64 ? head : 64;
     cuuint64_t dims[4] = {(cuuint64_t)d.head_size, (cuuint64_t)d.kv_heads, (cuuint64_t)d.block_size,
                           (cuuint64_t)d.num_blocks};
     cuuint64_t strides[3] = {(cuuint64_t)d.head_size * 2, (cuuint64_t)d.kv_heads * d.head_size * 2,
                              (cuuint64_t)d.block_size * d.kv_heads * d.head_size * 2};
     cuuint32_t box[4] = {(cuuint32_t)A, 1, (cuuint32_t)rows, 1};
     cuuint32_t estr[4] = {1, 1, 1, 1};
-    CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 4, const_cast<void*>(base), dims, strides,
-                    box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, swizzle_for(d.head_size),
+    CUresult r = fn(m, tma_type(d), 4, const_cast<void*>(base), dims, strides,
+                    box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, swizzle_for(head),
                     CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
     if (r != CUDA_SUCCESS) return fail(PA_ERR_CUDA, "cuTensorMapEncodeTiled(cache) failed: %d", (int)r);
     return PA_OK;
 }
 
 // Query [token_count, q_heads, head_size] seen as (head_size, q_heads,
-// token_count); a box is 128 / group tokens x group heads = 128 rows.
+// token_count); a box is 128 / group tokens (rounded down) x group heads,
+// at most 128 rows.
 pa_status make_query_map(CUtensorMap* m, const void* base, const pa_dims& d) {
     EncodeTiledFn fn = encode_fn();
     if (!fn) return fail(PA_ERR_CUDA, "cuTensorMapEncodeTiled entry point unavailable");
-    const int A = d.head_size < 64 ? d.head_size : 64;
+    const int head = pa::padded_head(d.head_size);
+    const int A = head < 64 ? head : 64;
     const int g = d.q_heads / d.kv_heads;
     cuuint64_t dims[3] = {(cuuint64_t)d.head_size, (cuuint64_t)d.q_heads, (cuuint64_t)d.token_count};
     cuuint64_t strides[2] = {(cuuint64_t)d.head_size * 2, (cuuint64_t)d.q_heads * d.head_size * 2};
     cuuint32_t box[3] = {(cuuint32_t)A, (cuuint32_t)g, (cuuint32_t)(pa::kPrefillRows / g)};
     cuuint32_t estr[3] = {1, 1, 1};
-    CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 3, const_cast<void*>(base), dims, strides,
-                    box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, swizzle_for(d.head_size),
+    CUresult r = fn(m, tma_type(d), 3, const_cast<void*>(base), dims, strides,
+                    box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, swizzle_for(head),
                     CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
     if (r != CUDA_SUCCESS) return fail(PA_ERR_CUDA, "cuTensorMapEncodeTiled(query) failed: %d", (int)r);
     return PA_OK;
@@ -160,12 +168,17 @@ pa_status check_dims(const pa_dims* dp) {
         return fail(PA_ERR_INVALID_ARGUMENT, "q_heads (%d) must be a positive multiple of kv_heads (%d)",
                     d.q_heads, d.kv_heads);
     const int g = d.q_heads / d.kv_heads;
-    if (!is_pow2(g) || g > 32)
-        return fail(PA_ERR_NOT_IMPLEMENTED, "q_heads / kv_heads = %d: only powers of two up to 32", g);
-    if (d.head_size <= 0 || d.head_size % 8 != 0)
-        return fail(PA_ERR_INVALID_ARGUMENT, "head_size %d must be a positive multiple of 8", d.head_size);
-    if (d.head_size != 16 && d.head_size != 32 && d.head_size != 64 && d.head_size != 128)
-        return fail(PA_ERR_NOT_IMPLEMENTED, "head_size %d: only 16, 32, 64, 128", d.head_size);
+    if (g > 32)
+        return fail(PA_ERR_NOT_IMPLEMENTED, "q_heads / kv_heads = %d: groups up to 32 are built", g);
+    if (d.head_size <= 0 || d.head_size % 8 != 0 || d.head_size > 256)
+        return fail(PA_ERR_INVALID_ARGUMENT, "head_size %d must be a multiple of 8 in [8, 256]",
+                    d.head_size);
+    if (d.softcap < 0.f || isnan(d.softcap) || isinf(d.softcap))
+        return fail(PA_ERR_INVALID_ARGUMENT, "softcap must be finite and >= 0");
+    if (d.local_window != 0 && d.local_window != 1)
+        return fail(PA_ERR_INVALID_ARGUMENT, "local_window must be 0 or 1");
+    if (d.local_window && d.local_window_size < 0)
+        return fail(PA_ERR_INVALID_ARGUMENT, "local_window_size must be >= 0");
     if (!is_pow2(d.block_size) || d.block_size < 16 || d.block_size > 256)
         return fail(PA_ERR_INVALID_ARGUMENT, "block_size %d must be a power of two in [16, 256]",
                     d.block_size);
@@ -255,8 +268,9 @@ pa_status pa_attention(const void* query, const void* key_cache, const void* val
     pa_status st = check_dims(dims);
     if (st != PA_OK) return st;
     const pa_dims& d = *dims;
-    if (d.dtype == PA_DTYPE_BF16)
-        return fail(PA_ERR_NOT_IMPLEMENTED, "bfloat16 attention is not implemented (f16 only)");
+    if (d.head_size > 128)
+        return fail(PA_ERR_NOT_IMPLEMENTED, "attention with head_size %d: sizes up to 128 are built",
+                    d.head_size);
     if (d.token_count == 0) return PA_OK;
     if (d.batch == 0) return fail(PA_ERR_INVALID_ARGUMENT, "token_count > 0 with batch 0");
     if (!(scale >= 0.f) || isinf(scale))
@@ -275,8 +289,16 @@ pa_status pa_attention(const void* query, const void* key_cache, const void* val
                     workspace_bytes, plan.workspace_bytes);
     if (plan.workspace_bytes > 0) PA_REQUIRE_PTR(workspace);
     if (scale == 0.f) scale = 1.f / sqrtf((float)d.head_size);
-    const float scale_log2 = scale * 1.4426950408889634f;
+    pa::ScoreMods mods{};
+    mods.scale = scale;
+    mods.scale_log2 = scale * 1.4426950408889634f;
+    mods.softcap = d.softcap;
+    mods.inv_softcap = d.softcap > 0.f ? 1.f / d.softcap : 0.f;
+    mods.window = d.local_window;
+    mods.window_size = d.local_window ? d.local_window_size : 0;
     const int g = d.q_heads / d.kv_heads;
+    const int head = pa::padded_head(d.head_size);
+    const bool bf16 = d.dtype == PA_DTYPE_BF16;
     const int kv_cap = d.max_blocks_per_seq * d.block_size;
     cudaStream_t s = static_cast<cudaStream_t>(stream);
 
@@ -291,13 +313,13 @@ pa_status pa_attention(const void* query, const void* key_cache, const void* val
         if ((st = make_cache_map(&tk, key_cache, d, rows)) != PA_OK) return st;
         if ((st = make_cache_map(&tv, value_cache, d, rows)) != PA_OK) return st;
         pa::DecodeParams p{};
-        p.query = static_cast<const __half*>(query);
-        p.key_cache = static_cast<const __half*>(key_cache);
-        p.value_cache = static_cast<const __half*>(value_cache);
-        p.out = static_cast<__half*>(out);
+        p.query = static_cast<const uint16_t*>(query);
+        p.key_cache = static_cast<const uint16_t*>(key_cache);
+        p.value_cache = static_cast<const uint16_t*>(value_cache);
+        p.out = static_cast<uint16_t*>(out);
         const size_t rows_total = (size_t)d.batch * d.kv_heads * plan.max_splits * (16 * plan.mtiles);
         p.part_o = static_cast<float*>(workspace);
-        p.part_lse = plan.workspace_bytes ? static_cast<float*>(workspace) + rows_total * d.head_size
+        p.part_lse = plan.workspace_bytes ? static_cast<float*>(workspace) + rows_total * head
                                           : nullptr;
         p.block_table = block_table;
         p.cu_seqlens_q = cu_seqlens_q;
@@ -309,6 +331,7 @@ pa_status pa_attention(const void* query, const void* key_cache, const void* val
         p.q_heads = d.q_heads;
         p.kv_heads = d.kv_heads;
         p.group = g;
+        p.head_size = d.head_size;
         p.block_size = d.block_size;
         p.max_blocks = d.max_blocks_per_seq;
         p.kv_cap = kv_cap;
@@ -318,23 +341,26 @@ pa_status pa_attention(const void* query, const void* key_cache, const void* val
         p.chunk = plan.chunk;
         p.max_splits = plan.max_splits;
         p.rmax = 16 * plan.mtiles;
-        p.scale_log2 = scale_log2;
+        p.mods = mods;
         {
             TraceScope tr(PA_KERNEL_DECODE, s);
-            cudaError_t e = pa::launch_decode(tk, tv, p, d.head_size, plan.mtiles, s);
+            cudaError_t e = pa::launch_decode(tk, tv, p, head, plan.mtiles, bf16, s);
             if (e != cudaSuccess) return cuda_fail(e, "decode launch");
         }
         if (plan.max_splits > 1) {
             TraceScope tr(PA_KERNEL_COMBINE, s);
-            cudaError_t e = pa::launch_combine(p, d.head_size, s);
+            cudaError_t e = pa::launch_combine(p, head, bf16, s);
             if (e != cudaSuccess) return cuda_fail(e, "combine launch");
         }
     }
 
     // Prefill part: sequences with q_len > prefill_min_q.
     if (d.max_seqlen_q_hint == 0 || d.max_seqlen_q_hint > prefill_min_q) {
+        // Query-tile pairs: 2 * (128 / group) tokens each; every prefill
+        // sequence adds at most one partly filled pair.
+        const long long pair_tokens = 2 * (pa::kPrefillRows / g);
         const long long longer = d.token_count / (prefill_min_q + 1);
-        const long long slots = (d.token_count * g + pa::kPrefillCtaRows - 1) / pa::kPrefillCtaRows +
+        const long long slots = (d.token_count + pair_tokens - 1) / pair_tokens +
                                 (longer < d.batch ? longer : d.batch);
         if (slots > 0) {
             if (slots * d.kv_heads >= (1ll << 31))
@@ -345,9 +371,9 @@ pa_status pa_attention(const void* query, const void* key_cache, const void* val
             if ((st = make_cache_map(&tk, key_cache, d, rows)) != PA_OK) return st;
             if ((st = make_cache_map(&tv, value_cache, d, rows)) != PA_OK) return st;
             pa::PrefillParams p{};
-            p.out = static_cast<__half*>(out);
-            p.key_cache = static_cast<const __half*>(key_cache);
-            p.value_cache = static_cast<const __half*>(value_cache);
+            p.out = static_cast<uint16_t*>(out);
+            p.key_cache = static_cast<const uint16_t*>(key_cache);
+            p.value_cache = static_cast<const uint16_t*>(value_cache);
             p.block_table = block_table;
             p.cu_seqlens_q = cu_seqlens_q;
             p.seqlens_kv = seqlens_kv;
@@ -358,6 +384,7 @@ pa_status pa_attention(const void* query, const void* key_cache, const void* val
             p.q_heads = d.q_heads;
             p.kv_heads = d.kv_heads;
             p.group = g;
+            p.head_size = d.head_size;
             p.block_size = d.block_size;
             p.max_blocks = d.max_blocks_per_seq;
             p.kv_cap = kv_cap;
@@ -365,9 +392,9 @@ pa_status pa_attention(const void* query, const void* key_cache, const void* val
             p.q_hint = d.max_seqlen_q_hint;
             p.decode_max_q = prefill_min_q;
             p.num_slots = (int)slots;
-            p.scale_log2 = scale_log2;
+            p.mods = mods;
             TraceScope tr(PA_KERNEL_PREFILL, s);
-            cudaError_t e = pa::launch_prefill(tq, tk, tv, p, d.head_size, s);
+            cudaError_t e = pa::launch_prefill(tq, tk, tv, p, head, bf16, s);
             if (e != cudaSuccess) return cuda_fail(e, "prefill launch");
         }
     }

@@ -6,6 +6,7 @@
 #pragma once
 
 #include <cuda.h>
+#include <cuda_bf16.h>
 #include <cuda_fp16.h>
 #include <stdint.h>
 
@@ -215,6 +216,44 @@ __device__ __forceinline__ uint32_t pack_half2(float lo, float hi) {
     return *reinterpret_cast<uint32_t*>(&h);
 }
 
+// D = A * B + D, m16n8k16, bf16 inputs, f32 accumulators.
+__device__ __forceinline__ void mma_16816_bf16(float* d, const uint32_t* a, uint32_t b0, uint32_t b1) {
+    asm volatile(
+        "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 "
+        "{%0, %1, %2, %3}, {%4, %5, %6, %7}, {%8, %9}, {%0, %1, %2, %3};"
+        : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+        : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
+}
+
+// The 16-bit element types of the attention inputs: f16 (__half) and bf16
+// (__nv_bfloat16).  pack2 rounds two fp32 values to nearest-even into one
+// 32-bit pair; mma is the m16n8k16 product of the type; zero is +0.
+template <typename T>
+struct Elem;
+
+template <>
+struct Elem<__half> {
+    static constexpr bool kBf16 = false;
+    static __device__ __forceinline__ uint32_t pack2(float lo, float hi) { return pack_half2(lo, hi); }
+    static __device__ __forceinline__ void mma(float* d, const uint32_t* a, uint32_t b0, uint32_t b1) {
+        mma_16816(d, a, b0, b1);
+    }
+};
+
+template <>
+struct Elem<__nv_bfloat16> {
+    static constexpr bool kBf16 = true;
+    static __device__ __forceinline__ uint32_t pack2(float lo, float hi) {
+        __nv_bfloat162 h = __floats2bfloat162_rn(lo, hi);
+        return *reinterpret_cast<uint32_t*>(&h);
+    }
+    static __device__ __forceinline__ void mma(float* d, const uint32_t* a, uint32_t b0, uint32_t b1) {
+        mma_16816_bf16(d, a, b0, b1);
+    }
+};
+
+
+
 // max(a, b, c) in one instruction (three-input form of max.f32, sm_100).
 __device__ __forceinline__ float fmax3(float a, float b, float c) {
     float d;
@@ -226,6 +265,18 @@ __device__ __forceinline__ float fast_exp2(float x) {
     float y;
     asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
     return y;
+}
+
+// Softcap score modifier in the softmax's log2 domain:
+//   c * tanh(s / c) * log2(e)
+// with tanh(y) = 1 - 2 / (e^(2y) + 1), e^(2y) taken as 2^(2y log2 e) on the
+// MUFU unit.  The exponent is clamped at 126 (tanh is 1 to fp32 precision
+// long before), so e^(2y) + 1 stays finite.  Absolute error of the tanh about
+// 1e-6: the score moves by under c * 1e-6.
+__device__ __forceinline__ float softcap_log2(float s, float cap, float inv_cap) {
+    const float e = fast_exp2(fminf(s * inv_cap * 2.8853900817779268f, 126.f));
+    const float t = 1.f - __fdividef(2.f, e + 1.f);
+    return cap * 1.4426950408889634f * t;
 }
 
 // ---------------------------------------------------------------- packed f32x2
@@ -257,11 +308,14 @@ __device__ __forceinline__ uint64_t f2_mul(uint64_t a, uint64_t b) {
 
 // ---------------------------------------------------------------- tcgen05
 
-// Instruction descriptor for tcgen05.mma kind::f16: f16 A and B, f32
-// accumulator, dense.  a_mn / b_mn select MN-major operands (else K-major).
-__host__ __device__ constexpr uint32_t umma_idesc_f16(int M, int N, bool a_mn, bool b_mn) {
+// Instruction descriptor for tcgen05.mma kind::f16: A and B both f16 (or
+// both bf16), f32 accumulator, dense.  a_mn / b_mn select MN-major operands
+// (else K-major).
+__host__ __device__ constexpr uint32_t umma_idesc_f16(int M, int N, bool a_mn, bool b_mn,
+                                                      bool bf16 = false) {
     return (1u << 4)                        // D format: f32
-         | (0u << 7) | (0u << 10)           // A, B format: f16
+         | ((bf16 ? 1u : 0u) << 7)          // A format: f16 (0) or bf16 (1)
+         | ((bf16 ? 1u : 0u) << 10)         // B format: the same as A
          | ((a_mn ? 1u : 0u) << 15)
          | ((b_mn ? 1u : 0u) << 16)
          | ((uint32_t)(N >> 3) << 17)

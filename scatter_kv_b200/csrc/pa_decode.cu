@@ -91,11 +91,32 @@ __device__ __forceinline__ uint32_t half2_mask(uint32_t v, bool lo_ok, bool hi_o
     return (lo_ok ? (v & 0xffffu) : 0u) | (hi_ok ? (v & 0xffff0000u) : 0u);
 }
 
-template <int HEAD, int MT, bool CPA>
+// Keys of sequence s that the decode CTAs stream: [k_first, T), split into
+// chunks of p.chunk in logical order.  Without a local window k_first is 0;
+// with one it is the first key any of the sequence's rows can see, rounded
+// down to the 32-key tile.
+__device__ __forceinline__ void decode_range(const SeqInfo& s, const DecodeParams& p, int& k_first,
+                                             int& n_splits) {
+    k_first = 0;
+    if (p.mods.window) {
+        const int lo = s.past - p.mods.window_size;
+        if (lo > 0) k_first = lo & ~(kDecodeKeys - 1);
+    }
+    n_splits = (s.kv_len - k_first + p.chunk - 1) / p.chunk;
+}
+
+// Output row r (of sequence s, KV head kvh) in the packed [token, q_heads,
+// head_size] layout.
+__device__ __forceinline__ long long out_row(const DecodeParams& p, const SeqInfo& s, int kvh, int r) {
+    return ((long long)(s.q_start + r / p.group) * p.q_heads + kvh * p.group + r % p.group) * p.head_size;
+}
+
+template <int HEAD, int MT, bool CPA, typename ET, bool CAP>
 __global__ void __launch_bounds__(Cfg<HEAD, MT, CPA>::THREADS, (HEAD >= 128 && !CPA) ? 2 : 3)
 decode_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_v,
               const DecodeParams p) {
     using C = Cfg<HEAD, MT, CPA>;
+    using E = Elem<ET>;
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>(
         (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -116,6 +137,7 @@ decode_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ 
     const int b = blockIdx.z, kvh = blockIdx.x, split = blockIdx.y;
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int g = p.group;
+    const int hs = p.head_size;
     // Status bits of a sequence are reported once, by CTA (split 0, kv head 0).
     const bool reporter = (split == 0 && kvh == 0 && threadIdx.x == 0);
 
@@ -134,11 +156,8 @@ decode_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ 
             if (reporter)
                 load_seq(p.cu_seqlens_q, p.seqlens_kv, b, p.batch, p.token_count, p.kv_cap,
                          p.kv_hint, p.q_hint, p.status, s);
-            for (int idx = threadIdx.x; idx < s.q_len * g * HEAD; idx += C::THREADS) {
-                const int r = idx / HEAD, d = idx % HEAD;
-                const long long o = ((long long)(s.q_start + r / g) * p.q_heads + kvh * g + r % g) * HEAD + d;
-                p.out[o] = __float2half_rn(0.f);
-            }
+            for (int idx = threadIdx.x; idx < s.q_len * g * hs; idx += C::THREADS)
+                p.out[out_row(p, s, kvh, idx / hs) + idx % hs] = 0;
         }
         return;
     }
@@ -149,17 +168,14 @@ decode_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ 
         if (reporter)
             load_seq(p.cu_seqlens_q, p.seqlens_kv, b, p.batch, p.token_count, p.kv_cap,
                      p.kv_hint, p.q_hint, p.status, s);
-        if (split == 0) {
-            for (int idx = threadIdx.x; idx < R * HEAD; idx += C::THREADS) {
-                const int r = idx / HEAD, d = idx % HEAD;
-                const long long o = ((long long)(s.q_start + r / g) * p.q_heads + kvh * g + r % g) * HEAD + d;
-                p.out[o] = __float2half_rn(0.f);
-            }
-        }
+        if (split == 0)
+            for (int idx = threadIdx.x; idx < R * hs; idx += C::THREADS)
+                p.out[out_row(p, s, kvh, idx / hs) + idx % hs] = 0;
         return;
     }
     const int T = s.kv_len;
-    const int n_splits = (T + p.chunk - 1) / p.chunk;
+    int k_first, n_splits;
+    decode_range(s, p, k_first, n_splits);
     if (split >= n_splits) return;
 
     if (threadIdx.x == 0) {
@@ -173,9 +189,24 @@ decode_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ 
         mbar_init(verdict, 1);
         fence_barrier_init();
     }
+    if (CPA && hs < HEAD) {
+        // Columns past the head size: zero in every stage, once (the copies
+        // never write them; TMA fills them with zeros by itself).
+        constexpr int CH = C::RB / 16;
+        for (int idx = threadIdx.x; idx < C::NST * 2 * C::BN * (HEAD / 8); idx += C::THREADS) {
+            const int jc = idx % (HEAD / 8);
+            if (jc * 8 < hs) continue;
+            const int r = (idx / (HEAD / 8)) % C::BN;
+            const int tt = idx / (HEAD / 8 * C::BN);          // stage * 2 + tensor
+            const int c = (jc * 8) / C::A, jj = jc % CH;
+            *reinterpret_cast<uint4*>(stages + tt * C::TILE_BYTES +
+                                      swz<C::RB>((uint32_t)((c * C::BN + r) * C::RB + jj * 16))) =
+                make_uint4(0, 0, 0, 0);
+        }
+    }
     __syncthreads();
 
-    const int k_begin = split * p.chunk;
+    const int k_begin = k_first + split * p.chunk;
     const int k_end = min(T, k_begin + p.chunk);
     const int ntiles = (k_end - k_begin + C::BN - 1) / C::BN;
     const int bs = p.block_size;
@@ -217,17 +248,19 @@ decode_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ 
             // is exactly pages k0/16 and k0/16 + 1.  Producer thread q copies
             // the 16-byte chunk q % CPR of rows q / CPR + i * RPI (a fixed
             // column per thread); rows at or past the split's end are not read
-            // (their block-table entries are not pages of this sequence).  Each
-            // thread arrives on the stage's mbarrier once its copies have landed.
+            // (their block-table entries are not pages of this sequence), nor
+            // are columns past the head size.  Each thread arrives on the
+            // stage's mbarrier once its copies have landed.
             constexpr int RPI = C::NPW * 32 / C::CPR;         // rows per pass of all producers
             static_assert((C::NPW * 32) % C::CPR == 0, "a fixed column per producer thread");
             const int q0 = pw * 32 + lane;
             const int r0 = q0 / C::CPR, jc = q0 % C::CPR;
             const int c = (jc * 8) / C::A, jj = jc % (C::A / 8);
+            const bool col_ok = jc * 8 < hs;
             const char* kc = reinterpret_cast<const char*>(p.key_cache);
             const char* vc = reinterpret_cast<const char*>(p.value_cache);
-            const long long row_bytes = (long long)p.kv_heads * HEAD * 2;
-            const long long colb = (long long)kvh * HEAD * 2 + jc * 16;
+            const long long row_bytes = (long long)p.kv_heads * hs * 2;
+            const long long colb = (long long)kvh * hs * 2 + jc * 16;
             for (int t = 0; t < ntiles; ++t) {
                 const int st = t % C::NST, u = t / C::NST;
                 bool go = true;
@@ -249,7 +282,7 @@ decode_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ 
 #pragma unroll
                 for (int i = 0; i < (C::BN + RPI - 1) / RPI; ++i) {
                     const int r = r0 + i * RPI;
-                    if (r < C::BN && k0 + r < k_end) {
+                    if (col_ok && r < C::BN && k0 + r < k_end) {
                         const int blk = (r >> 4) ? blk1 : blk0;
                         const long long goff = (long long)(blk * 16 + (r & 15)) * row_bytes + colb;
                         const uint32_t soff = swz<C::RB>((uint32_t)((c * C::BN + r) * C::RB + jj * 16));
@@ -296,27 +329,27 @@ decode_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ 
         // Rows held by this thread: r0 = mt*16 + quad, r1 = r0 + 8.
         int rows[2] = {mt * 16 + quad, mt * 16 + quad + 8};
         int lim[2];                        // last visible key (inclusive) per row
+        int lo[2];                         // first visible key per row
 #pragma unroll
         for (int h = 0; h < 2; ++h) {
             const int r = rows[h];
             lim[h] = (r < R) ? (s.past + r / g) : (T - 1);
+            lo[h] = p.mods.window ? lim[h] - p.mods.window_size : -(1 << 30);
         }
-        // Q fragments (A operand) straight from global memory.
+        // Q fragments (A operand) straight from global memory; columns past
+        // the head size are zero.
         uint32_t qf[HEAD / 16][4];
         {
-            const __half* q0 = nullptr;
-            const __half* q1 = nullptr;
-            if (rows[0] < R)
-                q0 = p.query + ((long long)(s.q_start + rows[0] / g) * p.q_heads + kvh * g + rows[0] % g) * HEAD;
-            if (rows[1] < R)
-                q1 = p.query + ((long long)(s.q_start + rows[1] / g) * p.q_heads + kvh * g + rows[1] % g) * HEAD;
+            const uint16_t* q0 = rows[0] < R ? p.query + out_row(p, s, kvh, rows[0]) : nullptr;
+            const uint16_t* q1 = rows[1] < R ? p.query + out_row(p, s, kvh, rows[1]) : nullptr;
 #pragma unroll
             for (int kk = 0; kk < HEAD / 16; ++kk) {
                 const int c = kk * 16 + 2 * qid;
-                qf[kk][0] = q0 ? *reinterpret_cast<const uint32_t*>(q0 + c) : 0u;
-                qf[kk][1] = q1 ? *reinterpret_cast<const uint32_t*>(q1 + c) : 0u;
-                qf[kk][2] = q0 ? *reinterpret_cast<const uint32_t*>(q0 + c + 8) : 0u;
-                qf[kk][3] = q1 ? *reinterpret_cast<const uint32_t*>(q1 + c + 8) : 0u;
+                const bool lo_ok = c < hs, hi_ok = c + 8 < hs;
+                qf[kk][0] = (q0 && lo_ok) ? *reinterpret_cast<const uint32_t*>(q0 + c) : 0u;
+                qf[kk][1] = (q1 && lo_ok) ? *reinterpret_cast<const uint32_t*>(q1 + c) : 0u;
+                qf[kk][2] = (q0 && hi_ok) ? *reinterpret_cast<const uint32_t*>(q0 + c + 8) : 0u;
+                qf[kk][3] = (q1 && hi_ok) ? *reinterpret_cast<const uint32_t*>(q1 + c + 8) : 0u;
             }
         }
         const long long pbase = (((long long)b * p.kv_heads + kvh) * p.max_splits + split) * p.rmax;
@@ -366,11 +399,11 @@ decode_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ 
                     const uint32_t off = (uint32_t)((c * C::BN + key) * C::RB + cc * 16);
                     uint32_t b0, b1, b2, b3;
                     ldsm_x4(kbase + swz<C::RB>(off), b0, b1, b2, b3);
-                    mma_16816(sacc[2 * np], qf[kk], b0, b1);
-                    mma_16816(sacc[2 * np + 1], qf[kk], b2, b3);
+                    E::mma(sacc[2 * np], qf[kk], b0, b1);
+                    E::mma(sacc[2 * np + 1], qf[kk], b2, b3);
                 }
             }
-            // Mask, scale to the log2 domain, online softmax.
+            // Scale (and cap) into the log2 domain, mask, online softmax.
             float mx[2] = {-INFINITY, -INFINITY};
 #pragma unroll
             for (int nt = 0; nt < 4; ++nt) {
@@ -378,8 +411,11 @@ decode_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ 
                 for (int e = 0; e < 4; ++e) {
                     const int h = e >> 1;
                     const int key = k0 + nt * 8 + 2 * qid + (e & 1);
-                    const bool vis = key < k_end && key <= lim[h];
-                    const float v = vis ? sacc[nt][e] * p.scale_log2 : -INFINITY;
+                    const bool vis = key < k_end && key <= lim[h] && key >= lo[h];
+                    const float sc = CAP ? softcap_log2(sacc[nt][e] * p.mods.scale, p.mods.softcap,
+                                                        p.mods.inv_softcap)
+                                         : sacc[nt][e] * p.mods.scale_log2;
+                    const float v = vis ? sc : -INFINITY;
                     sacc[nt][e] = v;
                     mx[h] = fmaxf(mx[h], v);
                 }
@@ -414,14 +450,14 @@ decode_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ 
                 oacc[i][2] *= alpha[1];
                 oacc[i][3] *= alpha[1];
             }
-            // P as A fragments (two k16 steps over the 32 keys).
+            // P as A fragments (two k16 steps over the 32 keys), in V's type.
             uint32_t pa[2][4];
 #pragma unroll
             for (int j = 0; j < 2; ++j) {
-                pa[j][0] = pack_half2(sacc[2 * j][0], sacc[2 * j][1]);
-                pa[j][1] = pack_half2(sacc[2 * j][2], sacc[2 * j][3]);
-                pa[j][2] = pack_half2(sacc[2 * j + 1][0], sacc[2 * j + 1][1]);
-                pa[j][3] = pack_half2(sacc[2 * j + 1][2], sacc[2 * j + 1][3]);
+                pa[j][0] = E::pack2(sacc[2 * j][0], sacc[2 * j][1]);
+                pa[j][1] = E::pack2(sacc[2 * j][2], sacc[2 * j][3]);
+                pa[j][2] = E::pack2(sacc[2 * j + 1][0], sacc[2 * j + 1][1]);
+                pa[j][3] = E::pack2(sacc[2 * j + 1][2], sacc[2 * j + 1][3]);
             }
             // O += P V.  Rows of V past the sequence end may hold anything
             // (NaN included): zero them in the fragments of the last tile.
@@ -443,8 +479,8 @@ decode_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ 
                         b1 = half2_mask(b1, kv0 + 8 < k_end, kv0 + 9 < k_end);
                         b3 = half2_mask(b3, kv0 + 8 < k_end, kv0 + 9 < k_end);
                     }
-                    mma_16816(oacc[2 * dp], pa[j], b0, b1);
-                    mma_16816(oacc[2 * dp + 1], pa[j], b2, b3);
+                    E::mma(oacc[2 * dp], pa[j], b0, b1);
+                    E::mma(oacc[2 * dp + 1], pa[j], b2, b3);
                 }
             }
             __syncwarp();
@@ -493,6 +529,7 @@ decode_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ 
         const bool direct = (n_splits == 1);
         for (int idx = threadIdx.x; idx < R * (HEAD / 4); idx += C::NCW * 32) {
             const int r = idx / (HEAD / 4), d4 = (idx % (HEAD / 4)) * 4;
+            if (direct && d4 >= hs) continue;
             float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
             for (int gg = 0; gg < C::NG; ++gg) {
                 const float4 v = *reinterpret_cast<const float4*>(scr + (gg * C::RMAX + r) * C::OST + d4);
@@ -502,11 +539,10 @@ decode_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ 
             const float inv = (L > 0.f) ? 1.f / L : 0.f;
             acc.x *= inv; acc.y *= inv; acc.z *= inv; acc.w *= inv;
             if (direct) {
-                const long long o = ((long long)(s.q_start + r / g) * p.q_heads + kvh * g + r % g) * HEAD + d4;
                 uint2 w;
-                w.x = pack_half2(acc.x, acc.y);
-                w.y = pack_half2(acc.z, acc.w);
-                *reinterpret_cast<uint2*>(p.out + o) = w;
+                w.x = E::pack2(acc.x, acc.y);
+                w.y = E::pack2(acc.z, acc.w);
+                *reinterpret_cast<uint2*>(p.out + out_row(p, s, kvh, r) + d4) = w;
             } else {
                 *reinterpret_cast<float4*>(p.part_o + (pbase + r) * HEAD + d4) = acc;
                 if (d4 == 0)
@@ -528,12 +564,13 @@ decode_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ 
 // One warp per output row (row r of KV head kvh of sequence b): merge the
 // row's splits in split order, O = sum_s w_s O_s / sum_s w_s with
 // w_s = 2^(lse_s - max lse).  Lane i owns columns [4i, 4i + 4).
-template <int HEAD>
+template <int HEAD, typename ET>
 __global__ void __launch_bounds__(128) combine_kernel(const DecodeParams p) {
+    using E = Elem<ET>;
     const int b = blockIdx.z, kvh = blockIdx.y;
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int r = blockIdx.x * 4 + warp;
-    const int g = p.group;
+    const int hs = p.head_size;
     const long long base = ((long long)b * p.kv_heads + kvh) * p.max_splits * p.rmax + r;
     const float* lse = p.part_lse + base;             // stride rmax per split
     // Lane sp's split lse, fetched together with the metadata (it does not
@@ -544,10 +581,11 @@ __global__ void __launch_bounds__(128) combine_kernel(const DecodeParams p) {
     if (!load_seq(p.cu_seqlens_q, p.seqlens_kv, b, p.batch, p.token_count, p.kv_cap, p.kv_hint,
                   p.q_hint, nullptr, s))
         return;
-    if (s.q_len == 0 || s.q_len > p.decode_max_q || r >= s.q_len * g) return;
-    const int n_splits = (s.kv_len + p.chunk - 1) / p.chunk;
+    if (s.q_len == 0 || s.q_len > p.decode_max_q || r >= s.q_len * p.group) return;
+    int k_first, n_splits;
+    decode_range(s, p, k_first, n_splits);
     if (n_splits == 1) return;                        // the decode kernel wrote the row
-    __half* orow = p.out + ((long long)(s.q_start + r / g) * p.q_heads + kvh * g + r % g) * HEAD;
+    uint16_t* orow = p.out + out_row(p, s, kvh, r);
     float M = -INFINITY;
     for (int sp = lane; sp < n_splits; sp += 32)
         M = fmaxf(M, sp < 32 ? lse_l : lse[(long long)sp * p.rmax]);
@@ -555,7 +593,7 @@ __global__ void __launch_bounds__(128) combine_kernel(const DecodeParams p) {
     for (int o = 16; o > 0; o >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, o));
     if (M == INFINITY) {
         // Some split found a bad block id: the sequence gets zero rows.
-        for (int d = lane; d < HEAD; d += 32) orow[d] = __float2half_rn(0.f);
+        for (int d = lane; d < hs; d += 32) orow[d] = 0;
         return;
     }
     // Split weights 2^(lse_s - M), lane sp holding split sp's (splits beyond 32
@@ -567,7 +605,7 @@ __global__ void __launch_bounds__(128) combine_kernel(const DecodeParams p) {
     for (int o = 16; o > 0; o >>= 1) L += __shfl_xor_sync(0xffffffffu, L, o);
     const float* po = p.part_o + base * HEAD + lane * 4;
     float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
-    const bool active = lane * 4 < HEAD;
+    const bool active = lane * 4 < hs;
 #pragma unroll 4
     for (int sp = 0; sp < n_splits; ++sp) {
         const float w = sp < 32 ? __shfl_sync(0xffffffffu, w_l, sp)
@@ -580,16 +618,16 @@ __global__ void __launch_bounds__(128) combine_kernel(const DecodeParams p) {
     if (!active) return;
     const float il = 1.f / L;
     uint2 wv;
-    wv.x = pack_half2(acc.x * il, acc.y * il);
-    wv.y = pack_half2(acc.z * il, acc.w * il);
+    wv.x = E::pack2(acc.x * il, acc.y * il);
+    wv.y = E::pack2(acc.z * il, acc.w * il);
     *reinterpret_cast<uint2*>(orow + lane * 4) = wv;
 }
 
-template <int HEAD, int MT, bool CPA>
+template <int HEAD, int MT, bool CPA, typename ET, bool CAP>
 cudaError_t launch_decode_t(const CUtensorMap& tm_k, const CUtensorMap& tm_v,
                             const DecodeParams& p, cudaStream_t stream) {
     using C = Cfg<HEAD, MT, CPA>;
-    auto kern = decode_kernel<HEAD, MT, CPA>;
+    auto kern = decode_kernel<HEAD, MT, CPA, ET, CAP>;
     cudaError_t e;
     if (CPA) {
         cudaFuncAttributes fa;
@@ -607,6 +645,29 @@ cudaError_t launch_decode_t(const CUtensorMap& tm_k, const CUtensorMap& tm_v,
     return cudaGetLastError();
 }
 
+template <int HEAD, typename ET, bool CAP>
+cudaError_t launch_decode_h(const CUtensorMap& tm_k, const CUtensorMap& tm_v, const DecodeParams& p,
+                            int mtiles, cudaStream_t stream) {
+    const bool cpa = p.block_size < kDecodeKeys;
+    if (cpa)
+        return mtiles == 1 ? launch_decode_t<HEAD, 1, true, ET, CAP>(tm_k, tm_v, p, stream)
+                           : launch_decode_t<HEAD, 2, true, ET, CAP>(tm_k, tm_v, p, stream);
+    return mtiles == 1 ? launch_decode_t<HEAD, 1, false, ET, CAP>(tm_k, tm_v, p, stream)
+                       : launch_decode_t<HEAD, 2, false, ET, CAP>(tm_k, tm_v, p, stream);
+}
+
+template <typename ET, bool CAP>
+cudaError_t launch_decode_d(const CUtensorMap& tm_k, const CUtensorMap& tm_v, const DecodeParams& p,
+                            int head, int mtiles, cudaStream_t stream) {
+    switch (head) {
+        case 16: return launch_decode_h<16, ET, CAP>(tm_k, tm_v, p, mtiles, stream);
+        case 32: return launch_decode_h<32, ET, CAP>(tm_k, tm_v, p, mtiles, stream);
+        case 64: return launch_decode_h<64, ET, CAP>(tm_k, tm_v, p, mtiles, stream);
+        case 128: return launch_decode_h<128, ET, CAP>(tm_k, tm_v, p, mtiles, stream);
+        default: return cudaErrorInvalidValue;
+    }
+}
+
 }  // namespace
 
 DecodePlan plan_decode(const pa_dims& d, int num_sms) {
@@ -620,6 +681,10 @@ DecodePlan plan_decode(const pa_dims& d, int num_sms) {
     pl.mtiles = (dq * g + 15) / 16;
     long long max_kv = (long long)d.max_blocks_per_seq * d.block_size;
     if (d.max_seqlen_kv_hint > 0 && d.max_seqlen_kv_hint < max_kv) max_kv = d.max_seqlen_kv_hint;
+    // With a local window a decode row sees at most window_size + 1 keys; the
+    // streamed range starts up to one tile earlier and spans the q_len rows.
+    if (d.local_window && (long long)d.local_window_size + dq + kDecodeKeys < max_kv)
+        max_kv = (long long)d.local_window_size + dq + kDecodeKeys;
     if (max_kv < 1) max_kv = 1;
     // Aim for about eight waves of two CTAs per SM if every sequence were as
     // long as the bound; chunks stay multiples of the key tile.
@@ -634,42 +699,42 @@ DecodePlan plan_decode(const pa_dims& d, int num_sms) {
     if (pl.max_splits > 1) {
         // [partial O: rows x head_size f32][partial lse: rows f32]
         const size_t rows = (size_t)d.batch * d.kv_heads * pl.max_splits * (16 * pl.mtiles);
-        pl.workspace_bytes = rows * (size_t)d.head_size * 4 + rows * 4;
+        pl.workspace_bytes = rows * (size_t)padded_head(d.head_size) * 4 + rows * 4;
         pl.workspace_bytes = (pl.workspace_bytes + 255) / 256 * 256;
     }
     return pl;
 }
 
-cudaError_t launch_decode(const CUtensorMap& tm_k, const CUtensorMap& tm_v,
-                          const DecodeParams& p, int head_size, int mtiles, cudaStream_t stream) {
-    const bool cpa = p.block_size < kDecodeKeys;
-#define PA_DECODE_CASE(H)                                                                      \
-    case H:                                                                                    \
-        if (cpa)                                                                               \
-            return mtiles == 1 ? launch_decode_t<H, 1, true>(tm_k, tm_v, p, stream)            \
-                               : launch_decode_t<H, 2, true>(tm_k, tm_v, p, stream);           \
-        return mtiles == 1 ? launch_decode_t<H, 1, false>(tm_k, tm_v, p, stream)               \
-                           : launch_decode_t<H, 2, false>(tm_k, tm_v, p, stream);
-    switch (head_size) {
-        PA_DECODE_CASE(16)
-        PA_DECODE_CASE(32)
-        PA_DECODE_CASE(64)
-        PA_DECODE_CASE(128)
-        default: return cudaErrorInvalidValue;
-    }
-#undef PA_DECODE_CASE
+int padded_head(int head_size) {
+    return head_size <= 16 ? 16 : head_size <= 32 ? 32 : head_size <= 64 ? 64 : 128;
 }
 
-cudaError_t launch_combine(const DecodeParams& p, int head_size, cudaStream_t stream) {
+cudaError_t launch_decode(const CUtensorMap& tm_k, const CUtensorMap& tm_v,
+                          const DecodeParams& p, int head, int mtiles, bool bf16, cudaStream_t stream) {
+    const bool cap = p.mods.softcap > 0.f;
+    if (bf16)
+        return cap ? launch_decode_d<__nv_bfloat16, true>(tm_k, tm_v, p, head, mtiles, stream)
+                   : launch_decode_d<__nv_bfloat16, false>(tm_k, tm_v, p, head, mtiles, stream);
+    return cap ? launch_decode_d<__half, true>(tm_k, tm_v, p, head, mtiles, stream)
+               : launch_decode_d<__half, false>(tm_k, tm_v, p, head, mtiles, stream);
+}
+
+template <typename ET>
+cudaError_t launch_combine_t(const DecodeParams& p, int head, cudaStream_t stream) {
     dim3 grid((p.rmax + 3) / 4, p.kv_heads, p.batch);
-    switch (head_size) {
-        case 16: combine_kernel<16><<<grid, 128, 0, stream>>>(p); break;
-        case 32: combine_kernel<32><<<grid, 128, 0, stream>>>(p); break;
-        case 64: combine_kernel<64><<<grid, 128, 0, stream>>>(p); break;
-        case 128: combine_kernel<128><<<grid, 128, 0, stream>>>(p); break;
+    switch (head) {
+        case 16: combine_kernel<16, ET><<<grid, 128, 0, stream>>>(p); break;
+        case 32: combine_kernel<32, ET><<<grid, 128, 0, stream>>>(p); break;
+        case 64: combine_kernel<64, ET><<<grid, 128, 0, stream>>>(p); break;
+        case 128: combine_kernel<128, ET><<<grid, 128, 0, stream>>>(p); break;
         default: return cudaErrorInvalidValue;
     }
     return cudaGetLastError();
+}
+
+cudaError_t launch_combine(const DecodeParams& p, int head, bool bf16, cudaStream_t stream) {
+    return bf16 ? launch_combine_t<__nv_bfloat16>(p, head, stream)
+                : launch_combine_t<__half>(p, head, stream);
 }
 
 }  // namespace pa

@@ -10,13 +10,25 @@
 
 namespace pa {
 
+// Score modifiers of one attention call (all off when zero-initialised).
+struct ScoreMods {
+    float scale;                  // multiplier of Q K^T (natural-log domain)
+    float scale_log2;             // scale * log2(e)
+    float softcap;                // > 0: c * tanh(s / c) on the scaled scores
+    float inv_softcap;            // 1 / softcap
+    int window;                   // 1: local window on
+    int window_size;              // query position P sees keys [P - window_size, P]
+};
+
 // Everything the decode (split-KV) kernels need besides the tensor maps.
+// 16-bit tensors (f16 or bf16) are held as uint16_t; the kernels read them
+// as their element type.
 struct DecodeParams {
-    const __half* query;
-    const __half* key_cache;      // [num_blocks, block_size, kv_heads, head_size]
-    const __half* value_cache;
-    __half* out;
-    float* part_o;                // [batch, kv_heads, max_splits, rmax, head_size]
+    const uint16_t* query;
+    const uint16_t* key_cache;    // [num_blocks, block_size, kv_heads, head_size]
+    const uint16_t* value_cache;
+    uint16_t* out;
+    float* part_o;                // [batch, kv_heads, max_splits, rmax, HEAD] (HEAD: padded size)
     float* part_lse;              // [batch, kv_heads, max_splits, rmax] (log2 domain)
     const int32_t* block_table;
     const int32_t* cu_seqlens_q;
@@ -28,6 +40,7 @@ struct DecodeParams {
     int q_heads;
     int kv_heads;
     int group;                    // q_heads / kv_heads
+    int head_size;                // elements per head row in memory (<= the kernel's HEAD)
     int block_size;
     int max_blocks;
     int kv_cap;                   // max_blocks_per_seq * block_size
@@ -37,13 +50,13 @@ struct DecodeParams {
     int chunk;                    // keys per split (multiple of the key tile)
     int max_splits;
     int rmax;                     // row capacity per (sequence, kv head) = 16 * m-tiles
-    float scale_log2;             // scale * log2(e)
+    ScoreMods mods;
 };
 
 struct PrefillParams {
-    __half* out;
-    const __half* key_cache;      // [num_blocks, block_size, kv_heads, head_size]
-    const __half* value_cache;
+    uint16_t* out;
+    const uint16_t* key_cache;    // [num_blocks, block_size, kv_heads, head_size]
+    const uint16_t* value_cache;
     const int32_t* block_table;
     const int32_t* cu_seqlens_q;
     const int32_t* seqlens_kv;
@@ -54,6 +67,7 @@ struct PrefillParams {
     int q_heads;
     int kv_heads;
     int group;
+    int head_size;                // elements per head row in memory (<= the kernel's HEAD)
     int block_size;
     int max_blocks;
     int kv_cap;
@@ -61,7 +75,7 @@ struct PrefillParams {
     int q_hint;
     int decode_max_q;             // sequences with q_len <= this are not prefill work
     int num_slots;                // query-tile pairs the grid covers per KV head (upper bound)
-    float scale_log2;
+    ScoreMods mods;
 };
 
 // The fused split-QKV + rotary + scatter pass (16-bit elements held as
@@ -108,6 +122,10 @@ struct DecodePlan {
 
 DecodePlan plan_decode(const pa_dims& d, int num_sms);
 
+// Head size the kernels are built for: the actual size rounded up to 16, 32,
+// 64 or 128 (columns past the actual size are zero in shared memory).
+int padded_head(int head_size);
+
 cudaError_t launch_scatter(const void* key, const void* value, const int32_t* slot_mapping,
                            void* key_cache, void* value_cache, const pa_dims& d,
                            int32_t* status, cudaStream_t stream, int num_sms);
@@ -119,8 +137,8 @@ cudaError_t launch_slot_mapping(const int32_t* block_table, const int32_t* cu,
 // Decode: split-KV partial attention, then (when any split count > 1) the
 // log-sum-exp combine.  Returns the CUDA error of the launches.
 cudaError_t launch_decode(const CUtensorMap& tm_k, const CUtensorMap& tm_v,
-                          const DecodeParams& p, int head_size, int mtiles, cudaStream_t stream);
-cudaError_t launch_combine(const DecodeParams& p, int head_size, cudaStream_t stream);
+                          const DecodeParams& p, int head, int mtiles, bool bf16, cudaStream_t stream);
+cudaError_t launch_combine(const DecodeParams& p, int head, bool bf16, cudaStream_t stream);
 
 // Size of the fixed scratch array behind pa_attention_noalloc, and the
 // lookup of its device address on the current device (once per device).
@@ -129,7 +147,7 @@ constexpr int kMaxDevices = 64;
 cudaError_t noalloc_scratch(void** ptr);
 
 cudaError_t launch_prefill(const CUtensorMap& tm_q, const CUtensorMap& tm_k,
-                           const CUtensorMap& tm_v, const PrefillParams& p, int head_size,
+                           const CUtensorMap& tm_v, const PrefillParams& p, int head, bool bf16,
                            cudaStream_t stream);
 
 // Key rows per decode stage; the cache tensor maps' box height is

@@ -131,9 +131,11 @@ struct Work {
 // the end of the grid, so SMs finish close together; measured 4-6% faster
 // than a sequence-major order, whose last CTAs included heavy pairs.  One
 // warp, 32 sequences per step; the first 32 sequences' lengths are read once
-// (one round trip for the usual batch), later ones once per rank.
+// (one round trip for the usual batch), later ones once per rank.  A pair
+// holds 2 * tokp tokens (tokp = 128 / group per query tile).
 __device__ bool find_work(const PrefillParams& p, long long slot, Work& w) {
     const int lane = threadIdx.x & 31;
+    const int pair_tokens = 2 * (kPrefillRows / p.group);
     auto lengths = [&](int b, int& c0, int& c1, int& kv, int& np) {
         c0 = c1 = kv = np = 0;
         if (b < p.batch) {
@@ -142,7 +144,7 @@ __device__ bool find_work(const PrefillParams& p, long long slot, Work& w) {
             kv = p.seqlens_kv[b];
             const int ql = c1 - c0;
             if (ql > p.decode_max_q && c0 >= 0 && (long long)c1 <= p.token_count)
-                np = (ql * p.group + kPrefillCtaRows - 1) / kPrefillCtaRows;
+                np = (ql + pair_tokens - 1) / pair_tokens;
         }
     };
     int c0f, c1f, kvf, npf;
@@ -175,6 +177,51 @@ __device__ bool find_work(const PrefillParams& p, long long slot, Work& w) {
     }
 }
 
+// Key tiles of one work item.  Half a (query tile a of the pair) covers
+// tokens [ia, ia + tokp) of the sequence, rows_valid[a] of its 128 rows; its
+// keys run from the first visible key of its first row (0, or P - w with a
+// local window) to the last visible key of its last row.  Tiles are counted
+// from jlo, the first tile either half needs; half a uses relative tiles
+// [js[a], ne[a]).
+struct TileRange {
+    int jlo;
+    int nrel;
+    int js[2];
+    int ne[2];
+    int rows_valid[2];
+};
+
+__device__ __forceinline__ TileRange tile_range(int past, int q_len, int pair, int tokp, int g,
+                                                const ScoreMods& m) {
+    TileRange t;
+    int first[2], end[2];
+    const int i0 = pair * 2 * tokp;
+    int jlo = 1 << 30, jhi = 0;
+#pragma unroll
+    for (int a = 0; a < 2; ++a) {
+        const int ia = i0 + a * tokp;
+        t.rows_valid[a] = max(0, min(tokp * g, (q_len - ia) * g));
+        const int last = min(q_len, ia + tokp) - 1;
+        first[a] = 0;
+        end[a] = 0;
+        if (t.rows_valid[a] > 0) {
+            end[a] = (past + last + 1 + kPrefillKeys - 1) / kPrefillKeys;
+            if (m.window) first[a] = max(0, past + ia - m.window_size) / kPrefillKeys;
+            jlo = min(jlo, first[a]);
+            jhi = max(jhi, end[a]);
+        }
+    }
+    if (jhi == 0) jlo = 0;
+    t.jlo = jlo;
+    t.nrel = jhi - jlo;
+#pragma unroll
+    for (int a = 0; a < 2; ++a) {
+        t.js[a] = t.rows_valid[a] > 0 ? first[a] - jlo : 0;
+        t.ne[a] = t.rows_valid[a] > 0 ? end[a] - jlo : 0;
+    }
+    return t;
+}
+
 // Bounded waits of the kernel.  With TMA producers the kernel's hot loop only
 // fits the SM's instruction cache with rolled polling loops (unrolled ones
 // cost about 6% of the kernel's time there); the cp.async path measures
@@ -188,11 +235,12 @@ __device__ __forceinline__ bool pwait_warp(uint64_t* bar, uint32_t parity) {
     return LEAN ? mbar_wait_warp_lean(bar, parity) : mbar_wait_warp(bar, parity);
 }
 
-template <int HEAD, bool CPA>
+template <int HEAD, bool CPA, typename ET, bool CAP>
 __global__ void __launch_bounds__(PCfg<HEAD, CPA>::THREADS, 1)
 prefill_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                const __grid_constant__ CUtensorMap tm_v, const PrefillParams p) {
     using C = PCfg<HEAD, CPA>;
+    using E = Elem<ET>;
     extern __shared__ __align__(1024) uint8_t smem[];
     uint64_t* bars = reinterpret_cast<uint64_t*>(smem + C::OFF_BAR);
     uint64_t* q_full = bars;
@@ -204,11 +252,13 @@ prefill_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
     uint64_t* drain = o_full + 2;            // every MMA issued so far is done (abort path)
     uint64_t* v_tail = drain + 1;            // TMA of the last V tile (zeroed before release)
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + C::NBAR);
-    // [0] b, [1] pair, [2] bad, [3] abort, [4] ring items issued, [6] kv head
+    // [0] b, [1] pair, [2] bad, [3] abort, [4] ring items issued, [6] kv head,
+    // [7] q_start, [8] q_len, [9] kv_len
     int* sh = reinterpret_cast<int*>(tmem_slot + 1);
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int g = p.group;
+    const int hs = p.head_size;
 
     if ((smem_u32(smem) & 1023u) != 0) {              // the swizzle needs 1024-B alignment
         if (threadIdx.x == 0) flag_status(p.status, PA_DEV_TIMEOUT);
@@ -221,6 +271,7 @@ prefill_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
     // known (its tensor map bounds every coordinate) and streams while warp 0
     // checks the block table.
     const int tokp = C::BM / g;                                  // tokens per half
+    const int qrows = tokp * g;                                  // rows per half Q's box fills
     if (warp == C::WARP_MMA) {
         tmem_alloc(tmem_slot, C::TMEM_COLS);
         tmem_relinquish();
@@ -259,7 +310,7 @@ prefill_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
                                p.q_hint, (first && lane == 0) ? p.status : nullptr, si);
             if (ok) {
                 if (lane == 0) {
-                    mbar_arrive_expect_tx(q_full, 2 * C::Q_BYTES);
+                    mbar_arrive_expect_tx(q_full, 2 * C::NA * qrows * C::RB);
 #pragma unroll
                     for (int a = 0; a < 2; ++a)
 #pragma unroll
@@ -267,27 +318,32 @@ prefill_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
                             tma_load_3d(smem + C::OFF_Q + a * C::Q_BYTES + c * C::BM * C::RB, &tm_q,
                                         q_full, c * C::A, w.kvh * g, si.q_start + (w.pair * 2 + a) * tokp);
                 }
-                // Block-table check (the row's ids in range), keeping page 0's id.
+                // Block-table check (the row's ids in range), keeping the id of
+                // the page that holds the first key tile.
+                const TileRange tr = tile_range(si.past, si.q_len, w.pair, tokp, g, p.mods);
+                const int key0 = tr.jlo * C::BN;
+                const int pg_first = key0 / p.block_size;
                 const int npages = (si.kv_len + p.block_size - 1) / p.block_size;
                 const int32_t* row = p.block_table + (long long)w.b * p.max_blocks;
                 bool badid = false;
                 int id0 = 0;
                 for (int pg = lane; pg < npages; pg += 32) {
                     const int id = row[pg];
-                    if (pg == 0) id0 = id;
+                    if (pg == pg_first) id0 = id;
                     badid |= id < 0 || (long long)id >= p.num_blocks;
                 }
+                id0 = __shfl_sync(0xffffffffu, id0, pg_first & 31);
                 ok = !__any_sync(0xffffffffu, badid);
                 if (!ok && first && lane == 0) flag_status(p.status, PA_DEV_BAD_BLOCK);
-                if (!CPA && ok && lane == 0) {
-                    // TMA path: key tile 0 (ring item 0, one page of at least 128
-                    // rows) is issued here too, with the arrivals of every producer;
-                    // the producers start at ring item 1.
+                if (!CPA && ok && lane == 0 && tr.nrel > 0) {
+                    // TMA path: the first key tile (ring item 0, within one page of
+                    // at least 128 rows) is issued here too, with the arrivals of
+                    // every producer; the producers start at ring item 1.
                     mbar_arrive_expect_tx(&full[0], (uint32_t)C::KV_BYTES);
 #pragma unroll
                     for (int c = 0; c < C::NA; ++c)
                         tma_load_4d(smem + C::OFF_RING + c * C::BN * C::RB, &tm_k, &full[0], c * C::A,
-                                    w.kvh, 0, id0);
+                                    w.kvh, key0 % p.block_size, id0);
                     if (C::NPROD > 1) mbar_arrive_cnt(&full[0], C::NPROD - 1);
                     sh[4] = 1;                           // ring items issued (abort drain)
                 }
@@ -303,6 +359,33 @@ prefill_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
             sh[8] = si.q_len;
             sh[9] = si.kv_len;
         }
+    } else if (warp >= 4 && warp < 8) {
+        // Shared memory that no copy writes, zeroed once (generic stores, made
+        // visible to the tensor cores): Q rows past the group's rows, and on the
+        // cp.async path the ring's columns past the head size (TMA fills those
+        // with zeros by itself).
+        const int t4 = threadIdx.x - 128;
+        for (int idx = t4; idx < 2 * C::NA * (C::BM - qrows) * (C::RB / 16); idx += 128) {
+            const int ch = idx % (C::RB / 16);
+            const int r = qrows + (idx / (C::RB / 16)) % (C::BM - qrows);
+            const int ac = idx / ((C::RB / 16) * (C::BM - qrows));     // half * NA + column block
+            *reinterpret_cast<uint4*>(smem + C::OFF_Q + (ac / C::NA) * C::Q_BYTES +
+                                      (ac % C::NA) * C::BM * C::RB +
+                                      swz<C::RB>((uint32_t)(r * C::RB + ch * 16))) = make_uint4(0, 0, 0, 0);
+        }
+        if (CPA && hs < HEAD) {
+            for (int idx = t4; idx < C::NS * C::BN * (HEAD / 8); idx += 128) {
+                const int jc = idx % (HEAD / 8);
+                if (jc * 8 < hs) continue;
+                const int r = (idx / (HEAD / 8)) % C::BN;
+                const int st = idx / (HEAD / 8 * C::BN);
+                const int c = (jc * 8) / C::A, jj = jc % (C::A / 8);
+                *reinterpret_cast<uint4*>(smem + C::OFF_RING + st * C::KV_BYTES +
+                                          swz<C::RB>((uint32_t)((c * C::BN + r) * C::RB + jj * 16))) =
+                    make_uint4(0, 0, 0, 0);
+            }
+        }
+        fence_proxy_async_smem();
     }
     tc_fence_before();
     __syncthreads();
@@ -317,25 +400,16 @@ prefill_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
     s.kv_len = sh[9];
     s.past = s.kv_len - s.q_len;
     const int i0 = pair * 2 * tokp;                              // first token of half 0
-    // Rows and key tiles of each half (a half past the sequence end has none).
-    int rows_valid[2], ntiles_h[2];
-#pragma unroll
-    for (int a = 0; a < 2; ++a) {
-        const int ia = i0 + a * tokp;
-        rows_valid[a] = max(0, min(C::BM, (s.q_len - ia) * g));
-        const int last = min(s.q_len, ia + tokp) - 1;
-        ntiles_h[a] = rows_valid[a] > 0 ? (s.past + last + 1 + C::BN - 1) / C::BN : 0;
-    }
-    const int ntiles = max(ntiles_h[0], ntiles_h[1]);
+    const TileRange tr = tile_range(s.past, s.q_len, pair, tokp, g, p.mods);
     const int T = s.kv_len;
     if (b < 0 || sh[2] != 0) {
         if (b >= 0) {
             // Invalid sequence or block table: its rows of `out` are zero.
-            const int rows = rows_valid[0] + rows_valid[1];
-            for (int idx = threadIdx.x; idx < rows * HEAD; idx += C::THREADS) {
-                const int r = idx / HEAD, d = idx % HEAD;
-                const long long o = ((long long)(s.q_start + i0 + r / g) * p.q_heads + kvh * g + r % g) * HEAD + d;
-                p.out[o] = __float2half_rn(0.f);
+            const int rows = tr.rows_valid[0] + tr.rows_valid[1];
+            for (int idx = threadIdx.x; idx < rows * hs; idx += C::THREADS) {
+                const int r = idx / hs, d = idx % hs;
+                const long long o = ((long long)(s.q_start + i0 + r / g) * p.q_heads + kvh * g + r % g) * hs + d;
+                p.out[o] = 0;
             }
             // Q's copy lands before the CTA's shared memory is released.
             if (sh[2] == 2 && threadIdx.x == 0) pwait<!CPA>(q_full, 0);
@@ -349,22 +423,25 @@ prefill_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
     const int bs = p.block_size;
     const int32_t* bt = p.block_table + (long long)b * p.max_blocks;
     const int box = bs < C::BN ? bs : C::BN;
+    const int nrel = tr.nrel;
+    const int kbase = tr.jlo * C::BN;                            // first key of relative tile 0
 
     if (warp == 8 || warp >= 10) {
         // -------------------------------------------------------------- producers
         regs_dec<C::REGS_OTHER>();
         const int pw = warp == 8 ? 0 : warp - 9;       // producer index 0, 1, 2
-        // Ring item u: K_{u/2} (u even) or V_{u/2} (u odd), in stage u % NS.
-        // Key tile j covers keys [128 j, 128 j + 128): the pages (or the part of
-        // one page) holding them, up to the last page that starts before T.
-        // Box b = page * NA + column block goes to producer b % NPROD.
+        // Ring item u: K_{u/2} (u even) or V_{u/2} (u odd) of relative tile
+        // u / 2, in stage u % NS.  Relative tile j covers keys [kbase + 128 j,
+        // kbase + 128 j + 128): the pages (or the part of one page) holding
+        // them, up to the last page that starts before T.  Box b = page * NA +
+        // column block goes to producer b % NPROD.
         // Block ids of the sequence, 32 pages at a time in registers (lane i
         // holds page win_base + i); the next window is fetched a whole window
         // ahead, so issuing a tile never waits on a block-table load.
         const int npages = (T + bs - 1) / bs;
-        int win_base = 0;
-        int win_id = lane < npages ? bt[lane] : 0;
-        int nxt_id = 32 + lane < npages ? bt[32 + lane] : 0;
+        int win_base = (kbase / bs) & ~31;
+        int win_id = win_base + lane < npages ? bt[win_base + lane] : 0;
+        int nxt_id = win_base + 32 + lane < npages ? bt[win_base + 32 + lane] : 0;
         auto page_id = [&](int page) -> int {          // warp-uniform, pages ascending
             while (page >= win_base + 32) {
                 win_base += 32;
@@ -374,24 +451,25 @@ prefill_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
             return __shfl_sync(0xffffffffu, win_id, page - win_base);
         };
         // cp.async path: producer thread q = pw * 32 + lane copies chunk q % CPR
-        // of rows q / CPR + i * RPI (a fixed column per thread).
+        // of rows q / CPR + i * RPI (a fixed column per thread); chunks past the
+        // head size stay zero.
         const int qt = pw * 32 + lane;
         const int r0 = qt / C::CPR, jc = qt % C::CPR;
         const int cb = (jc * 8) / C::A, jj = jc % (C::A / 8);
+        const bool col_ok = jc * 8 < hs;
         const int lbs = 31 - __clz(bs);
-        const long long row_bytes = (long long)p.kv_heads * HEAD * 2;
-        const long long colb = (long long)kvh * HEAD * 2 + jc * 16;
+        const long long row_bytes = (long long)p.kv_heads * hs * 2;
+        const long long colb = (long long)kvh * hs * 2 + jc * 16;
         int tile_ids = 0;
         int next_ids = 0;
         if (CPA) {
-            const int np0 = (min(C::BN, T) + bs - 1) / bs;
-            next_ids = lane < np0 ? bt[lane] : 0;          // becomes tile 0's ids at u = 0
+            const int np0 = (min(kbase + C::BN, T) - kbase + bs - 1) / bs;
+            next_ids = lane < np0 ? bt[(kbase >> lbs) + lane] : 0;   // tile 0's ids at u = 0
         }
-        for (int u = CPA ? 0 : 1; u < 2 * ntiles; ++u) {
+        for (int u = CPA ? 0 : 1; u < 2 * nrel; ++u) {
             const int st = u % C::NS;
-            const int j = u >> 1;
             const bool is_v = (u & 1) != 0;
-            const int k0 = j * C::BN;
+            const int k0 = kbase + (u >> 1) * C::BN;
             // The last V tile (rows past T to be zeroed) is producer 0's alone
             // on the TMA path.
             const bool tail = is_v && (k0 + C::BN > T);
@@ -425,7 +503,7 @@ prefill_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
                     const int r = r0 + i * C::RPI;
                     const int key = k0 + r;
                     const int blk = __shfl_sync(0xffffffffu, tile_ids, r < C::BN ? (r >> lbs) : 0);
-                    if (r < C::BN) {
+                    if (r < C::BN && col_ok) {
                         const uint32_t soff = swz<C::RB>((uint32_t)((cb * C::BN + r) * C::RB + jj * 16));
                         if (key < T) {
                             const long long row = ((long long)blk << lbs) + (key & (bs - 1));
@@ -492,8 +570,8 @@ prefill_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
         // -------------------------------------------------------------- MMA issuer
         regs_dec<C::REGS_OTHER>();
         if (lane == 0) {
-            constexpr uint32_t idesc_s = umma_idesc_f16(C::BM, C::BN, false, false);
-            constexpr uint32_t idesc_o = umma_idesc_f16(C::BM, HEAD, false, true);
+            constexpr uint32_t idesc_s = umma_idesc_f16(C::BM, C::BN, false, false, E::kBf16);
+            constexpr uint32_t idesc_o = umma_idesc_f16(C::BM, HEAD, false, true, E::kBf16);
             // Descriptors of the bases; k-steps add byte offsets / 16 to the
             // start-address field (addresses stay below 256 KB).
             const uint64_t dq0 = umma_sdesc(smem_u32(sQ), 16, 8 * C::RB, C::LAYOUT);
@@ -521,43 +599,44 @@ prefill_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
                     umma_f16_ts(o_col, p_col + kk * 8, db, idesc_o, (!first || kk > 0) ? 1u : 0u);
                 }
             };
-            const int nt0 = ntiles_h[0], nt1 = ntiles_h[1];
-            bool alive = pwait<!CPA>(q_full, 0) && (ntiles == 0 || pwait<!CPA>(&full[0], 0));
-            if (alive && ntiles > 0) {
+            // Half a takes part in relative tile j when js[a] <= j < ne[a].
+            const int js0 = tr.js[0], ne0 = tr.ne[0], js1 = tr.js[1], ne1 = tr.ne[1];
+            bool alive = pwait<!CPA>(q_full, 0) && (nrel == 0 || pwait<!CPA>(&full[0], 0));
+            if (alive && nrel > 0) {
                 tc_fence_after();
-                if (nt0 > 0) issue_s(0, 0);
-                if (nt1 > 0) issue_s(1, 0);
+                if (js0 == 0 && ne0 > 0) issue_s(0, 0);
+                if (js1 == 0 && ne1 > 0) issue_s(1, 0);
                 umma_commit(&empty[0]);                  // K_0 read by both S products
             }
-            for (int j = 0; alive && j < ntiles; ++j) {
+            for (int j = 0; alive && j < nrel; ++j) {
                 const int uv = 2 * j + 1, sv = uv % C::NS;
                 const int uk = 2 * j + 2, sk = uk % C::NS;      // K_{j+1}
-                const bool more = j + 1 < ntiles;
+                const bool more = j + 1 < nrel;
                 // Both ring items of this step first (loaded tiles ago, as a rule), so
                 // that the two products of a group issue back to back.
                 if (!pwait<!CPA>(&full[sv], (uv / C::NS) & 1)) { alive = false; break; }
                 if (more && !pwait<!CPA>(&full[sk], (uk / C::NS) & 1)) { alive = false; break; }
                 // Half 0 group: P_0,j V_j, then S_0,j+1.
-                if (j < nt0) {
-                    if (!pwait<!CPA>(&p_full[0], j & 1)) { alive = false; break; }
+                if (js0 <= j && j < ne0) {
+                    if (!pwait<!CPA>(&p_full[0], (j - js0) & 1)) { alive = false; break; }
                     tc_fence_after();
-                    issue_pv(0, sv, j == 0);
-                    if (j == nt0 - 1) umma_commit(&o_full[0]);
+                    issue_pv(0, sv, j == js0);
+                    if (j == ne0 - 1) umma_commit(&o_full[0]);
                 }
-                if (more && j + 1 < nt0) {
+                if (more && js0 <= j + 1 && j + 1 < ne0) {
                     tc_fence_after();
                     issue_s(0, sk);
                 }
                 // Half 1 group: P_1,j V_j, then S_1,j+1.
-                if (j < nt1) {
-                    if (!pwait<!CPA>(&p_full[1], j & 1)) { alive = false; break; }
+                if (js1 <= j && j < ne1) {
+                    if (!pwait<!CPA>(&p_full[1], (j - js1) & 1)) { alive = false; break; }
                     tc_fence_after();
-                    issue_pv(1, sv, j == 0);
-                    if (j == nt1 - 1) umma_commit(&o_full[1]);
+                    issue_pv(1, sv, j == js1);
+                    if (j == ne1 - 1) umma_commit(&o_full[1]);
                 }
                 umma_commit(&empty[sv]);                 // V_j read by both P V products
                 if (more) {
-                    if (j + 1 < nt1) issue_s(1, sk);
+                    if (js1 <= j + 1 && j + 1 < ne1) issue_s(1, sk);
                     umma_commit(&empty[sk]);             // K_{j+1} read by both S products
                 }
             }
@@ -578,26 +657,31 @@ prefill_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
         const uint32_t lane_base = (uint32_t)((warp & 3) * 32) << 16;
         const int ia = i0 + a * tokp;                    // first token of this half
         const int tok = ia + r / g;                      // token of this row within the sequence
-        const int my_rows = a ? rows_valid[1] : rows_valid[0];
+        const int my_rows = tr.rows_valid[a];
         const int lim = (r < my_rows) ? s.past + tok : T - 1;   // last visible key
+        const int lo = (p.mods.window && r < my_rows) ? lim - p.mods.window_size : -(1 << 30);
         const int full_vis = s.past + ia;                // every row of the half sees keys <= this
-        const int nt = a ? ntiles_h[1] : ntiles_h[0];
+        // Every row of the half sees keys >= this (window only).
+        const int lo_max = p.mods.window ? s.past + min(s.q_len, ia + tokp) - 1 - p.mods.window_size
+                                         : -(1 << 30);
+        const int js = tr.js[a];
+        const int nt = tr.ne[a] - js;                    // tiles of this half
         const uint32_t scol = tmem + lane_base + (uint32_t)(a * 128);
         const uint32_t ocol = tmem + lane_base + C::COL_O + (uint32_t)(a * 128);
         float m_used = -INFINITY, l = 0.f;
         bool alive = true;
-        for (int j = 0; j < nt; ++j) {
-            if (!pwait_warp<!CPA>(&s_full[a], j & 1)) { alive = false; break; }
+        for (int jj = 0; jj < nt; ++jj) {
+            if (!pwait_warp<!CPA>(&s_full[a], jj & 1)) { alive = false; break; }
             tc_fence_after();
             uint32_t sv[C::BN];
 #pragma unroll
             for (int c = 0; c < C::BN; c += 32) tmem_ld32(scol + c, sv + c);
             tmem_wait_ld();
-            const int k0 = j * C::BN;
-            if (k0 + C::BN - 1 > full_vis) {
+            const int k0 = kbase + (js + jj) * C::BN;
+            if (k0 + C::BN - 1 > full_vis || k0 < lo_max) {
 #pragma unroll
                 for (int c = 0; c < C::BN; ++c)
-                    sv[c] = (k0 + c) <= lim ? sv[c] : __float_as_uint(-INFINITY);
+                    sv[c] = ((k0 + c) <= lim && (k0 + c) >= lo) ? sv[c] : __float_as_uint(-INFINITY);
             }
             // Row max: 8 independent chains of three-input maxima.
             float m8[8];
@@ -608,8 +692,13 @@ prefill_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
 #pragma unroll
                 for (int i = 0; i < 8; ++i)
                     m8[i] = fmax3(m8[i], __uint_as_float(sv[c + i]), __uint_as_float(sv[c + 8 + i]));
-            const float mx = p.scale_log2 *
+            const float mraw =
                 fmax3(fmax3(m8[0], m8[1], m8[2]), fmax3(m8[3], m8[4], m8[5]), fmaxf(m8[6], m8[7]));
+            // The score modifiers are increasing: the row max maps to the max.
+            const float mx = CAP ? (mraw == -INFINITY ? -INFINITY
+                                                      : softcap_log2(mraw * p.mods.scale, p.mods.softcap,
+                                                                     p.mods.inv_softcap))
+                                 : p.mods.scale_log2 * mraw;
             // Lazy rescale: a row moves its exponent base only when its max grows
             // by more than 8; the warp rescales O when any of its rows does.
             const bool grow = mx > m_used + 8.f;
@@ -618,7 +707,7 @@ prefill_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
                 const float alpha = grow ? ((m_used == -INFINITY) ? 0.f : fast_exp2(m_used - m_new)) : 1.f;
                 l *= alpha;
                 m_used = m_new;
-                if (j > 0) {
+                if (jj > 0) {
                     // s_full's commit for this tile also covered P_a V_{j-1}: O is
                     // final up to tile j-1 and no MMA writes it until P_a is ready.
 #pragma unroll
@@ -635,24 +724,32 @@ prefill_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
             const float base = (m_used == -INFINITY) ? 0.f : m_used;
             // Column pairs run on the packed f32x2 pipe: x = s * scale - base and
             // the row sums (two independent pair accumulators).
-            const uint64_t scale2 = f2_pack(p.scale_log2, p.scale_log2);
+            const uint64_t scale2 = f2_pack(p.mods.scale_log2, p.mods.scale_log2);
             const uint64_t nbase2 = f2_pack(-base, -base);
             uint64_t rs2[2] = {f2_pack(0.f, 0.f), f2_pack(0.f, 0.f)};
-            // P over S, 64 keys at a time: 64 f16 = 32 columns of this row's
-            // lane, over S columns already read into registers.
+            // P over S, 64 keys at a time: 64 16-bit values = 32 columns of this
+            // row's lane, over S columns already read into registers.
 #pragma unroll
             for (int h = 0; h < C::BN; h += 64) {
                 uint32_t pk[32];
 #pragma unroll
                 for (int c = h; c < h + 64; c += 2) {
-                    const uint64_t x2 = f2_fma(f2_pack(__uint_as_float(sv[c]), __uint_as_float(sv[c + 1])),
-                                               scale2, nbase2);
                     float x0, x1;
-                    f2_unpack(x2, x0, x1);
+                    if (CAP) {
+                        const float s0 = __uint_as_float(sv[c]), s1 = __uint_as_float(sv[c + 1]);
+                        x0 = (s0 == -INFINITY ? -INFINITY
+                                              : softcap_log2(s0 * p.mods.scale, p.mods.softcap, p.mods.inv_softcap)) - base;
+                        x1 = (s1 == -INFINITY ? -INFINITY
+                                              : softcap_log2(s1 * p.mods.scale, p.mods.softcap, p.mods.inv_softcap)) - base;
+                    } else {
+                        const uint64_t x2 = f2_fma(f2_pack(__uint_as_float(sv[c]), __uint_as_float(sv[c + 1])),
+                                                   scale2, nbase2);
+                        f2_unpack(x2, x0, x1);
+                    }
                     const float p0 = fast_exp2(x0);
                     const float p1 = fast_exp2(x1);
                     rs2[(c >> 1) & 1] = f2_add(rs2[(c >> 1) & 1], f2_pack(p0, p1));
-                    pk[(c - h) / 2] = pack_half2(p0, p1);
+                    pk[(c - h) / 2] = E::pack2(p0, p1);
                 }
                 tmem_st32(scol + h / 2, pk);
             }
@@ -667,11 +764,11 @@ prefill_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
             __syncwarp();
             if (lane == 0) mbar_arrive(&p_full[a]);
         }
-        // Epilogue: O / l -> f16 rows of `out`.
+        // Epilogue: O / l -> rows of `out` (the head's first hs columns).
         if (alive && nt > 0 && pwait_warp<!CPA>(&o_full[a], 0)) {
             tc_fence_after();
             const float inv = (l > 0.f) ? 1.f / l : 0.f;
-            __half* orow = p.out + ((long long)(s.q_start + tok) * p.q_heads + kvh * g + r % g) * HEAD;
+            uint16_t* orow = p.out + ((long long)(s.q_start + tok) * p.q_heads + kvh * g + r % g) * hs;
             // O in EPB-column batches, one round trip to tensor memory each: the
             // whole row on the TMA path; 16 columns on the cp.async path, which
             // measured faster with them.
@@ -685,11 +782,12 @@ prefill_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
                 if (r < my_rows) {
 #pragma unroll
                     for (int c0 = 0; c0 < EPB; c0 += 8) {
+                        if (h0 + c0 >= hs) continue;
                         uint4 w0;
-                        w0.x = pack_half2(__uint_as_float(ov[c0]) * inv, __uint_as_float(ov[c0 + 1]) * inv);
-                        w0.y = pack_half2(__uint_as_float(ov[c0 + 2]) * inv, __uint_as_float(ov[c0 + 3]) * inv);
-                        w0.z = pack_half2(__uint_as_float(ov[c0 + 4]) * inv, __uint_as_float(ov[c0 + 5]) * inv);
-                        w0.w = pack_half2(__uint_as_float(ov[c0 + 6]) * inv, __uint_as_float(ov[c0 + 7]) * inv);
+                        w0.x = E::pack2(__uint_as_float(ov[c0]) * inv, __uint_as_float(ov[c0 + 1]) * inv);
+                        w0.y = E::pack2(__uint_as_float(ov[c0 + 2]) * inv, __uint_as_float(ov[c0 + 3]) * inv);
+                        w0.z = E::pack2(__uint_as_float(ov[c0 + 4]) * inv, __uint_as_float(ov[c0 + 5]) * inv);
+                        w0.w = E::pack2(__uint_as_float(ov[c0 + 6]) * inv, __uint_as_float(ov[c0 + 7]) * inv);
                         *reinterpret_cast<uint4*>(orow + h0 + c0) = w0;
                     }
                 }
@@ -709,7 +807,7 @@ prefill_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
         pwait<!CPA>(q_full, 0);
         const int issued = sh[4];
         for (int u = issued - C::NS > 0 ? issued - C::NS : 0; u < issued; ++u) {
-            const bool tail = (u & 1) && ((u >> 1) * C::BN + C::BN > T);
+            const bool tail = (u & 1) && (kbase + (u >> 1) * C::BN + C::BN > T);
             if (tail) pwait<!CPA>(v_tail, 0);
             else pwait<!CPA>(&full[u % C::NS], (u / C::NS) & 1);
         }
@@ -721,11 +819,11 @@ prefill_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
     }
 }
 
-template <int HEAD, bool CPA>
+template <int HEAD, bool CPA, typename ET, bool CAP>
 cudaError_t launch_prefill_t(const CUtensorMap& tm_q, const CUtensorMap& tm_k,
                              const CUtensorMap& tm_v, const PrefillParams& p, cudaStream_t stream) {
     using C = PCfg<HEAD, CPA>;
-    auto kern = prefill_kernel<HEAD, CPA>;
+    auto kern = prefill_kernel<HEAD, CPA, ET, CAP>;
     // The register split inside the kernel assumes this launch budget; with
     // any other, setmaxnreg.inc could wait for registers that never come.
     cudaFuncAttributes fa;
@@ -739,24 +837,37 @@ cudaError_t launch_prefill_t(const CUtensorMap& tm_q, const CUtensorMap& tm_k,
     return cudaGetLastError();
 }
 
+template <int HEAD, typename ET, bool CAP>
+cudaError_t launch_prefill_h(const CUtensorMap& tm_q, const CUtensorMap& tm_k,
+                             const CUtensorMap& tm_v, const PrefillParams& p, cudaStream_t stream) {
+    return p.block_size < kPrefillKeys ? launch_prefill_t<HEAD, true, ET, CAP>(tm_q, tm_k, tm_v, p, stream)
+                                       : launch_prefill_t<HEAD, false, ET, CAP>(tm_q, tm_k, tm_v, p, stream);
+}
+
+template <typename ET, bool CAP>
+cudaError_t launch_prefill_d(const CUtensorMap& tm_q, const CUtensorMap& tm_k,
+                             const CUtensorMap& tm_v, const PrefillParams& p, int head,
+                             cudaStream_t stream) {
+    switch (head) {
+        case 16: return launch_prefill_h<16, ET, CAP>(tm_q, tm_k, tm_v, p, stream);
+        case 32: return launch_prefill_h<32, ET, CAP>(tm_q, tm_k, tm_v, p, stream);
+        case 64: return launch_prefill_h<64, ET, CAP>(tm_q, tm_k, tm_v, p, stream);
+        case 128: return launch_prefill_h<128, ET, CAP>(tm_q, tm_k, tm_v, p, stream);
+        default: return cudaErrorInvalidValue;
+    }
+}
+
 }  // namespace
 
 cudaError_t launch_prefill(const CUtensorMap& tm_q, const CUtensorMap& tm_k,
-                           const CUtensorMap& tm_v, const PrefillParams& p, int head_size,
+                           const CUtensorMap& tm_v, const PrefillParams& p, int head, bool bf16,
                            cudaStream_t stream) {
-    const bool cpa = p.block_size < kPrefillKeys;
-#define PA_PREFILL_CASE(H)                                                               \
-    case H:                                                                              \
-        return cpa ? launch_prefill_t<H, true>(tm_q, tm_k, tm_v, p, stream)              \
-                   : launch_prefill_t<H, false>(tm_q, tm_k, tm_v, p, stream);
-    switch (head_size) {
-        PA_PREFILL_CASE(16)
-        PA_PREFILL_CASE(32)
-        PA_PREFILL_CASE(64)
-        PA_PREFILL_CASE(128)
-        default: return cudaErrorInvalidValue;
-    }
-#undef PA_PREFILL_CASE
+    const bool cap = p.mods.softcap > 0.f;
+    if (bf16)
+        return cap ? launch_prefill_d<__nv_bfloat16, true>(tm_q, tm_k, tm_v, p, head, stream)
+                   : launch_prefill_d<__nv_bfloat16, false>(tm_q, tm_k, tm_v, p, head, stream);
+    return cap ? launch_prefill_d<__half, true>(tm_q, tm_k, tm_v, p, head, stream)
+               : launch_prefill_d<__half, false>(tm_q, tm_k, tm_v, p, head, stream);
 }
 
 }  // namespace pa

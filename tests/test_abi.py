@@ -52,9 +52,12 @@ FAKE = 1 << 20          # aligned non-null address; never dereferenced (calls fa
 
 @pytest.mark.parametrize("kw,status", [
     (dict(q_heads=6, kv_heads=4), 1),            # not a multiple
-    (dict(q_heads=12, kv_heads=4), 2),           # group 3: not built
+    (dict(q_heads=48, kv_heads=1), 2),           # group 48: not built (decode rows <= 32)
     (dict(head_size=20), 1),                     # not a multiple of 8
-    (dict(head_size=96), 2),                     # valid per the pages, not built
+    (dict(head_size=264), 1),                    # beyond 256
+    (dict(head_size=192), 2),                    # valid, attention not built past 128
+    (dict(softcap=-1.0), 1),
+    (dict(window=-2), 1),
     (dict(block_size=24), 1),
     (dict(block_size=512), 1),
     (dict(num_blocks=1 << 28, block_size=16), 1),  # slots overflow int32
@@ -65,14 +68,6 @@ def test_dims_rejected_before_launch(pa, kw, status):
     with pytest.raises(pa.PagedAttentionError) as e:
         pa.pa_attention(FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, 0.0, FAKE, d, None, 0, None, 0)
     assert e.value.status == status
-
-
-def test_bf16_attention_is_not_implemented(pa):
-    d = _dims(pa, dtype=pa.PA_DTYPE_BF16)
-    with pytest.raises(pa.PagedAttentionError) as e:
-        pa.pa_attention(FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, 0.0, FAKE, d, FAKE, 1 << 30, None, 0)
-    assert e.value.status == pa.PA_ERR_NOT_IMPLEMENTED
-    assert "bfloat16" in str(e.value)
 
 
 def _rotary(pa, rd, inter=0, maxpos=64):

@@ -33,6 +33,7 @@ class Spec:
     num_blocks: int             # physical pages in the pool
     dist: str = "normal"        # "normal" -> N(0,1), "uniform" -> U[-1,1]
     seed: int = 0
+    elem: str = "f16"           # "f16": float16 arrays; "bf16": bfloat16 bit patterns as uint16
     extra: dict = field(default_factory=dict)
 
     @property
@@ -120,25 +121,46 @@ CONFIG_KEYS = {
 
 
 def custom(q_lens, past, q_heads, kv_heads, head_size, block_size, num_blocks=None,
-           dist="normal", seed=7, name="custom") -> Spec:
+           dist="normal", seed=7, name="custom", elem="f16") -> Spec:
     q = np.asarray(q_lens, dtype=np.int64)
     p = np.asarray(past, dtype=np.int64)
-    s = Spec(name, q, p, q_heads, kv_heads, head_size, block_size, 0, dist=dist, seed=seed)
+    s = Spec(name, q, p, q_heads, kv_heads, head_size, block_size, 0, dist=dist, seed=seed,
+             elem=elem)
     need = _pool(s.pages_per_seq)
     s.num_blocks = max(need, 1) if num_blocks is None else int(num_blocks)
     assert s.num_blocks >= need
     return s
 
 
-def _draw(rng, n, dist, chunk=1 << 24):
-    out = np.empty(n, dtype=np.float16)
+def _to_bf16_bits(x: np.ndarray) -> np.ndarray:
+    """float32 -> bfloat16 bit patterns (uint16), rounded to nearest-even by torch."""
+    import torch
+    return torch.from_numpy(np.ascontiguousarray(x, dtype=np.float32)).to(torch.bfloat16) \
+        .view(torch.int16).numpy().view(np.uint16)
+
+
+BF16_NAN = np.uint16(0x7FC0)
+
+
+def _draw(rng, n, dist, elem="f16", chunk=1 << 24):
+    out = np.empty(n, dtype=np.uint16 if elem == "bf16" else np.float16)
     for lo in range(0, n, chunk):
         hi = min(n, lo + chunk)
         if dist == "uniform":
-            out[lo:hi] = rng.uniform(-1.0, 1.0, size=hi - lo)
+            v = rng.uniform(-1.0, 1.0, size=hi - lo)
         else:
-            out[lo:hi] = rng.standard_normal(size=hi - lo, dtype=np.float32)
+            v = rng.standard_normal(size=hi - lo, dtype=np.float32)
+        out[lo:hi] = _to_bf16_bits(v) if elem == "bf16" else v
     return out
+
+
+def fill_value(elem: str, fill: float):
+    """`fill` in the element type's storage (bf16: its bit pattern)."""
+    if elem != "bf16":
+        return fill
+    if np.isnan(fill):
+        return BF16_NAN
+    return _to_bf16_bits(np.array([fill], dtype=np.float32))[0]
 
 
 def generate(spec: Spec, fill: float = 0.0, seed: int | None = None, block_order=None) -> dict:
@@ -148,7 +170,8 @@ def generate(spec: Spec, fill: float = 0.0, seed: int | None = None, block_order
     (the new tokens), key_cache/value_cache [num_blocks, block_size, kv_heads,
     d], block_table int32 [batch, max_blocks_per_seq] (-1 past a sequence's
     pages), cu_seqlens_q int32 [batch + 1], seqlens_kv int32 [batch], all
-    float16 where floating point.  ``block_order`` overrides the seeded pool
+    float16 where floating point (bfloat16 bit patterns as uint16 when
+    ``spec.elem`` is "bf16").  ``block_order`` overrides the seeded pool
     permutation (used by the page-permutation tests).
     """
     rng = np.random.Generator(np.random.PCG64(spec.seed if seed is None else seed))
@@ -167,16 +190,18 @@ def generate(spec: Spec, fill: float = 0.0, seed: int | None = None, block_order
         nxt += n
     T = spec.token_count
     qh, kvh, d, bs = spec.q_heads, spec.kv_heads, spec.head_size, spec.block_size
-    query = _draw(rng, T * qh * d, spec.dist).reshape(T, qh, d)
-    key = _draw(rng, T * kvh * d, spec.dist).reshape(T, kvh, d)
-    value = _draw(rng, T * kvh * d, spec.dist).reshape(T, kvh, d)
-    key_cache = np.full((spec.num_blocks, bs, kvh, d), fill, dtype=np.float16)
-    value_cache = np.full((spec.num_blocks, bs, kvh, d), fill, dtype=np.float16)
+    el = spec.elem
+    query = _draw(rng, T * qh * d, spec.dist, el).reshape(T, qh, d)
+    key = _draw(rng, T * kvh * d, spec.dist, el).reshape(T, kvh, d)
+    value = _draw(rng, T * kvh * d, spec.dist, el).reshape(T, kvh, d)
+    cdt = np.uint16 if el == "bf16" else np.float16
+    key_cache = np.full((spec.num_blocks, bs, kvh, d), fill_value(el, fill), dtype=cdt)
+    value_cache = np.full((spec.num_blocks, bs, kvh, d), fill_value(el, fill), dtype=cdt)
     used = block_table[block_table >= 0]
     per_page = bs * kvh * d
     for cache in (key_cache, value_cache):
         flat = cache.reshape(spec.num_blocks, per_page)
-        vals = _draw(rng, used.size * per_page, spec.dist).reshape(used.size, per_page)
+        vals = _draw(rng, used.size * per_page, spec.dist, el).reshape(used.size, per_page)
         flat[used] = vals
     cu = np.zeros(spec.batch + 1, dtype=np.int32)
     cu[1:] = np.cumsum(spec.q_lens)
