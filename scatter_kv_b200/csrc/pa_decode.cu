@@ -95,10 +95,11 @@ __device__ __forceinline__ uint32_t half2_mask(uint32_t v, bool lo_ok, bool hi_o
 // chunks of p.chunk in logical order.  Without a local window k_first is 0;
 // with one it is the first key any of the sequence's rows can see, rounded
 // down to the 32-key tile.
+template <bool GEN>
 __device__ __forceinline__ void decode_range(const SeqInfo& s, const DecodeParams& p, int& k_first,
                                              int& n_splits) {
     k_first = 0;
-    if (p.mods.window) {
+    if (GEN && p.mods.window) {
         const int lo = s.past - p.mods.window_size;
         if (lo > 0) k_first = lo & ~(kDecodeKeys - 1);
     }
@@ -111,7 +112,20 @@ __device__ __forceinline__ long long out_row(const DecodeParams& p, const SeqInf
     return ((long long)(s.q_start + r / p.group) * p.q_heads + kvh * p.group + r % p.group) * p.head_size;
 }
 
-template <int HEAD, int MT, bool CPA, typename ET, bool CAP>
+// Rows [0, rows) of KV head kvh of sequence s set to zero (invalid
+// metadata), 16 bytes per store.
+__device__ __forceinline__ void zero_rows(const DecodeParams& p, const SeqInfo& s, int kvh, int rows,
+                                       int threads) {
+    const int per_row = p.head_size / 8;
+#pragma unroll 1
+    for (int r = threadIdx.x / per_row; r < rows; r += threads / per_row) {
+        const int c = threadIdx.x % per_row;
+        if (threadIdx.x < (threads / per_row) * per_row)
+            *reinterpret_cast<uint4*>(p.out + out_row(p, s, kvh, r) + c * 8) = make_uint4(0, 0, 0, 0);
+    }
+}
+
+template <int HEAD, int MT, bool CPA, typename ET, bool GEN>
 __global__ void __launch_bounds__(Cfg<HEAD, MT, CPA>::THREADS, (HEAD >= 128 && !CPA) ? 2 : 3)
 decode_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_v,
               const DecodeParams p) {
@@ -137,7 +151,7 @@ decode_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ 
     const int b = blockIdx.z, kvh = blockIdx.x, split = blockIdx.y;
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int g = p.group;
-    const int hs = p.head_size;
+    const int hs = GEN ? p.head_size : HEAD;   // the general build pads heads
     // Status bits of a sequence are reported once, by CTA (split 0, kv head 0).
     const bool reporter = (split == 0 && kvh == 0 && threadIdx.x == 0);
 
@@ -156,8 +170,7 @@ decode_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ 
             if (reporter)
                 load_seq(p.cu_seqlens_q, p.seqlens_kv, b, p.batch, p.token_count, p.kv_cap,
                          p.kv_hint, p.q_hint, p.status, s);
-            for (int idx = threadIdx.x; idx < s.q_len * g * hs; idx += C::THREADS)
-                p.out[out_row(p, s, kvh, idx / hs) + idx % hs] = 0;
+            zero_rows(p, s, kvh, s.q_len * g, C::THREADS);
         }
         return;
     }
@@ -168,14 +181,12 @@ decode_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ 
         if (reporter)
             load_seq(p.cu_seqlens_q, p.seqlens_kv, b, p.batch, p.token_count, p.kv_cap,
                      p.kv_hint, p.q_hint, p.status, s);
-        if (split == 0)
-            for (int idx = threadIdx.x; idx < R * hs; idx += C::THREADS)
-                p.out[out_row(p, s, kvh, idx / hs) + idx % hs] = 0;
+        if (split == 0) zero_rows(p, s, kvh, R, C::THREADS);
         return;
     }
     const int T = s.kv_len;
     int k_first, n_splits;
-    decode_range(s, p, k_first, n_splits);
+    decode_range<GEN>(s, p, k_first, n_splits);
     if (split >= n_splits) return;
 
     if (threadIdx.x == 0) {
@@ -193,6 +204,7 @@ decode_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ 
         // Columns past the head size: zero in every stage, once (the copies
         // never write them; TMA fills them with zeros by itself).
         constexpr int CH = C::RB / 16;
+#pragma unroll 1
         for (int idx = threadIdx.x; idx < C::NST * 2 * C::BN * (HEAD / 8); idx += C::THREADS) {
             const int jc = idx % (HEAD / 8);
             if (jc * 8 < hs) continue;
@@ -334,7 +346,7 @@ decode_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ 
         for (int h = 0; h < 2; ++h) {
             const int r = rows[h];
             lim[h] = (r < R) ? (s.past + r / g) : (T - 1);
-            lo[h] = p.mods.window ? lim[h] - p.mods.window_size : -(1 << 30);
+            lo[h] = (GEN && p.mods.window) ? lim[h] - p.mods.window_size : -(1 << 30);
         }
         // Q fragments (A operand) straight from global memory; columns past
         // the head size are zero.
@@ -411,8 +423,10 @@ decode_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ 
                 for (int e = 0; e < 4; ++e) {
                     const int h = e >> 1;
                     const int key = k0 + nt * 8 + 2 * qid + (e & 1);
-                    const bool vis = key < k_end && key <= lim[h] && key >= lo[h];
-                    const float sc = CAP ? softcap_log2(sacc[nt][e] * p.mods.scale, p.mods.softcap,
+                    bool vis = key < k_end && key <= lim[h];
+                    if (GEN) vis = vis && key >= lo[h];
+                    const float sc = (GEN && p.mods.softcap > 0.f)
+                                         ? softcap_log2(sacc[nt][e] * p.mods.scale, p.mods.softcap,
                                                         p.mods.inv_softcap)
                                          : sacc[nt][e] * p.mods.scale_log2;
                     const float v = vis ? sc : -INFINITY;
@@ -583,7 +597,7 @@ __global__ void __launch_bounds__(128) combine_kernel(const DecodeParams p) {
         return;
     if (s.q_len == 0 || s.q_len > p.decode_max_q || r >= s.q_len * p.group) return;
     int k_first, n_splits;
-    decode_range(s, p, k_first, n_splits);
+    decode_range<true>(s, p, k_first, n_splits);
     if (n_splits == 1) return;                        // the decode kernel wrote the row
     uint16_t* orow = p.out + out_row(p, s, kvh, r);
     float M = -INFINITY;
@@ -623,11 +637,11 @@ __global__ void __launch_bounds__(128) combine_kernel(const DecodeParams p) {
     *reinterpret_cast<uint2*>(orow + lane * 4) = wv;
 }
 
-template <int HEAD, int MT, bool CPA, typename ET, bool CAP>
+template <int HEAD, int MT, bool CPA, typename ET, bool GEN>
 cudaError_t launch_decode_t(const CUtensorMap& tm_k, const CUtensorMap& tm_v,
                             const DecodeParams& p, cudaStream_t stream) {
     using C = Cfg<HEAD, MT, CPA>;
-    auto kern = decode_kernel<HEAD, MT, CPA, ET, CAP>;
+    auto kern = decode_kernel<HEAD, MT, CPA, ET, GEN>;
     cudaError_t e;
     if (CPA) {
         cudaFuncAttributes fa;
@@ -645,25 +659,25 @@ cudaError_t launch_decode_t(const CUtensorMap& tm_k, const CUtensorMap& tm_v,
     return cudaGetLastError();
 }
 
-template <int HEAD, typename ET, bool CAP>
+template <int HEAD, typename ET, bool GEN>
 cudaError_t launch_decode_h(const CUtensorMap& tm_k, const CUtensorMap& tm_v, const DecodeParams& p,
                             int mtiles, cudaStream_t stream) {
     const bool cpa = p.block_size < kDecodeKeys;
     if (cpa)
-        return mtiles == 1 ? launch_decode_t<HEAD, 1, true, ET, CAP>(tm_k, tm_v, p, stream)
-                           : launch_decode_t<HEAD, 2, true, ET, CAP>(tm_k, tm_v, p, stream);
-    return mtiles == 1 ? launch_decode_t<HEAD, 1, false, ET, CAP>(tm_k, tm_v, p, stream)
-                       : launch_decode_t<HEAD, 2, false, ET, CAP>(tm_k, tm_v, p, stream);
+        return mtiles == 1 ? launch_decode_t<HEAD, 1, true, ET, GEN>(tm_k, tm_v, p, stream)
+                           : launch_decode_t<HEAD, 2, true, ET, GEN>(tm_k, tm_v, p, stream);
+    return mtiles == 1 ? launch_decode_t<HEAD, 1, false, ET, GEN>(tm_k, tm_v, p, stream)
+                       : launch_decode_t<HEAD, 2, false, ET, GEN>(tm_k, tm_v, p, stream);
 }
 
-template <typename ET, bool CAP>
+template <typename ET, bool GEN>
 cudaError_t launch_decode_d(const CUtensorMap& tm_k, const CUtensorMap& tm_v, const DecodeParams& p,
                             int head, int mtiles, cudaStream_t stream) {
     switch (head) {
-        case 16: return launch_decode_h<16, ET, CAP>(tm_k, tm_v, p, mtiles, stream);
-        case 32: return launch_decode_h<32, ET, CAP>(tm_k, tm_v, p, mtiles, stream);
-        case 64: return launch_decode_h<64, ET, CAP>(tm_k, tm_v, p, mtiles, stream);
-        case 128: return launch_decode_h<128, ET, CAP>(tm_k, tm_v, p, mtiles, stream);
+        case 16: return launch_decode_h<16, ET, GEN>(tm_k, tm_v, p, mtiles, stream);
+        case 32: return launch_decode_h<32, ET, GEN>(tm_k, tm_v, p, mtiles, stream);
+        case 64: return launch_decode_h<64, ET, GEN>(tm_k, tm_v, p, mtiles, stream);
+        case 128: return launch_decode_h<128, ET, GEN>(tm_k, tm_v, p, mtiles, stream);
         default: return cudaErrorInvalidValue;
     }
 }
@@ -711,11 +725,14 @@ int padded_head(int head_size) {
 
 cudaError_t launch_decode(const CUtensorMap& tm_k, const CUtensorMap& tm_v,
                           const DecodeParams& p, int head, int mtiles, bool bf16, cudaStream_t stream) {
-    const bool cap = p.mods.softcap > 0.f;
+    // The general build takes the score modifiers (softcap, local window)
+    // and a head size below the kernel's at run time; the plain build, for
+    // the common case, has none of their code.
+    const bool gen = p.mods.softcap > 0.f || p.mods.window || p.head_size != head;
     if (bf16)
-        return cap ? launch_decode_d<__nv_bfloat16, true>(tm_k, tm_v, p, head, mtiles, stream)
+        return gen ? launch_decode_d<__nv_bfloat16, true>(tm_k, tm_v, p, head, mtiles, stream)
                    : launch_decode_d<__nv_bfloat16, false>(tm_k, tm_v, p, head, mtiles, stream);
-    return cap ? launch_decode_d<__half, true>(tm_k, tm_v, p, head, mtiles, stream)
+    return gen ? launch_decode_d<__half, true>(tm_k, tm_v, p, head, mtiles, stream)
                : launch_decode_d<__half, false>(tm_k, tm_v, p, head, mtiles, stream);
 }
 

@@ -191,6 +191,7 @@ struct TileRange {
     int rows_valid[2];
 };
 
+template <bool GEN>
 __device__ __forceinline__ TileRange tile_range(int past, int q_len, int pair, int tokp, int g,
                                                 const ScoreMods& m) {
     TileRange t;
@@ -206,7 +207,7 @@ __device__ __forceinline__ TileRange tile_range(int past, int q_len, int pair, i
         end[a] = 0;
         if (t.rows_valid[a] > 0) {
             end[a] = (past + last + 1 + kPrefillKeys - 1) / kPrefillKeys;
-            if (m.window) first[a] = max(0, past + ia - m.window_size) / kPrefillKeys;
+            if (GEN && m.window) first[a] = max(0, past + ia - m.window_size) / kPrefillKeys;
             jlo = min(jlo, first[a]);
             jhi = max(jhi, end[a]);
         }
@@ -235,7 +236,7 @@ __device__ __forceinline__ bool pwait_warp(uint64_t* bar, uint32_t parity) {
     return LEAN ? mbar_wait_warp_lean(bar, parity) : mbar_wait_warp(bar, parity);
 }
 
-template <int HEAD, bool CPA, typename ET, bool CAP>
+template <int HEAD, bool CPA, typename ET, bool GEN>
 __global__ void __launch_bounds__(PCfg<HEAD, CPA>::THREADS, 1)
 prefill_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                const __grid_constant__ CUtensorMap tm_v, const PrefillParams p) {
@@ -258,7 +259,7 @@ prefill_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int g = p.group;
-    const int hs = p.head_size;
+    const int hs = GEN ? p.head_size : HEAD;   // the general build pads heads
 
     if ((smem_u32(smem) & 1023u) != 0) {              // the swizzle needs 1024-B alignment
         if (threadIdx.x == 0) flag_status(p.status, PA_DEV_TIMEOUT);
@@ -320,7 +321,7 @@ prefill_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
                 }
                 // Block-table check (the row's ids in range), keeping the id of
                 // the page that holds the first key tile.
-                const TileRange tr = tile_range(si.past, si.q_len, w.pair, tokp, g, p.mods);
+                const TileRange tr = tile_range<GEN>(si.past, si.q_len, w.pair, tokp, g, p.mods);
                 const int key0 = tr.jlo * C::BN;
                 const int pg_first = key0 / p.block_size;
                 const int npages = (si.kv_len + p.block_size - 1) / p.block_size;
@@ -359,31 +360,22 @@ prefill_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
             sh[8] = si.q_len;
             sh[9] = si.kv_len;
         }
-    } else if (warp >= 4 && warp < 8) {
-        // Shared memory that no copy writes, zeroed once (generic stores, made
-        // visible to the tensor cores): Q rows past the group's rows, and on the
-        // cp.async path the ring's columns past the head size (TMA fills those
-        // with zeros by itself).
+    } else if (CPA && warp >= 4 && warp < 8 && hs < HEAD) {
+        // The ring's columns past the head size: no copy writes them (TMA
+        // fills them with zeros by itself), so they are zeroed once here and
+        // made visible to the tensor cores.  (Q rows past the group's rows
+        // need nothing: they only feed output rows that are never written.)
         const int t4 = threadIdx.x - 128;
-        for (int idx = t4; idx < 2 * C::NA * (C::BM - qrows) * (C::RB / 16); idx += 128) {
-            const int ch = idx % (C::RB / 16);
-            const int r = qrows + (idx / (C::RB / 16)) % (C::BM - qrows);
-            const int ac = idx / ((C::RB / 16) * (C::BM - qrows));     // half * NA + column block
-            *reinterpret_cast<uint4*>(smem + C::OFF_Q + (ac / C::NA) * C::Q_BYTES +
-                                      (ac % C::NA) * C::BM * C::RB +
-                                      swz<C::RB>((uint32_t)(r * C::RB + ch * 16))) = make_uint4(0, 0, 0, 0);
-        }
-        if (CPA && hs < HEAD) {
-            for (int idx = t4; idx < C::NS * C::BN * (HEAD / 8); idx += 128) {
-                const int jc = idx % (HEAD / 8);
-                if (jc * 8 < hs) continue;
-                const int r = (idx / (HEAD / 8)) % C::BN;
-                const int st = idx / (HEAD / 8 * C::BN);
-                const int c = (jc * 8) / C::A, jj = jc % (C::A / 8);
-                *reinterpret_cast<uint4*>(smem + C::OFF_RING + st * C::KV_BYTES +
-                                          swz<C::RB>((uint32_t)((c * C::BN + r) * C::RB + jj * 16))) =
-                    make_uint4(0, 0, 0, 0);
-            }
+#pragma unroll 1
+        for (int idx = t4; idx < C::NS * C::BN * (HEAD / 8); idx += 128) {
+            const int jc = idx % (HEAD / 8);
+            if (jc * 8 < hs) continue;
+            const int r = (idx / (HEAD / 8)) % C::BN;
+            const int st = idx / (HEAD / 8 * C::BN);
+            const int c = (jc * 8) / C::A, jj = jc % (C::A / 8);
+            *reinterpret_cast<uint4*>(smem + C::OFF_RING + st * C::KV_BYTES +
+                                      swz<C::RB>((uint32_t)((c * C::BN + r) * C::RB + jj * 16))) =
+                make_uint4(0, 0, 0, 0);
         }
         fence_proxy_async_smem();
     }
@@ -400,16 +392,18 @@ prefill_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
     s.kv_len = sh[9];
     s.past = s.kv_len - s.q_len;
     const int i0 = pair * 2 * tokp;                              // first token of half 0
-    const TileRange tr = tile_range(s.past, s.q_len, pair, tokp, g, p.mods);
+    const TileRange tr = tile_range<GEN>(s.past, s.q_len, pair, tokp, g, p.mods);
     const int T = s.kv_len;
     if (b < 0 || sh[2] != 0) {
         if (b >= 0) {
             // Invalid sequence or block table: its rows of `out` are zero.
             const int rows = tr.rows_valid[0] + tr.rows_valid[1];
-            for (int idx = threadIdx.x; idx < rows * hs; idx += C::THREADS) {
-                const int r = idx / hs, d = idx % hs;
-                const long long o = ((long long)(s.q_start + i0 + r / g) * p.q_heads + kvh * g + r % g) * hs + d;
-                p.out[o] = 0;
+#pragma unroll 1
+            for (int r = warp; r < rows; r += C::THREADS / 32) {
+                uint16_t* orow = p.out + ((long long)(s.q_start + i0 + r / g) * p.q_heads + kvh * g + r % g) * hs;
+#pragma unroll 1
+                for (int d = lane * 8; d < hs; d += 256)
+                    *reinterpret_cast<uint4*>(orow + d) = make_uint4(0, 0, 0, 0);
             }
             // Q's copy lands before the CTA's shared memory is released.
             if (sh[2] == 2 && threadIdx.x == 0) pwait<!CPA>(q_full, 0);
@@ -657,15 +651,17 @@ prefill_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
         const uint32_t lane_base = (uint32_t)((warp & 3) * 32) << 16;
         const int ia = i0 + a * tokp;                    // first token of this half
         const int tok = ia + r / g;                      // token of this row within the sequence
-        const int my_rows = tr.rows_valid[a];
+        const int my_rows = a ? tr.rows_valid[1] : tr.rows_valid[0];
         const int lim = (r < my_rows) ? s.past + tok : T - 1;   // last visible key
-        const int lo = (p.mods.window && r < my_rows) ? lim - p.mods.window_size : -(1 << 30);
+        const bool win = GEN && p.mods.window;
+        const bool cap = GEN && p.mods.softcap > 0.f;
+        const int lo = (win && r < my_rows) ? lim - p.mods.window_size : -(1 << 30);
         const int full_vis = s.past + ia;                // every row of the half sees keys <= this
         // Every row of the half sees keys >= this (window only).
-        const int lo_max = p.mods.window ? s.past + min(s.q_len, ia + tokp) - 1 - p.mods.window_size
-                                         : -(1 << 30);
-        const int js = tr.js[a];
-        const int nt = tr.ne[a] - js;                    // tiles of this half
+        const int lo_max = win ? s.past + min(s.q_len, ia + tokp) - 1 - p.mods.window_size
+                               : -(1 << 30);
+        const int js = a ? tr.js[1] : tr.js[0];
+        const int nt = (a ? tr.ne[1] : tr.ne[0]) - js;   // tiles of this half
         const uint32_t scol = tmem + lane_base + (uint32_t)(a * 128);
         const uint32_t ocol = tmem + lane_base + C::COL_O + (uint32_t)(a * 128);
         float m_used = -INFINITY, l = 0.f;
@@ -678,10 +674,16 @@ prefill_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
             for (int c = 0; c < C::BN; c += 32) tmem_ld32(scol + c, sv + c);
             tmem_wait_ld();
             const int k0 = kbase + (js + jj) * C::BN;
-            if (k0 + C::BN - 1 > full_vis || k0 < lo_max) {
+            if (GEN && win) {
+                if (k0 + C::BN - 1 > full_vis || k0 < lo_max) {
+#pragma unroll
+                    for (int c = 0; c < C::BN; ++c)
+                        sv[c] = ((k0 + c) <= lim && (k0 + c) >= lo) ? sv[c] : __float_as_uint(-INFINITY);
+                }
+            } else if (k0 + C::BN - 1 > full_vis) {
 #pragma unroll
                 for (int c = 0; c < C::BN; ++c)
-                    sv[c] = ((k0 + c) <= lim && (k0 + c) >= lo) ? sv[c] : __float_as_uint(-INFINITY);
+                    sv[c] = (k0 + c) <= lim ? sv[c] : __float_as_uint(-INFINITY);
             }
             // Row max: 8 independent chains of three-input maxima.
             float m8[8];
@@ -695,7 +697,7 @@ prefill_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
             const float mraw =
                 fmax3(fmax3(m8[0], m8[1], m8[2]), fmax3(m8[3], m8[4], m8[5]), fmaxf(m8[6], m8[7]));
             // The score modifiers are increasing: the row max maps to the max.
-            const float mx = CAP ? (mraw == -INFINITY ? -INFINITY
+            const float mx = cap ? (mraw == -INFINITY ? -INFINITY
                                                       : softcap_log2(mraw * p.mods.scale, p.mods.softcap,
                                                                      p.mods.inv_softcap))
                                  : p.mods.scale_log2 * mraw;
@@ -724,9 +726,22 @@ prefill_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
             const float base = (m_used == -INFINITY) ? 0.f : m_used;
             // Column pairs run on the packed f32x2 pipe: x = s * scale - base and
             // the row sums (two independent pair accumulators).
-            const uint64_t scale2 = f2_pack(p.mods.scale_log2, p.mods.scale_log2);
             const uint64_t nbase2 = f2_pack(-base, -base);
             uint64_t rs2[2] = {f2_pack(0.f, 0.f), f2_pack(0.f, 0.f)};
+            // Softcap: the capped score replaces S in place (masked keys stay
+            // -inf), and from here on the scale is 1.
+            float sc2 = p.mods.scale_log2;
+            if (GEN && cap) {
+#pragma unroll
+                for (int c = 0; c < C::BN; ++c) {
+                    const float sc = __uint_as_float(sv[c]);
+                    sv[c] = __float_as_uint(sc == -INFINITY ? -INFINITY
+                                                            : softcap_log2(sc * p.mods.scale, p.mods.softcap,
+                                                                           p.mods.inv_softcap));
+                }
+                sc2 = 1.f;
+            }
+            const uint64_t scale2 = f2_pack(sc2, sc2);
             // P over S, 64 keys at a time: 64 16-bit values = 32 columns of this
             // row's lane, over S columns already read into registers.
 #pragma unroll
@@ -735,17 +750,9 @@ prefill_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
 #pragma unroll
                 for (int c = h; c < h + 64; c += 2) {
                     float x0, x1;
-                    if (CAP) {
-                        const float s0 = __uint_as_float(sv[c]), s1 = __uint_as_float(sv[c + 1]);
-                        x0 = (s0 == -INFINITY ? -INFINITY
-                                              : softcap_log2(s0 * p.mods.scale, p.mods.softcap, p.mods.inv_softcap)) - base;
-                        x1 = (s1 == -INFINITY ? -INFINITY
-                                              : softcap_log2(s1 * p.mods.scale, p.mods.softcap, p.mods.inv_softcap)) - base;
-                    } else {
-                        const uint64_t x2 = f2_fma(f2_pack(__uint_as_float(sv[c]), __uint_as_float(sv[c + 1])),
-                                                   scale2, nbase2);
-                        f2_unpack(x2, x0, x1);
-                    }
+                    const uint64_t x2 = f2_fma(f2_pack(__uint_as_float(sv[c]), __uint_as_float(sv[c + 1])),
+                                               scale2, nbase2);
+                    f2_unpack(x2, x0, x1);
                     const float p0 = fast_exp2(x0);
                     const float p1 = fast_exp2(x1);
                     rs2[(c >> 1) & 1] = f2_add(rs2[(c >> 1) & 1], f2_pack(p0, p1));
@@ -819,11 +826,11 @@ prefill_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
     }
 }
 
-template <int HEAD, bool CPA, typename ET, bool CAP>
+template <int HEAD, bool CPA, typename ET, bool GEN>
 cudaError_t launch_prefill_t(const CUtensorMap& tm_q, const CUtensorMap& tm_k,
                              const CUtensorMap& tm_v, const PrefillParams& p, cudaStream_t stream) {
     using C = PCfg<HEAD, CPA>;
-    auto kern = prefill_kernel<HEAD, CPA, ET, CAP>;
+    auto kern = prefill_kernel<HEAD, CPA, ET, GEN>;
     // The register split inside the kernel assumes this launch budget; with
     // any other, setmaxnreg.inc could wait for registers that never come.
     cudaFuncAttributes fa;
@@ -837,22 +844,22 @@ cudaError_t launch_prefill_t(const CUtensorMap& tm_q, const CUtensorMap& tm_k,
     return cudaGetLastError();
 }
 
-template <int HEAD, typename ET, bool CAP>
+template <int HEAD, typename ET, bool GEN>
 cudaError_t launch_prefill_h(const CUtensorMap& tm_q, const CUtensorMap& tm_k,
                              const CUtensorMap& tm_v, const PrefillParams& p, cudaStream_t stream) {
-    return p.block_size < kPrefillKeys ? launch_prefill_t<HEAD, true, ET, CAP>(tm_q, tm_k, tm_v, p, stream)
-                                       : launch_prefill_t<HEAD, false, ET, CAP>(tm_q, tm_k, tm_v, p, stream);
+    return p.block_size < kPrefillKeys ? launch_prefill_t<HEAD, true, ET, GEN>(tm_q, tm_k, tm_v, p, stream)
+                                       : launch_prefill_t<HEAD, false, ET, GEN>(tm_q, tm_k, tm_v, p, stream);
 }
 
-template <typename ET, bool CAP>
+template <typename ET, bool GEN>
 cudaError_t launch_prefill_d(const CUtensorMap& tm_q, const CUtensorMap& tm_k,
                              const CUtensorMap& tm_v, const PrefillParams& p, int head,
                              cudaStream_t stream) {
     switch (head) {
-        case 16: return launch_prefill_h<16, ET, CAP>(tm_q, tm_k, tm_v, p, stream);
-        case 32: return launch_prefill_h<32, ET, CAP>(tm_q, tm_k, tm_v, p, stream);
-        case 64: return launch_prefill_h<64, ET, CAP>(tm_q, tm_k, tm_v, p, stream);
-        case 128: return launch_prefill_h<128, ET, CAP>(tm_q, tm_k, tm_v, p, stream);
+        case 16: return launch_prefill_h<16, ET, GEN>(tm_q, tm_k, tm_v, p, stream);
+        case 32: return launch_prefill_h<32, ET, GEN>(tm_q, tm_k, tm_v, p, stream);
+        case 64: return launch_prefill_h<64, ET, GEN>(tm_q, tm_k, tm_v, p, stream);
+        case 128: return launch_prefill_h<128, ET, GEN>(tm_q, tm_k, tm_v, p, stream);
         default: return cudaErrorInvalidValue;
     }
 }
@@ -862,11 +869,16 @@ cudaError_t launch_prefill_d(const CUtensorMap& tm_q, const CUtensorMap& tm_k,
 cudaError_t launch_prefill(const CUtensorMap& tm_q, const CUtensorMap& tm_k,
                            const CUtensorMap& tm_v, const PrefillParams& p, int head, bool bf16,
                            cudaStream_t stream) {
-    const bool cap = p.mods.softcap > 0.f;
+    // The general build takes the score modifiers (softcap, local window), a
+    // head size below the kernel's and a group that does not divide the
+    // 128-row tile at run time; the plain build, for the common case, has
+    // none of their code.
+    const bool gen = p.mods.softcap > 0.f || p.mods.window || p.head_size != head ||
+                     kPrefillRows % p.group != 0;
     if (bf16)
-        return cap ? launch_prefill_d<__nv_bfloat16, true>(tm_q, tm_k, tm_v, p, head, stream)
+        return gen ? launch_prefill_d<__nv_bfloat16, true>(tm_q, tm_k, tm_v, p, head, stream)
                    : launch_prefill_d<__nv_bfloat16, false>(tm_q, tm_k, tm_v, p, head, stream);
-    return cap ? launch_prefill_d<__half, true>(tm_q, tm_k, tm_v, p, head, stream)
+    return gen ? launch_prefill_d<__half, true>(tm_q, tm_k, tm_v, p, head, stream)
                : launch_prefill_d<__half, false>(tm_q, tm_k, tm_v, p, head, stream);
 }
 

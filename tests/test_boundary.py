@@ -83,8 +83,8 @@ def test_hint_exceeded():
     import pa_harness
     orig = pa_harness.dims_for
 
-    def short_hint(s, xx, hints=True):
-        d = orig(s, xx, hints)
+    def short_hint(s, xx, hints=True, *args, **kwargs):
+        d = orig(s, xx, hints, *args, **kwargs)
         d.max_seqlen_kv_hint = int(s.seqlens_kv[2]) - 1
         return d
     pa_harness.dims_for = short_hint
