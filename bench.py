@@ -495,6 +495,79 @@ def measure_workload(args, spec, wl_key, world, dev, steps, e2e=True, cpu=True):
     return rec
 
 
+def measure_qkv_rotary(args, spec, world, dev, steps):
+    """The fused split-QKV + rotary + scatter pass over one batch of new
+    tokens (packed QKV of the workload's shape, rotary on all head_size
+    dimensions, split pairing), timed alone: CUDA-graph replays, L2 flushed
+    between them.  HBM-bound: its algorithmic bytes are the packed QKV read,
+    Q written, K and V written into the cache, the cos/sin rows read and the
+    slots written."""
+    import torch
+    import scatter_kv_b200 as pa
+
+    x = workloads.generate(spec)
+    T, qh, kvh, d = spec.token_count, spec.q_heads, spec.kv_heads, spec.head_size
+    rng = np.random.default_rng(spec.seed)
+    qkv = torch.from_numpy(rng.standard_normal((T, qh + 2 * kvh, d), dtype=np.float32)
+                           .astype(np.float16)).to(dev)
+    maxpos = int(spec.seqlens_kv.max())
+    ang = np.arange(maxpos)[:, None] * (10000.0 ** (-2.0 * np.arange(d // 2) / d))[None, :]
+    cos = torch.from_numpy(np.cos(ang).astype(np.float16)).to(dev)
+    sin = torch.from_numpy(np.sin(ang).astype(np.float16)).to(dev)
+    meta = {k: torch.from_numpy(np.ascontiguousarray(x[k])).to(dev)
+            for k in ("block_table", "cu_seqlens_q", "seqlens_kv", "key_cache", "value_cache")}
+    dims = pa.make_dims(batch=spec.batch, token_count=T, q_heads=qh, kv_heads=kvh, head_size=d,
+                        num_blocks=spec.num_blocks, block_size=spec.block_size,
+                        max_blocks_per_seq=x["block_table"].shape[1])
+    rot = pa.pa_rotary()
+    rot.rotary_dim, rot.interleaved, rot.max_position = d, 0, maxpos
+    q_out = torch.empty((T, qh, d), dtype=torch.float16, device=dev)
+    slots = torch.empty(T, dtype=torch.int32, device=dev)
+    status = torch.zeros(1, dtype=torch.int32, device=dev)
+    qp, kp, vp, stride = pa.packed_qkv_views(qkv, dims)
+    stream = torch.cuda.Stream(device=dev)
+    flush = torch.empty(2 * L2_BYTES // 4, dtype=torch.int32, device=dev)
+    scrub = torch.zeros(2 * L2_BYTES // 4, dtype=torch.int32, device=dev)
+    scrub_out = torch.empty((), dtype=torch.int64, device=dev)
+
+    def call():
+        pa.pa_split_qkv_rotary_scatter(qp, kp, vp, stride, stride, cos, sin, rot,
+                                       meta["block_table"], meta["cu_seqlens_q"],
+                                       meta["seqlens_kv"], q_out, meta["key_cache"],
+                                       meta["value_cache"], slots, dims, status, stream)
+
+    with torch.cuda.stream(stream):
+        for _ in range(3):
+            call()
+        stream.synchronize()
+        if int(status.item()) != 0:
+            raise RuntimeError(f"device status {int(status.item()):#x} in the fused QKV pass")
+        graph = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(graph, stream=stream):
+            call()
+        ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+              for _ in range(steps)]
+        barrier(world, dev)
+        torch.cuda.synchronize()
+        for k in range(steps):
+            flush.fill_(k)
+            torch.sum(scrub, 0, dtype=torch.int64, out=scrub_out)
+            ev[k][0].record(stream)
+            graph.replay()
+            ev[k][1].record(stream)
+        torch.cuda.synchronize()
+        barrier(world, dev)
+    ms = max_over_ranks(sum(a.elapsed_time(b) for a, b in ev), world, dev) / steps
+    nbytes = (T * (qh + 2 * kvh) * d * 2 + T * qh * d * 2 + 2 * T * kvh * d * 2 + T * d * 2
+              + 4 * T)
+    gbs = nbytes / (ms * 1e-3) / 1e9
+    peaks = load_peaks()
+    return {"workload": spec.name + ", packed QKV, rotary_dim = head_size, split pairing",
+            "us": ms * 1e3, "bytes": nbytes, "GB/s": gbs, "frac": gbs / peaks["hbm_gbs"],
+            "frac_nominal": gbs / NOMINAL_HBM_GBS, "peak_source": f"{peaks['source']} copy bandwidth",
+            "timing": "CUDA-graph replays of the one call, L2 flushed between them"}
+
+
 def run_gpu(args, spec, rank, world, local):
     import torch
 
@@ -511,6 +584,9 @@ def run_gpu(args, spec, rank, world, local):
             o = workloads.CONFIGS[workloads.CONFIG_KEYS[key]]()
             others[key] = measure_workload(args, o, key, world, dev, max(10, args.steps // 2),
                                            e2e=True)
+        others["fused_split_qkv_rotary_scatter"] = measure_qkv_rotary(
+            args, workloads.CONFIGS[workloads.CONFIG_KEYS["prefill"]](), world, dev,
+            max(10, args.steps // 2))
     if rank != 0:
         return None
     line = {

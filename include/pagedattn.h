@@ -161,7 +161,9 @@ typedef struct {
  *   sin, x2 cos + x1 sin) with cos / sin = cache[p][m] for pair index m;
  *   elements from rotary_dim on are copied.  fp32 arithmetic, rounded to
  *   nearest-even.
- *   query_out: [token_count, q_heads, head_size] (rotated Q), written.
+ *   query_out: [token_count, q_heads, head_size] (rotated Q), written; or
+ *          NULL, in which case query is not read (it may be NULL too) and the
+ *          call is the slot mapping and the scatter of K and V in one kernel.
  *   key_cache, value_cache: as for pa_scatter_kv; rotated K and V land in
  *          slot block_table[b][p / block_size] * block_size + p % block_size.
  *   slot_mapping: optional [token_count] int32 output of those slots (-1

@@ -309,13 +309,21 @@ def allocate(dims: pa_dims, device="cuda", out=None):
 
 
 def step(query, key, value, key_cache, value_cache, block_table, cu_seqlens_q, seqlens_kv,
-         scale, dims: pa_dims, buffers: Workspace, stream=None):
+         scale, dims: pa_dims, buffers: Workspace, stream=None, fused: bool = True):
     """One pass of the hot path: slot mapping, scatter of the new K/V, then
-    attention.  Returns ``buffers.out``."""
-    pa_compute_slot_mapping(block_table, cu_seqlens_q, seqlens_kv, buffers.slot_mapping, dims,
-                            buffers.status, stream)
-    pa_scatter_kv(key, value, buffers.slot_mapping, key_cache, value_cache, dims, buffers.status,
-                  stream)
+    attention.  ``fused``: slot mapping and scatter in one kernel
+    (pa_split_qkv_rotary_scatter without a query output); otherwise
+    pa_compute_slot_mapping then pa_scatter_kv.  Both write
+    ``buffers.slot_mapping``.  Returns ``buffers.out``."""
+    if fused:
+        pa_split_qkv_rotary_scatter(None, key, value, 0, 0, None, None, None, block_table,
+                                    cu_seqlens_q, seqlens_kv, None, key_cache, value_cache,
+                                    buffers.slot_mapping, dims, buffers.status, stream)
+    else:
+        pa_compute_slot_mapping(block_table, cu_seqlens_q, seqlens_kv, buffers.slot_mapping, dims,
+                                buffers.status, stream)
+        pa_scatter_kv(key, value, buffers.slot_mapping, key_cache, value_cache, dims,
+                      buffers.status, stream)
     pa_attention(query, key_cache, value_cache, block_table, cu_seqlens_q, seqlens_kv, scale,
                  buffers.out, dims, buffers.workspace, None, buffers.status, stream)
     return buffers.out

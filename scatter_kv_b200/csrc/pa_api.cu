@@ -451,10 +451,12 @@ pa_status pa_split_qkv_rotary_scatter(const void* query, const void* key, const 
         return fail(PA_ERR_INVALID_ARGUMENT,
                     "token strides (%lld, %lld) must cover the heads and be multiples of 8 elements",
                     qs, ks);
-    PA_REQUIRE_PTR(query);
+    if (query_out != nullptr) {
+        PA_REQUIRE_PTR(query);
+        PA_REQUIRE_PTR(query_out);
+    }
     PA_REQUIRE_PTR(key);
     PA_REQUIRE_PTR(value);
-    PA_REQUIRE_PTR(query_out);
     PA_REQUIRE_PTR(key_cache);
     PA_REQUIRE_PTR(value_cache);
     PA_REQUIRE_IPTR(block_table);

@@ -44,6 +44,20 @@ __device__ __forceinline__ uint32_t swz(uint32_t o) {
     return o ^ (((o >> 7) & mask) << 4);
 }
 
+// ---------------------------------------------------------------- dependent launch
+// Programmatic dependent launch: the library's kernels are launched so that
+// each may start while the previous kernel on the stream is finishing.  A
+// kernel lets its successor launch (launch_dependents; the successor's CTAs
+// then take SM slots as they free up) and waits for its predecessor's
+// completion and memory (wait) before it reads any global input.  Both are
+// no-ops for a kernel launched without the attribute.
+__device__ __forceinline__ void pdl_launch_dependents() {
+    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+__device__ __forceinline__ void pdl_wait() {
+    asm volatile("griddepcontrol.wait;" ::: "memory");
+}
+
 // ---------------------------------------------------------------- mbarrier
 
 __device__ __forceinline__ void mbar_init(uint64_t* bar, uint32_t count) {

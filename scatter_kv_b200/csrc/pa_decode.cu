@@ -155,6 +155,8 @@ decode_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ 
     // Status bits of a sequence are reported once, by CTA (split 0, kv head 0).
     const bool reporter = (split == 0 && kvh == 0 && threadIdx.x == 0);
 
+    pdl_launch_dependents();
+    pdl_wait();
     SeqInfo s;
     const bool ok = load_seq(p.cu_seqlens_q, p.seqlens_kv, b, p.batch, p.token_count, p.kv_cap,
                              p.kv_hint, p.q_hint, nullptr, s);
@@ -587,6 +589,8 @@ __global__ void __launch_bounds__(128) combine_kernel(const DecodeParams p) {
     const int hs = p.head_size;
     const long long base = ((long long)b * p.kv_heads + kvh) * p.max_splits * p.rmax + r;
     const float* lse = p.part_lse + base;             // stride rmax per split
+    pdl_launch_dependents();
+    pdl_wait();
     // Lane sp's split lse, fetched together with the metadata (it does not
     // depend on it; splits past the sequence's count are ignored below).
     const float lse_l = lane < p.max_splits ? lse[(long long)lane * p.rmax] : -INFINITY;
@@ -654,9 +658,8 @@ cudaError_t launch_decode_t(const CUtensorMap& tm_k, const CUtensorMap& tm_v,
     e = cudaFuncSetAttribute(kern, cudaFuncAttributePreferredSharedMemoryCarveout,
                              cudaSharedmemCarveoutMaxShared);
     if (e != cudaSuccess) return e;
-    dim3 grid(p.kv_heads, p.max_splits, p.batch);
-    kern<<<grid, C::THREADS, C::SMEM, stream>>>(tm_k, tm_v, p);
-    return cudaGetLastError();
+    return launch_pdl(kern, dim3(p.kv_heads, p.max_splits, p.batch), dim3(C::THREADS), C::SMEM,
+                      stream, tm_k, tm_v, p);
 }
 
 template <int HEAD, typename ET, bool GEN>
@@ -738,15 +741,14 @@ cudaError_t launch_decode(const CUtensorMap& tm_k, const CUtensorMap& tm_v,
 
 template <typename ET>
 cudaError_t launch_combine_t(const DecodeParams& p, int head, cudaStream_t stream) {
-    dim3 grid((p.rmax + 3) / 4, p.kv_heads, p.batch);
+    const dim3 grid((p.rmax + 3) / 4, p.kv_heads, p.batch);
     switch (head) {
-        case 16: combine_kernel<16, ET><<<grid, 128, 0, stream>>>(p); break;
-        case 32: combine_kernel<32, ET><<<grid, 128, 0, stream>>>(p); break;
-        case 64: combine_kernel<64, ET><<<grid, 128, 0, stream>>>(p); break;
-        case 128: combine_kernel<128, ET><<<grid, 128, 0, stream>>>(p); break;
+        case 16: return launch_pdl(combine_kernel<16, ET>, grid, dim3(128), 0, stream, p);
+        case 32: return launch_pdl(combine_kernel<32, ET>, grid, dim3(128), 0, stream, p);
+        case 64: return launch_pdl(combine_kernel<64, ET>, grid, dim3(128), 0, stream, p);
+        case 128: return launch_pdl(combine_kernel<128, ET>, grid, dim3(128), 0, stream, p);
         default: return cudaErrorInvalidValue;
     }
-    return cudaGetLastError();
 }
 
 cudaError_t launch_combine(const DecodeParams& p, int head, bool bf16, cudaStream_t stream) {

@@ -273,6 +273,7 @@ prefill_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
     // checks the block table.
     const int tokp = C::BM / g;                                  // tokens per half
     const int qrows = tokp * g;                                  // rows per half Q's box fills
+    pdl_launch_dependents();
     if (warp == C::WARP_MMA) {
         tmem_alloc(tmem_slot, C::TMEM_COLS);
         tmem_relinquish();
@@ -299,6 +300,7 @@ prefill_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
             tma_prefetch_desc(&tm_v);
         }
         __syncwarp();
+        pdl_wait();                                  // inputs of earlier kernels are ready
         Work w;
         const bool has = find_work(p, (long long)blockIdx.x, w);
         // sh[2]: 0 valid, 1 invalid, 2 invalid with Q's TMA in flight.
@@ -379,6 +381,7 @@ prefill_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
         }
         fence_proxy_async_smem();
     }
+    pdl_wait();
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
@@ -840,8 +843,7 @@ cudaError_t launch_prefill_t(const CUtensorMap& tm_q, const CUtensorMap& tm_k,
     e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM);
     if (e != cudaSuccess) return e;
     const long long ctas = (long long)p.num_slots * p.kv_heads;
-    kern<<<(unsigned)ctas, C::THREADS, C::SMEM, stream>>>(tm_q, tm_k, tm_v, p);
-    return cudaGetLastError();
+    return launch_pdl(kern, dim3((unsigned)ctas), dim3(C::THREADS), C::SMEM, stream, tm_q, tm_k, tm_v, p);
 }
 
 template <int HEAD, typename ET, bool GEN>

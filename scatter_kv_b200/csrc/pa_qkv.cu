@@ -101,6 +101,8 @@ qkv_rotary_scatter_kernel(const QkvParams p) {
     __shared__ int s_pos[kTokPerCta];
     __shared__ int s_ok[kTokPerCta];             // 0: the token's metadata is invalid
 
+    pdl_launch_dependents();
+    pdl_wait();
     const long long t0 = (long long)blockIdx.x * kTokPerCta;
     const bool staged = p.batch <= kQkvMaxStaged;
     if (staged)
@@ -154,7 +156,10 @@ qkv_rotary_scatter_kernel(const QkvParams p) {
     const int rg = p.rotary_dim / 16;                 // rotated vector groups per row (8 pairs each)
     const int pt = (p.head_size - p.rotary_dim) / 8;  // pass-through vectors per row
     const int per_row = rg + pt;
-    const int uq = p.q_heads * per_row, uk = p.kv_heads * per_row, uv = p.kv_heads * d8;
+    // Without a query output the pass only scatters K and V (slot mapping and
+    // scatter in one kernel).
+    const int uq = p.query_out != nullptr ? p.q_heads * per_row : 0;
+    const int uk = p.kv_heads * per_row, uv = p.kv_heads * d8;
     const int per_tok = uq + uk + uv;
     const int ntok = (int)min((long long)kTokPerCta, p.token_count - t0);
     const int half = p.rotary_dim / 2;
@@ -239,10 +244,10 @@ cudaError_t launch_qkv_rotary_scatter(const QkvParams& p, bool bf16, cudaStream_
     const long long blocks = (p.token_count + kTokPerCta - 1) / kTokPerCta;
     if (blocks <= 0) return cudaSuccess;
     if (bf16)
-        qkv_rotary_scatter_kernel<__nv_bfloat16><<<(unsigned)blocks, kQkvThreads, 0, stream>>>(p);
-    else
-        qkv_rotary_scatter_kernel<__half><<<(unsigned)blocks, kQkvThreads, 0, stream>>>(p);
-    return cudaGetLastError();
+        return launch_pdl(qkv_rotary_scatter_kernel<__nv_bfloat16>, dim3((unsigned)blocks),
+                          dim3(kQkvThreads), 0, stream, p);
+    return launch_pdl(qkv_rotary_scatter_kernel<__half>, dim3((unsigned)blocks), dim3(kQkvThreads), 0,
+                      stream, p);
 }
 
 }  // namespace pa

@@ -42,6 +42,8 @@ scatter_kv_kernel(const uint4* __restrict__ key, const uint4* __restrict__ value
                   const int32_t* __restrict__ slot_mapping, uint4* __restrict__ key_cache,
                   uint4* __restrict__ value_cache, long long token_count, int vec_per_token,
                   long long num_slots, int32_t* status) {
+    pdl_launch_dependents();
+    pdl_wait();
     const long long total = token_count * vec_per_token;
     const long long stride = (long long)gridDim.x * kScatterThreads * kScatterUnroll;
     for (long long base = (long long)blockIdx.x * kScatterThreads * kScatterUnroll + threadIdx.x;
@@ -88,6 +90,8 @@ slot_mapping_kernel(const int32_t* __restrict__ block_table, const int32_t* __re
                     int batch, long long token_count, int max_blocks, int block_size,
                     long long num_blocks, int32_t* status) {
     extern __shared__ int32_t s_cu[];    // cu_seqlens_q[1 .. batch] (when batch <= kSlotMaxStaged)
+    pdl_launch_dependents();
+    pdl_wait();
     const bool staged = batch <= kSlotMaxStaged;
     if (staged)
         for (int i = threadIdx.x; i < batch; i += kSlotThreads) s_cu[i] = cu[i + 1];
@@ -131,11 +135,10 @@ cudaError_t launch_scatter(const void* key, const void* value, const int32_t* sl
     const long long cap = (long long)num_sms * 8;
     if (blocks > cap) blocks = cap;
     if (blocks < 1) blocks = 1;
-    scatter_kv_kernel<<<(unsigned)blocks, kScatterThreads, 0, stream>>>(
-        static_cast<const uint4*>(key), static_cast<const uint4*>(value), slot_mapping,
-        static_cast<uint4*>(key_cache), static_cast<uint4*>(value_cache), d.token_count,
-        vec_per_token, d.num_blocks * d.block_size, status);
-    return cudaGetLastError();
+    return launch_pdl(scatter_kv_kernel, dim3((unsigned)blocks), dim3(kScatterThreads), 0, stream,
+                      static_cast<const uint4*>(key), static_cast<const uint4*>(value), slot_mapping,
+                      static_cast<uint4*>(key_cache), static_cast<uint4*>(value_cache), d.token_count,
+                      vec_per_token, d.num_blocks * (long long)d.block_size, status);
 }
 
 cudaError_t launch_slot_mapping(const int32_t* block_table, const int32_t* cu,
@@ -144,10 +147,9 @@ cudaError_t launch_slot_mapping(const int32_t* block_table, const int32_t* cu,
     const int threads = kSlotThreads;
     long long blocks = (d.token_count + threads - 1) / threads;
     const size_t smem = d.batch <= kSlotMaxStaged ? (size_t)d.batch * 4 : 0;
-    slot_mapping_kernel<<<(unsigned)blocks, threads, smem, stream>>>(
-        block_table, cu, seqlens_kv, slot_mapping, d.batch, d.token_count, d.max_blocks_per_seq,
-        d.block_size, d.num_blocks, status);
-    return cudaGetLastError();
+    return launch_pdl(slot_mapping_kernel, dim3((unsigned)blocks), dim3(threads), smem, stream,
+                      block_table, cu, seqlens_kv, slot_mapping, d.batch, d.token_count,
+                      d.max_blocks_per_seq, d.block_size, d.num_blocks, status);
 }
 
 }  // namespace pa

@@ -62,7 +62,7 @@ def dims_for(spec: workloads.Spec, x: dict, hints: bool = True, softcap: float =
 
 
 def run_gpu(spec: workloads.Spec, x: dict, hints: bool = True, scale: float | None = None,
-            repeat: int = 1, softcap: float = 0.0, window=None):
+            repeat: int = 1, softcap: float = 0.0, window=None, fused: bool = True):
     """Slot mapping + scatter + attention on the GPU.  Returns (out as numpy
     float16 -- bf16 bit patterns as uint16 for bf16 inputs --, device tensors
     dict, status word, slot mapping as numpy)."""
@@ -75,7 +75,8 @@ def run_gpu(spec: workloads.Spec, x: dict, hints: bool = True, scale: float | No
     outs = []
     for _ in range(repeat):
         pa.step(dv["query"], dv["key"], dv["value"], dv["key_cache"], dv["value_cache"],
-                dv["block_table"], dv["cu_seqlens_q"], dv["seqlens_kv"], sc, dims, bufs)
+                dv["block_table"], dv["cu_seqlens_q"], dv["seqlens_kv"], sc, dims, bufs,
+                fused=fused)
         torch.cuda.synchronize()
         outs.append(host_bits(bufs.out, spec.elem))
     status = int(bufs.status[0].item())

@@ -99,6 +99,12 @@ def test_split_qkv_rotary_needs_caches_only_with_rotation(pa):
         pa.pa_split_qkv_rotary_scatter(FAKE, FAKE, FAKE, 0, 0, None, FAKE, _rotary(pa, 64), FAKE,
                                        FAKE, FAKE, FAKE, FAKE, FAKE, None, d, None, 0)
     assert "cos_cache" in str(e.value)
+    # Without a query output the query may be NULL (scatter only); the other
+    # tensors may not.
+    with pytest.raises(pa.PagedAttentionError) as e:
+        pa.pa_split_qkv_rotary_scatter(None, None, FAKE, 0, 0, None, None, None, FAKE, FAKE, FAKE,
+                                       None, FAKE, FAKE, None, d, None, 0)
+    assert "key" in str(e.value)
     # token_count 0: nothing to do, nothing read.
     pa.pa_split_qkv_rotary_scatter(None, None, None, 0, 0, None, None, None, None, None, None,
                                    None, None, None, None, _dims(pa, token_count=0), None, 0)

@@ -237,3 +237,40 @@ def test_min_seqlen_hint_routes_every_sequence_to_prefill():
     for b in (2, 4):
         rows = slice(cu[b], cu[b + 1])
         assert np.array_equal(outs[0][rows].view(np.uint16), outs[1][rows].view(np.uint16))
+
+
+def test_back_to_back_calls_sharing_a_workspace():
+    """Calls on one stream may overlap their launches (each kernel waits for
+    the previous one before touching memory): three attention calls queued
+    without a host sync, sharing one split-KV workspace, give the same bits
+    as calls made one at a time."""
+    import torch
+    import scatter_kv_b200 as pa
+    from pa_harness import dims_for, to_dev
+    specs = [workloads.custom([1, 2, 1, 3], [3000, 2500, 900, 4000], 16, 4, 128, 16, seed=s)
+             for s in (21, 22)]
+    xs = [workloads.generate(s) for s in specs]
+    dvs = [to_dev(x) for x in xs]
+    dims = [dims_for(s, x) for s, x in zip(specs, xs)]
+    need = max(pa.pa_attention_workspace_size(d) for d in dims)
+    ws = torch.empty(need, dtype=torch.uint8, device="cuda")
+    st = torch.zeros(1, dtype=torch.int32, device="cuda")
+
+    def attend(i, out):
+        dv = dvs[i]
+        pa.pa_attention(dv["query"], dv["key_cache"], dv["value_cache"], dv["block_table"],
+                        dv["cu_seqlens_q"], dv["seqlens_kv"], 0.0, out, dims[i], ws, need, st)
+
+    ref = []
+    for i in range(2):
+        out = torch.empty_like(dvs[i]["query"])
+        attend(i, out)
+        torch.cuda.synchronize()
+        ref.append(out.clone())
+    outs = [torch.empty_like(dvs[i % 2]["query"]) for i in range(3)]
+    for i in range(3):
+        attend(i % 2, outs[i])
+    torch.cuda.synchronize()
+    assert int(st.item()) == 0
+    for i in range(3):
+        assert torch.equal(outs[i].view(torch.int16), ref[i % 2].view(torch.int16))

@@ -208,3 +208,22 @@ def test_position_past_the_caches_is_flagged():
     kc = dv["key_cache"].view(-1, 2, 64)
     untouched = np.setdiff1d(np.arange(kc.shape[0]), s[:3])
     assert torch.equal(kc[untouched].view(torch.int16), kc0.view(-1, 2, 64)[untouched].view(torch.int16))
+
+
+@pytest.mark.parametrize("cfg", [1, 3])
+def test_scatter_only_pass_equals_slot_mapping_then_scatter(cfg):
+    """Without a query output the fused pass is slot mapping plus scatter in
+    one kernel: the step built on it gives the same slots, caches and
+    attention output, bit for bit, as pa_compute_slot_mapping followed by
+    pa_scatter_kv."""
+    spec = workloads.CONFIGS[cfg]()
+    x = workloads.generate(spec)
+    from pa_harness import run_gpu
+    a, dva, sa, slots_a = run_gpu(spec, x, fused=True)
+    b, dvb, sb, slots_b = run_gpu(spec, x, fused=False)
+    assert sa == sb == 0
+    assert np.array_equal(slots_a, slots_b)
+    assert np.array_equal(a.view(np.uint16), b.view(np.uint16))
+    import torch
+    for name in ("key_cache", "value_cache"):
+        assert torch.equal(dva[name].view(torch.int16), dvb[name].view(torch.int16))
