@@ -309,7 +309,7 @@ def allocate(dims: pa_dims, device="cuda", out=None):
 
 
 def step(query, key, value, key_cache, value_cache, block_table, cu_seqlens_q, seqlens_kv,
-         scale, dims: pa_dims, buffers: Workspace, stream=None, fused: bool = True):
+         scale, dims: pa_dims, buffers: Workspace, stream=None, fused: bool = False):
     """One pass of the hot path: slot mapping, scatter of the new K/V, then
     attention.  ``fused``: slot mapping and scatter in one kernel
     (pa_split_qkv_rotary_scatter without a query output); otherwise

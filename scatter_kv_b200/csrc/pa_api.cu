@@ -497,7 +497,8 @@ pa_status pa_split_qkv_rotary_scatter(const void* query, const void* key, const 
     p.kv_cap = d.max_blocks_per_seq * d.block_size;
     cudaStream_t s = static_cast<cudaStream_t>(stream);
     TraceScope tr(PA_KERNEL_QKV_ROTARY, s);
-    cudaError_t e = pa::launch_qkv_rotary_scatter(p, d.dtype == PA_DTYPE_BF16, s);
+    cudaError_t e = pa::launch_qkv_rotary_scatter(p, d.dtype == PA_DTYPE_BF16, s,
+                                                  num_sms_of_current_device());
     return e == cudaSuccess ? PA_OK : cuda_fail(e, "split-QKV rotary scatter launch");
 }
 

@@ -131,7 +131,8 @@ struct QkvParams {
     int kv_cap;
 };
 
-cudaError_t launch_qkv_rotary_scatter(const QkvParams& p, bool bf16, cudaStream_t stream);
+cudaError_t launch_qkv_rotary_scatter(const QkvParams& p, bool bf16, cudaStream_t stream,
+                                      int num_sms);
 
 struct DecodePlan {
     int decode_max_q;

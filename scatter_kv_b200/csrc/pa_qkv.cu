@@ -19,7 +19,7 @@
 //     rotated K and unchanged V go to cache block slot / block_size, row
 //     slot % block_size, slot = block_table[b][p / bs] * bs + p % bs.
 //
-// Work: a CTA takes kTokPerCta consecutive tokens.  Its first threads find
+// Work: a CTA takes up to kTokPerCta consecutive tokens.  Its first threads find
 // each token's sequence (binary search over cu_seqlens_q staged in shared
 // memory), position and slot; then all threads stream the tokens' rows in
 // 16-byte vectors, consecutive threads on consecutive vectors of a row.  A
@@ -40,7 +40,7 @@ namespace pa {
 namespace {
 
 constexpr int kQkvThreads = 256;
-constexpr int kTokPerCta = 8;
+constexpr int kTokPerCta = 8;          // at most; see launch_qkv_rotary_scatter
 constexpr int kQkvMaxStaged = 4096;    // cu_seqlens_q entries staged in shared memory
 
 template <typename T>
@@ -95,7 +95,7 @@ __device__ __forceinline__ void rotate(float x1, float x2, float c, float s, flo
 
 template <typename T>
 __global__ void __launch_bounds__(kQkvThreads)
-qkv_rotary_scatter_kernel(const QkvParams p) {
+qkv_rotary_scatter_kernel(const QkvParams p, int tok_per_cta) {
     __shared__ int s_cu[kQkvMaxStaged];
     __shared__ long long s_slot[kTokPerCta];     // -1: no cache write
     __shared__ int s_pos[kTokPerCta];
@@ -103,12 +103,12 @@ qkv_rotary_scatter_kernel(const QkvParams p) {
 
     pdl_launch_dependents();
     pdl_wait();
-    const long long t0 = (long long)blockIdx.x * kTokPerCta;
+    const long long t0 = (long long)blockIdx.x * tok_per_cta;
     const bool staged = p.batch <= kQkvMaxStaged;
     if (staged)
         for (int i = threadIdx.x; i < p.batch; i += kQkvThreads) s_cu[i] = p.cu_seqlens_q[i + 1];
     __syncthreads();
-    if (threadIdx.x < kTokPerCta) {
+    if (threadIdx.x < tok_per_cta) {
         const long long t = t0 + threadIdx.x;
         long long slot = -1;
         int pos = 0, ok = 0;
@@ -161,7 +161,7 @@ qkv_rotary_scatter_kernel(const QkvParams p) {
     const int uq = p.query_out != nullptr ? p.q_heads * per_row : 0;
     const int uk = p.kv_heads * per_row, uv = p.kv_heads * d8;
     const int per_tok = uq + uk + uv;
-    const int ntok = (int)min((long long)kTokPerCta, p.token_count - t0);
+    const int ntok = (int)min((long long)tok_per_cta, p.token_count - t0);
     const int half = p.rotary_dim / 2;
     const uint4 zero = make_uint4(0, 0, 0, 0);
 
@@ -240,14 +240,20 @@ qkv_rotary_scatter_kernel(const QkvParams p) {
 
 }  // namespace
 
-cudaError_t launch_qkv_rotary_scatter(const QkvParams& p, bool bf16, cudaStream_t stream) {
-    const long long blocks = (p.token_count + kTokPerCta - 1) / kTokPerCta;
+cudaError_t launch_qkv_rotary_scatter(const QkvParams& p, bool bf16, cudaStream_t stream,
+                                      int num_sms) {
+    // Tokens per CTA: up to kTokPerCta, fewer when that leaves the grid under
+    // two CTAs per SM (small decode batches: one token per CTA).
+    long long tpc = (p.token_count + 2LL * num_sms - 1) / (2LL * num_sms);
+    if (tpc < 1) tpc = 1;
+    if (tpc > kTokPerCta) tpc = kTokPerCta;
+    const long long blocks = (p.token_count + tpc - 1) / tpc;
     if (blocks <= 0) return cudaSuccess;
     if (bf16)
         return launch_pdl(qkv_rotary_scatter_kernel<__nv_bfloat16>, dim3((unsigned)blocks),
-                          dim3(kQkvThreads), 0, stream, p);
+                          dim3(kQkvThreads), 0, stream, p, (int)tpc);
     return launch_pdl(qkv_rotary_scatter_kernel<__half>, dim3((unsigned)blocks), dim3(kQkvThreads), 0,
-                      stream, p);
+                      stream, p, (int)tpc);
 }
 
 }  // namespace pa

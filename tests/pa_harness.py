@@ -62,7 +62,7 @@ def dims_for(spec: workloads.Spec, x: dict, hints: bool = True, softcap: float =
 
 
 def run_gpu(spec: workloads.Spec, x: dict, hints: bool = True, scale: float | None = None,
-            repeat: int = 1, softcap: float = 0.0, window=None, fused: bool = True):
+            repeat: int = 1, softcap: float = 0.0, window=None, fused: bool = False):
     """Slot mapping + scatter + attention on the GPU.  Returns (out as numpy
     float16 -- bf16 bit patterns as uint16 for bf16 inputs --, device tensors
     dict, status word, slot mapping as numpy)."""
