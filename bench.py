@@ -253,26 +253,39 @@ def _strip_comments(src: str) -> str:
     return "\n".join(ln for ln in lines if ln)
 
 
-def kernel_source_hash() -> str:
-    """Hash of the kernel sources' code: a profile taken on them stays valid
-    through comment-only edits, and any code change invalidates it."""
+# Sources each profiled kernel is built from: a profile stays tied to them.
+KERNEL_SOURCES = {
+    "decode_split_kv": ("pa_decode.cu", "pa_common.cuh", "pa_internal.h"),
+    "decode_combine": ("pa_decode.cu", "pa_common.cuh", "pa_internal.h"),
+    "prefill_tcgen05": ("pa_prefill.cu", "pa_common.cuh", "pa_internal.h"),
+    "scatter_kv": ("pa_scatter.cu", "pa_common.cuh", "pa_internal.h"),
+    "slot_mapping": ("pa_scatter.cu", "pa_common.cuh", "pa_internal.h"),
+    "qkv_rotary_scatter": ("pa_qkv.cu", "pa_common.cuh", "pa_internal.h"),
+}
+
+
+def kernel_source_hash(files=None) -> str:
+    """Hash of the code of the given kernel sources (default: all of them): a
+    profile taken on them stays valid through comment-only edits, and any
+    code change invalidates it."""
     h = hashlib.sha256()
-    for name in sorted(os.listdir(os.path.join(ROOT, "scatter_kv_b200", "csrc"))):
-        with open(os.path.join(ROOT, "scatter_kv_b200", "csrc", name), encoding="utf-8") as f:
+    csrc = os.path.join(ROOT, "scatter_kv_b200", "csrc")
+    for name in sorted(files if files is not None else os.listdir(csrc)):
+        with open(os.path.join(csrc, name), encoding="utf-8") as f:
             h.update(name.encode() + _strip_comments(f.read()).encode())
     return h.hexdigest()[:16]
 
 
 def profiled_traffic(kernel: str, workload: str):
     """dram bytes per launch from a committed ncu summary, if it was taken
-    on the current kernel sources (else None)."""
+    on the kernel's current sources (else None)."""
     path = os.path.join(ROOT, "profiles", f"{kernel}_{workload}.md")
     if not os.path.exists(path):
         return None
     text = open(path).read()
     m = re.search(r"traffic_bytes_per_launch:\s*([0-9.eE+]+)", text)
     h = re.search(r"source_hash:\s*([0-9a-f]+)", text)
-    if not m or not h or h.group(1) != kernel_source_hash():
+    if not m or not h or h.group(1) != kernel_source_hash(KERNEL_SOURCES.get(kernel)):
         return None
     return float(m.group(1))
 

@@ -46,3 +46,17 @@ def test_algorithmic_counts_split_between_kernels():
     assert c["prefill_flops"] == 4 * 8 * 16 * sum(range(6, 16))
     assert not c["decode"] and bench.unit_of(spec) == "TFLOP/s"
     assert bench.unit_of(workloads.custom([1, 3], [9, 9], 8, 2, 16, 16)) == "GB/s"
+
+
+def test_profile_hash_covers_only_the_kernels_sources(tmp_path, monkeypatch):
+    csrc = tmp_path / "scatter_kv_b200" / "csrc"
+    csrc.mkdir(parents=True)
+    for n in ("pa_decode.cu", "pa_common.cuh", "pa_internal.h", "pa_prefill.cu"):
+        (csrc / n).write_text(f"int {n.split('.')[0]};\n")
+    monkeypatch.setattr(bench, "ROOT", str(tmp_path))
+    files = bench.KERNEL_SOURCES["decode_split_kv"]
+    h0 = bench.kernel_source_hash(files)
+    (csrc / "pa_prefill.cu").write_text("int changed;\n")
+    assert bench.kernel_source_hash(files) == h0
+    (csrc / "pa_common.cuh").write_text("int changed;\n")
+    assert bench.kernel_source_hash(files) != h0
