@@ -64,6 +64,11 @@ def _load():
         lib.oracle_rotary.argtypes = [P, i64, ctypes.c_int, ctypes.c_int, i64, P, P, P,
                                       ctypes.c_int, ctypes.c_int, ctypes.c_int, P]
         lib.oracle_max_threads.restype = ctypes.c_int
+        lib.oracle_quantize_int4.argtypes = [ctypes.c_float, ctypes.c_float]
+        lib.oracle_quantize_int4.restype = ctypes.c_int
+        lib.oracle_scatter_kv_int4.argtypes = [P, P, P, P, P, P, P, i64, ctypes.c_int, ctypes.c_int,
+                                               ctypes.c_int]
+        lib.oracle_dequantize_int4.argtypes = [P, P, i64, ctypes.c_int, ctypes.c_int, P]
         _lib = lib
     return _lib
 
@@ -211,4 +216,41 @@ def rotary(x, positions, cos_cache, sin_cache, rotary_dim: int, interleaved: boo
         base = x.ctypes.data_as(ctypes.c_void_p)
         lib.oracle_rotary(base, T, H, d, x.strides[0] // x.itemsize, _ptr(pos), _ptr(cc), _ptr(sc),
                           rotary_dim, 1 if interleaved else 0, dtype, _ptr(out))
+    return out
+
+
+def quantize_int4(x: float, scale: float) -> int:
+    """Code of one value: round(x / scale) (binary32, ties to even) clamped to [-8, 7]."""
+    return int(_load().oracle_quantize_int4(float(x), float(scale)))
+
+
+def scatter_kv_int4(key, value, slot_mapping, k_scale, v_scale, key_cache, value_cache,
+                    bf16: bool = False) -> None:
+    """In place: quantise token t's K/V rows with the per-channel scales
+    [kv_heads, head_size] and pack them into INT4 cache slot slot_mapping[t]
+    (caches uint8 [num_blocks, block_size, kv_heads, head_size // 2])."""
+    lib = _load()
+    dtype = _elem_type(key, bf16)
+    assert key_cache.dtype == value_cache.dtype == np.uint8
+    assert key_cache.flags.c_contiguous and value_cache.flags.c_contiguous
+    key = _c(key, key.dtype)
+    value = _c(value, value.dtype)
+    T, kvh, d = key.shape
+    assert key_cache.shape[2:] == (kvh, d // 2)
+    ks = _c(k_scale, np.float32).reshape(kvh, d)
+    vs = _c(v_scale, np.float32).reshape(kvh, d)
+    slots = _c(slot_mapping, np.int32)
+    lib.oracle_scatter_kv_int4(_ptr(key), _ptr(value), _ptr(slots), _ptr(ks), _ptr(vs),
+                               _ptr(key_cache), _ptr(value_cache), T, kvh, d, dtype)
+
+
+def dequantize_int4(cache, scale) -> np.ndarray:
+    """float64 [num_blocks, block_size, kv_heads, head_size] values of an INT4 cache."""
+    lib = _load()
+    nb, bs, kvh, half = cache.shape
+    d = 2 * half
+    c = _c(cache, np.uint8)
+    sc = _c(scale, np.float32).reshape(kvh, d)
+    out = np.empty((nb, bs, kvh, d), dtype=np.float64)
+    lib.oracle_dequantize_int4(_ptr(c), _ptr(sc), nb * bs, kvh, d, _ptr(out))
     return out

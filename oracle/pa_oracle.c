@@ -321,6 +321,76 @@ void oracle_rotary(const void *x, int64_t token_count, int heads, int head_size,
     }
 }
 
+/* INT4 KV cache (the packed-INT4 PagedAttention of the "[WebGPU] Implement
+ * SparseAttentionIndexer" PR's file list: INT4 cache reads and writes,
+ * per-channel scaling; the byte format is not on the pages).  Reading taken:
+ * a cache row of one KV head holds head_size signed 4-bit codes, two per
+ * byte -- channel 2j in the low nibble of byte j, channel 2j+1 in the high
+ * nibble, two's complement in [-8, 7]; every channel c of KV head h has one
+ * fp32 scale s[h][c] (separate for K and V), and a code q stands for q * s.
+ * Quantisation rounds x / s to the nearest integer, ties to even, and
+ * clamps to [-8, 7]; the quotient is taken in binary32 (x is a 16-bit value,
+ * exact in binary32; the division is IEEE, correctly rounded), the
+ * precision the GPU takes the same decision in. */
+int oracle_quantize_int4(float x, float s)
+{
+    float r = rintf(x / s);
+    if (r > 7.0f) r = 7.0f;
+    if (r < -8.0f) r = -8.0f;
+    return (int)r;
+}
+
+/* Code of channel c from a packed row. */
+static int int4_code(const uint8_t *row, int c)
+{
+    int nib = (c & 1) ? (row[c >> 1] >> 4) : (row[c >> 1] & 0xf);
+    return nib >= 8 ? nib - 16 : nib;
+}
+
+/* Scatter with quantisation: token t's K and V rows ([token_count, kv_heads,
+ * head_size] 16-bit values of type dtype) are quantised with the
+ * per-channel scales k_scale / v_scale [kv_heads, head_size] and packed
+ * into cache slot slot_mapping[t] (negative: skipped) of the INT4 caches
+ * [num_blocks, block_size, kv_heads, head_size / 2]. */
+void oracle_scatter_kv_int4(const void *key, const void *value, const int32_t *slot_mapping,
+                            const float *k_scale, const float *v_scale, uint8_t *key_cache,
+                            uint8_t *value_cache, int64_t token_count, int kv_heads, int head_size,
+                            int dtype)
+{
+    fill_half_table();
+    int64_t row_bytes = (int64_t)kv_heads * head_size / 2;
+    for (int64_t t = 0; t < token_count; ++t) {
+        int32_t slot = slot_mapping[t];
+        if (slot < 0) continue;
+        for (int h = 0; h < kv_heads; ++h) {
+            for (int c = 0; c < head_size; c += 2) {
+                int64_t src = (t * kv_heads + h) * (int64_t)head_size + c;
+                int64_t dst = slot * row_bytes + ((int64_t)h * head_size + c) / 2;
+                int k0 = oracle_quantize_int4((float)load(key, src, dtype), k_scale[h * head_size + c]);
+                int k1 = oracle_quantize_int4((float)load(key, src + 1, dtype), k_scale[h * head_size + c + 1]);
+                int v0 = oracle_quantize_int4((float)load(value, src, dtype), v_scale[h * head_size + c]);
+                int v1 = oracle_quantize_int4((float)load(value, src + 1, dtype), v_scale[h * head_size + c + 1]);
+                key_cache[dst] = (uint8_t)((k0 & 0xf) | ((k1 & 0xf) << 4));
+                value_cache[dst] = (uint8_t)((v0 & 0xf) | ((v1 & 0xf) << 4));
+            }
+        }
+    }
+}
+
+/* The value every cache element stands for: out[slot][h][c] = code * s[h][c]
+ * (fp64, exact), for all num_slots = num_blocks * block_size rows. */
+void oracle_dequantize_int4(const uint8_t *cache, const float *scale, int64_t num_slots,
+                            int kv_heads, int head_size, double *out)
+{
+    int64_t row_bytes = (int64_t)kv_heads * head_size / 2;
+    for (int64_t r = 0; r < num_slots; ++r)
+        for (int h = 0; h < kv_heads; ++h)
+            for (int c = 0; c < head_size; ++c)
+                out[(r * kv_heads + h) * (int64_t)head_size + c] =
+                    (double)int4_code(cache + r * row_bytes + (int64_t)h * head_size / 2, c) *
+                    (double)scale[h * head_size + c];
+}
+
 int oracle_max_threads(void)
 {
 #ifdef _OPENMP

@@ -255,3 +255,72 @@ def test_rotary_reads_strided_packed_rows():
     got = oracle.rotary(k_view, pos, cos, sin, 16, False)
     want = oracle.rotary(np.ascontiguousarray(k_view), pos, cos, sin, 16, False)
     assert np.array_equal(got, want)
+
+
+# ---------------------------------------------------------------- INT4 cache
+
+def test_int4_codes_round_trip_and_round_ties_to_even():
+    for s in (1.0, 0.25, 4.0):
+        for k in range(-8, 8):
+            assert oracle.quantize_int4(k * s, s) == k
+    # Ties: 2.5 -> 2 and 3.5 -> 4 (to even), -2.5 -> -2; half-away rounding gives 3, 4, -3.
+    assert [oracle.quantize_int4(v, 0.5) for v in (1.25, 1.75, -1.25)] == [2, 4, -2]
+    # Clamping at both ends, including a tie that rounds past 7.
+    assert [oracle.quantize_int4(v, 1.0) for v in (100.0, 7.5, -8.5, -100.0)] == [7, 7, -8, -8]
+
+
+def test_int4_packing_by_hand():
+    """Codes (3, -2, 7, -8) of one head row pack into bytes 0xE3, 0x87 (low
+    nibble = even channel), written at the token's slot only."""
+    key = np.array([[[3.0, -2.0, 7.0, -8.0]]], dtype=np.float16)
+    value = -key
+    kc = np.zeros((2, 2, 1, 2), dtype=np.uint8)
+    vc = np.zeros_like(kc)
+    ones = np.ones((1, 4), dtype=np.float32)
+    oracle.scatter_kv_int4(key, value, np.array([3], np.int32), ones, ones, kc, vc)
+    assert list(kc.reshape(-1, 2)[3]) == [0xE3, 0x87]
+    assert list(vc.reshape(-1, 2)[3]) == [0x2D, 0x79]      # codes (-3, 2, -7, 7): 8 clamps to 7
+    assert not kc.reshape(-1, 2)[:3].any()
+    deq = oracle.dequantize_int4(kc, np.full((1, 4), 0.5, np.float32))
+    assert list(deq.reshape(-1, 4)[3]) == [1.5, -1.0, 3.5, -4.0]
+
+
+def test_int4_error_bound_and_exact_grid():
+    """Dequantised codes lie within half a scale step of in-range inputs, and
+    inputs on the grid come back exactly."""
+    rng = np.random.default_rng(13)
+    kvh, d = 2, 16
+    scale = rng.uniform(0.05, 0.5, size=(kvh, d)).astype(np.float32)
+    x = (rng.uniform(-7.4, 7.4, size=(50, kvh, d)) * scale).astype(np.float16)
+    kc = np.zeros((50, 1, kvh, d // 2), dtype=np.uint8)
+    vc = np.zeros_like(kc)
+    slots = np.arange(50, dtype=np.int32)
+    oracle.scatter_kv_int4(x, x, slots, scale, scale, kc, vc)
+    deq = oracle.dequantize_int4(kc, scale)[:, 0]
+    assert (np.abs(deq - x.astype(np.float64)) <= scale.astype(np.float64) / 2 * (1 + 1e-6)).all()
+    grid = (rng.integers(-8, 8, size=(50, kvh, d)) * 0.25).astype(np.float16)
+    quarter = np.full((kvh, d), 0.25, np.float32)
+    oracle.scatter_kv_int4(grid, grid, slots, quarter, quarter, kc, vc)
+    assert np.array_equal(oracle.dequantize_int4(vc, quarter)[:, 0], grid.astype(np.float64))
+
+
+def test_int4_attention_on_grid_values_equals_plain_attention():
+    """Attention over an INT4 cache is attention over the values its codes
+    stand for: with K and V on the quantisation grid, it equals the plain
+    oracle on the f16 cache, bit for bit."""
+    rng = np.random.default_rng(14)
+    q_lens, past, qh, kvh, d, bs = [3, 1], [20, 9], 4, 2, 16, 8
+    P = _random_problem(rng, q_lens, past, qh, kvh, d, bs, dtype=np.float16)
+    s = np.float32(0.5)
+    kc = (np.clip(np.rint(np.nan_to_num(P["kc"].astype(np.float32)) / s), -8, 7) * s).astype(np.float16)
+    vc = (np.clip(np.rint(np.nan_to_num(P["vc"].astype(np.float32)) / s), -8, 7) * s).astype(np.float16)
+    nb = kc.shape[0]
+    slots = np.arange(nb * bs, dtype=np.int32)
+    k4 = np.zeros((nb, bs, kvh, d // 2), np.uint8)
+    v4 = np.zeros_like(k4)
+    scale = np.full((kvh, d), s, np.float32)
+    oracle.scatter_kv_int4(kc.reshape(-1, kvh, d), vc.reshape(-1, kvh, d), slots, scale, scale, k4, v4)
+    want = oracle.attention(P["query"], kc, vc, P["table"], P["cu"], P["skv"], 0.25)
+    got = oracle.attention(P["query"].astype(np.float64), oracle.dequantize_int4(k4, scale),
+                           oracle.dequantize_int4(v4, scale), P["table"], P["cu"], P["skv"], 0.25)
+    assert np.array_equal(got, want)
