@@ -358,16 +358,34 @@ def kernel_roofline(name: str, avg_ms: float, counts: dict, peaks: dict, workloa
     return rec
 
 
-def measure_workload(args, spec, wl_key, world, dev, steps, e2e=True, cpu=True):
+def measure_workload(args, spec, wl_key, world, dev, steps, e2e=True, cpu=True, int4=False):
     """Time one workload: CUDA-graph replays of the whole step (value),
     traced eager steps (per-kernel times), and optionally the end-to-end step
-    through the public API with host buffers."""
+    through the public API with host buffers.  int4: the same batch over INT4
+    caches (random codes, per-channel scales), scatter and attention through
+    the INT4 entry points."""
     import torch
     import scatter_kv_b200 as pa
 
     counts = algorithmic_counts(spec)
     peaks = load_peaks()
     x = workloads.generate(spec)
+    if int4:
+        rng = np.random.default_rng(spec.seed)
+        shape = (spec.num_blocks, spec.block_size, spec.kv_heads, spec.head_size // 2)
+        x["key_cache"] = rng.integers(0, 256, size=shape, dtype=np.uint8)
+        x["value_cache"] = rng.integers(0, 256, size=shape, dtype=np.uint8)
+        x["k_scale"] = rng.uniform(0.1, 0.3, size=(spec.kv_heads, spec.head_size)).astype(np.float32)
+        x["v_scale"] = rng.uniform(0.1, 0.3, size=(spec.kv_heads, spec.head_size)).astype(np.float32)
+        # A quarter of the K/V bytes, plus every (sequence, KV head)'s scales.
+        scale_bytes = 2 * spec.batch * spec.kv_heads * spec.head_size * 4
+        counts["kv_bytes"] //= 4
+        counts["decode_bytes"] = counts["kv_bytes"] + counts["q_bytes"] + scale_bytes
+        counts["scatter_bytes"] = (2 * spec.token_count * spec.kv_heads * spec.head_size * 2
+                                   + 2 * spec.token_count * spec.kv_heads * spec.head_size // 2
+                                   + 4 * spec.token_count)
+        counts["step_bytes"] = (counts["kv_bytes"] + 2 * counts["q_bytes"] + scale_bytes
+                                + counts["scatter_bytes"])
     d = {k: torch.from_numpy(np.ascontiguousarray(v)).to(dev) for k, v in x.items()}
     dims = pa.make_dims(batch=spec.batch, token_count=spec.token_count, q_heads=spec.q_heads,
                         kv_heads=spec.kv_heads, head_size=spec.head_size,
@@ -390,6 +408,16 @@ def measure_workload(args, spec, wl_key, world, dev, steps, e2e=True, cpu=True):
         torch.sum(scrub, 0, dtype=torch.int64, out=scrub_out)
 
     def step():
+        if int4:
+            pa.pa_compute_slot_mapping(d["block_table"], d["cu_seqlens_q"], d["seqlens_kv"],
+                                       bufs.slot_mapping, dims, bufs.status, stream)
+            pa.pa_scatter_kv_int4(d["key"], d["value"], bufs.slot_mapping, d["k_scale"],
+                                  d["v_scale"], d["key_cache"], d["value_cache"], dims, bufs.status,
+                                  stream)
+            pa.pa_attention_int4(d["query"], d["key_cache"], d["value_cache"], d["k_scale"],
+                                 d["v_scale"], d["block_table"], d["cu_seqlens_q"], d["seqlens_kv"],
+                                 scale, bufs.out, dims, bufs.workspace, None, bufs.status, stream)
+            return
         pa.step(d["query"], d["key"], d["value"], d["key_cache"], d["value_cache"],
                 d["block_table"], d["cu_seqlens_q"], d["seqlens_kv"], scale, dims, bufs, stream)
 
@@ -499,7 +527,10 @@ def measure_workload(args, spec, wl_key, world, dev, steps, e2e=True, cpu=True):
     if e2e:
         rec["e2e"] = {"value": per_sec(ms_e2e / steps * 1e-3), "unit": unit,
                       "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h}
-    if cpu and world == 1 and not args.no_cpu_baseline:
+    if int4:
+        rec["config"]["kv_cache"] = "INT4, two codes per byte, fp32 per-channel scales"
+        e2e = False
+    if cpu and world == 1 and not args.no_cpu_baseline and not int4:
         r = time_oracle(spec, x_with_scatter(x, spec), args.cpu_seconds)
         rec["cpu_baseline"] = {"value": r["gbs"] if unit == "GB/s" else r["tflops"], "unit": unit,
                                "cores": r["cores"], "kind": "oracle", "sample": r["sample"]}
@@ -597,6 +628,9 @@ def run_gpu(args, spec, rank, world, local):
             o = workloads.CONFIGS[workloads.CONFIG_KEYS[key]]()
             others[key] = measure_workload(args, o, key, world, dev, max(10, args.steps // 2),
                                            e2e=True)
+        others["long_decode_int4"] = measure_workload(
+            args, workloads.CONFIGS[workloads.CONFIG_KEYS["long_decode"]](), "long_decode_int4",
+            world, dev, max(10, args.steps // 2), e2e=False, int4=True)
         others["fused_split_qkv_rotary_scatter"] = measure_qkv_rotary(
             args, workloads.CONFIGS[workloads.CONFIG_KEYS["prefill"]](), world, dev,
             max(10, args.steps // 2))

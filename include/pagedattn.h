@@ -234,6 +234,42 @@ pa_status pa_attention_noalloc(const void* query, const void* key_cache, const v
                                const int32_t* seqlens_kv, float scale, void* out,
                                const pa_dims* dims, int32_t* dev_status, void* stream);
 
+/* INT4 KV cache.  The "[WebGPU] Implement SparseAttentionIndexer" PR's file
+ * list adds packed INT4 PagedAttention (INT4 cache reads and writes,
+ * per-channel scaling, INT4 dequantisation); the byte format is not given
+ * there, so this library defines it:
+ *   key_cache, value_cache: [num_blocks, block_size, kv_heads, head_size / 2]
+ *          bytes; byte j of a head row holds channel 2j in its low nibble and
+ *          channel 2j + 1 in its high nibble, as two's complement codes in
+ *          [-8, 7].
+ *   k_scale, v_scale: [kv_heads, head_size] fp32 device arrays, positive and
+ *          finite: code q of channel c of KV head h stands for q * scale[h][c].
+ * The caches hold a quarter of the f16 bytes; decode, which streams them, is
+ * bound by those bytes. */
+
+/* pa_scatter_kv_int4 -- pa_scatter_kv into INT4 caches: every value x of the
+ * new K/V rows (dims->dtype, f16 or bf16) is stored as
+ * clamp(round(x / scale), -8, 7), the quotient taken in fp32 and rounded to
+ * nearest-even.  head_size must be a multiple of 16.  Slots as for
+ * pa_scatter_kv. */
+pa_status pa_scatter_kv_int4(const void* key, const void* value, const int32_t* slot_mapping,
+                             const float* k_scale, const float* v_scale, void* key_cache,
+                             void* value_cache, const pa_dims* dims, int32_t* dev_status,
+                             void* stream);
+
+/* pa_attention_int4 -- pa_attention over INT4 caches, for decode batches:
+ * max_seqlen_q_hint must be set and no larger than the decode cut-off
+ * (min(4, 32 / group)); head sizes 32, 64 and 128; no softcap or window
+ * (PA_ERR_NOT_IMPLEMENTED otherwise).  The result is attention over the
+ * values the codes stand for.  Query and output in dims->dtype; workspace
+ * from pa_attention_workspace_size(dims).  A sequence longer than the hint
+ * is flagged PA_DEV_HINT_EXCEEDED and gets zero rows. */
+pa_status pa_attention_int4(const void* query, const void* key_cache, const void* value_cache,
+                            const float* k_scale, const float* v_scale, const int32_t* block_table,
+                            const int32_t* cu_seqlens_q, const int32_t* seqlens_kv, float scale,
+                            void* out, const pa_dims* dims, void* workspace,
+                            size_t workspace_bytes, int32_t* dev_status, void* stream);
+
 /* pa_get_status -- synchronise `stream` and copy *dev_status to *host_code.
  * For tests and debugging; it blocks the host. */
 pa_status pa_get_status(const int32_t* dev_status, int32_t* host_code, void* stream);

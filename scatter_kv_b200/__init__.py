@@ -90,6 +90,7 @@ EXPORTS = [
     "pa_scatter_kv", "pa_compute_slot_mapping", "pa_attention_workspace_size", "pa_attention",
     "pa_get_status", "pa_status_string", "pa_last_error", "pa_trace_enable", "pa_trace_read",
     "pa_kernel_name", "pa_attention_noalloc", "pa_split_qkv_rotary_scatter",
+    "pa_scatter_kv_int4", "pa_attention_int4",
 ]
 
 # Bytes of the fixed scratch array behind pa_attention_noalloc.
@@ -118,6 +119,11 @@ def _load():
                                                 ctypes.POINTER(pa_rotary), P, P, P, P, P, P, P,
                                                 D, P, P]
     lib.pa_split_qkv_rotary_scatter.restype = ctypes.c_int
+    lib.pa_scatter_kv_int4.argtypes = [P, P, P, P, P, P, P, D, P, P]
+    lib.pa_scatter_kv_int4.restype = ctypes.c_int
+    lib.pa_attention_int4.argtypes = [P, P, P, P, P, P, P, P, ctypes.c_float, P, D, P,
+                                      ctypes.c_size_t, P, P]
+    lib.pa_attention_int4.restype = ctypes.c_int
     lib.pa_get_status.argtypes = [P, I32P, P]
     lib.pa_get_status.restype = ctypes.c_int
     lib.pa_status_string.argtypes = [ctypes.c_int]
@@ -253,6 +259,26 @@ def pa_split_qkv_rotary_scatter(query, key, value, q_token_stride, kv_token_stri
         _ptr(block_table), _ptr(cu_seqlens_q), _ptr(seqlens_kv), _ptr(query_out), _ptr(key_cache),
         _ptr(value_cache), _ptr(slot_mapping), ctypes.byref(dims), _ptr(dev_status),
         _stream(stream)))
+
+
+def pa_scatter_kv_int4(key, value, slot_mapping, k_scale, v_scale, key_cache, value_cache,
+                       dims: pa_dims, dev_status=None, stream=None) -> None:
+    _check(lib.pa_scatter_kv_int4(_ptr(key), _ptr(value), _ptr(slot_mapping), _ptr(k_scale),
+                                  _ptr(v_scale), _ptr(key_cache), _ptr(value_cache),
+                                  ctypes.byref(dims), _ptr(dev_status), _stream(stream)))
+
+
+def pa_attention_int4(query, key_cache, value_cache, k_scale, v_scale, block_table, cu_seqlens_q,
+                      seqlens_kv, scale, out, dims: pa_dims, workspace=None, workspace_bytes=None,
+                      dev_status=None, stream=None) -> None:
+    if workspace_bytes is None:
+        workspace_bytes = 0 if workspace is None or isinstance(workspace, int) else \
+            workspace.numel() * workspace.element_size()
+    _check(lib.pa_attention_int4(_ptr(query), _ptr(key_cache), _ptr(value_cache), _ptr(k_scale),
+                                 _ptr(v_scale), _ptr(block_table), _ptr(cu_seqlens_q),
+                                 _ptr(seqlens_kv), float(scale), _ptr(out), ctypes.byref(dims),
+                                 _ptr(workspace), int(workspace_bytes), _ptr(dev_status),
+                                 _stream(stream)))
 
 
 def packed_qkv_views(qkv, dims: pa_dims):

@@ -502,6 +502,117 @@ pa_status pa_split_qkv_rotary_scatter(const void* query, const void* key, const 
     return e == cudaSuccess ? PA_OK : cuda_fail(e, "split-QKV rotary scatter launch");
 }
 
+pa_status pa_scatter_kv_int4(const void* key, const void* value, const int32_t* slot_mapping,
+                             const float* k_scale, const float* v_scale, void* key_cache,
+                             void* value_cache, const pa_dims* dims, int32_t* dev_status,
+                             void* stream) {
+    g_last_error[0] = 0;
+    pa_status st = check_dims(dims);
+    if (st != PA_OK) return st;
+    if (dims->head_size % 16 != 0)
+        return fail(PA_ERR_NOT_IMPLEMENTED, "INT4 caches: head_size %d is not a multiple of 16",
+                    dims->head_size);
+    if (dims->token_count == 0) return PA_OK;
+    PA_REQUIRE_PTR(key);
+    PA_REQUIRE_PTR(value);
+    PA_REQUIRE_IPTR(slot_mapping);
+    PA_REQUIRE_PTR(k_scale);
+    PA_REQUIRE_PTR(v_scale);
+    PA_REQUIRE_PTR(key_cache);
+    PA_REQUIRE_PTR(value_cache);
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    TraceScope tr(PA_KERNEL_SCATTER, s);
+    cudaError_t e = pa::launch_scatter_int4(key, value, slot_mapping, k_scale, v_scale, key_cache,
+                                            value_cache, *dims, dev_status, s,
+                                            num_sms_of_current_device());
+    return e == cudaSuccess ? PA_OK : cuda_fail(e, "INT4 scatter launch");
+}
+
+pa_status pa_attention_int4(const void* query, const void* key_cache, const void* value_cache,
+                            const float* k_scale, const float* v_scale, const int32_t* block_table,
+                            const int32_t* cu_seqlens_q, const int32_t* seqlens_kv, float scale,
+                            void* out, const pa_dims* dims, void* workspace,
+                            size_t workspace_bytes, int32_t* dev_status, void* stream) {
+    g_last_error[0] = 0;
+    pa_status st = check_dims(dims);
+    if (st != PA_OK) return st;
+    const pa_dims& d = *dims;
+    if (d.head_size != 32 && d.head_size != 64 && d.head_size != 128)
+        return fail(PA_ERR_NOT_IMPLEMENTED, "INT4 attention: head sizes 32, 64 and 128 are built");
+    if (d.softcap > 0.f || d.local_window)
+        return fail(PA_ERR_NOT_IMPLEMENTED, "INT4 attention: no softcap or local window");
+    const int nsm = num_sms_of_current_device();
+    const pa::DecodePlan plan = pa::plan_decode(d, nsm);
+    if (d.max_seqlen_q_hint <= 0 || d.max_seqlen_q_hint > plan.decode_max_q)
+        return fail(PA_ERR_NOT_IMPLEMENTED,
+                    "INT4 attention serves decode batches: max_seqlen_q_hint must be set and at most "
+                    "%d for these heads", plan.decode_max_q);
+    if (d.token_count == 0) return PA_OK;
+    if (d.batch == 0) return fail(PA_ERR_INVALID_ARGUMENT, "token_count > 0 with batch 0");
+    if (!(scale >= 0.f) || isinf(scale))
+        return fail(PA_ERR_INVALID_ARGUMENT, "scale must be finite and >= 0");
+    PA_REQUIRE_PTR(query);
+    PA_REQUIRE_PTR(key_cache);
+    PA_REQUIRE_PTR(value_cache);
+    PA_REQUIRE_PTR(k_scale);
+    PA_REQUIRE_PTR(v_scale);
+    PA_REQUIRE_PTR(out);
+    PA_REQUIRE_IPTR(block_table);
+    PA_REQUIRE_IPTR(cu_seqlens_q);
+    PA_REQUIRE_IPTR(seqlens_kv);
+    if (workspace_bytes < plan.workspace_bytes)
+        return fail(PA_ERR_INVALID_ARGUMENT, "workspace of %zu bytes is smaller than the %zu needed",
+                    workspace_bytes, plan.workspace_bytes);
+    if (plan.workspace_bytes > 0) PA_REQUIRE_PTR(workspace);
+    if (scale == 0.f) scale = 1.f / sqrtf((float)d.head_size);
+    pa::DecodeParams p{};
+    p.query = static_cast<const uint16_t*>(query);
+    p.key_cache = static_cast<const uint16_t*>(key_cache);
+    p.value_cache = static_cast<const uint16_t*>(value_cache);
+    p.out = static_cast<uint16_t*>(out);
+    const size_t rows_total = (size_t)d.batch * d.kv_heads * plan.max_splits * (16 * plan.mtiles);
+    p.part_o = static_cast<float*>(workspace);
+    p.part_lse = plan.workspace_bytes ? static_cast<float*>(workspace) + rows_total * d.head_size
+                                      : nullptr;
+    p.block_table = block_table;
+    p.cu_seqlens_q = cu_seqlens_q;
+    p.seqlens_kv = seqlens_kv;
+    p.status = dev_status;
+    p.token_count = d.token_count;
+    p.num_blocks = d.num_blocks;
+    p.batch = d.batch;
+    p.q_heads = d.q_heads;
+    p.kv_heads = d.kv_heads;
+    p.group = d.q_heads / d.kv_heads;
+    p.head_size = d.head_size;
+    p.block_size = d.block_size;
+    p.max_blocks = d.max_blocks_per_seq;
+    p.kv_cap = d.max_blocks_per_seq * d.block_size;
+    p.kv_hint = d.max_seqlen_kv_hint;
+    p.q_hint = d.max_seqlen_q_hint;
+    p.decode_max_q = plan.decode_max_q;
+    p.chunk = plan.chunk;
+    p.max_splits = plan.max_splits;
+    p.rmax = 16 * plan.mtiles;
+    p.mods.scale = scale;
+    p.mods.scale_log2 = scale * 1.4426950408889634f;
+    p.k_scale = k_scale;
+    p.v_scale = v_scale;
+    const bool bf16 = d.dtype == PA_DTYPE_BF16;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    {
+        TraceScope tr(PA_KERNEL_DECODE, s);
+        cudaError_t e = pa::launch_decode_int4(p, d.head_size, plan.mtiles, bf16, s);
+        if (e != cudaSuccess) return cuda_fail(e, "INT4 decode launch");
+    }
+    if (plan.max_splits > 1) {
+        TraceScope tr(PA_KERNEL_COMBINE, s);
+        cudaError_t e = pa::launch_combine(p, d.head_size, bf16, s);
+        if (e != cudaSuccess) return cuda_fail(e, "combine launch");
+    }
+    return PA_OK;
+}
+
 pa_status pa_get_status(const int32_t* dev_status, int32_t* host_code, void* stream) {
     g_last_error[0] = 0;
     if (dev_status == nullptr || host_code == nullptr)

@@ -249,6 +249,9 @@ template <>
 struct Elem<__half> {
     static constexpr bool kBf16 = false;
     static __device__ __forceinline__ uint32_t pack2(float lo, float hi) { return pack_half2(lo, hi); }
+    static __device__ __forceinline__ float2 unpack2(uint32_t v) {
+        return __half22float2(*reinterpret_cast<const __half2*>(&v));
+    }
     static __device__ __forceinline__ void mma(float* d, const uint32_t* a, uint32_t b0, uint32_t b1) {
         mma_16816(d, a, b0, b1);
     }
@@ -260,6 +263,9 @@ struct Elem<__nv_bfloat16> {
     static __device__ __forceinline__ uint32_t pack2(float lo, float hi) {
         __nv_bfloat162 h = __floats2bfloat162_rn(lo, hi);
         return *reinterpret_cast<uint32_t*>(&h);
+    }
+    static __device__ __forceinline__ float2 unpack2(uint32_t v) {
+        return __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&v));
     }
     static __device__ __forceinline__ void mma(float* d, const uint32_t* a, uint32_t b0, uint32_t b1) {
         mma_16816_bf16(d, a, b0, b1);

@@ -55,6 +55,12 @@ constexpr int kDecodeLaunchRegs = 80;
 constexpr int kDecRegsCons = 136, kDecRegsProd = 24;
 static_assert(128 * (kDecRegsCons + kDecRegsProd) == 256 * kDecodeLaunchRegs,
               "register split must equal the launch budget");
+// INT4 pages: two CTAs per SM at 128 registers; the consumers take 168, the
+// producers (which hold four tiles of loads in registers) 88.
+constexpr int kQ4LaunchRegs = 128;
+constexpr int kQ4RegsCons = 168, kQ4RegsProd = 88;
+static_assert(128 * (kQ4RegsCons + kQ4RegsProd) == 256 * kQ4LaunchRegs,
+              "register split must equal the launch budget");
 
 template <int HEAD, int MT, bool CPA>
 struct Cfg {
@@ -125,8 +131,41 @@ __device__ __forceinline__ void zero_rows(const DecodeParams& p, const SeqInfo& 
     }
 }
 
-template <int HEAD, int MT, bool CPA, typename ET, bool GEN>
-__global__ void __launch_bounds__(Cfg<HEAD, MT, CPA>::THREADS, (HEAD >= 128 && !CPA) ? 2 : 3)
+// INT4 pages (Q4): two signed 4-bit codes per byte, the low nibble the even
+// channel; a code q of channel c stands for q * scale[kv head][c].  The
+// producer converts the codes of a 16-byte chunk (32 channels of one key) to
+// 16-bit values exactly: byte b's two nibbles are placed in the low bits of
+// the two halves of a 32-bit word, their sign bits flipped, over the
+// exponent of 1024 (f16) or 128 (bf16), where the spacing of representable
+// values is 1 -- so each half reads 1024 + (n ^ 8) (or 128 + (n ^ 8)) and
+// one subtraction leaves n as a signed integer.
+template <typename ET>
+__device__ __forceinline__ uint32_t int4_pair(uint32_t w, uint32_t w_hi, int byte) {
+    // Byte `byte` of w into bits 0-7, the same byte of w >> 4 into bits 16-23.
+    const uint32_t t = __byte_perm(w, w_hi, (uint32_t)(byte | (byte << 4) | ((4 + byte) << 8) | ((4 + byte) << 12)));
+    if (Elem<ET>::kBf16) {
+        const uint32_t v = (t & 0x000F000Fu) ^ 0x43084308u;          // 128 + (n ^ 8), both halves
+        __nv_bfloat162 h = *reinterpret_cast<const __nv_bfloat162*>(&v);
+        h = __hsub2(h, __floats2bfloat162_rn(136.f, 136.f));
+        return *reinterpret_cast<uint32_t*>(&h);
+    } else {
+        const uint32_t v = (t & 0x000F000Fu) ^ 0x64086408u;          // 1024 + (n ^ 8), both halves
+        __half2 h = *reinterpret_cast<const __half2*>(&v);
+        h = __hsub2(h, __floats2half2_rn(1032.f, 1032.f));
+        return *reinterpret_cast<uint32_t*>(&h);
+    }
+}
+
+__device__ __forceinline__ uint4 ld_nc16(const void* p) {
+    uint4 v;
+    asm volatile("ld.global.nc.L1::no_allocate.v4.u32 {%0, %1, %2, %3}, [%4];"
+                 : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w) : "l"(p));
+    return v;
+}
+
+template <int HEAD, int MT, bool CPA, typename ET, bool GEN, bool Q4 = false>
+__global__ void __launch_bounds__(Cfg<HEAD, MT, CPA>::THREADS,
+                                  Q4 ? 2 : ((HEAD >= 128 && !CPA) ? 2 : 3))
 decode_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_v,
               const DecodeParams p) {
     using C = Cfg<HEAD, MT, CPA>;
@@ -228,7 +267,8 @@ decode_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ 
 
     if (warp >= C::NCW) {
         // ------------------------------------------------------------ producers
-        if (CPA) asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(kDecRegsProd));
+        if (Q4) asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(kQ4RegsProd));
+        else if (CPA) asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(kDecRegsProd));
         const int pw = warp - C::NCW;
         // The split's block ids, fetched once by the first producer warp, so
         // issuing a tile never waits on a dependent global load.  They are
@@ -257,7 +297,81 @@ decode_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ 
             const int i = page - pg0;
             return i < C::MAX_IDS ? sids[i] : bt[page];
         };
-        if (CPA && !bad) {
+        if constexpr (Q4) {
+            if (!bad) {
+                // INT4 pages (any block size): producer thread q loads the 16-byte
+                // chunk q % CPR4 (32 channels) of key row q / CPR4 of every tile,
+                // D tiles ahead in registers, and writes its 64 bytes of 16-bit
+                // values where the swizzled stage layout puts them; each thread
+                // arrives on the stage once its stores are done.
+                constexpr int CPR4 = HEAD / 32;
+                static_assert(HEAD >= 32 && (C::NPW * 32) / CPR4 >= C::BN, "one pass covers a tile");
+                constexpr int D = 4;
+                const int q0 = pw * 32 + lane;
+                const int r = q0 / CPR4, jc = q0 % CPR4;
+                const bool active = r < C::BN;
+                const int lbs = 31 - __clz(bs);
+                const char* kc = reinterpret_cast<const char*>(p.key_cache);
+                const char* vc = reinterpret_cast<const char*>(p.value_cache);
+                const long long row_bytes = (long long)p.kv_heads * (HEAD / 2);
+                const long long colb = (long long)kvh * (HEAD / 2) + jc * 16;
+                uint4 kr[D], vr[D];
+                auto issue = [&](int t, uint4& kx, uint4& vx) {
+                    kx = vx = make_uint4(0, 0, 0, 0);
+                    const int key = k_begin + t * C::BN + r;
+                    if (active && t < ntiles && key < k_end) {
+                        const long long g = ((long long)block_of(key >> lbs) * bs + (key & (bs - 1))) * row_bytes + colb;
+                        kx = ld_nc16(kc + g);
+                        vx = ld_nc16(vc + g);
+                    }
+                };
+                auto put = [&](uint8_t* tile, const uint4& x) {
+                    const uint32_t w[4] = {x.x, x.y, x.z, x.w};
+#pragma unroll
+                    for (int i = 0; i < 4; ++i) {
+                        const uint32_t hi = w[i] >> 4;
+                        uint4 o;
+                        o.x = int4_pair<ET>(w[i], hi, 0);
+                        o.y = int4_pair<ET>(w[i], hi, 1);
+                        o.z = int4_pair<ET>(w[i], hi, 2);
+                        o.w = int4_pair<ET>(w[i], hi, 3);
+                        const int ch = jc * 32 + i * 8;
+                        const int cb = ch / C::A, jj = (ch % C::A) / 8;
+                        *reinterpret_cast<uint4*>(tile + swz<C::RB>((uint32_t)((cb * C::BN + r) * C::RB + jj * 16))) = o;
+                    }
+                };
+#pragma unroll
+                for (int j = 0; j < D; ++j) issue(j, kr[j], vr[j]);
+                bool stop = false;
+                for (int t0 = 0; t0 < ntiles && !stop; t0 += D) {
+#pragma unroll
+                    for (int j = 0; j < D; ++j) {
+                        const int t = t0 + j;
+                        if (t >= ntiles) break;
+                        const int st = t % C::NST, u = t / C::NST;
+                        bool go = true;
+                        if (lane == 0 && u > 0) go = mbar_wait(&empty[st], (u - 1) & 1);
+                        go = __shfl_sync(0xffffffffu, go, 0);
+                        if (!go) {
+                            if (lane == 0) {
+                                flag_status(p.status, PA_DEV_TIMEOUT);
+                                atomicExch(&sflag[1], 1);
+                            }
+                            stop = true;
+                            break;
+                        }
+                        if (__shfl_sync(0xffffffffu, *(volatile int*)&sflag[1], 0)) { stop = true; break; }
+                        uint8_t* kt = stages + st * C::STAGE_BYTES;
+                        if (active) {
+                            put(kt, kr[j]);
+                            put(kt + C::TILE_BYTES, vr[j]);
+                        }
+                        mbar_arrive(&full[st]);
+                        issue(t + D, kr[j], vr[j]);
+                    }
+                }
+            }
+        } else if (CPA && !bad) {
             // 16-key pages (the only size that takes this path): a 32-key tile
             // is exactly pages k0/16 and k0/16 + 1.  Producer thread q copies
             // the 16-byte chunk q % CPR of rows q / CPR + i * RPI (a fixed
@@ -336,7 +450,8 @@ decode_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ 
         }
     } else {
         // ------------------------------------------------------------ consumers
-        if (CPA) asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(kDecRegsCons));
+        if (Q4) asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(kQ4RegsCons));
+        else if (CPA) asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(kDecRegsCons));
         const int mt = warp % MT;          // which 16 query rows
         const int grp = warp / MT;         // which tiles
         const int quad = lane >> 2, qid = lane & 3;
@@ -364,6 +479,17 @@ decode_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ 
                 qf[kk][1] = (q1 && lo_ok) ? *reinterpret_cast<const uint32_t*>(q1 + c) : 0u;
                 qf[kk][2] = (q0 && hi_ok) ? *reinterpret_cast<const uint32_t*>(q0 + c + 8) : 0u;
                 qf[kk][3] = (q1 && hi_ok) ? *reinterpret_cast<const uint32_t*>(q1 + c + 8) : 0u;
+                if constexpr (Q4) {
+                    // The K scales fold into Q: S = sum_c (Q[c] * ks[c]) * code[c].
+                    const float2 s0 = *reinterpret_cast<const float2*>(p.k_scale + kvh * HEAD + c);
+                    const float2 s1 = *reinterpret_cast<const float2*>(p.k_scale + kvh * HEAD + c + 8);
+#pragma unroll
+                    for (int e = 0; e < 4; ++e) {
+                        const float2 sc = (e < 2) ? s0 : s1;
+                        const float2 qv = Elem<ET>::unpack2(qf[kk][e]);
+                        qf[kk][e] = E::pack2(qv.x * sc.x, qv.y * sc.y);
+                    }
+                }
             }
         }
         const long long pbase = (((long long)b * p.kv_heads + kvh) * p.max_splits + split) * p.rmax;
@@ -554,6 +680,11 @@ decode_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ 
             const float L = row_l[r];
             const float inv = (L > 0.f) ? 1.f / L : 0.f;
             acc.x *= inv; acc.y *= inv; acc.z *= inv; acc.w *= inv;
+            if constexpr (Q4) {
+                // V's per-channel scales factor out of the P V sum.
+                const float4 vs = *reinterpret_cast<const float4*>(p.v_scale + kvh * HEAD + d4);
+                acc.x *= vs.x; acc.y *= vs.y; acc.z *= vs.z; acc.w *= vs.w;
+            }
             if (direct) {
                 uint2 w;
                 w.x = E::pack2(acc.x, acc.y);
@@ -641,17 +772,18 @@ __global__ void __launch_bounds__(128) combine_kernel(const DecodeParams p) {
     *reinterpret_cast<uint2*>(orow + lane * 4) = wv;
 }
 
-template <int HEAD, int MT, bool CPA, typename ET, bool GEN>
+template <int HEAD, int MT, bool CPA, typename ET, bool GEN, bool Q4 = false>
 cudaError_t launch_decode_t(const CUtensorMap& tm_k, const CUtensorMap& tm_v,
                             const DecodeParams& p, cudaStream_t stream) {
     using C = Cfg<HEAD, MT, CPA>;
-    auto kern = decode_kernel<HEAD, MT, CPA, ET, GEN>;
+    auto kern = decode_kernel<HEAD, MT, CPA, ET, GEN, Q4>;
     cudaError_t e;
     if (CPA) {
+        // The register split inside the kernel assumes this launch budget.
         cudaFuncAttributes fa;
         e = cudaFuncGetAttributes(&fa, kern);
         if (e != cudaSuccess) return e;
-        if (fa.numRegs != kDecodeLaunchRegs) return cudaErrorInvalidKernelImage;
+        if (fa.numRegs != (Q4 ? kQ4LaunchRegs : kDecodeLaunchRegs)) return cudaErrorInvalidKernelImage;
     }
     e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM);
     if (e != cudaSuccess) return e;
@@ -671,6 +803,13 @@ cudaError_t launch_decode_h(const CUtensorMap& tm_k, const CUtensorMap& tm_v, co
                            : launch_decode_t<HEAD, 2, true, ET, GEN>(tm_k, tm_v, p, stream);
     return mtiles == 1 ? launch_decode_t<HEAD, 1, false, ET, GEN>(tm_k, tm_v, p, stream)
                        : launch_decode_t<HEAD, 2, false, ET, GEN>(tm_k, tm_v, p, stream);
+}
+
+template <int HEAD, typename ET>
+cudaError_t launch_decode_q4_h(const CUtensorMap& tm, const DecodeParams& p, int mtiles,
+                               cudaStream_t stream) {
+    return mtiles == 1 ? launch_decode_t<HEAD, 1, true, ET, false, true>(tm, tm, p, stream)
+                       : launch_decode_t<HEAD, 2, true, ET, false, true>(tm, tm, p, stream);
 }
 
 template <typename ET, bool GEN>
@@ -737,6 +876,20 @@ cudaError_t launch_decode(const CUtensorMap& tm_k, const CUtensorMap& tm_v,
                    : launch_decode_d<__nv_bfloat16, false>(tm_k, tm_v, p, head, mtiles, stream);
     return gen ? launch_decode_d<__half, true>(tm_k, tm_v, p, head, mtiles, stream)
                : launch_decode_d<__half, false>(tm_k, tm_v, p, head, mtiles, stream);
+}
+
+cudaError_t launch_decode_int4(const DecodeParams& p, int head, int mtiles, bool bf16,
+                               cudaStream_t stream) {
+    CUtensorMap unused{};                 // the INT4 producer reads pages without TMA
+    switch (head) {
+        case 32: return bf16 ? launch_decode_q4_h<32, __nv_bfloat16>(unused, p, mtiles, stream)
+                             : launch_decode_q4_h<32, __half>(unused, p, mtiles, stream);
+        case 64: return bf16 ? launch_decode_q4_h<64, __nv_bfloat16>(unused, p, mtiles, stream)
+                             : launch_decode_q4_h<64, __half>(unused, p, mtiles, stream);
+        case 128: return bf16 ? launch_decode_q4_h<128, __nv_bfloat16>(unused, p, mtiles, stream)
+                              : launch_decode_q4_h<128, __half>(unused, p, mtiles, stream);
+        default: return cudaErrorInvalidValue;
+    }
 }
 
 template <typename ET>

@@ -72,6 +72,8 @@ struct DecodeParams {
     int max_splits;
     int rmax;                     // row capacity per (sequence, kv head) = 16 * m-tiles
     ScoreMods mods;
+    const float* k_scale;         // INT4 caches: per-channel scales [kv_heads, head_size]
+    const float* v_scale;
 };
 
 struct PrefillParams {
@@ -161,6 +163,13 @@ cudaError_t launch_slot_mapping(const int32_t* block_table, const int32_t* cu,
 cudaError_t launch_decode(const CUtensorMap& tm_k, const CUtensorMap& tm_v,
                           const DecodeParams& p, int head, int mtiles, bool bf16, cudaStream_t stream);
 cudaError_t launch_combine(const DecodeParams& p, int head, bool bf16, cudaStream_t stream);
+// Decode over INT4 caches (head sizes 32, 64, 128; any block size).
+cudaError_t launch_decode_int4(const DecodeParams& p, int head, int mtiles, bool bf16,
+                               cudaStream_t stream);
+cudaError_t launch_scatter_int4(const void* key, const void* value, const int32_t* slot_mapping,
+                                const float* k_scale, const float* v_scale, void* key_cache,
+                                void* value_cache, const pa_dims& d, int32_t* status,
+                                cudaStream_t stream, int num_sms);
 
 // Size of the fixed scratch array behind pa_attention_noalloc, and the
 // lookup of its device address on the current device (once per device).

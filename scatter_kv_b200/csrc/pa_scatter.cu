@@ -124,7 +124,77 @@ slot_mapping_kernel(const int32_t* __restrict__ block_table, const int32_t* __re
     slot_mapping[t] = slot;
 }
 
+// Scatter into INT4 caches: each thread quantises 16 channels of one token's
+// head row of K and of V -- code = round(x / scale) (binary32 division,
+// nearest-even) clamped to [-8, 7] -- and writes them as 8 packed bytes, the
+// low nibble the even channel.
+template <typename ET>
+__global__ void __launch_bounds__(kScatterThreads)
+scatter_kv_int4_kernel(const uint16_t* __restrict__ key, const uint16_t* __restrict__ value,
+                       const int32_t* __restrict__ slot_mapping, const float* __restrict__ k_scale,
+                       const float* __restrict__ v_scale, uint8_t* __restrict__ key_cache,
+                       uint8_t* __restrict__ value_cache, long long token_count, int kv_heads,
+                       int head_size, long long num_slots, int32_t* status) {
+    pdl_launch_dependents();
+    pdl_wait();
+    const int per_head = head_size / 16;
+    const int per_token = kv_heads * per_head;
+    const long long total = token_count * per_token;
+    for (long long i = (long long)blockIdx.x * kScatterThreads + threadIdx.x; i < total;
+         i += (long long)gridDim.x * kScatterThreads) {
+        const long long t = i / per_token;
+        const int u = (int)(i - t * per_token);
+        const int h = u / per_head, c0 = (u - h * per_head) * 16;
+        const long long src = (t * kv_heads + h) * head_size + c0;
+        const uint4 k0 = *reinterpret_cast<const uint4*>(key + src);
+        const uint4 k1 = *reinterpret_cast<const uint4*>(key + src + 8);
+        const uint4 v0 = *reinterpret_cast<const uint4*>(value + src);
+        const uint4 v1 = *reinterpret_cast<const uint4*>(value + src + 8);
+        const int slot = __ldg(slot_mapping + t);
+        if (slot < 0) continue;
+        if ((long long)slot >= num_slots) {
+            if (u == 0) flag_status(status, PA_DEV_BAD_SLOT);
+            continue;
+        }
+        auto quant = [&](const uint4& a, const uint4& b, const float* sc) {
+            const uint32_t w[8] = {a.x, a.y, a.z, a.w, b.x, b.y, b.z, b.w};
+            uint32_t packed[2] = {0u, 0u};
+#pragma unroll
+            for (int j = 0; j < 8; ++j) {
+                const float2 x = Elem<ET>::unpack2(w[j]);
+                const float2 s = *reinterpret_cast<const float2*>(sc + 2 * j);
+                const float q0 = fminf(fmaxf(rintf(__fdiv_rn(x.x, s.x)), -8.f), 7.f);
+                const float q1 = fminf(fmaxf(rintf(__fdiv_rn(x.y, s.y)), -8.f), 7.f);
+                const uint32_t byte = ((uint32_t)(int)q0 & 0xFu) | (((uint32_t)(int)q1 & 0xFu) << 4);
+                packed[j >> 2] |= byte << (8 * (j & 3));
+            }
+            return make_uint2(packed[0], packed[1]);
+        };
+        const long long dst = ((long long)slot * kv_heads + h) * (head_size / 2) + c0 / 2;
+        *reinterpret_cast<uint2*>(key_cache + dst) = quant(k0, k1, k_scale + h * head_size + c0);
+        *reinterpret_cast<uint2*>(value_cache + dst) = quant(v0, v1, v_scale + h * head_size + c0);
+    }
+}
+
 }  // namespace
+
+cudaError_t launch_scatter_int4(const void* key, const void* value, const int32_t* slot_mapping,
+                                const float* k_scale, const float* v_scale, void* key_cache,
+                                void* value_cache, const pa_dims& d, int32_t* status,
+                                cudaStream_t stream, int num_sms) {
+    const long long total = d.token_count * d.kv_heads * (d.head_size / 16);
+    long long blocks = (total + kScatterThreads - 1) / kScatterThreads;
+    const long long cap = (long long)num_sms * 8;
+    if (blocks > cap) blocks = cap;
+    if (blocks < 1) blocks = 1;
+    auto kern = d.dtype == PA_DTYPE_BF16 ? scatter_kv_int4_kernel<__nv_bfloat16>
+                                         : scatter_kv_int4_kernel<__half>;
+    return launch_pdl(kern, dim3((unsigned)blocks), dim3(kScatterThreads), 0, stream,
+                      static_cast<const uint16_t*>(key), static_cast<const uint16_t*>(value),
+                      slot_mapping, k_scale, v_scale, static_cast<uint8_t*>(key_cache),
+                      static_cast<uint8_t*>(value_cache), d.token_count, d.kv_heads, d.head_size,
+                      d.num_blocks * (long long)d.block_size, status);
+}
 
 cudaError_t launch_scatter(const void* key, const void* value, const int32_t* slot_mapping,
                            void* key_cache, void* value_cache, const pa_dims& d,
