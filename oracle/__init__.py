@@ -64,6 +64,10 @@ def _load():
         lib.oracle_rotary.argtypes = [P, i64, ctypes.c_int, ctypes.c_int, i64, P, P, P,
                                       ctypes.c_int, ctypes.c_int, ctypes.c_int, P]
         lib.oracle_max_threads.restype = ctypes.c_int
+        lib.oracle_sparse_attention.argtypes = [P, P, P, P, P, P, ctypes.c_int, i64, ctypes.c_int,
+                                                ctypes.c_int, ctypes.c_int, ctypes.c_int,
+                                                ctypes.c_int, P, ctypes.c_int, ctypes.c_int,
+                                                ctypes.c_double, ctypes.c_int, P, P, P]
         lib.oracle_quantize_int4.argtypes = [ctypes.c_float, ctypes.c_float]
         lib.oracle_quantize_int4.restype = ctypes.c_int
         lib.oracle_scatter_kv_int4.argtypes = [P, P, P, P, P, P, P, i64, ctypes.c_int, ctypes.c_int,
@@ -253,4 +257,34 @@ def dequantize_int4(cache, scale) -> np.ndarray:
     sc = _c(scale, np.float32).reshape(kvh, d)
     out = np.empty((nb, bs, kvh, d), dtype=np.float64)
     lib.oracle_dequantize_int4(_ptr(c), _ptr(sc), nb * bs, kvh, d, _ptr(out))
+    return out
+
+
+def sparse_attention(query, key_cache, value_cache, block_table, cu_seqlens_q, seqlens_kv,
+                     selected, local_window: int, scale: float, bf16: bool = False) -> np.ndarray:
+    """Local-plus-selected attention: token t and KV head h see keys
+    [P - local_window, P] plus the selected positions selected[t, h, :] that
+    are in [0, P] (int32 [token_count, kv_heads, num_selected]; -1 pads),
+    each key once.  Returns float64 [token_count, q_heads, head_size]."""
+    lib = _load()
+    dtype = _elem_type(query, bf16)
+    q = _c(query, query.dtype)
+    kc = key_cache if key_cache.flags.c_contiguous else np.ascontiguousarray(key_cache)
+    vc = value_cache if value_cache.flags.c_contiguous else np.ascontiguousarray(value_cache)
+    bt = _c(block_table, np.int32)
+    cu = _c(cu_seqlens_q, np.int32)
+    skv = _c(seqlens_kv, np.int32)
+    sel = _c(selected, np.int32)
+    T, qh, d = q.shape
+    nb, bs, kvh, _ = kc.shape
+    assert sel.shape[:2] == (T, kvh) and local_window >= 0
+    max_keys = max(1, int(skv.max()) if skv.size else 1)
+    mark = np.empty(max_keys, dtype=np.uint8)
+    scores = np.empty(max_keys, dtype=np.float64)
+    out = np.empty((T, qh, d), dtype=np.float64)
+    if T:
+        lib.oracle_sparse_attention(_ptr(q), _ptr(kc), _ptr(vc), _ptr(bt), _ptr(cu), _ptr(skv),
+                                    len(skv), T, qh, kvh, d, bs, bt.shape[1], _ptr(sel),
+                                    sel.shape[2], int(local_window), float(scale), dtype,
+                                    _ptr(mark), _ptr(scores), _ptr(out))
     return out

@@ -391,6 +391,68 @@ void oracle_dequantize_int4(const uint8_t *cache, const float *scale, int64_t nu
                     (double)scale[h * head_size + c];
 }
 
+/* Sparse paged attention, local plus selected ("[WebGPU] Implement
+ * SparseAttentionIndexer" follow-up, "Motivation and Context": selections
+ * reference request-local positions in the main paged cache, executed as
+ * local-plus-selected attention).  Reading taken: query token t (sequence b,
+ * position P = past_len_b + i) and KV head h see the union of the local
+ * window -- keys [max(0, P - local_window), P] -- and the selected positions
+ * selected[t][h][0 .. num_selected) that are >= 0 and <= P; each key counts
+ * once.  Query heads of one KV head's group share its selection.  The
+ * scores, softmax and V average are those of oracle_attention, over that
+ * key set in increasing position order.  out: [token_count, q_heads,
+ * head_size] doubles; mark: scratch of max_keys bytes. */
+void oracle_sparse_attention(const void *query, const void *key_cache, const void *value_cache,
+                             const int32_t *block_table, const int32_t *cu_seqlens_q,
+                             const int32_t *seqlens_kv, int batch, int64_t token_count,
+                             int q_heads, int kv_heads, int head_size, int block_size,
+                             int max_blocks_per_seq, const int32_t *selected, int num_selected,
+                             int local_window, double scale, int dtype, uint8_t *mark,
+                             double *scores, double *out)
+{
+    fill_half_table();
+    int group = q_heads / kv_heads;
+    for (int64_t t = 0; t < token_count; ++t) {
+        int b = seq_of_token(cu_seqlens_q, batch, t);
+        int64_t q_len = cu_seqlens_q[b + 1] - cu_seqlens_q[b];
+        int64_t P = seqlens_kv[b] - q_len + (t - cu_seqlens_q[b]);
+        for (int h = 0; h < q_heads; ++h) {
+            int kvh = h / group;
+            memset(mark, 0, (size_t)(P + 1));
+            for (int64_t j = P - local_window < 0 ? 0 : P - local_window; j <= P; ++j) mark[j] = 1;
+            for (int s = 0; s < num_selected; ++s) {
+                int32_t e = selected[(t * kv_heads + kvh) * (int64_t)num_selected + s];
+                if (e >= 0 && e <= P) mark[e] = 1;
+            }
+            int64_t qbase = (t * q_heads + h) * (int64_t)head_size;
+            double m = -INFINITY;
+            for (int64_t j = 0; j <= P; ++j) {
+                if (!mark[j]) continue;
+                int64_t block = block_table[(int64_t)b * max_blocks_per_seq + j / block_size];
+                int64_t kbase = ((block * block_size + j % block_size) * kv_heads + kvh) * (int64_t)head_size;
+                double sc = 0.0;
+                for (int d = 0; d < head_size; ++d)
+                    sc += load(query, qbase + d, dtype) * load(key_cache, kbase + d, dtype);
+                sc *= scale;
+                scores[j] = sc;
+                if (sc > m) m = sc;
+            }
+            double denom = 0.0;
+            double *y = out + qbase;
+            for (int d = 0; d < head_size; ++d) y[d] = 0.0;
+            for (int64_t j = 0; j <= P; ++j) {
+                if (!mark[j]) continue;
+                double pj = exp(scores[j] - m);
+                denom += pj;
+                int64_t block = block_table[(int64_t)b * max_blocks_per_seq + j / block_size];
+                int64_t vbase = ((block * block_size + j % block_size) * kv_heads + kvh) * (int64_t)head_size;
+                for (int d = 0; d < head_size; ++d) y[d] += pj * load(value_cache, vbase + d, dtype);
+            }
+            for (int d = 0; d < head_size; ++d) y[d] /= denom;
+        }
+    }
+}
+
 int oracle_max_threads(void)
 {
 #ifdef _OPENMP

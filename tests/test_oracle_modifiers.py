@@ -324,3 +324,78 @@ def test_int4_attention_on_grid_values_equals_plain_attention():
     got = oracle.attention(P["query"].astype(np.float64), oracle.dequantize_int4(k4, scale),
                            oracle.dequantize_int4(v4, scale), P["table"], P["cu"], P["skv"], 0.25)
     assert np.array_equal(got, want)
+
+
+# ---------------------------------------------------------------- sparse (local + selected)
+
+def _sel(T, kvh, rows):
+    """selected [T, kvh, S] from per-(token, head) lists, -1 padded."""
+    S = max(1, max((len(r) for r in rows.values()), default=1))
+    a = np.full((T, kvh, S), -1, np.int32)
+    for (t, h), r in rows.items():
+        a[t, h, :len(r)] = r
+    return a
+
+
+def test_sparse_without_selections_is_the_local_window():
+    rng = np.random.default_rng(15)
+    P = _random_problem(rng, [3, 1, 5], [20, 9, 30], 4, 2, 16, 8)
+    T = int(P["cu"][-1])
+    for w in (0, 3, 100):
+        a = oracle.sparse_attention(P["query"], P["kc"], P["vc"], P["table"], P["cu"], P["skv"],
+                                    np.full((T, 2, 4), -1, np.int32), w, 0.25)
+        b = oracle.attention(P["query"], P["kc"], P["vc"], P["table"], P["cu"], P["skv"], 0.25,
+                             window=w)
+        assert np.array_equal(a, b)
+
+
+def test_sparse_selecting_every_earlier_key_is_causal_attention():
+    rng = np.random.default_rng(16)
+    P = _random_problem(rng, [2, 3], [12, 5], 4, 2, 16, 4)
+    T = int(P["cu"][-1])
+    every = np.broadcast_to(np.arange(40, dtype=np.int32), (T, 2, 40)).copy()
+    a = oracle.sparse_attention(P["query"], P["kc"], P["vc"], P["table"], P["cu"], P["skv"],
+                                every, 1, 0.25)
+    b = oracle.attention(P["query"], P["kc"], P["vc"], P["table"], P["cu"], P["skv"], 0.25)
+    assert np.array_equal(a, b)
+
+
+def test_sparse_closed_forms_and_dense_reference():
+    """Window 0 plus one selected key far back: the row averages exactly two
+    value rows with softmax weights of their two scores; a duplicate or a
+    future selection changes nothing; and a numpy dense reference with an
+    explicit mask agrees on a random selection."""
+    rng = np.random.default_rng(17)
+    q_lens, past, qh, kvh, d = [2, 1], [30, 12], 4, 2, 16
+    P = _random_problem(rng, q_lens, past, qh, kvh, d, 8)
+    T = int(P["cu"][-1])
+    sel = _sel(T, kvh, {(t, h): [3, 3, 50] for t in range(T) for h in range(kvh)})
+    got = oracle.sparse_attention(P["query"], P["kc"], P["vc"], P["table"], P["cu"], P["skv"],
+                                  sel, 0, 0.25)
+    cu = P["cu"]
+    for t in range(T):
+        b = 0 if t < cu[1] else 1
+        pos = past[b] + t - cu[b]
+        for h in range(qh):
+            k, v = P["k_seqs"][b][:, h // 2], P["v_seqs"][b][:, h // 2]
+            s = np.array([P["query"][t, h] @ k[3], P["query"][t, h] @ k[pos]]) * 0.25
+            w = np.exp(s - s.max())
+            np.testing.assert_allclose(got[t, h], (w[0] * v[3] + w[1] * v[pos]) / w.sum(), atol=1e-12)
+    # Random selections against a dense masked reference.
+    sel = rng.integers(-1, 45, size=(T, kvh, 7)).astype(np.int32)
+    got = oracle.sparse_attention(P["query"], P["kc"], P["vc"], P["table"], P["cu"], P["skv"],
+                                  sel, 2, 0.25)
+    for t in range(T):
+        b = 0 if t < cu[1] else 1
+        pos = past[b] + t - cu[b]
+        for h in range(qh):
+            keep = np.zeros(pos + 1, bool)
+            keep[max(0, pos - 2):] = True
+            for e in sel[t, h // 2]:
+                if 0 <= e <= pos:
+                    keep[e] = True
+            k = P["k_seqs"][b][:pos + 1, h // 2][keep]
+            v = P["v_seqs"][b][:pos + 1, h // 2][keep]
+            s = k @ P["query"][t, h] * 0.25
+            w = np.exp(s - s.max())
+            np.testing.assert_allclose(got[t, h], w @ v / w.sum(), atol=1e-12)
