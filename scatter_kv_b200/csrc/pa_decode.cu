@@ -521,6 +521,13 @@ decode_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ 
                 atomicExch(&sflag[1], 1);
                 break;
             }
+            if (MT > 1 && mt * 16 >= R) {
+                // This warp's 16 rows are all padding (a short q_len): release
+                // the stage without computing on it.
+                __syncwarp();
+                if (lane == 0) mbar_arrive(&empty[st]);
+                continue;
+            }
             const uint32_t kbase = smem_u32(stages + st * C::STAGE_BYTES);
             const uint32_t vbase = kbase + C::TILE_BYTES;
             const int k0 = k_begin + t * C::BN;
