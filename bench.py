@@ -261,6 +261,7 @@ KERNEL_SOURCES = {
     "scatter_kv": ("pa_scatter.cu", "pa_common.cuh", "pa_internal.h"),
     "slot_mapping": ("pa_scatter.cu", "pa_common.cuh", "pa_internal.h"),
     "qkv_rotary_scatter": ("pa_qkv.cu", "pa_common.cuh", "pa_internal.h"),
+    "sparse_local_selected": ("pa_sparse.cu", "pa_common.cuh", "pa_internal.h"),
 }
 
 
@@ -612,6 +613,79 @@ def measure_qkv_rotary(args, spec, world, dev, steps):
             "timing": "CUDA-graph replays of the one call, L2 flushed between them"}
 
 
+def measure_sparse(args, spec, world, dev, steps, num_selected=1024, window=128):
+    """Sparse paged attention (local window + selected positions) on the
+    decode-heavy batch: every (token, KV head) selects num_selected sorted
+    positions below its window.  HBM-bound: its algorithmic bytes are the
+    K/V rows of every selected and window key, read once per KV head, plus
+    Q read and O written.  Timed alone: CUDA-graph replays, L2 flushed."""
+    import torch
+    import scatter_kv_b200 as pa
+
+    x = workloads.generate(spec)
+    rng = np.random.default_rng(spec.seed)
+    T, kvh, d = spec.token_count, spec.kv_heads, spec.head_size
+    cu = x["cu_seqlens_q"]
+    sel = np.full((T, kvh, num_selected), -1, np.int32)
+    nkeys = 0
+    for b in range(spec.batch):
+        for t in range(int(cu[b]), int(cu[b + 1])):
+            P = int(spec.past[b]) + t - int(cu[b])
+            lo = max(0, P - window)
+            for h in range(kvh):
+                k = min(num_selected, lo)
+                sel[t, h, :k] = np.sort(rng.choice(lo, size=k, replace=False)) if k else []
+                nkeys += k + (P - lo + 1)
+    dd = {k: torch.from_numpy(np.ascontiguousarray(x[k])).to(dev)
+          for k in ("query", "key_cache", "value_cache", "block_table", "cu_seqlens_q", "seqlens_kv")}
+    seld = torch.from_numpy(sel).to(dev)
+    dims = pa.make_dims(batch=spec.batch, token_count=T, q_heads=spec.q_heads, kv_heads=kvh,
+                        head_size=d, num_blocks=spec.num_blocks, block_size=spec.block_size,
+                        max_blocks_per_seq=x["block_table"].shape[1])
+    out = torch.empty((T, spec.q_heads, d), dtype=torch.float16, device=dev)
+    status = torch.zeros(1, dtype=torch.int32, device=dev)
+    stream = torch.cuda.Stream(device=dev)
+    flush = torch.empty(2 * L2_BYTES // 4, dtype=torch.int32, device=dev)
+    scrub = torch.zeros(2 * L2_BYTES // 4, dtype=torch.int32, device=dev)
+    scrub_out = torch.empty((), dtype=torch.int64, device=dev)
+
+    def call():
+        pa.pa_sparse_attention(dd["query"], dd["key_cache"], dd["value_cache"], dd["block_table"],
+                               dd["cu_seqlens_q"], dd["seqlens_kv"], seld, num_selected, window,
+                               0.0, out, dims, status, stream)
+
+    with torch.cuda.stream(stream):
+        for _ in range(3):
+            call()
+        stream.synchronize()
+        if int(status.item()) != 0:
+            raise RuntimeError(f"device status {int(status.item()):#x} in sparse attention")
+        graph = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(graph, stream=stream):
+            call()
+        ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+              for _ in range(steps)]
+        barrier(world, dev)
+        torch.cuda.synchronize()
+        for k in range(steps):
+            flush.fill_(k)
+            torch.sum(scrub, 0, dtype=torch.int64, out=scrub_out)
+            ev[k][0].record(stream)
+            graph.replay()
+            ev[k][1].record(stream)
+        torch.cuda.synchronize()
+        barrier(world, dev)
+    ms = max_over_ranks(sum(a.elapsed_time(b) for a, b in ev), world, dev) / steps
+    nbytes = nkeys * d * 2 * 2 + 2 * T * spec.q_heads * d * 2
+    gbs = nbytes / (ms * 1e-3) / 1e9
+    peaks = load_peaks()
+    return {"workload": f"{spec.name}, {num_selected} selected positions + window {window} "
+                        "per (token, KV head)",
+            "us": ms * 1e3, "bytes": nbytes, "GB/s": gbs, "frac": gbs / peaks["hbm_gbs"],
+            "frac_nominal": gbs / NOMINAL_HBM_GBS, "peak_source": f"{peaks['source']} copy bandwidth",
+            "timing": "CUDA-graph replays of the one call, L2 flushed between them"}
+
+
 def run_gpu(args, spec, rank, world, local):
     import torch
 
@@ -631,6 +705,9 @@ def run_gpu(args, spec, rank, world, local):
         others["long_decode_int4"] = measure_workload(
             args, workloads.CONFIGS[workloads.CONFIG_KEYS["long_decode"]](), "long_decode_int4",
             world, dev, max(10, args.steps // 2), e2e=False, int4=True)
+        others["sparse_local_selected"] = measure_sparse(
+            args, workloads.CONFIGS[workloads.CONFIG_KEYS["decode"]](), world, dev,
+            max(10, args.steps // 2))
         others["fused_split_qkv_rotary_scatter"] = measure_qkv_rotary(
             args, workloads.CONFIGS[workloads.CONFIG_KEYS["prefill"]](), world, dev,
             max(10, args.steps // 2))

@@ -64,7 +64,9 @@ enum {
     PA_DEV_TIMEOUT        = 1 << 5,  /* a bounded in-kernel wait gave up (never expected) */
     PA_DEV_HINT_EXCEEDED  = 1 << 6,  /* a sequence is longer than max_seqlen_q_hint or
                                         max_seqlen_kv_hint */
-    PA_DEV_BAD_POSITION   = 1 << 7   /* a token's position is past the rotary caches' rows */
+    PA_DEV_BAD_POSITION   = 1 << 7,  /* a token's position is past the rotary caches' rows */
+    PA_DEV_BAD_SELECTION  = 1 << 8   /* sparse attention: selected positions not strictly
+                                        increasing, or -1 padding before a position */
 };
 
 /* Problem dimensions, all host-known.  token_count = cu_seqlens_q[batch].
@@ -270,6 +272,33 @@ pa_status pa_attention_int4(const void* query, const void* key_cache, const void
                             void* out, const pa_dims* dims, void* workspace,
                             size_t workspace_bytes, int32_t* dev_status, void* stream);
 
+/* pa_sparse_attention -- sparse paged attention, local plus selected.  The
+ * "[WebGPU] Implement SparseAttentionIndexer" follow-up ("Motivation and
+ * Context") has selections that reference request-local positions in the
+ * main paged cache, run as local-plus-selected attention; scores and
+ * softmax as in the FlexAttention doc's "FlexAttention Computation".
+ * Token t of sequence b sits at position P = seqlens_kv[b] - q_len_b + i.
+ * For KV head h it attends to keys [max(0, P - local_window), P] and to the
+ * positions selected[t][h][0 .. num_selected) that are >= 0 and <= P; a
+ * key counts once.  The query heads of KV head h's group share its
+ * selection.
+ *   query, key_cache, value_cache, block_table, cu_seqlens_q, seqlens_kv,
+ *          scale, out: as for pa_attention (out written for every token).
+ *   selected: [token_count, kv_heads, num_selected] int32 device array
+ *          (may be NULL when num_selected is 0).  Its non-negative entries
+ *          must be strictly increasing, with -1 padding only after them;
+ *          otherwise the token's rows are zero and PA_DEV_BAD_SELECTION is
+ *          set.
+ *   local_window: >= 0 (0: the token's own key only).
+ * num_selected + local_window + 1 may not exceed 8192, and head sizes 16,
+ * 32, 64 and 128 are built (PA_ERR_NOT_IMPLEMENTED otherwise); the dims'
+ * softcap and local window must be off.  No workspace. */
+pa_status pa_sparse_attention(const void* query, const void* key_cache, const void* value_cache,
+                              const int32_t* block_table, const int32_t* cu_seqlens_q,
+                              const int32_t* seqlens_kv, const int32_t* selected,
+                              int32_t num_selected, int32_t local_window, float scale, void* out,
+                              const pa_dims* dims, int32_t* dev_status, void* stream);
+
 /* pa_get_status -- synchronise `stream` and copy *dev_status to *host_code.
  * For tests and debugging; it blocks the host. */
 pa_status pa_get_status(const int32_t* dev_status, int32_t* host_code, void* stream);
@@ -299,7 +328,8 @@ enum {
     PA_KERNEL_COMBINE = 3,
     PA_KERNEL_PREFILL = 4,
     PA_KERNEL_QKV_ROTARY = 5,
-    PA_KERNEL_COUNT = 6
+    PA_KERNEL_SPARSE = 6,
+    PA_KERNEL_COUNT = 7
 };
 
 pa_status pa_trace_enable(int on);

@@ -38,6 +38,7 @@ PA_DEV_BAD_SLOT = 1 << 4
 PA_DEV_TIMEOUT = 1 << 5
 PA_DEV_HINT_EXCEEDED = 1 << 6
 PA_DEV_BAD_POSITION = 1 << 7
+PA_DEV_BAD_SELECTION = 1 << 8
 
 PA_KERNEL_SCATTER = 0
 PA_KERNEL_SLOT_MAPPING = 1
@@ -45,6 +46,7 @@ PA_KERNEL_DECODE = 2
 PA_KERNEL_COMBINE = 3
 PA_KERNEL_PREFILL = 4
 PA_KERNEL_QKV_ROTARY = 5
+PA_KERNEL_SPARSE = 6
 PA_TRACE_CAPACITY = 4096
 
 
@@ -90,7 +92,7 @@ EXPORTS = [
     "pa_scatter_kv", "pa_compute_slot_mapping", "pa_attention_workspace_size", "pa_attention",
     "pa_get_status", "pa_status_string", "pa_last_error", "pa_trace_enable", "pa_trace_read",
     "pa_kernel_name", "pa_attention_noalloc", "pa_split_qkv_rotary_scatter",
-    "pa_scatter_kv_int4", "pa_attention_int4",
+    "pa_scatter_kv_int4", "pa_attention_int4", "pa_sparse_attention",
 ]
 
 # Bytes of the fixed scratch array behind pa_attention_noalloc.
@@ -124,6 +126,9 @@ def _load():
     lib.pa_attention_int4.argtypes = [P, P, P, P, P, P, P, P, ctypes.c_float, P, D, P,
                                       ctypes.c_size_t, P, P]
     lib.pa_attention_int4.restype = ctypes.c_int
+    lib.pa_sparse_attention.argtypes = [P, P, P, P, P, P, P, ctypes.c_int32, ctypes.c_int32,
+                                        ctypes.c_float, P, D, P, P]
+    lib.pa_sparse_attention.restype = ctypes.c_int
     lib.pa_get_status.argtypes = [P, I32P, P]
     lib.pa_get_status.restype = ctypes.c_int
     lib.pa_status_string.argtypes = [ctypes.c_int]
@@ -279,6 +284,16 @@ def pa_attention_int4(query, key_cache, value_cache, k_scale, v_scale, block_tab
                                  _ptr(seqlens_kv), float(scale), _ptr(out), ctypes.byref(dims),
                                  _ptr(workspace), int(workspace_bytes), _ptr(dev_status),
                                  _stream(stream)))
+
+
+def pa_sparse_attention(query, key_cache, value_cache, block_table, cu_seqlens_q, seqlens_kv,
+                        selected, num_selected, local_window, scale, out, dims: pa_dims,
+                        dev_status=None, stream=None) -> None:
+    _check(lib.pa_sparse_attention(_ptr(query), _ptr(key_cache), _ptr(value_cache),
+                                   _ptr(block_table), _ptr(cu_seqlens_q), _ptr(seqlens_kv),
+                                   _ptr(selected), int(num_selected), int(local_window),
+                                   float(scale), _ptr(out), ctypes.byref(dims), _ptr(dev_status),
+                                   _stream(stream)))
 
 
 def packed_qkv_views(qkv, dims: pa_dims):

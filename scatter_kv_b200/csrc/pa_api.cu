@@ -613,6 +613,69 @@ pa_status pa_attention_int4(const void* query, const void* key_cache, const void
     return PA_OK;
 }
 
+pa_status pa_sparse_attention(const void* query, const void* key_cache, const void* value_cache,
+                              const int32_t* block_table, const int32_t* cu_seqlens_q,
+                              const int32_t* seqlens_kv, const int32_t* selected,
+                              int32_t num_selected, int32_t local_window, float scale, void* out,
+                              const pa_dims* dims, int32_t* dev_status, void* stream) {
+    g_last_error[0] = 0;
+    pa_status st = check_dims(dims);
+    if (st != PA_OK) return st;
+    const pa_dims& d = *dims;
+    if (d.head_size != 16 && d.head_size != 32 && d.head_size != 64 && d.head_size != 128)
+        return fail(PA_ERR_NOT_IMPLEMENTED, "sparse attention: head sizes 16, 32, 64, 128 are built");
+    if (d.softcap > 0.f || d.local_window)
+        return fail(PA_ERR_NOT_IMPLEMENTED,
+                    "sparse attention takes its window as an argument; no softcap or dims window");
+    if (num_selected < 0 || local_window < 0)
+        return fail(PA_ERR_INVALID_ARGUMENT, "num_selected and local_window must be >= 0");
+    if ((long long)num_selected + local_window + 1 > pa::kSparseMaxKeys)
+        return fail(PA_ERR_NOT_IMPLEMENTED,
+                    "sparse attention: num_selected + local_window + 1 = %lld keys, more than %d",
+                    (long long)num_selected + local_window + 1, pa::kSparseMaxKeys);
+    if (d.token_count == 0) return PA_OK;
+    if (d.batch == 0) return fail(PA_ERR_INVALID_ARGUMENT, "token_count > 0 with batch 0");
+    if (d.kv_heads > 65535) return fail(PA_ERR_NOT_IMPLEMENTED, "kv_heads > 65535");
+    if (!(scale >= 0.f) || isinf(scale))
+        return fail(PA_ERR_INVALID_ARGUMENT, "scale must be finite and >= 0");
+    PA_REQUIRE_PTR(query);
+    PA_REQUIRE_PTR(key_cache);
+    PA_REQUIRE_PTR(value_cache);
+    PA_REQUIRE_PTR(out);
+    PA_REQUIRE_IPTR(block_table);
+    PA_REQUIRE_IPTR(cu_seqlens_q);
+    PA_REQUIRE_IPTR(seqlens_kv);
+    if (num_selected > 0) PA_REQUIRE_IPTR(selected);
+    if (scale == 0.f) scale = 1.f / sqrtf((float)d.head_size);
+    pa::SparseParams p{};
+    p.query = static_cast<const uint16_t*>(query);
+    p.key_cache = static_cast<const uint16_t*>(key_cache);
+    p.value_cache = static_cast<const uint16_t*>(value_cache);
+    p.out = static_cast<uint16_t*>(out);
+    p.block_table = block_table;
+    p.cu_seqlens_q = cu_seqlens_q;
+    p.seqlens_kv = seqlens_kv;
+    p.selected = selected;
+    p.status = dev_status;
+    p.token_count = d.token_count;
+    p.num_blocks = d.num_blocks;
+    p.batch = d.batch;
+    p.q_heads = d.q_heads;
+    p.kv_heads = d.kv_heads;
+    p.group = d.q_heads / d.kv_heads;
+    p.head_size = d.head_size;
+    p.block_size = d.block_size;
+    p.max_blocks = d.max_blocks_per_seq;
+    p.kv_cap = d.max_blocks_per_seq * d.block_size;
+    p.num_selected = num_selected;
+    p.local_window = local_window;
+    p.scale_log2 = scale * 1.4426950408889634f;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    TraceScope tr(PA_KERNEL_SPARSE, s);
+    cudaError_t e = pa::launch_sparse(p, d.dtype == PA_DTYPE_BF16, s);
+    return e == cudaSuccess ? PA_OK : cuda_fail(e, "sparse attention launch");
+}
+
 pa_status pa_get_status(const int32_t* dev_status, int32_t* host_code, void* stream) {
     g_last_error[0] = 0;
     if (dev_status == nullptr || host_code == nullptr)
@@ -664,6 +727,7 @@ const char* pa_kernel_name(int32_t kernel) {
         case PA_KERNEL_COMBINE: return "decode_combine";
         case PA_KERNEL_PREFILL: return "prefill_tcgen05";
         case PA_KERNEL_QKV_ROTARY: return "qkv_rotary_scatter";
+        case PA_KERNEL_SPARSE: return "sparse_local_selected";
     }
     return "unknown";
 }

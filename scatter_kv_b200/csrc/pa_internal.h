@@ -136,6 +136,35 @@ struct QkvParams {
 cudaError_t launch_qkv_rotary_scatter(const QkvParams& p, bool bf16, cudaStream_t stream,
                                       int num_sms);
 
+// Sparse paged attention (local plus selected), one CTA per (KV head, token).
+constexpr int kSparseMaxKeys = 8192;  // keys one (token, KV head) may see: selections + window
+struct SparseParams {
+    const uint16_t* query;        // [token_count, q_heads, head_size]
+    const uint16_t* key_cache;    // [num_blocks, block_size, kv_heads, head_size]
+    const uint16_t* value_cache;
+    uint16_t* out;
+    const int32_t* block_table;
+    const int32_t* cu_seqlens_q;
+    const int32_t* seqlens_kv;
+    const int32_t* selected;      // [token_count, kv_heads, num_selected]
+    int32_t* status;
+    long long token_count;
+    long long num_blocks;
+    int batch;
+    int q_heads;
+    int kv_heads;
+    int group;
+    int head_size;
+    int block_size;
+    int max_blocks;
+    int kv_cap;
+    int num_selected;
+    int local_window;
+    float scale_log2;
+};
+
+cudaError_t launch_sparse(const SparseParams& p, bool bf16, cudaStream_t stream);
+
 struct DecodePlan {
     int decode_max_q;
     int mtiles;                   // 1 or 2 (16 query rows each)
