@@ -165,7 +165,8 @@ sparse_kernel(const SparseParams p) {
     __syncthreads();
     if (b < 0 || sh[3] != 0) {
         // Invalid metadata, selection or block id: this token's rows are zero.
-        if (b >= 0 && kvh == 0 && threadIdx.x == 0)
+        // Selections are per (token, KV head): every CTA reports its own.
+        if (b >= 0 && threadIdx.x == 0)
             flag_status(p.status, (sh[3] & 1) ? PA_DEV_BAD_SELECTION : PA_DEV_BAD_BLOCK);
         const int per_row = p.head_size / 8;
         for (int i = threadIdx.x; i < R * per_row; i += C::THREADS) {
