@@ -268,9 +268,6 @@ pa_status pa_attention(const void* query, const void* key_cache, const void* val
     pa_status st = check_dims(dims);
     if (st != PA_OK) return st;
     const pa_dims& d = *dims;
-    if (d.head_size > 128)
-        return fail(PA_ERR_NOT_IMPLEMENTED, "attention with head_size %d: sizes up to 128 are built",
-                    d.head_size);
     if (d.token_count == 0) return PA_OK;
     if (d.batch == 0) return fail(PA_ERR_INVALID_ARGUMENT, "token_count > 0 with batch 0");
     if (!(scale >= 0.f) || isinf(scale))
@@ -356,9 +353,11 @@ pa_status pa_attention(const void* query, const void* key_cache, const void* val
 
     // Prefill part: sequences with q_len > prefill_min_q.
     if (d.max_seqlen_q_hint == 0 || d.max_seqlen_q_hint > prefill_min_q) {
-        // Query-tile pairs: 2 * (128 / group) tokens each; every prefill
-        // sequence adds at most one partly filled pair.
-        const long long pair_tokens = 2 * (pa::kPrefillRows / g);
+        // Work items: query-tile pairs of 2 * (128 / group) tokens (one tile of
+        // 128 / group tokens at head size 256); every prefill sequence adds at
+        // most one partly filled item.
+        const bool wide = head > 128;
+        const long long pair_tokens = (wide ? 1 : 2) * (pa::kPrefillRows / g);
         const long long longer = d.token_count / (prefill_min_q + 1);
         const long long slots = (d.token_count + pair_tokens - 1) / pair_tokens +
                                 (longer < d.batch ? longer : d.batch);
@@ -366,7 +365,8 @@ pa_status pa_attention(const void* query, const void* key_cache, const void* val
             if (slots * d.kv_heads >= (1ll << 31))
                 return fail(PA_ERR_NOT_IMPLEMENTED, "too many query tiles (%lld)", slots);
             CUtensorMap tq, tk, tv;
-            const int rows = d.block_size < pa::kPrefillKeys ? d.block_size : pa::kPrefillKeys;
+            const int keys = wide ? pa::kPrefill256Keys : pa::kPrefillKeys;
+            const int rows = d.block_size < keys ? d.block_size : keys;
             if ((st = make_query_map(&tq, query, d)) != PA_OK) return st;
             if ((st = make_cache_map(&tk, key_cache, d, rows)) != PA_OK) return st;
             if ((st = make_cache_map(&tv, value_cache, d, rows)) != PA_OK) return st;
@@ -394,7 +394,8 @@ pa_status pa_attention(const void* query, const void* key_cache, const void* val
             p.num_slots = (int)slots;
             p.mods = mods;
             TraceScope tr(PA_KERNEL_PREFILL, s);
-            cudaError_t e = pa::launch_prefill(tq, tk, tv, p, head, bf16, s);
+            cudaError_t e = wide ? pa::launch_prefill256(tq, tk, tv, p, bf16, s)
+                                 : pa::launch_prefill(tq, tk, tv, p, head, bf16, s);
             if (e != cudaSuccess) return cuda_fail(e, "prefill launch");
         }
     }

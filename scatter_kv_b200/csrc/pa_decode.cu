@@ -55,6 +55,24 @@ constexpr int kDecodeLaunchRegs = 80;
 constexpr int kDecRegsCons = 136, kDecRegsProd = 24;
 static_assert(128 * (kDecRegsCons + kDecRegsProd) == 256 * kDecodeLaunchRegs,
               "register split must equal the launch budget");
+// Head size 256 holds twice the Q fragments and O accumulators: one CTA per
+// SM (its 4 stages take 128 KB), launched with 128 registers a thread, the
+// consumers raised to 232.
+constexpr int kDec256LaunchRegs = 128;
+constexpr int kDec256RegsCons = 232, kDec256RegsProd = 24;
+static_assert(128 * (kDec256RegsCons + kDec256RegsProd) == 256 * kDec256LaunchRegs,
+              "register split must equal the launch budget");
+
+template <int HEAD>
+__host__ __device__ constexpr int dec_launch_regs() { return HEAD > 128 ? kDec256LaunchRegs : kDecodeLaunchRegs; }
+template <int HEAD>
+__host__ __device__ constexpr int dec_regs_cons() { return HEAD > 128 ? kDec256RegsCons : kDecRegsCons; }
+template <int HEAD>
+__host__ __device__ constexpr int dec_regs_prod() { return HEAD > 128 ? kDec256RegsProd : kDecRegsProd; }
+template <int HEAD, bool CPA, bool Q4>
+__host__ __device__ constexpr int dec_ctas_per_sm() {
+    return Q4 ? 2 : HEAD > 128 ? (CPA ? 2 : 1) : ((HEAD >= 128 && !CPA) ? 2 : 3);
+}
 // INT4 pages: two CTAs per SM at 128 registers; the consumers take 168, the
 // producers (which hold four tiles of loads in registers) 88.
 constexpr int kQ4LaunchRegs = 128;
@@ -164,8 +182,7 @@ __device__ __forceinline__ uint4 ld_nc16(const void* p) {
 }
 
 template <int HEAD, int MT, bool CPA, typename ET, bool GEN, bool Q4 = false>
-__global__ void __launch_bounds__(Cfg<HEAD, MT, CPA>::THREADS,
-                                  Q4 ? 2 : ((HEAD >= 128 && !CPA) ? 2 : 3))
+__global__ void __launch_bounds__(Cfg<HEAD, MT, CPA>::THREADS, (dec_ctas_per_sm<HEAD, CPA, Q4>()))
 decode_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_v,
               const DecodeParams p) {
     using C = Cfg<HEAD, MT, CPA>;
@@ -268,7 +285,7 @@ decode_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ 
     if (warp >= C::NCW) {
         // ------------------------------------------------------------ producers
         if (Q4) asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(kQ4RegsProd));
-        else if (CPA) asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(kDecRegsProd));
+        else if (CPA) asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(dec_regs_prod<HEAD>()));
         const int pw = warp - C::NCW;
         // The split's block ids, fetched once by the first producer warp, so
         // issuing a tile never waits on a dependent global load.  They are
@@ -451,7 +468,7 @@ decode_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ 
     } else {
         // ------------------------------------------------------------ consumers
         if (Q4) asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(kQ4RegsCons));
-        else if (CPA) asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(kDecRegsCons));
+        else if (CPA) asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(dec_regs_cons<HEAD>()));
         const int mt = warp % MT;          // which 16 query rows
         const int grp = warp / MT;         // which tiles
         const int quad = lane >> 2, qid = lane & 3;
@@ -759,24 +776,33 @@ __global__ void __launch_bounds__(128) combine_kernel(const DecodeParams p) {
     for (int sp = lane + 32; sp < n_splits; sp += 32) L += fast_exp2(lse[(long long)sp * p.rmax] - M);
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) L += __shfl_xor_sync(0xffffffffu, L, o);
+    // Column groups of 128 (one for head sizes up to 128, two for 256).
+    constexpr int NCG = HEAD > 128 ? HEAD / 128 : 1;
     const float* po = p.part_o + base * HEAD + lane * 4;
-    float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
-    const bool active = lane * 4 < hs;
+    float4 acc[NCG];
+#pragma unroll
+    for (int cg = 0; cg < NCG; ++cg) acc[cg] = make_float4(0.f, 0.f, 0.f, 0.f);
 #pragma unroll 4
     for (int sp = 0; sp < n_splits; ++sp) {
         const float w = sp < 32 ? __shfl_sync(0xffffffffu, w_l, sp)
                                 : fast_exp2(lse[(long long)sp * p.rmax] - M);
-        if (active) {
-            const float4 v = *reinterpret_cast<const float4*>(po + (long long)sp * p.rmax * HEAD);
-            acc.x += w * v.x; acc.y += w * v.y; acc.z += w * v.z; acc.w += w * v.w;
+#pragma unroll
+        for (int cg = 0; cg < NCG; ++cg) {
+            if (cg * 128 + lane * 4 < hs) {
+                const float4 v = *reinterpret_cast<const float4*>(po + (long long)sp * p.rmax * HEAD + cg * 128);
+                acc[cg].x += w * v.x; acc[cg].y += w * v.y; acc[cg].z += w * v.z; acc[cg].w += w * v.w;
+            }
         }
     }
-    if (!active) return;
     const float il = 1.f / L;
-    uint2 wv;
-    wv.x = E::pack2(acc.x * il, acc.y * il);
-    wv.y = E::pack2(acc.z * il, acc.w * il);
-    *reinterpret_cast<uint2*>(orow + lane * 4) = wv;
+#pragma unroll
+    for (int cg = 0; cg < NCG; ++cg) {
+        if (cg * 128 + lane * 4 >= hs) continue;
+        uint2 wv;
+        wv.x = E::pack2(acc[cg].x * il, acc[cg].y * il);
+        wv.y = E::pack2(acc[cg].z * il, acc[cg].w * il);
+        *reinterpret_cast<uint2*>(orow + cg * 128 + lane * 4) = wv;
+    }
 }
 
 template <int HEAD, int MT, bool CPA, typename ET, bool GEN, bool Q4 = false>
@@ -790,7 +816,7 @@ cudaError_t launch_decode_t(const CUtensorMap& tm_k, const CUtensorMap& tm_v,
         cudaFuncAttributes fa;
         e = cudaFuncGetAttributes(&fa, kern);
         if (e != cudaSuccess) return e;
-        if (fa.numRegs != (Q4 ? kQ4LaunchRegs : kDecodeLaunchRegs)) return cudaErrorInvalidKernelImage;
+        if (fa.numRegs != (Q4 ? kQ4LaunchRegs : dec_launch_regs<HEAD>())) return cudaErrorInvalidKernelImage;
     }
     e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM);
     if (e != cudaSuccess) return e;
@@ -827,6 +853,7 @@ cudaError_t launch_decode_d(const CUtensorMap& tm_k, const CUtensorMap& tm_v, co
         case 32: return launch_decode_h<32, ET, GEN>(tm_k, tm_v, p, mtiles, stream);
         case 64: return launch_decode_h<64, ET, GEN>(tm_k, tm_v, p, mtiles, stream);
         case 128: return launch_decode_h<128, ET, GEN>(tm_k, tm_v, p, mtiles, stream);
+        case 256: return launch_decode_h<256, ET, GEN>(tm_k, tm_v, p, mtiles, stream);
         default: return cudaErrorInvalidValue;
     }
 }
@@ -869,7 +896,8 @@ DecodePlan plan_decode(const pa_dims& d, int num_sms) {
 }
 
 int padded_head(int head_size) {
-    return head_size <= 16 ? 16 : head_size <= 32 ? 32 : head_size <= 64 ? 64 : 128;
+    return head_size <= 16 ? 16 : head_size <= 32 ? 32 : head_size <= 64 ? 64
+         : head_size <= 128 ? 128 : 256;
 }
 
 cudaError_t launch_decode(const CUtensorMap& tm_k, const CUtensorMap& tm_v,
@@ -907,6 +935,7 @@ cudaError_t launch_combine_t(const DecodeParams& p, int head, cudaStream_t strea
         case 32: return launch_pdl(combine_kernel<32, ET>, grid, dim3(128), 0, stream, p);
         case 64: return launch_pdl(combine_kernel<64, ET>, grid, dim3(128), 0, stream, p);
         case 128: return launch_pdl(combine_kernel<128, ET>, grid, dim3(128), 0, stream, p);
+        case 256: return launch_pdl(combine_kernel<256, ET>, grid, dim3(128), 0, stream, p);
         default: return cudaErrorInvalidValue;
     }
 }

@@ -218,5 +218,12 @@ constexpr int kPrefillKeys = 128;
 constexpr int kPrefillRows = 128;      // query rows per tensor-core tile
 constexpr int kPrefillCtaRows = 256;   // query rows per prefill CTA (two tiles)
 constexpr int kPrefillLaunchRegs = 168; // registers per thread of the 384-thread prefill CTA
+constexpr int kPrefill256Keys = 64;    // keys per tile of the head-size-256 prefill kernel
+
+// Prefill for head sizes 136 .. 256 (padded to 256): one 128-row query tile
+// per CTA; cache tensor maps with boxes of min(block_size, kPrefill256Keys) rows.
+cudaError_t launch_prefill256(const CUtensorMap& tm_q, const CUtensorMap& tm_k,
+                              const CUtensorMap& tm_v, const PrefillParams& p, bool bf16,
+                              cudaStream_t stream);
 
 }  // namespace pa

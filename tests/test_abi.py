@@ -55,7 +55,6 @@ FAKE = 1 << 20          # aligned non-null address; never dereferenced (calls fa
     (dict(q_heads=48, kv_heads=1), 2),           # group 48: not built (decode rows <= 32)
     (dict(head_size=20), 1),                     # not a multiple of 8
     (dict(head_size=264), 1),                    # beyond 256
-    (dict(head_size=192), 2),                    # valid, attention not built past 128
     (dict(softcap=-1.0), 1),
     (dict(window=-2), 1),
     (dict(block_size=24), 1),
