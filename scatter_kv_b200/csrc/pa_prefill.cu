@@ -457,6 +457,23 @@ prefill_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
         const int lbs = 31 - __clz(bs);
         const long long row_bytes = (long long)p.kv_heads * hs * 2;
         const long long colb = (long long)kvh * hs * 2 + jc * 16;
+        // Whole tiles (every key below T) go by 16-row units instead: unit v
+        // holds tile rows 16 v .. 16 v + 15, all in one page (pages hold 16 or
+        // more keys), and goes to producer warp v % NPROD.  Lane l copies
+        // chunk l % CPR of unit rows l / CPR + k * URPL: its shared-memory
+        // offsets are the same in every unit (the swizzle repeats every 8
+        // rows), so a copy costs one address add.
+        constexpr int URPL = C::CPR < 32 ? 32 / C::CPR : 1;     // unit rows per warp pass
+        constexpr int UPL = 16 / URPL;                           // copies per lane per unit
+        const int ucj = lane % C::CPR;
+        const bool ucol_ok = ucj * 8 < hs;
+        uint32_t usoff[UPL];
+#pragma unroll
+        for (int k = 0; k < UPL; ++k)
+            usoff[k] = swz<C::RB>((uint32_t)((((ucj * 8) / C::A) * C::BN + lane / C::CPR + k * URPL) * C::RB +
+                                             (ucj % (C::A / 8)) * 16));
+        const long long ucolb = (long long)kvh * hs * 2 + ucj * 16 + (long long)(lane / C::CPR) * row_bytes;
+        const long long ustep = (long long)URPL * row_bytes;
         int tile_ids = 0;
         int next_ids = 0;
         if (CPA) {
@@ -495,6 +512,20 @@ prefill_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
                 }
                 const char* cache = reinterpret_cast<const char*>(is_v ? p.value_cache : p.key_cache);
                 const uint32_t sdst = smem_u32(dst);
+                if (k0 + C::BN <= T) {
+#pragma unroll 1
+                    for (int v = pw; v < C::BN / 16; v += C::NPROD) {
+                        const int blk = __shfl_sync(0xffffffffu, tile_ids, (16 * v) >> lbs);
+                        const char* src = cache + (((long long)blk << lbs) + ((16 * v) & (bs - 1))) * row_bytes + ucolb;
+                        const uint32_t sv = sdst + (uint32_t)(v * 16 * C::RB);
+                        if (ucol_ok) {
+#pragma unroll
+                            for (int k = 0; k < UPL; ++k) cp_async16(sv + usoff[k], src + k * ustep);
+                        }
+                    }
+                    cp_async_arrive(&full[st]);
+                    continue;
+                }
 #pragma unroll 2
                 for (int i = 0; i < (C::BN + C::RPI - 1) / C::RPI; ++i) {
                     const int r = r0 + i * C::RPI;

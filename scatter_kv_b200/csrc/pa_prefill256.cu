@@ -306,6 +306,33 @@ prefill256_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
         const bool col_ok = jc * 8 < hs;
         const long long row_bytes = (long long)p.kv_heads * hs * 2;
         const long long colb = (long long)kvh * hs * 2 + jc * 16;
+        // cp.async path, whole tiles (every key below T): 16-row units, unit v
+        // (tile rows 16 v .. 16 v + 15, one page) to producer warp v % NPROD;
+        // lane l copies chunk l of the 16 rows, at the same swizzled offsets
+        // in every unit.  Block ids come from 32-page windows in registers
+        // (lane i holds page base + i), the next one fetched a window ahead;
+        // the previous window stays for the V tiles, which trail the K tiles
+        // by two tiles.
+        const int ucj = lane;
+        const bool ucol_ok = ucj * 8 < hs;
+        const uint32_t usoff0 = (uint32_t)((((ucj * 8) / C::A) * C::BN) * C::RB + (ucj % (C::A / 8)) * 16);
+        const long long ucolb = (long long)kvh * hs * 2 + ucj * 16;
+        const int npages = (T + bs - 1) / bs;
+        int wb = (kbase >> lbs) & ~31;
+        int w_prev = 0;
+        int w_cur = (CPA && wb + lane < npages) ? bt[wb + lane] : 0;
+        int w_next = (CPA && wb + 32 + lane < npages) ? bt[wb + 32 + lane] : 0;
+        auto page_id = [&](int page) -> int {          // warp-uniform; page >= wb - 32
+            while (page >= wb + 32) {
+                wb += 32;
+                w_prev = w_cur;
+                w_cur = w_next;
+                w_next = wb + 32 + lane < npages ? bt[wb + 32 + lane] : 0;
+            }
+            const int a = __shfl_sync(0xffffffffu, w_cur, (page - wb) & 31);
+            const int c = __shfl_sync(0xffffffffu, w_prev, (page - wb) & 31);
+            return page >= wb ? a : c;
+        };
         for (int u = 0; u < nitems; ++u) {
             int j;
             bool is_v;
@@ -327,11 +354,27 @@ prefill256_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
             if (__shfl_sync(0xffffffffu, *(volatile int*)&sh[3], 0)) break;
             uint8_t* dst = ring + st * C::KV_BYTES;
             if (CPA) {
-                // Pages of 16 or 32 keys: lane l holds the block id of page k0 / bs + l.
-                const int npg = (min(k0 + C::BN, T) - k0 + bs - 1) / bs;
-                const int ids = lane < npg ? bt[(k0 >> lbs) + lane] : 0;
                 const char* cache = reinterpret_cast<const char*>(is_v ? p.value_cache : p.key_cache);
                 const uint32_t sdst = smem_u32(dst);
+                if (k0 + C::BN <= T) {
+#pragma unroll 1
+                    for (int v = pw; v < C::BN / 16; v += C::NPROD) {
+                        const int blk = page_id((k0 + 16 * v) >> lbs);
+                        const char* src = cache + (((long long)blk << lbs) + ((k0 + 16 * v) & (bs - 1))) * row_bytes + ucolb;
+                        const uint32_t sv = sdst + (uint32_t)(v * 16 * C::RB);
+                        if (ucol_ok) {
+#pragma unroll
+                            for (int k = 0; k < 16; ++k)
+                                cp_async16(sv + swz<C::RB>(usoff0 + (uint32_t)(k * C::RB)), src + k * row_bytes);
+                        }
+                    }
+                    cp_async_arrive(&full[st]);
+                    continue;
+                }
+                // The tile holding T: row by row, lane l holding the block id
+                // of page k0 / bs + l.
+                const int npg = (min(k0 + C::BN, T) - k0 + bs - 1) / bs;
+                const int ids = lane < npg ? bt[(k0 >> lbs) + lane] : 0;
 #pragma unroll 2
                 for (int i = 0; i < (C::BN + C::RPI - 1) / C::RPI; ++i) {
                     const int r = r0 + i * C::RPI;
