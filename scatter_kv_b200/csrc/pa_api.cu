@@ -259,12 +259,70 @@ pa_status pa_attention_workspace_size(const pa_dims* dims, size_t* bytes) {
     return PA_OK;
 }
 
-pa_status pa_attention(const void* query, const void* key_cache, const void* value_cache,
-                       const int32_t* block_table, const int32_t* cu_seqlens_q,
-                       const int32_t* seqlens_kv, float scale, void* out, const pa_dims* dims,
-                       void* workspace, size_t workspace_bytes, int32_t* dev_status,
-                       void* stream) {
-    g_last_error[0] = 0;
+}  // extern "C"
+
+namespace {
+
+// ------------------------------------------------------------------ side stream
+
+// Side stream for the decode part of a batch that also has prefill work.  The
+// two parts write disjoint rows of `out` and only read the caches, so they
+// may run at the same time: the split-KV decode CTAs (HBM-bound, small) then
+// fill SMs that the prefill kernel (tensor-bound, one CTA per SM) leaves
+// idle, and the combine runs beside the prefill.  The side stream forks from
+// the caller's stream with an event and joins it again before the call
+// returns, so the caller sees one stream; the fork-join pattern is valid
+// under stream capture.  One per device and CUDA context, created on first
+// use (never during a capture: until created, calls run both parts on the
+// caller's stream).  The lock is held from fork to join so that concurrent
+// callers pair their own records and waits.
+struct SideStream {
+    std::mutex mu;
+    CUcontext ctx = nullptr;
+    cudaStream_t stream = nullptr;
+    cudaEvent_t fork = nullptr;
+    cudaEvent_t join = nullptr;
+};
+SideStream g_side[pa::kMaxDevices];
+
+SideStream* side_stream_for(cudaStream_t user, std::unique_lock<std::mutex>& lock) {
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= pa::kMaxDevices) return nullptr;
+    SideStream& ss = g_side[dev];
+    lock = std::unique_lock<std::mutex>(ss.mu);
+    const CUcontext ctx = pa::current_context();
+    if (ctx == nullptr) return nullptr;
+    if (ss.ctx != ctx) {
+        // First use on this device, or its context was reset (the old
+        // handles died with it).
+        cudaStreamCaptureStatus cs = cudaStreamCaptureStatusNone;
+        if (cudaStreamIsCapturing(user, &cs) != cudaSuccess || cs != cudaStreamCaptureStatusNone) {
+            cudaGetLastError();
+            return nullptr;
+        }
+        cudaStream_t st = nullptr;
+        cudaEvent_t ef = nullptr, ej = nullptr;
+        if (cudaStreamCreateWithFlags(&st, cudaStreamNonBlocking) != cudaSuccess ||
+            cudaEventCreateWithFlags(&ef, cudaEventDisableTiming) != cudaSuccess ||
+            cudaEventCreateWithFlags(&ej, cudaEventDisableTiming) != cudaSuccess) {
+            cudaGetLastError();
+            if (ef) cudaEventDestroy(ef);
+            if (st) cudaStreamDestroy(st);
+            return nullptr;
+        }
+        ss.stream = st;
+        ss.fork = ef;
+        ss.join = ej;
+        ss.ctx = ctx;
+    }
+    return &ss;
+}
+
+pa_status attention_impl(const void* query, const void* key_cache, const void* value_cache,
+                         const int32_t* block_table, const int32_t* cu_seqlens_q,
+                         const int32_t* seqlens_kv, float scale, void* out, const pa_dims* dims,
+                         void* workspace, size_t workspace_bytes, int32_t* dev_status,
+                         void* stream, bool allow_fork) {
     pa_status st = check_dims(dims);
     if (st != PA_OK) return st;
     const pa_dims& d = *dims;
@@ -304,7 +362,9 @@ pa_status pa_attention(const void* query, const void* key_cache, const void* val
     // prefill kernel instead (it handles any q_len), and no decode runs.
     const bool run_decode = d.min_seqlen_q_hint <= plan.decode_max_q;
     const int prefill_min_q = run_decode ? plan.decode_max_q : 0;   // prefill takes q_len > this
-    if (run_decode) {
+    const bool run_prefill = d.max_seqlen_q_hint == 0 || d.max_seqlen_q_hint > prefill_min_q;
+    auto decode_part = [&](cudaStream_t s) -> pa_status {
+        pa_status st = PA_OK;
         CUtensorMap tk, tv;
         const int rows = d.block_size < pa::kDecodeKeys ? d.block_size : pa::kDecodeKeys;
         if ((st = make_cache_map(&tk, key_cache, d, rows)) != PA_OK) return st;
@@ -349,10 +409,12 @@ pa_status pa_attention(const void* query, const void* key_cache, const void* val
             cudaError_t e = pa::launch_combine(p, head, bf16, s);
             if (e != cudaSuccess) return cuda_fail(e, "combine launch");
         }
-    }
+        return PA_OK;
+    };
 
     // Prefill part: sequences with q_len > prefill_min_q.
-    if (d.max_seqlen_q_hint == 0 || d.max_seqlen_q_hint > prefill_min_q) {
+    auto prefill_part = [&](cudaStream_t s) -> pa_status {
+        pa_status st = PA_OK;
         // Work items: query-tile pairs of 2 * (128 / group) tokens (one tile of
         // 128 / group tokens at head size 256); every prefill sequence adds at
         // most one partly filled item.
@@ -398,8 +460,42 @@ pa_status pa_attention(const void* query, const void* key_cache, const void* val
                                  : pa::launch_prefill(tq, tk, tv, p, head, bf16, s);
             if (e != cudaSuccess) return cuda_fail(e, "prefill launch");
         }
+        return PA_OK;
+    };
+
+    std::unique_lock<std::mutex> side_lock;
+    SideStream* side = (allow_fork && run_decode && run_prefill) ? side_stream_for(s, side_lock) : nullptr;
+    if (side == nullptr) {
+        if (run_decode && (st = decode_part(s)) != PA_OK) return st;
+        return run_prefill ? prefill_part(s) : PA_OK;
     }
-    return PA_OK;
+    cudaError_t e = cudaEventRecord(side->fork, s);
+    if (e == cudaSuccess) e = cudaStreamWaitEvent(side->stream, side->fork, 0);
+    if (e != cudaSuccess) return cuda_fail(e, "fork to the side stream");
+    const pa_status st_dec = decode_part(side->stream);
+    // The join is enqueued whatever happened above, so that the caller's
+    // stream (or capture) never holds an open fork.
+    pa_status st_pre = PA_OK;
+    e = cudaEventRecord(side->join, side->stream);
+    if (e == cudaSuccess && st_dec == PA_OK) st_pre = prefill_part(s);
+    const cudaError_t ej = e == cudaSuccess ? cudaStreamWaitEvent(s, side->join, 0) : e;
+    if (st_dec != PA_OK) return st_dec;
+    if (ej != cudaSuccess) return cuda_fail(ej, "join of the side stream");
+    return st_pre;
+}
+
+}  // namespace
+
+extern "C" {
+
+pa_status pa_attention(const void* query, const void* key_cache, const void* value_cache,
+                       const int32_t* block_table, const int32_t* cu_seqlens_q,
+                       const int32_t* seqlens_kv, float scale, void* out, const pa_dims* dims,
+                       void* workspace, size_t workspace_bytes, int32_t* dev_status,
+                       void* stream) {
+    g_last_error[0] = 0;
+    return attention_impl(query, key_cache, value_cache, block_table, cu_seqlens_q, seqlens_kv,
+                          scale, out, dims, workspace, workspace_bytes, dev_status, stream, true);
 }
 
 pa_status pa_attention_noalloc(const void* query, const void* key_cache, const void* value_cache,
@@ -420,8 +516,9 @@ pa_status pa_attention_noalloc(const void* query, const void* key_cache, const v
         cudaError_t e = pa::noalloc_scratch(&scratch);
         if (e != cudaSuccess) return cuda_fail(e, "cudaGetSymbolAddress(noalloc scratch)");
     }
-    return pa_attention(query, key_cache, value_cache, block_table, cu_seqlens_q, seqlens_kv, scale,
-                        out, dims, scratch, need, dev_status, stream);
+    // No side stream here: creating one is an allocation.
+    return attention_impl(query, key_cache, value_cache, block_table, cu_seqlens_q, seqlens_kv,
+                          scale, out, dims, scratch, need, dev_status, stream, false);
 }
 
 pa_status pa_split_qkv_rotary_scatter(const void* query, const void* key, const void* value,

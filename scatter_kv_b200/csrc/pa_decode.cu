@@ -978,6 +978,13 @@ CtxGetCurrentFn ctx_get_current_fn() {
 }
 }  // namespace
 
+CUcontext current_context() {
+    CtxGetCurrentFn get_ctx = ctx_get_current_fn();
+    CUcontext ctx = nullptr;
+    if (get_ctx == nullptr || get_ctx(&ctx) != CUDA_SUCCESS) return nullptr;
+    return ctx;
+}
+
 cudaError_t noalloc_scratch(void** ptr) {
     static std::mutex mu;
     static void* addr[kMaxDevices] = {nullptr};

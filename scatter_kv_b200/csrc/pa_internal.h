@@ -205,6 +205,8 @@ cudaError_t launch_scatter_int4(const void* key, const void* value, const int32_
 constexpr size_t kNoAllocScratchBytes = size_t(8) << 20;
 constexpr int kMaxDevices = 64;
 cudaError_t noalloc_scratch(void** ptr);
+// The CUDA context current on this thread (null if none or unknown).
+CUcontext current_context();
 
 cudaError_t launch_prefill(const CUtensorMap& tm_q, const CUtensorMap& tm_k,
                            const CUtensorMap& tm_v, const PrefillParams& p, int head, bool bf16,
