@@ -204,7 +204,13 @@ pa_status pa_attention_workspace_size(const pa_dims* dims, size_t* bytes);
  *   workspace: device buffer of at least pa_attention_workspace_size() bytes
  *          (may be NULL when that is 0); contents need no initialisation.
  * Sequences with q_len_b <= 4 take the split-KV decode kernels, longer ones
- * the tensor-core prefill kernel; both write disjoint rows of `out`. */
+ * the tensor-core prefill kernel; both write disjoint rows of `out`.
+ * Streams: all work is ordered after what `stream` holds at the call and
+ * before what it is given next.  When a batch may hold both kinds of
+ * sequence, the decode kernels run on a library-owned side stream of the
+ * device (created on the first such call outside a stream capture), forked
+ * from `stream` by an event and joined back into it before the call returns;
+ * under stream capture this records a fork-join in the graph. */
 pa_status pa_attention(const void* query, const void* key_cache, const void* value_cache,
                        const int32_t* block_table, const int32_t* cu_seqlens_q,
                        const int32_t* seqlens_kv, float scale, void* out, const pa_dims* dims,
