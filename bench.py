@@ -262,6 +262,8 @@ KERNEL_SOURCES = {
     "slot_mapping": ("pa_scatter.cu", "pa_common.cuh", "pa_internal.h"),
     "qkv_rotary_scatter": ("pa_qkv.cu", "pa_common.cuh", "pa_internal.h"),
     "sparse_local_selected": ("pa_sparse.cu", "pa_common.cuh", "pa_internal.h"),
+    # head sizes 136 .. 256: the one-tile-per-CTA prefill kernel
+    "prefill_tcgen05@d256": ("pa_prefill256.cu", "pa_common.cuh", "pa_internal.h"),
 }
 
 
@@ -286,7 +288,8 @@ def profiled_traffic(kernel: str, workload: str):
     text = open(path).read()
     m = re.search(r"traffic_bytes_per_launch:\s*([0-9.eE+]+)", text)
     h = re.search(r"source_hash:\s*([0-9a-f]+)", text)
-    if not m or not h or h.group(1) != kernel_source_hash(KERNEL_SOURCES.get(kernel)):
+    key = kernel + "@d256" if workload.endswith("_d256") else kernel
+    if not m or not h or h.group(1) != kernel_source_hash(KERNEL_SOURCES.get(key)):
         return None
     return float(m.group(1))
 
@@ -617,6 +620,7 @@ def measure_qkv_rotary(args, spec, world, dev, steps):
     return {"workload": spec.name + ", packed QKV, rotary_dim = head_size, split pairing",
             "us": ms * 1e3, "bytes": nbytes, "GB/s": gbs, "frac": gbs / peaks["hbm_gbs"],
             "frac_nominal": gbs / NOMINAL_HBM_GBS, "peak_source": f"{peaks['source']} copy bandwidth",
+            "traffic": profiled_traffic("qkv_rotary_scatter", "prefill"),
             "timing": "CUDA-graph replays of the one call, L2 flushed between them"}
 
 
@@ -690,6 +694,7 @@ def measure_sparse(args, spec, world, dev, steps, num_selected=1024, window=128)
                         "per (token, KV head)",
             "us": ms * 1e3, "bytes": nbytes, "GB/s": gbs, "frac": gbs / peaks["hbm_gbs"],
             "frac_nominal": gbs / NOMINAL_HBM_GBS, "peak_source": f"{peaks['source']} copy bandwidth",
+            "traffic": profiled_traffic("sparse_local_selected", "decode"),
             "timing": "CUDA-graph replays of the one call, L2 flushed between them"}
 
 
@@ -698,6 +703,21 @@ def run_gpu(args, spec, rank, world, local):
 
     torch.cuda.set_device(local)
     dev = torch.device("cuda", local)
+    if args.only and args.part != "step":
+        # One other part alone (for profiling): its record as the line.
+        if args.part == "int4":
+            rec = measure_workload(args, spec, args.workload + "_int4", world, dev, args.steps,
+                                   e2e=False, int4=True)
+        elif args.part == "sparse":
+            rec = measure_sparse(args, spec, world, dev, args.steps)
+        elif args.part == "d256":
+            rec = measure_workload(args, workloads.spec_prefill_mha_d256(), "prefill_d256", world,
+                                   dev, args.steps, e2e=False, cpu=False)
+        else:
+            rec = measure_qkv_rotary(args, spec, world, dev, args.steps)
+        if rank == 0:
+            print(json.dumps({"part": args.part, **rec}), flush=True)
+        return rec
     main = measure_workload(args, spec, args.workload, world, dev, args.steps)
     # The other full-size workloads, measured in the same process and reported
     # in the same line (each with its own clocks, roofline and CPU baseline).
@@ -715,6 +735,9 @@ def run_gpu(args, spec, rank, world, local):
         others["sparse_local_selected"] = measure_sparse(
             args, workloads.CONFIGS[workloads.CONFIG_KEYS["decode"]](), world, dev,
             max(10, args.steps // 2))
+        others["prefill_d256"] = measure_workload(args, workloads.spec_prefill_mha_d256(),
+                                                  "prefill_d256", world, dev,
+                                                  max(10, args.steps // 2), e2e=True)
         others["fused_split_qkv_rotary_scatter"] = measure_qkv_rotary(
             args, workloads.CONFIGS[workloads.CONFIG_KEYS["prefill"]](), world, dev,
             max(10, args.steps // 2))
@@ -759,6 +782,11 @@ def main(argv=None):
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--only", action="store_true",
                     help="measure only --workload (default: every full-size workload)")
+    ap.add_argument("--part", default="step", choices=["step", "int4", "sparse", "qkv_rotary", "d256"],
+                    help="with --only: the part to measure on --workload's batch (step: the "
+                         "whole step; int4: INT4-cache scatter + decode; sparse: sparse "
+                         "attention; qkv_rotary: the fused split-QKV pass; d256: causal "
+                         "prefill at head size 256)")
     args = ap.parse_args(argv)
     if args.warmup < 3 and args.impl == "ours":
         args.warmup = 3

@@ -107,6 +107,17 @@ def spec_long_decode(rng_seed: int = 1004) -> Spec:
     return s
 
 
+def spec_prefill_mha_d256(rng_seed: int = 1005) -> Spec:
+    """The causal prefill MHA shape at head size 256: 8 sequences, q_len =
+    total_kv = 2048, 16/16 heads, bs 256 (a head size the pages' XQA kernels
+    are built for; not one of the five benchmark configurations)."""
+    q = np.full(8, 2048, dtype=np.int64)
+    past = np.zeros(8, dtype=np.int64)
+    s = Spec("causal prefill MHA, head size 256", q, past, 16, 16, 256, 256, 0, seed=rng_seed)
+    s.num_blocks = _pool(s.pages_per_seq)
+    return s
+
+
 CONFIGS = {
     0: spec_tiny,
     1: spec_decode_gqa,
