@@ -482,6 +482,8 @@ decode_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ 
             lim[h] = (r < R) ? (s.past + r / g) : (T - 1);
             lo[h] = (GEN && p.mods.window) ? lim[h] - p.mods.window_size : -(1 << 30);
         }
+        // With a window, every valid row sees keys at or after this one.
+        const int max_lo = (GEN && p.mods.window) ? s.past + (R - 1) / g - p.mods.window_size : 0;
         // Q fragments (A operand) straight from global memory; columns past
         // the head size are zero.
         uint32_t qf[HEAD / 16][4];
@@ -567,55 +569,99 @@ decode_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ 
                     E::mma(sacc[2 * np + 1], qf[kk], b2, b3);
                 }
             }
-            // Scale (and cap) into the log2 domain, mask, online softmax.
+            // Online softmax in the log2 domain.  A tile that lies wholly in
+            // every row's visible range (keys <= past, inside the split and,
+            // with a window, at or after every row's first key) skips the
+            // per-key mask and takes the max of the raw scores (the scale is
+            // positive).  The exponent base m_run of a row moves only when the
+            // row's max passes it by more than 8 (P stays below 2^8), and the
+            // warp rescales O only when one of its rows moves.
+            const bool cap = GEN && p.mods.softcap > 0.f;
+            const bool interior = !Q4 && !cap && k0 + C::BN <= k_end && k0 + C::BN - 1 <= s.past &&
+                                  (!GEN || !p.mods.window || k0 >= max_lo);
             float mx[2] = {-INFINITY, -INFINITY};
+            if (interior) {
 #pragma unroll
-            for (int nt = 0; nt < 4; ++nt) {
+                for (int nt = 0; nt < 4; ++nt) {
+                    mx[0] = fmax3(mx[0], sacc[nt][0], sacc[nt][1]);
+                    mx[1] = fmax3(mx[1], sacc[nt][2], sacc[nt][3]);
+                }
+            } else {
 #pragma unroll
-                for (int e = 0; e < 4; ++e) {
-                    const int h = e >> 1;
-                    const int key = k0 + nt * 8 + 2 * qid + (e & 1);
-                    bool vis = key < k_end && key <= lim[h];
-                    if (GEN) vis = vis && key >= lo[h];
-                    const float sc = (GEN && p.mods.softcap > 0.f)
-                                         ? softcap_log2(sacc[nt][e] * p.mods.scale, p.mods.softcap,
-                                                        p.mods.inv_softcap)
-                                         : sacc[nt][e] * p.mods.scale_log2;
-                    const float v = vis ? sc : -INFINITY;
-                    sacc[nt][e] = v;
-                    mx[h] = fmaxf(mx[h], v);
+                for (int nt = 0; nt < 4; ++nt) {
+#pragma unroll
+                    for (int e = 0; e < 4; ++e) {
+                        const int h = e >> 1;
+                        const int key = k0 + nt * 8 + 2 * qid + (e & 1);
+                        bool vis = key < k_end && key <= lim[h];
+                        if (GEN) vis = vis && key >= lo[h];
+                        const float sc = cap ? softcap_log2(sacc[nt][e] * p.mods.scale, p.mods.softcap,
+                                                            p.mods.inv_softcap)
+                                             : sacc[nt][e] * p.mods.scale_log2;
+                        const float v = vis ? sc : -INFINITY;
+                        sacc[nt][e] = v;
+                        mx[h] = fmaxf(mx[h], v);
+                    }
                 }
             }
-            float alpha[2];
+            bool grow[2];
 #pragma unroll
             for (int h = 0; h < 2; ++h) {
                 mx[h] = fmaxf(mx[h], __shfl_xor_sync(0xffffffffu, mx[h], 1));
                 mx[h] = fmaxf(mx[h], __shfl_xor_sync(0xffffffffu, mx[h], 2));
-                const float m_new = fmaxf(m_run[h], mx[h]);
-                const float base = (m_new == -INFINITY) ? 0.f : m_new;
-                alpha[h] = fast_exp2(m_run[h] - base);
-                m_run[h] = m_new;
-                mx[h] = base;
+                if (interior) mx[h] *= p.mods.scale_log2;
+                grow[h] = mx[h] > m_run[h] + 8.f;
             }
+            if constexpr (Q4) {
+                // INT4 build: the base follows the max on every tile (the lazy
+                // form costs this build spills).
+                float alpha[2];
+#pragma unroll
+                for (int h = 0; h < 2; ++h) {
+                    const float m_new = fmaxf(m_run[h], mx[h]);
+                    alpha[h] = fast_exp2(m_run[h] - ((m_new == -INFINITY) ? 0.f : m_new));
+                    m_run[h] = m_new;
+                    l_run[h] *= alpha[h];
+                }
+#pragma unroll
+                for (int i = 0; i < HEAD / 8; ++i) {
+                    oacc[i][0] *= alpha[0];
+                    oacc[i][1] *= alpha[0];
+                    oacc[i][2] *= alpha[1];
+                    oacc[i][3] *= alpha[1];
+                }
+            } else if (__any_sync(0xffffffffu, grow[0] || grow[1])) {
+                float alpha[2];
+#pragma unroll
+                for (int h = 0; h < 2; ++h) {
+                    const float m_new = grow[h] ? mx[h] : m_run[h];
+                    alpha[h] = grow[h] ? ((m_run[h] == -INFINITY) ? 0.f : fast_exp2(m_run[h] - m_new)) : 1.f;
+                    m_run[h] = m_new;
+                    l_run[h] *= alpha[h];
+                }
+#pragma unroll
+                for (int i = 0; i < HEAD / 8; ++i) {
+                    oacc[i][0] *= alpha[0];
+                    oacc[i][1] *= alpha[0];
+                    oacc[i][2] *= alpha[1];
+                    oacc[i][3] *= alpha[1];
+                }
+            }
+            const float sc2 = interior ? p.mods.scale_log2 : 1.f;
+            const float nb0 = (m_run[0] == -INFINITY) ? 0.f : -m_run[0];
+            const float nb1 = (m_run[1] == -INFINITY) ? 0.f : -m_run[1];
             float psum[2] = {0.f, 0.f};
 #pragma unroll
             for (int nt = 0; nt < 4; ++nt) {
 #pragma unroll
                 for (int e = 0; e < 4; ++e) {
-                    const float pe = fast_exp2(sacc[nt][e] - mx[e >> 1]);
+                    const float pe = fast_exp2(fmaf(sacc[nt][e], sc2, (e >> 1) ? nb1 : nb0));
                     sacc[nt][e] = pe;
                     psum[e >> 1] += pe;
                 }
             }
-#pragma unroll
-            for (int h = 0; h < 2; ++h) l_run[h] = l_run[h] * alpha[h] + psum[h];
-#pragma unroll
-            for (int i = 0; i < HEAD / 8; ++i) {
-                oacc[i][0] *= alpha[0];
-                oacc[i][1] *= alpha[0];
-                oacc[i][2] *= alpha[1];
-                oacc[i][3] *= alpha[1];
-            }
+            l_run[0] += psum[0];
+            l_run[1] += psum[1];
             // P as A fragments (two k16 steps over the 32 keys), in V's type.
             uint32_t pa[2][4];
 #pragma unroll

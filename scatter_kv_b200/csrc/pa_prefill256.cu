@@ -72,13 +72,18 @@ struct Item {
     int b, kvh, tile, c0, c1, kv;
 };
 
-// CTA x -> (sequence, KV head, query tile), longest work first (a
-// sequence's last tile has the most keys): every sequence's rank-0 tile,
-// then every rank-1 tile, and so on.
+// CTA x -> (sequence, KV head, query tile), sequence-major: the items of one
+// (sequence, KV head) are adjacent, its longest tile (the last, with the
+// most keys) first.  The CTAs in flight then cover a few (sequence, KV head)
+// pairs at a time and share their K/V tiles through L2 (at 256 columns a
+// query tile's K/V stream is twice that of the 128-wide kernel, and an order
+// that mixes all pairs re-reads it from DRAM); the light tiles of the last
+// pairs end the grid.  One warp, 32 sequences per step.
 __device__ bool find_item(const PrefillParams& p, long long slot, int tokp, Item& w) {
     const int lane = threadIdx.x & 31;
-    auto lengths = [&](int b, int& c0, int& c1, int& kv, int& nt) {
-        c0 = c1 = kv = nt = 0;
+    for (int b0 = 0; b0 < p.batch; b0 += 32) {
+        const int b = b0 + lane;
+        int c0 = 0, c1 = 0, kv = 0, nt = 0;
         if (b < p.batch) {
             c0 = p.cu_seqlens_q[b];
             c1 = p.cu_seqlens_q[b + 1];
@@ -87,34 +92,29 @@ __device__ bool find_item(const PrefillParams& p, long long slot, int tokp, Item
             if (ql > p.decode_max_q && c0 >= 0 && (long long)c1 <= p.token_count)
                 nt = (ql + tokp - 1) / tokp;
         }
-    };
-    int c0f, c1f, kvf, ntf;
-    lengths(lane, c0f, c1f, kvf, ntf);
-    for (int r = 0;; ++r) {
-        bool more = false;
-        for (int b0 = 0; b0 < p.batch; b0 += 32) {
-            int c0 = c0f, c1 = c1f, kv = kvf, nt = ntf;
-            if (b0 > 0) lengths(b0 + lane, c0, c1, kv, nt);
-            const unsigned m = __ballot_sync(0xffffffffu, nt > r);
-            more = more || m != 0u;
-            const long long total = (long long)__popc(m) * p.kv_heads;
-            if (slot < total) {
-                const int k = (int)(slot / p.kv_heads);
-                unsigned mm = m;
-                for (int i = 0; i < k; ++i) mm &= mm - 1u;
-                const int lb = __ffs(mm) - 1;
-                w.b = b0 + lb;
-                w.kvh = (int)(slot % p.kv_heads);
-                w.tile = __shfl_sync(0xffffffffu, nt, lb) - 1 - r;
-                w.c0 = __shfl_sync(0xffffffffu, c0, lb);
-                w.c1 = __shfl_sync(0xffffffffu, c1, lb);
-                w.kv = __shfl_sync(0xffffffffu, kv, lb);
-                return true;
-            }
-            slot -= total;
+        const long long items = (long long)nt * p.kv_heads;
+        long long incl = items;
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+            const long long t = __shfl_up_sync(0xffffffffu, incl, o);
+            if (lane >= o) incl += t;
         }
-        if (!more) return false;
+        const long long total = __shfl_sync(0xffffffffu, incl, 31);
+        if (slot < total) {
+            const int lb = __ffs(__ballot_sync(0xffffffffu, incl > slot)) - 1;
+            const long long rel = slot - __shfl_sync(0xffffffffu, incl - items, lb);
+            const int ntb = __shfl_sync(0xffffffffu, nt, lb);
+            w.b = b0 + lb;
+            w.kvh = (int)(rel / ntb);
+            w.tile = ntb - 1 - (int)(rel % ntb);
+            w.c0 = __shfl_sync(0xffffffffu, c0, lb);
+            w.c1 = __shfl_sync(0xffffffffu, c1, lb);
+            w.kv = __shfl_sync(0xffffffffu, kv, lb);
+            return true;
+        }
+        slot -= total;
     }
+    return false;
 }
 
 // Ring item u of a CTA with nt key tiles: K_0, K_1, then V_j, K_{j+2} for
