@@ -73,10 +73,10 @@ template <int HEAD, bool CPA, bool Q4>
 __host__ __device__ constexpr int dec_ctas_per_sm() {
     return Q4 ? 2 : HEAD > 128 ? (CPA ? 2 : 1) : ((HEAD >= 128 && !CPA) ? 2 : 3);
 }
-// INT4 pages: two CTAs per SM at 128 registers; the consumers take 168, the
-// producers (which hold four tiles of loads in registers) 88.
+// INT4 pages: two CTAs per SM at 128 registers; the consumers take 160, the
+// producers (which hold four tiles of loads in registers) 96.
 constexpr int kQ4LaunchRegs = 128;
-constexpr int kQ4RegsCons = 168, kQ4RegsProd = 88;
+constexpr int kQ4RegsCons = 160, kQ4RegsProd = 96;
 static_assert(128 * (kQ4RegsCons + kQ4RegsProd) == 256 * kQ4LaunchRegs,
               "register split must equal the launch budget");
 
@@ -150,29 +150,57 @@ __device__ __forceinline__ void zero_rows(const DecodeParams& p, const SeqInfo& 
 }
 
 // INT4 pages (Q4): two signed 4-bit codes per byte, the low nibble the even
-// channel; a code q of channel c stands for q * scale[kv head][c].  The
-// producer converts the codes of a 16-byte chunk (32 channels of one key) to
-// 16-bit values exactly: byte b's two nibbles are placed in the low bits of
-// the two halves of a 32-bit word, their sign bits flipped, over the
-// exponent of 1024 (f16) or 128 (bf16), where the spacing of representable
-// values is 1 -- so each half reads 1024 + (n ^ 8) (or 128 + (n ^ 8)) and
-// one subtraction leaves n as a signed integer.
+// channel; a code q of channel c stands for q * scale[kv head][c].
+
+// The 8 codes of one 32-bit word (channels c .. c + 7, low nibble first) as
+// 16-bit values, in the order c, c+4, c+1, c+5, c+2, c+6, c+3, c+7 (pairs
+// (c+i, c+i+4) per 32-bit lane).  One AND-XOR per pair puts the two codes,
+// sign bits flipped, under the exponent of 1024 (f16; 128 for bf16) where
+// the spacing is 1, and one subtraction leaves them signed.  In f16 the odd
+// nibbles are taken in place, at 16 times the spacing, and one FMA scales
+// them back (both steps exact); bf16's 7-bit mantissa has no room for that,
+// so its odd nibbles are shifted down first.  Stages hold INT4 tiles in this
+// order: the consumers read Q and write O through the same permutation.
 template <typename ET>
-__device__ __forceinline__ uint32_t int4_pair(uint32_t w, uint32_t w_hi, int byte) {
-    // Byte `byte` of w into bits 0-7, the same byte of w >> 4 into bits 16-23.
-    const uint32_t t = __byte_perm(w, w_hi, (uint32_t)(byte | (byte << 4) | ((4 + byte) << 8) | ((4 + byte) << 12)));
+__device__ __forceinline__ uint4 int4_word(uint32_t w) {
+    uint4 o;
     if (Elem<ET>::kBf16) {
-        const uint32_t v = (t & 0x000F000Fu) ^ 0x43084308u;          // 128 + (n ^ 8), both halves
-        __nv_bfloat162 h = *reinterpret_cast<const __nv_bfloat162*>(&v);
-        h = __hsub2(h, __floats2bfloat162_rn(136.f, 136.f));
-        return *reinterpret_cast<uint32_t*>(&h);
+        const __nv_bfloat162 off = __floats2bfloat162_rn(136.f, 136.f);
+        uint32_t t[4];
+        t[0] = (w & 0x000F000Fu) ^ 0x43084308u;
+        t[1] = ((w >> 4) & 0x000F000Fu) ^ 0x43084308u;
+        t[2] = ((w >> 8) & 0x000F000Fu) ^ 0x43084308u;
+        t[3] = ((w >> 12) & 0x000F000Fu) ^ 0x43084308u;
+        uint32_t r[4];
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+            __nv_bfloat162 h = __hsub2(*reinterpret_cast<const __nv_bfloat162*>(&t[i]), off);
+            r[i] = *reinterpret_cast<uint32_t*>(&h);
+        }
+        o = make_uint4(r[0], r[1], r[2], r[3]);
     } else {
-        const uint32_t v = (t & 0x000F000Fu) ^ 0x64086408u;          // 1024 + (n ^ 8), both halves
-        __half2 h = *reinterpret_cast<const __half2*>(&v);
-        h = __hsub2(h, __floats2half2_rn(1032.f, 1032.f));
-        return *reinterpret_cast<uint32_t*>(&h);
+        const __half2 off = __floats2half2_rn(1032.f, 1032.f);
+        const __half2 sc = __floats2half2_rn(0.0625f, 0.0625f);
+        const __half2 off16 = __floats2half2_rn(-72.f, -72.f);
+        const uint32_t w8 = w >> 8;
+        uint32_t t[4];
+        t[0] = (w & 0x000F000Fu) ^ 0x64086408u;
+        t[1] = (w & 0x00F000F0u) ^ 0x64806480u;
+        t[2] = (w8 & 0x000F000Fu) ^ 0x64086408u;
+        t[3] = (w8 & 0x00F000F0u) ^ 0x64806480u;
+        __half2 h[4];
+        h[0] = __hsub2(*reinterpret_cast<const __half2*>(&t[0]), off);
+        h[1] = __hfma2(*reinterpret_cast<const __half2*>(&t[1]), sc, off16);
+        h[2] = __hsub2(*reinterpret_cast<const __half2*>(&t[2]), off);
+        h[3] = __hfma2(*reinterpret_cast<const __half2*>(&t[3]), sc, off16);
+        o = make_uint4(*reinterpret_cast<uint32_t*>(&h[0]), *reinterpret_cast<uint32_t*>(&h[1]),
+                       *reinterpret_cast<uint32_t*>(&h[2]), *reinterpret_cast<uint32_t*>(&h[3]));
     }
+    return o;
 }
+
+// Channel held at position p of an INT4 stage row (see int4_word).
+__host__ __device__ constexpr int int4_channel(int p) { return (p & ~7) + ((p & 7) >> 1) + 4 * (p & 1); }
 
 __device__ __forceinline__ uint4 ld_nc16(const void* p) {
     uint4 v;
@@ -346,12 +374,7 @@ decode_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ 
                     const uint32_t w[4] = {x.x, x.y, x.z, x.w};
 #pragma unroll
                     for (int i = 0; i < 4; ++i) {
-                        const uint32_t hi = w[i] >> 4;
-                        uint4 o;
-                        o.x = int4_pair<ET>(w[i], hi, 0);
-                        o.y = int4_pair<ET>(w[i], hi, 1);
-                        o.z = int4_pair<ET>(w[i], hi, 2);
-                        o.w = int4_pair<ET>(w[i], hi, 3);
+                        const uint4 o = int4_word<ET>(w[i]);
                         const int ch = jc * 32 + i * 8;
                         const int cb = ch / C::A, jj = (ch % C::A) / 8;
                         *reinterpret_cast<uint4*>(tile + swz<C::RB>((uint32_t)((cb * C::BN + r) * C::RB + jj * 16))) = o;
@@ -493,21 +516,29 @@ decode_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ 
 #pragma unroll
             for (int kk = 0; kk < HEAD / 16; ++kk) {
                 const int c = kk * 16 + 2 * qid;
-                const bool lo_ok = c < hs, hi_ok = c + 8 < hs;
-                qf[kk][0] = (q0 && lo_ok) ? *reinterpret_cast<const uint32_t*>(q0 + c) : 0u;
-                qf[kk][1] = (q1 && lo_ok) ? *reinterpret_cast<const uint32_t*>(q1 + c) : 0u;
-                qf[kk][2] = (q0 && hi_ok) ? *reinterpret_cast<const uint32_t*>(q0 + c + 8) : 0u;
-                qf[kk][3] = (q1 && hi_ok) ? *reinterpret_cast<const uint32_t*>(q1 + c + 8) : 0u;
                 if constexpr (Q4) {
-                    // The K scales fold into Q: S = sum_c (Q[c] * ks[c]) * code[c].
-                    const float2 s0 = *reinterpret_cast<const float2*>(p.k_scale + kvh * HEAD + c);
-                    const float2 s1 = *reinterpret_cast<const float2*>(p.k_scale + kvh * HEAD + c + 8);
+                    // INT4 stages hold channels permuted (int4_channel): Q takes
+                    // the same order, and the K scales fold into it:
+                    // S = sum_c (Q[c] * ks[c]) * code[c].
+                    const float* ks = p.k_scale + kvh * HEAD;
 #pragma unroll
                     for (int e = 0; e < 4; ++e) {
-                        const float2 sc = (e < 2) ? s0 : s1;
-                        const float2 qv = Elem<ET>::unpack2(qf[kk][e]);
-                        qf[kk][e] = E::pack2(qv.x * sc.x, qv.y * sc.y);
+                        const uint16_t* qr = (e & 1) ? q1 : q0;
+                        const int pos = c + ((e & 2) ? 8 : 0);
+                        const int c0 = int4_channel(pos), c1 = int4_channel(pos + 1);
+                        if (qr) {
+                            const float2 qv = Elem<ET>::unpack2((uint32_t)qr[c0] | ((uint32_t)qr[c1] << 16));
+                            qf[kk][e] = E::pack2(qv.x * ks[c0], qv.y * ks[c1]);
+                        } else {
+                            qf[kk][e] = 0u;
+                        }
                     }
+                } else {
+                    const bool lo_ok = c < hs, hi_ok = c + 8 < hs;
+                    qf[kk][0] = (q0 && lo_ok) ? *reinterpret_cast<const uint32_t*>(q0 + c) : 0u;
+                    qf[kk][1] = (q1 && lo_ok) ? *reinterpret_cast<const uint32_t*>(q1 + c) : 0u;
+                    qf[kk][2] = (q0 && hi_ok) ? *reinterpret_cast<const uint32_t*>(q0 + c + 8) : 0u;
+                    qf[kk][3] = (q1 && hi_ok) ? *reinterpret_cast<const uint32_t*>(q1 + c + 8) : 0u;
                 }
             }
         }
@@ -729,11 +760,21 @@ decode_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ 
                 row_l[r] = L;
                 row_m[r] = M;
             }
-            float* dst = scr + (grp * C::RMAX + r) * C::OST + 2 * qid;
+            if constexpr (Q4) {
+                // Positions 2 qid, 2 qid + 1 of each 8 hold channels qid, qid + 4.
+                float* dst = scr + (grp * C::RMAX + r) * C::OST + qid;
 #pragma unroll
-            for (int i = 0; i < HEAD / 8; ++i) {
-                float2 v = make_float2(oacc[i][2 * h] * f, oacc[i][2 * h + 1] * f);
-                *reinterpret_cast<float2*>(dst + i * 8) = v;
+                for (int i = 0; i < HEAD / 8; ++i) {
+                    dst[i * 8] = oacc[i][2 * h] * f;
+                    dst[i * 8 + 4] = oacc[i][2 * h + 1] * f;
+                }
+            } else {
+                float* dst = scr + (grp * C::RMAX + r) * C::OST + 2 * qid;
+#pragma unroll
+                for (int i = 0; i < HEAD / 8; ++i) {
+                    float2 v = make_float2(oacc[i][2 * h] * f, oacc[i][2 * h + 1] * f);
+                    *reinterpret_cast<float2*>(dst + i * 8) = v;
+                }
             }
         }
         asm volatile("bar.sync 1, %0;" ::"r"(C::NCW * 32));
