@@ -269,7 +269,7 @@ pa_status pa_scatter_kv_int4(const void* key, const void* value, const int32_t* 
 
 /* pa_attention_int4 -- pa_attention over INT4 caches, for decode batches:
  * max_seqlen_q_hint must be set and no larger than the decode cut-off
- * (min(4, 32 / group)); head sizes 32, 64 and 128; no softcap or window
+ * (min(4, 32 / group)); head sizes 32, 64, 128 and 256; no softcap or window
  * (PA_ERR_NOT_IMPLEMENTED otherwise).  The result is attention over the
  * values the codes stand for.  Query and output in dims->dtype; workspace
  * from pa_attention_workspace_size(dims).  A sequence longer than the hint

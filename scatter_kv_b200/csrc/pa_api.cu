@@ -635,8 +635,8 @@ pa_status pa_attention_int4(const void* query, const void* key_cache, const void
     pa_status st = check_dims(dims);
     if (st != PA_OK) return st;
     const pa_dims& d = *dims;
-    if (d.head_size != 32 && d.head_size != 64 && d.head_size != 128)
-        return fail(PA_ERR_NOT_IMPLEMENTED, "INT4 attention: head sizes 32, 64 and 128 are built");
+    if (d.head_size != 32 && d.head_size != 64 && d.head_size != 128 && d.head_size != 256)
+        return fail(PA_ERR_NOT_IMPLEMENTED, "INT4 attention: head sizes 32, 64, 128 and 256 are built");
     if (d.softcap > 0.f || d.local_window)
         return fail(PA_ERR_NOT_IMPLEMENTED, "INT4 attention: no softcap or local window");
     const int nsm = num_sms_of_current_device();

@@ -71,10 +71,12 @@ template <int HEAD>
 __host__ __device__ constexpr int dec_regs_prod() { return HEAD > 128 ? kDec256RegsProd : kDecRegsProd; }
 template <int HEAD, bool CPA, bool Q4>
 __host__ __device__ constexpr int dec_ctas_per_sm() {
-    return Q4 ? 2 : HEAD > 128 ? (CPA ? 2 : 1) : ((HEAD >= 128 && !CPA) ? 2 : 3);
+    return Q4 ? (HEAD > 128 ? 1 : 2) : HEAD > 128 ? (CPA ? 2 : 1) : ((HEAD >= 128 && !CPA) ? 2 : 3);
 }
 // INT4 pages: two CTAs per SM at 128 registers; the consumers take 160, the
-// producers (which hold four tiles of loads in registers) 96.
+// producers (which hold four tiles of loads in registers) 96.  At head size
+// 256 one CTA per SM, without a split (the consumers hold twice the Q
+// fragments and O accumulators).
 constexpr int kQ4LaunchRegs = 128;
 constexpr int kQ4RegsCons = 160, kQ4RegsProd = 96;
 static_assert(128 * (kQ4RegsCons + kQ4RegsProd) == 256 * kQ4LaunchRegs,
@@ -312,7 +314,9 @@ decode_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ 
 
     if (warp >= C::NCW) {
         // ------------------------------------------------------------ producers
-        if (Q4) asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(kQ4RegsProd));
+        if (Q4) {
+            if (HEAD <= 128) asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(kQ4RegsProd));
+        }
         else if (CPA) asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(dec_regs_prod<HEAD>()));
         const int pw = warp - C::NCW;
         // The split's block ids, fetched once by the first producer warp, so
@@ -345,12 +349,15 @@ decode_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ 
         if constexpr (Q4) {
             if (!bad) {
                 // INT4 pages (any block size): producer thread q loads the 16-byte
-                // chunk q % CPR4 (32 channels) of key row q / CPR4 of every tile,
-                // D tiles ahead in registers, and writes its 64 bytes of 16-bit
-                // values where the swizzled stage layout puts them; each thread
-                // arrives on the stage once its stores are done.
+                // chunk q % CPR4 (32 channels) of key rows q / CPR4 + i * RPP of
+                // every tile (NP4 passes; two at head size 256), D tiles ahead in
+                // registers, and writes its 64 bytes of 16-bit values per row
+                // where the swizzled stage layout puts them; each thread arrives
+                // on the stage once its stores are done.
                 constexpr int CPR4 = HEAD / 32;
-                static_assert(HEAD >= 32 && (C::NPW * 32) / CPR4 >= C::BN, "one pass covers a tile");
+                constexpr int RPP = (C::NPW * 32) / CPR4;        // key rows per pass
+                constexpr int NP4 = RPP >= C::BN ? 1 : C::BN / RPP;
+                static_assert(HEAD >= 32 && RPP * NP4 >= C::BN, "the passes cover a tile");
                 constexpr int D = 4;
                 const int q0 = pw * 32 + lane;
                 const int r = q0 / CPR4, jc = q0 % CPR4;
@@ -360,24 +367,31 @@ decode_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ 
                 const char* vc = reinterpret_cast<const char*>(p.value_cache);
                 const long long row_bytes = (long long)p.kv_heads * (HEAD / 2);
                 const long long colb = (long long)kvh * (HEAD / 2) + jc * 16;
-                uint4 kr[D], vr[D];
-                auto issue = [&](int t, uint4& kx, uint4& vx) {
-                    kx = vx = make_uint4(0, 0, 0, 0);
-                    const int key = k_begin + t * C::BN + r;
-                    if (active && t < ntiles && key < k_end) {
-                        const long long g = ((long long)block_of(key >> lbs) * bs + (key & (bs - 1))) * row_bytes + colb;
-                        kx = ld_nc16(kc + g);
-                        vx = ld_nc16(vc + g);
+                uint4 kr[D][NP4], vr[D][NP4];
+                auto issue = [&](int t, uint4* kx, uint4* vx) {
+#pragma unroll
+                    for (int pp = 0; pp < NP4; ++pp) {
+                        kx[pp] = vx[pp] = make_uint4(0, 0, 0, 0);
+                        const int key = k_begin + t * C::BN + r + pp * RPP;
+                        if (active && t < ntiles && key < k_end) {
+                            const long long g = ((long long)block_of(key >> lbs) * bs + (key & (bs - 1))) * row_bytes + colb;
+                            kx[pp] = ld_nc16(kc + g);
+                            vx[pp] = ld_nc16(vc + g);
+                        }
                     }
                 };
-                auto put = [&](uint8_t* tile, const uint4& x) {
-                    const uint32_t w[4] = {x.x, x.y, x.z, x.w};
+                auto put = [&](uint8_t* tile, const uint4* x) {
 #pragma unroll
-                    for (int i = 0; i < 4; ++i) {
-                        const uint4 o = int4_word<ET>(w[i]);
-                        const int ch = jc * 32 + i * 8;
-                        const int cb = ch / C::A, jj = (ch % C::A) / 8;
-                        *reinterpret_cast<uint4*>(tile + swz<C::RB>((uint32_t)((cb * C::BN + r) * C::RB + jj * 16))) = o;
+                    for (int pp = 0; pp < NP4; ++pp) {
+                        const uint32_t w[4] = {x[pp].x, x[pp].y, x[pp].z, x[pp].w};
+                        const int row = r + pp * RPP;
+#pragma unroll
+                        for (int i = 0; i < 4; ++i) {
+                            const uint4 o = int4_word<ET>(w[i]);
+                            const int ch = jc * 32 + i * 8;
+                            const int cb = ch / C::A, jj = (ch % C::A) / 8;
+                            *reinterpret_cast<uint4*>(tile + swz<C::RB>((uint32_t)((cb * C::BN + row) * C::RB + jj * 16))) = o;
+                        }
                     }
                 };
 #pragma unroll
@@ -490,7 +504,9 @@ decode_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ 
         }
     } else {
         // ------------------------------------------------------------ consumers
-        if (Q4) asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(kQ4RegsCons));
+        if (Q4) {
+            if (HEAD <= 128) asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(kQ4RegsCons));
+        }
         else if (CPA) asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(dec_regs_cons<HEAD>()));
         const int mt = warp % MT;          // which 16 query rows
         const int grp = warp / MT;         // which tiles
@@ -898,7 +914,7 @@ cudaError_t launch_decode_t(const CUtensorMap& tm_k, const CUtensorMap& tm_v,
     using C = Cfg<HEAD, MT, CPA>;
     auto kern = decode_kernel<HEAD, MT, CPA, ET, GEN, Q4>;
     cudaError_t e;
-    if (CPA) {
+    if (CPA && !(Q4 && HEAD > 128)) {
         // The register split inside the kernel assumes this launch budget.
         cudaFuncAttributes fa;
         e = cudaFuncGetAttributes(&fa, kern);
@@ -1010,6 +1026,8 @@ cudaError_t launch_decode_int4(const DecodeParams& p, int head, int mtiles, bool
                              : launch_decode_q4_h<64, __half>(unused, p, mtiles, stream);
         case 128: return bf16 ? launch_decode_q4_h<128, __nv_bfloat16>(unused, p, mtiles, stream)
                               : launch_decode_q4_h<128, __half>(unused, p, mtiles, stream);
+        case 256: return bf16 ? launch_decode_q4_h<256, __nv_bfloat16>(unused, p, mtiles, stream)
+                              : launch_decode_q4_h<256, __half>(unused, p, mtiles, stream);
         default: return cudaErrorInvalidValue;
     }
 }

@@ -134,6 +134,10 @@ CASES = [
     ([2, 1, 3], [500, 6000, 77], 16, 2, 64, 16, "f16"),
     ([1, 3], [999, 64], 8, 8, 32, 128, "f16"),
     ([1, 1, 2, 4], [700, 3000, 45, 9000], 32, 8, 128, 16, "bf16"),
+    # head size 256 (the pages' INT4 XQA kernels are built for it)
+    ([1, 2, 4, 1], [2500, 300, 6000, 33], 16, 2, 256, 16, "f16"),
+    ([3, 1], [4100, 900], 32, 4, 256, 256, "bf16"),
+    ([1, 1, 1], [1500, 70, 8000], 8, 8, 256, 64, "f16"),
 ]
 
 
