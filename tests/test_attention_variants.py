@@ -95,3 +95,14 @@ def test_groups_not_powers_of_two(qh, kvh, bs):
 def test_group_of_three_without_hints():
     spec = workloads.custom([1, 77, 3], [4000, 10, 500], 24, 8, 64, 16, seed=9)
     _check(spec, hints=False)
+
+
+@pytest.mark.parametrize("bs", [16, 32, 64])
+@pytest.mark.parametrize("heads,d", [((32, 8), 128), ((16, 16), 64), ((8, 2), 32)])
+def test_cp_async_page_sizes(bs, heads, d):
+    """Pages smaller than the prefill kernel's 128-key tile take its cp.async
+    producers: whole tiles by 16-row units (one page each), the tile holding
+    the sequence end row by row.  Long pasts give many whole tiles."""
+    q, past = [300, 1, 700, 129, 2], [1000, 4000, 0, 517, 60]
+    spec = workloads.custom(q, past, heads[0], heads[1], d, bs, seed=bs + d)
+    _check(spec)

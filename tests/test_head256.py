@@ -85,3 +85,22 @@ def test_head256_growing_keys(bs):
 def test_head256_long_prefill_without_hints():
     spec = workloads.custom([700, 513], [1500, 0], 16, 2, 256, 128, seed=3)
     _check(spec, hints=False)
+
+
+def test_head256_full_size_prefill_sampled_rows_and_bit_identity():
+    """The head-256 causal prefill workload at full size (8 x 2048 tokens,
+    16/16 heads, 256-key pages): 2048 sampled rows (every sequence's first
+    and last token included) against the oracle, with unused cache rows
+    poisoned, and the same bits on a second run."""
+    from pa_harness import sample_rows
+    spec = workloads.spec_prefill_mha_d256()
+    x = workloads.generate(spec)
+    poison_unused(spec, x)
+    outs, _, status, _ = run_gpu(spec, x, repeat=2)
+    assert status == 0
+    assert np.array_equal(outs[0].view(np.uint16), outs[1].view(np.uint16))
+    rows = sample_rows(spec, 2048, seed=7)
+    want, _, _, _ = oracle_step(spec, x, rows=rows)
+    got = outs[0][rows[:, 0], rows[:, 1]]
+    mx, mn = tolerances(spec)
+    assert_close(got, want, mx, mn, what="head-256 prefill, sampled rows")
