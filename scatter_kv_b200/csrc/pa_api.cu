@@ -318,6 +318,17 @@ SideStream* side_stream_for(cudaStream_t user, std::unique_lock<std::mutex>& loc
     return &ss;
 }
 
+// Driver-API calls (the tensor-map encoder) need a current context.  A host
+// thread whose first CUDA work is this library's call may have none yet (the
+// runtime binds the device's primary context lazily): make it current.
+cudaError_t ensure_context() {
+    if (pa::current_context() != nullptr) return cudaSuccess;
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e == cudaSuccess) e = cudaSetDevice(dev);
+    return e;
+}
+
 pa_status attention_impl(const void* query, const void* key_cache, const void* value_cache,
                          const int32_t* block_table, const int32_t* cu_seqlens_q,
                          const int32_t* seqlens_kv, float scale, void* out, const pa_dims* dims,
@@ -337,6 +348,10 @@ pa_status attention_impl(const void* query, const void* key_cache, const void* v
     PA_REQUIRE_IPTR(block_table);
     PA_REQUIRE_IPTR(cu_seqlens_q);
     PA_REQUIRE_IPTR(seqlens_kv);
+    {
+        const cudaError_t e = ensure_context();
+        if (e != cudaSuccess) return cuda_fail(e, "no CUDA context for the calling thread");
+    }
     const int nsm = num_sms_of_current_device();
     const pa::DecodePlan plan = pa::plan_decode(d, nsm);
     if (workspace_bytes < plan.workspace_bytes)

@@ -100,3 +100,57 @@ def test_bad_cu_seqlens_flagged():
     x["cu_seqlens_q"][-1] -= 1       # last sequence ends before token_count
     got, _, status, _ = run_gpu(spec, x)
     assert status & pa.PA_DEV_BAD_CU_SEQLENS
+
+
+@pytest.mark.gpu
+def test_side_stream_from_two_host_threads():
+    """Mixed batches (decode and prefill sequences, so the decode part forks
+    to the library's side stream) from two host threads on two streams at
+    once, 20 calls each: every result equals the serial one bit for bit."""
+    import threading
+
+    import torch
+    import scatter_kv_b200 as pa
+    from pa_harness import dims_for, host_bits, to_dev
+
+    specs = [workloads.custom([1, 3, 90, 1, 200], [700, 2000, 30, 5, 400], 16, 4, 128, 16, seed=61),
+             workloads.custom([2, 150, 1], [3000, 0, 900], 32, 8, 128, 16, seed=62)]
+    runs = []
+    for spec in specs:
+        x = workloads.generate(spec)
+        dv = to_dev(x)
+        dims = dims_for(spec, x)
+        bufs = pa.allocate(dims)
+        pa.step(dv["query"], dv["key"], dv["value"], dv["key_cache"], dv["value_cache"],
+                dv["block_table"], dv["cu_seqlens_q"], dv["seqlens_kv"], 0.0, dims, bufs)
+        torch.cuda.synchronize()
+        runs.append((spec, dv, dims, bufs, host_bits(bufs.out, spec.elem)))
+    errors = []
+
+    def worker(i):
+        try:
+            spec, dv, dims, bufs, ref = runs[i]
+            s = torch.cuda.Stream()
+            outs = []
+            with torch.cuda.stream(s):
+                for _ in range(20):
+                    pa.pa_attention(dv["query"], dv["key_cache"], dv["value_cache"], dv["block_table"],
+                                    dv["cu_seqlens_q"], dv["seqlens_kv"], 0.0, bufs.out, dims,
+                                    bufs.workspace, None, bufs.status, s)
+                    outs.append(bufs.out.clone())
+            s.synchronize()
+            for o in outs:
+                if not np.array_equal(host_bits(o, spec.elem).view(np.uint16), ref.view(np.uint16)):
+                    errors.append(f"thread {i}: result differs")
+                    break
+            if int(bufs.status[0].item()) != 0:
+                errors.append(f"thread {i}: status {int(bufs.status[0].item()):#x}")
+        except Exception as e:          # noqa: BLE001 -- reported below
+            errors.append(f"thread {i}: {e!r}")
+
+    threads = [threading.Thread(target=worker, args=(i,)) for i in range(2)]
+    for t in threads:
+        t.start()
+    for t in threads:
+        t.join()
+    assert not errors, errors
