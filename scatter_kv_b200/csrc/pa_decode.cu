@@ -97,6 +97,7 @@ struct Cfg {
     // pass at once and read a stage whose previous tile is still in use.)
     static constexpr int NST = 4;
     static_assert(NST % NG == 0, "each stage must belong to one consumer group");
+    static_assert(NST % NCW == 0, "with one-warp groups too (short sequences in two-row-tile builds)");
     static constexpr int NPW = CPA ? 4 : 1;             // producer warps (cp.async: a warpgroup)
     static constexpr int THREADS = 32 * (NCW + NPW);
     // setmaxnreg (cp.async path) acts on whole warpgroups: consumers are one,
@@ -508,8 +509,15 @@ decode_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ 
             if (HEAD <= 128) asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(kQ4RegsCons));
         }
         else if (CPA) asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(dec_regs_cons<HEAD>()));
-        const int mt = warp % MT;          // which 16 query rows
-        const int grp = warp / MT;         // which tiles
+        // Groups: MT warps (one per 16 query rows) share every NG-th tile.  When
+        // a two-row-tile build meets a sequence of at most 16 rows, every warp
+        // takes the 16 rows and tiles of its own (NCW groups of one warp; each
+        // stage still belongs to one group, NST being a multiple of NCW).
+        const bool shortq = MT > 1 && R <= 16;
+        const int mt = shortq ? 0 : warp % MT;             // which 16 query rows
+        const int grp = shortq ? warp : warp / MT;         // which tiles
+        const int ng = shortq ? C::NCW : C::NG;            // groups
+        const int gst = shortq ? 16 : C::RMAX;             // a group's row stride in the merge
         const int quad = lane >> 2, qid = lane & 3;
         // Rows held by this thread: r0 = mt*16 + quad, r1 = r0 + 8.
         int rows[2] = {mt * 16 + quad, mt * 16 + quad + 8};
@@ -580,7 +588,7 @@ decode_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ 
         // A split with a bad block id runs no tile: its rows come out as zero
         // when the sequence has one split; otherwise it writes an lse of +inf,
         // on which the combine zeroes the sequence's rows.
-        for (int t = split_bad ? ntiles : grp; t < ntiles; t += C::NG) {
+        for (int t = split_bad ? ntiles : grp; t < ntiles; t += ng) {
             const int st = t % C::NST, u = t / C::NST;
             if (!mbar_wait_warp(&full[st], u & 1)) {
                 flag_status(p.status, PA_DEV_TIMEOUT);
@@ -743,7 +751,7 @@ decode_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ 
                 }
             }
             __syncwarp();
-            if (lane == 0) mbar_arrive(&empty[st]);
+            if (lane == 0) mbar_arrive_cnt(&empty[st], shortq ? MT : 1);
         }
 
         // ---------------------------------------------------- merge the groups
@@ -756,8 +764,8 @@ decode_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ 
         if (qid == 0) {
 #pragma unroll
             for (int h = 0; h < 2; ++h) {
-                red_m[grp * C::RMAX + rows[h]] = m_run[h];
-                red_l[grp * C::RMAX + rows[h]] = l_run[h];
+                red_m[grp * gst + rows[h]] = m_run[h];
+                red_l[grp * gst + rows[h]] = l_run[h];
             }
         }
         asm volatile("bar.sync 1, %0;" ::"r"(C::NCW * 32));
@@ -766,26 +774,26 @@ decode_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ 
         for (int h = 0; h < 2; ++h) {
             const int r = rows[h];
             float M = -INFINITY;
-            for (int gg = 0; gg < C::NG; ++gg) M = fmaxf(M, red_m[gg * C::RMAX + r]);
+            for (int gg = 0; gg < ng; ++gg) M = fmaxf(M, red_m[gg * gst + r]);
             const float base = (M == -INFINITY) ? 0.f : M;
             const float f = fast_exp2(m_run[h] - base);
             if (grp == 0 && qid == 0) {
                 float L = 0.f;
-                for (int gg = 0; gg < C::NG; ++gg)
-                    L += red_l[gg * C::RMAX + r] * fast_exp2(red_m[gg * C::RMAX + r] - base);
+                for (int gg = 0; gg < ng; ++gg)
+                    L += red_l[gg * gst + r] * fast_exp2(red_m[gg * gst + r] - base);
                 row_l[r] = L;
                 row_m[r] = M;
             }
             if constexpr (Q4) {
                 // Positions 2 qid, 2 qid + 1 of each 8 hold channels qid, qid + 4.
-                float* dst = scr + (grp * C::RMAX + r) * C::OST + qid;
+                float* dst = scr + (grp * gst + r) * C::OST + qid;
 #pragma unroll
                 for (int i = 0; i < HEAD / 8; ++i) {
                     dst[i * 8] = oacc[i][2 * h] * f;
                     dst[i * 8 + 4] = oacc[i][2 * h + 1] * f;
                 }
             } else {
-                float* dst = scr + (grp * C::RMAX + r) * C::OST + 2 * qid;
+                float* dst = scr + (grp * gst + r) * C::OST + 2 * qid;
 #pragma unroll
                 for (int i = 0; i < HEAD / 8; ++i) {
                     float2 v = make_float2(oacc[i][2 * h] * f, oacc[i][2 * h + 1] * f);
@@ -800,8 +808,8 @@ decode_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ 
             const int r = idx / (HEAD / 4), d4 = (idx % (HEAD / 4)) * 4;
             if (direct && d4 >= hs) continue;
             float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
-            for (int gg = 0; gg < C::NG; ++gg) {
-                const float4 v = *reinterpret_cast<const float4*>(scr + (gg * C::RMAX + r) * C::OST + d4);
+            for (int gg = 0; gg < ng; ++gg) {
+                const float4 v = *reinterpret_cast<const float4*>(scr + (gg * gst + r) * C::OST + d4);
                 acc.x += v.x; acc.y += v.y; acc.z += v.z; acc.w += v.w;
             }
             const float L = row_l[r];

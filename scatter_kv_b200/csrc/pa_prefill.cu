@@ -480,6 +480,7 @@ prefill_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
             const int np0 = (min(kbase + C::BN, T) - kbase + bs - 1) / bs;
             next_ids = lane < np0 ? bt[(kbase >> lbs) + lane] : 0;   // tile 0's ids at u = 0
         }
+        CpAsyncArrivals arr;
         for (int u = CPA ? 0 : 1; u < 2 * nrel; ++u) {
             const int st = u % C::NS;
             const bool is_v = (u & 1) != 0;
@@ -523,7 +524,7 @@ prefill_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
                             for (int k = 0; k < UPL; ++k) cp_async16(sv + usoff[k], src + k * ustep);
                         }
                     }
-                    cp_async_arrive(&full[st]);
+                    arr.item_done(full, st);
                     continue;
                 }
 #pragma unroll 2
@@ -543,13 +544,12 @@ prefill_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
                     }
                 }
                 if (tail) {
-                    // Zero stores are generic-proxy writes: land the copies, make
-                    // both visible to the tensor core, then arrive.
-                    cp_async_wait_all();
-                    fence_proxy_async_smem();
+                    // Zero stores are generic-proxy writes too: land everything,
+                    // fence, then arrive.
+                    arr.flush(full);
                     mbar_arrive(&full[st]);
                 } else {
-                    cp_async_arrive(&full[st]);
+                    arr.item_done(full, st);
                 }
                 continue;
             }
@@ -593,7 +593,7 @@ prefill_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
                 if (lane == 0) mbar_arrive_cnt(&full[st], C::NPROD);
             }
         }
-        if (CPA) cp_async_wait_all();
+        if (CPA) arr.flush(full);
     } else if (warp == C::WARP_MMA) {
         // -------------------------------------------------------------- MMA issuer
         regs_dec<C::REGS_OTHER>();

@@ -333,6 +333,7 @@ prefill256_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
             const int c = __shfl_sync(0xffffffffu, w_prev, (page - wb) & 31);
             return page >= wb ? a : c;
         };
+        CpAsyncArrivals arr;
         for (int u = 0; u < nitems; ++u) {
             int j;
             bool is_v;
@@ -368,7 +369,7 @@ prefill256_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
                                 cp_async16(sv + swz<C::RB>(usoff0 + (uint32_t)(k * C::RB)), src + k * row_bytes);
                         }
                     }
-                    cp_async_arrive(&full[st]);
+                    arr.item_done(full, st);
                     continue;
                 }
                 // The tile holding T: row by row, lane l holding the block id
@@ -391,11 +392,12 @@ prefill256_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
                     }
                 }
                 if (tail) {
-                    cp_async_wait_all();
-                    fence_proxy_async_smem();
+                    // Zero stores are generic-proxy writes too: land everything,
+                    // fence, then arrive.
+                    arr.flush(full);
                     mbar_arrive(&full[st]);
                 } else {
-                    cp_async_arrive(&full[st]);
+                    arr.item_done(full, st);
                 }
                 continue;
             }
@@ -433,7 +435,7 @@ prefill256_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
                 if (lane == 0) mbar_arrive_cnt(&full[st], C::NPROD);
             }
         }
-        if (CPA) cp_async_wait_all();
+        if (CPA) arr.flush(full);
     } else if (warp == C::WARP_MMA) {
         // -------------------------------------------------------------- MMA issuer
         if (lane == 0) {
