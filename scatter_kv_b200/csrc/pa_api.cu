@@ -348,16 +348,16 @@ pa_status attention_impl(const void* query, const void* key_cache, const void* v
     PA_REQUIRE_IPTR(block_table);
     PA_REQUIRE_IPTR(cu_seqlens_q);
     PA_REQUIRE_IPTR(seqlens_kv);
-    {
-        const cudaError_t e = ensure_context();
-        if (e != cudaSuccess) return cuda_fail(e, "no CUDA context for the calling thread");
-    }
     const int nsm = num_sms_of_current_device();
     const pa::DecodePlan plan = pa::plan_decode(d, nsm);
     if (workspace_bytes < plan.workspace_bytes)
         return fail(PA_ERR_INVALID_ARGUMENT, "workspace of %zu bytes is smaller than the %zu needed",
                     workspace_bytes, plan.workspace_bytes);
     if (plan.workspace_bytes > 0) PA_REQUIRE_PTR(workspace);
+    {
+        const cudaError_t e = ensure_context();
+        if (e != cudaSuccess) return cuda_fail(e, "no CUDA context for the calling thread");
+    }
     if (scale == 0.f) scale = 1.f / sqrtf((float)d.head_size);
     pa::ScoreMods mods{};
     mods.scale = scale;
