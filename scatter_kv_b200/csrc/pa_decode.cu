@@ -668,8 +668,8 @@ decode_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ 
                 grow[h] = mx[h] > m_run[h] + 8.f;
             }
             if constexpr (Q4) {
-                // INT4 build: the base follows the max on every tile (the lazy
-                // form costs this build spills).
+                // INT4 instantiation: the base follows the max on every tile
+                // (there the lazy form spills registers).
                 float alpha[2];
 #pragma unroll
                 for (int h = 0; h < 2; ++h) {
