@@ -73,7 +73,8 @@ enum {
  * head_size a multiple of 8 in [8, 256] (the kernels are built for 16, 32,
  * 64, 128 and 256 columns; other sizes run in the next larger build, their
  * extra columns zero); block_size a power of two in [16, 256]; q_heads a
- * multiple of kv_heads with q_heads / kv_heads <= 32;
+ * multiple of kv_heads with q_heads / kv_heads <= 128 (groups above 32 run
+ * every sequence, decode ones included, in the prefill kernel);
  * num_blocks * block_size < 2^31.
  * The hints are optional upper bounds (0 = unknown): max_seqlen_q_hint
  * bounds every q_len_b, max_seqlen_kv_hint every seqlens_kv[b].  They size

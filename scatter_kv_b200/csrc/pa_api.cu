@@ -168,8 +168,9 @@ pa_status check_dims(const pa_dims* dp) {
         return fail(PA_ERR_INVALID_ARGUMENT, "q_heads (%d) must be a positive multiple of kv_heads (%d)",
                     d.q_heads, d.kv_heads);
     const int g = d.q_heads / d.kv_heads;
-    if (g > 32)
-        return fail(PA_ERR_NOT_IMPLEMENTED, "q_heads / kv_heads = %d: groups up to 32 are built", g);
+    if (g > pa::kPrefillRows)
+        return fail(PA_ERR_NOT_IMPLEMENTED, "q_heads / kv_heads = %d: groups up to %d are built", g,
+                    pa::kPrefillRows);
     if (d.head_size <= 0 || d.head_size % 8 != 0 || d.head_size > 256)
         return fail(PA_ERR_INVALID_ARGUMENT, "head_size %d must be a multiple of 8 in [8, 256]",
                     d.head_size);
@@ -375,7 +376,7 @@ pa_status attention_impl(const void* query, const void* key_cache, const void* v
     // Decode (split-KV) part: sequences with q_len <= plan.decode_max_q.  A
     // lower bound on q_len above the cut-off sends every sequence to the
     // prefill kernel instead (it handles any q_len), and no decode runs.
-    const bool run_decode = d.min_seqlen_q_hint <= plan.decode_max_q;
+    const bool run_decode = plan.decode_max_q > 0 && d.min_seqlen_q_hint <= plan.decode_max_q;
     const int prefill_min_q = run_decode ? plan.decode_max_q : 0;   // prefill takes q_len > this
     const bool run_prefill = d.max_seqlen_q_hint == 0 || d.max_seqlen_q_hint > prefill_min_q;
     auto decode_part = [&](cudaStream_t s) -> pa_status {
@@ -740,6 +741,8 @@ pa_status pa_sparse_attention(const void* query, const void* key_cache, const vo
     if (d.softcap > 0.f || d.local_window)
         return fail(PA_ERR_NOT_IMPLEMENTED,
                     "sparse attention takes its window as an argument; no softcap or dims window");
+    if (d.q_heads / d.kv_heads > 32)
+        return fail(PA_ERR_NOT_IMPLEMENTED, "sparse attention: groups up to 32 are built");
     if (num_selected < 0 || local_window < 0)
         return fail(PA_ERR_INVALID_ARGUMENT, "num_selected and local_window must be >= 0");
     if ((long long)num_selected + local_window + 1 > pa::kSparseMaxKeys)

@@ -974,6 +974,15 @@ cudaError_t launch_decode_d(const CUtensorMap& tm_k, const CUtensorMap& tm_v, co
 DecodePlan plan_decode(const pa_dims& d, int num_sms) {
     DecodePlan pl{};
     const int g = d.q_heads / d.kv_heads;
+    if (g > 32) {
+        // A query row block of more than 32 rows per KV head does not fit the
+        // decode tile: every sequence goes to the prefill kernel.
+        pl.decode_max_q = 0;
+        pl.mtiles = 1;
+        pl.chunk = kDecodeKeys;
+        pl.max_splits = 1;
+        return pl;
+    }
     int dq = kDecodeMaxQ;
     if (32 / g < dq) dq = 32 / g;
     if (d.max_seqlen_q_hint > 0 && d.max_seqlen_q_hint < dq) dq = d.max_seqlen_q_hint;

@@ -52,7 +52,7 @@ FAKE = 1 << 20          # aligned non-null address; never dereferenced (calls fa
 
 @pytest.mark.parametrize("kw,status", [
     (dict(q_heads=6, kv_heads=4), 1),            # not a multiple
-    (dict(q_heads=48, kv_heads=1), 2),           # group 48: not built (decode rows <= 32)
+    (dict(q_heads=256, kv_heads=1), 2),          # group 256: not built (prefill rows <= 128)
     (dict(head_size=20), 1),                     # not a multiple of 8
     (dict(head_size=264), 1),                    # beyond 256
     (dict(softcap=-1.0), 1),

@@ -106,3 +106,15 @@ def test_cp_async_page_sizes(bs, heads, d):
     q, past = [300, 1, 700, 129, 2], [1000, 4000, 0, 517, 60]
     spec = workloads.custom(q, past, heads[0], heads[1], d, bs, seed=bs + d)
     _check(spec)
+
+
+@pytest.mark.parametrize("qh,kvh", [(48, 1), (64, 1), (128, 2), (96, 1), (128, 1)])
+@pytest.mark.parametrize("bs", [16, 256])
+def test_groups_above_32(qh, kvh, bs):
+    """Groups of more than 32 query heads per KV head (MQA with many heads):
+    every sequence, decode ones included, runs in the prefill kernel (query
+    tiles of 128 / group tokens)."""
+    q, past = [1, 3, 2, 45, 160], [1200, 30, 0, 500, 64]
+    spec = workloads.custom(q, past, qh, kvh, 128, bs, seed=qh + kvh + bs)
+    _check(spec)
+    _check(spec, hints=False)

@@ -59,7 +59,7 @@ def test_head256_softcap_and_window(bs):
     _check(spec, softcap=20.0, window=333)
 
 
-@pytest.mark.parametrize("qh,kvh", [(6, 2), (10, 2), (8, 8), (32, 1)])
+@pytest.mark.parametrize("qh,kvh", [(6, 2), (10, 2), (8, 8), (32, 1), (64, 1)])
 def test_head256_groups(qh, kvh):
     q, past = [1, 2, 45, 160], [1200, 30, 0, 500]
     spec = workloads.custom(q, past, qh, kvh, 256, 16, seed=qh * 10 + kvh)
