@@ -55,8 +55,8 @@ struct QCfg {
     static constexpr int OFF_Q = 0;
     static constexpr int OFF_RING = OFF_Q + Q_BYTES;
     static constexpr int OFF_BAR = OFF_RING + NS * KV_BYTES;
-    // q_full, full/empty x NS, s_full[2], p_full, o_ready, o_full, drain, v_tail
-    static constexpr int NBAR = 1 + 2 * NS + 2 + 1 + 1 + 1 + 1 + 1;
+    // q_full, full/empty x NS, s_full[2], p_full[2], o_ready, o_full, drain, v_tail
+    static constexpr int NBAR = 1 + 2 * NS + 2 + 2 + 1 + 1 + 1 + 1;
     static constexpr int SMEM = OFF_BAR + NBAR * 8 + 64;
     static constexpr int THREADS = 256;
     static constexpr int WARP_SETUP = 4, WARP_MMA = 5;
@@ -149,8 +149,12 @@ prefill256_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
     uint64_t* full = q_full + 1;             // [NS]
     uint64_t* empty = full + C::NS;          // [NS]
     uint64_t* s_full = empty + C::NS;        // [2] S of a buffer ready
-    uint64_t* p_full = s_full + 2;           // P of the current tile written (4 warps)
-    uint64_t* o_ready = p_full + 1;          // a P V product done (one phase per tile)
+    // [2] P of tile j written by the 4 softmax warps, in p_full[j % 2]: with S
+    // double-buffered a warp may finish tile j + 1 before a slower one finishes
+    // tile j, so consecutive tiles count on different barriers (tile j + 2 needs
+    // S_{j+2}, which comes after P_j V_j: no warp gets two tiles ahead).
+    uint64_t* p_full = s_full + 2;
+    uint64_t* o_ready = p_full + 2;          // a P V product done (one phase per tile)
     uint64_t* o_full = o_ready + 1;          // the last P V done
     uint64_t* drain = o_full + 1;
     uint64_t* v_tail = drain + 1;
@@ -185,7 +189,8 @@ prefill256_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
             }
             mbar_init(&s_full[0], 1);
             mbar_init(&s_full[1], 1);
-            mbar_init(p_full, 4);
+            mbar_init(&p_full[0], 4);
+            mbar_init(&p_full[1], 4);
             mbar_init(o_ready, 1);
             mbar_init(o_full, 1);
             mbar_init(drain, 1);
@@ -476,7 +481,7 @@ prefill256_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
             }
             for (int j = 0; alive && j < nt; ++j) {
                 const int buf = j & 1;
-                if (!qwait<!CPA>(p_full, j & 1)) { alive = false; break; }
+                if (!qwait<!CPA>(&p_full[j & 1], (j >> 1) & 1)) { alive = false; break; }
                 if (!qwait<!CPA>(&full[u % C::NS], (u / C::NS) & 1)) { alive = false; break; }
                 tc_fence_after();
                 issue_pv(buf, u % C::NS, j == 0);
@@ -602,7 +607,7 @@ prefill256_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
             tmem_wait_st();
             tc_fence_before();
             __syncwarp();
-            if (lane == 0) mbar_arrive(p_full);
+            if (lane == 0) mbar_arrive(&p_full[buf]);
         }
         // Epilogue: O / l -> the row of `out` (its first hs columns).
         if (alive && nt > 0 && mbar_wait_warp_lean(o_full, 0)) {
