@@ -60,3 +60,56 @@ def test_profile_hash_covers_only_the_kernels_sources(tmp_path, monkeypatch):
     assert bench.kernel_source_hash(files) == h0
     (csrc / "pa_common.cuh").write_text("int changed;\n")
     assert bench.kernel_source_hash(files) != h0
+
+
+def test_committed_profiles_are_well_formed():
+    """Every ncu summary under profiles/ names a kernel the bench reports,
+    records the source hash and the DRAM traffic the bench reads, and gives
+    commands with --clock-control none.  (Whether the hash still matches the
+    kernel's sources is the bench's business: it reports no traffic then.)"""
+    import os
+    import re
+    pdir = os.path.join(bench.ROOT, "profiles")
+    names = sorted(f for f in os.listdir(pdir) if f.endswith(".md"))
+    assert names
+    for f in names:
+        assert any(f.startswith(k + "_") for k in bench.KERNEL_SOURCES if "@" not in k), f
+        text = open(os.path.join(pdir, f)).read()
+        assert re.search(r"source_hash:\s*[0-9a-f]{16}", text), f
+        assert re.search(r"traffic_bytes_per_launch:\s*[0-9.]+", text), f
+        for line in text.splitlines():
+            if line.startswith("ncu "):
+                assert "--clock-control none" in line, (f, line)
+
+
+def test_head256_profiles_hash_the_head256_kernel(tmp_path, monkeypatch):
+    csrc = tmp_path / "scatter_kv_b200" / "csrc"
+    csrc.mkdir(parents=True)
+    for n in ("pa_prefill.cu", "pa_prefill256.cu", "pa_common.cuh", "pa_internal.h"):
+        (csrc / n).write_text(f"int {n.split('.')[0]};\n")
+    pdir = tmp_path / "profiles"
+    pdir.mkdir()
+    monkeypatch.setattr(bench, "ROOT", str(tmp_path))
+    h = bench.kernel_source_hash(bench.KERNEL_SOURCES["prefill_tcgen05@d256"])
+    (pdir / "prefill_tcgen05_prefill_d256.md").write_text(
+        f"source_hash: {h}\ntraffic_bytes_per_launch: 123\n")
+    assert bench.profiled_traffic("prefill_tcgen05", "prefill_d256") == 123.0
+    (csrc / "pa_prefill.cu").write_text("int changed;\n")          # the 128-wide kernel: no effect
+    assert bench.profiled_traffic("prefill_tcgen05", "prefill_d256") == 123.0
+    (csrc / "pa_prefill256.cu").write_text("int changed;\n")
+    assert bench.profiled_traffic("prefill_tcgen05", "prefill_d256") is None
+
+
+def test_part_option_is_parsed():
+    seen = {}
+
+    def fake_run_gpu(args, spec, rank, world, local):
+        seen["part"], seen["only"], seen["workload"] = args.part, args.only, args.workload
+
+    orig = bench.run_gpu
+    bench.run_gpu = fake_run_gpu
+    try:
+        bench.main(["--only", "--part", "d256", "--workload", "prefill", "--steps", "1"])
+    finally:
+        bench.run_gpu = orig
+    assert seen == {"part": "d256", "only": True, "workload": "prefill"}
