@@ -158,6 +158,8 @@ CASES = [
     ([1, 1, 1], [5, 0, 17], 8, 2, 8, 8),
     ([2, 0, 3], [4, 6, 1], 4, 1, 8, 4),          # a zero-length sequence in the middle
     ([16, 4, 1], [16, 28, 63], 4, 4, 16, 16),
+    ([1, 3, 2], [9, 0, 5], 64, 1, 8, 4),          # MQA, a group of 64
+    ([2, 1], [3, 6], 96, 2, 8, 2),                # a group of 48
 ]
 
 
