@@ -345,6 +345,16 @@ pa_status pa_trace_enable(int on);
 int pa_trace_read(pa_trace_record* records, int max_records);
 const char* pa_kernel_name(int32_t kernel);
 
+/* pa_selftest_wait_timeout -- the failure path of the bounded waits, for
+ * tests.  Every mbarrier wait in the library's kernels gives up after a
+ * fixed limit (2 s), sets PA_DEV_TIMEOUT in the status word and lets its
+ * kernel return, so a lost arrival ends as a status bit, not a hang, and the
+ * CUDA context stays usable.  This call launches one small kernel on
+ * `stream` whose waits can never succeed (nothing arrives on its barrier):
+ * after about 2 s it sets PA_DEV_TIMEOUT in *dev_status and exits.  It reads
+ * and writes nothing else. */
+pa_status pa_selftest_wait_timeout(int32_t* dev_status, void* stream);
+
 #ifdef __cplusplus
 }
 #endif

@@ -92,7 +92,7 @@ EXPORTS = [
     "pa_scatter_kv", "pa_compute_slot_mapping", "pa_attention_workspace_size", "pa_attention",
     "pa_get_status", "pa_status_string", "pa_last_error", "pa_trace_enable", "pa_trace_read",
     "pa_kernel_name", "pa_attention_noalloc", "pa_split_qkv_rotary_scatter",
-    "pa_scatter_kv_int4", "pa_attention_int4", "pa_sparse_attention",
+    "pa_scatter_kv_int4", "pa_attention_int4", "pa_sparse_attention", "pa_selftest_wait_timeout",
 ]
 
 # Bytes of the fixed scratch array behind pa_attention_noalloc.
@@ -117,6 +117,8 @@ def _load():
     lib.pa_attention.restype = ctypes.c_int
     lib.pa_attention_noalloc.argtypes = [P, P, P, P, P, P, ctypes.c_float, P, D, P, P]
     lib.pa_attention_noalloc.restype = ctypes.c_int
+    lib.pa_selftest_wait_timeout.argtypes = [P, P]
+    lib.pa_selftest_wait_timeout.restype = ctypes.c_int
     lib.pa_split_qkv_rotary_scatter.argtypes = [P, P, P, ctypes.c_int64, ctypes.c_int64, P, P,
                                                 ctypes.POINTER(pa_rotary), P, P, P, P, P, P, P,
                                                 D, P, P]
@@ -312,6 +314,11 @@ def pa_get_status(dev_status, stream=None) -> int:
     code = ctypes.c_int32(0)
     _check(lib.pa_get_status(_ptr(dev_status), ctypes.byref(code), _stream(stream)))
     return int(code.value)
+
+
+def pa_selftest_wait_timeout(dev_status, stream=None) -> None:
+    """Launch the kernel whose bounded waits must time out (see the header)."""
+    _check(lib.pa_selftest_wait_timeout(_ptr(dev_status), _stream(stream)))
 
 
 def pa_trace_enable(on: bool = True) -> None:

@@ -514,6 +514,13 @@ pa_status pa_attention(const void* query, const void* key_cache, const void* val
                           scale, out, dims, workspace, workspace_bytes, dev_status, stream, true);
 }
 
+pa_status pa_selftest_wait_timeout(int32_t* dev_status, void* stream) {
+    g_last_error[0] = 0;
+    PA_REQUIRE_IPTR(dev_status);
+    const cudaError_t e = pa::launch_wait_timeout_selftest(dev_status, static_cast<cudaStream_t>(stream));
+    return e == cudaSuccess ? PA_OK : cuda_fail(e, "wait-timeout self-test launch");
+}
+
 pa_status pa_attention_noalloc(const void* query, const void* key_cache, const void* value_cache,
                                const int32_t* block_table, const int32_t* cu_seqlens_q,
                                const int32_t* seqlens_kv, float scale, void* out,

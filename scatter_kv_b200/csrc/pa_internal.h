@@ -208,6 +208,10 @@ cudaError_t noalloc_scratch(void** ptr);
 // The CUDA context current on this thread (null if none or unknown).
 CUcontext current_context();
 
+// A kernel whose three kinds of bounded mbarrier wait can never succeed:
+// each gives up after its limit and flags PA_DEV_TIMEOUT in *status.
+cudaError_t launch_wait_timeout_selftest(int32_t* status, cudaStream_t stream);
+
 cudaError_t launch_prefill(const CUtensorMap& tm_q, const CUtensorMap& tm_k,
                            const CUtensorMap& tm_v, const PrefillParams& p, int head, bool bf16,
                            cudaStream_t stream);
