@@ -108,13 +108,15 @@ typedef struct {
 /* pa_scatter_kv -- write the new tokens' keys and values into the paged caches.
  * PR "[WebGPU] Initial PagedAttention implementation (1/n)", "Description"
  * (scatter K/V into the paged cache); the cache update is in place.
- *   key, value:   [token_count, kv_heads, head_size] f16, read only.
+ *   key, value:   [token_count, kv_heads, head_size] in dims->dtype (f16 or
+ *                 bf16), read only.
  *   slot_mapping: [token_count] int32; token t goes to block slot / block_size,
  *                 row slot % block_size.  A negative slot skips the token; a
  *                 slot >= num_blocks * block_size is skipped and flagged
  *                 PA_DEV_BAD_SLOT.  Duplicate slots: which write lands is
  *                 unspecified.
- *   key_cache, value_cache: [num_blocks, block_size, kv_heads, head_size] f16,
+ *   key_cache, value_cache: [num_blocks, block_size, kv_heads, head_size] in
+ *                 dims->dtype,
  *                 updated in place.
  * token_count == 0 is a valid no-op.  Bytes are copied unchanged. */
 pa_status pa_scatter_kv(const void* key, const void* value, const int32_t* slot_mapping,
@@ -195,13 +197,13 @@ pa_status pa_attention_workspace_size(const pa_dims* dims, size_t* bytes);
  * implementation (1/n)", "FlashAttention: optional seqlens_q input": query i
  * of sequence b (q_len_b = cu_seqlens_q[b+1] - cu_seqlens_q[b]) attends to
  * logical key positions [0, seqlens_kv[b] - q_len_b + i].
- *   query: [token_count, q_heads, head_size] f16, packed by sequence.
+ *   query: [token_count, q_heads, head_size] in dims->dtype, packed by sequence.
  *   key_cache, value_cache: as for pa_scatter_kv (read only here; call
  *          pa_scatter_kv first, on the same stream).  Cache rows that no
  *          sequence's visible keys map to are never used, whatever they hold.
  *   block_table, cu_seqlens_q, seqlens_kv: as for pa_compute_slot_mapping.
  *   scale: multiplier of Q K^T; 0 selects 1 / sqrt(head_size).
- *   out:   [token_count, q_heads, head_size] f16, written for every token.
+ *   out:   [token_count, q_heads, head_size] in dims->dtype, written for every token.
  *   workspace: device buffer of at least pa_attention_workspace_size() bytes
  *          (may be NULL when that is 0); contents need no initialisation.
  * Sequences with q_len_b <= 4 take the split-KV decode kernels, longer ones
