@@ -144,6 +144,20 @@ def test_workspace_size_and_undersized_workspace(pa):
     assert "workspace" in str(e.value)
     # A short maximum length needs a single split and no workspace at all.
     assert pa.pa_attention_workspace_size(_dims(pa, max_blocks_per_seq=2)) == 0
+    # Groups above 32 run no decode kernel, so they need no split workspace.
+    assert pa.pa_attention_workspace_size(_dims(pa, q_heads=64, kv_heads=1, max_blocks_per_seq=512)) == 0
+    assert pa.pa_attention_workspace_size(_dims(pa, q_heads=128, kv_heads=1, max_blocks_per_seq=512)) == 0
+
+
+def test_int4_and_sparse_reject_groups_above_32(pa):
+    d = _dims(pa, q_heads=64, kv_heads=1, head_size=128, max_seqlen_q=1)
+    with pytest.raises(pa.PagedAttentionError) as e:
+        pa.pa_attention_int4(FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, 0.0, FAKE, d, None, 0,
+                             None, 0)
+    assert e.value.status == pa.PA_ERR_NOT_IMPLEMENTED
+    with pytest.raises(pa.PagedAttentionError) as e:
+        pa.pa_sparse_attention(FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, 4, 8, 0.0, FAKE, d, None, 0)
+    assert e.value.status == pa.PA_ERR_NOT_IMPLEMENTED
 
 
 def test_status_strings(pa):
